@@ -1,0 +1,487 @@
+"""Benchmark of the fused-convolution hot path on B200.
+
+One step = one pass of both fused operations over their full-size synthetic
+workloads, inputs resident in device memory:
+
+  op A  conv2d x[128,8,384,384] (Cout 64, 3x3, stride 1, no pad) -> AvgPool2d(4)
+        -> sigmoid -> sum -> out[128]
+  op B  depthwise(K 9, stride 1, pad 4) + pointwise(256 -> 512) conv1d
+        x[32,256,4096] -> out[32,512,4096]
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fcv|reference]
+Under torchrun each rank runs its own replica of the step (the batch items are
+independent; there is no data-path collective) and rank 0 prints one JSON line
+with the whole-job throughput.  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload instead (rank 0 only).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from direct_convolution_chip_b200 import workloads as wl  # noqa: E402
+
+METRIC = "fused-conv GFLOP/s (2·MACs/s) and % of B200 roofline per config"
+UNIT = "GFLOP/s"
+SPEC_FMA_LANES_PER_SM = 128       # FP32 FMA units per SM
+SPEC_SM_MAX_MHZ = 1965.0          # clocks.max.sm
+TF32_OVER_BF16 = 1.1 / 2.25       # nominal dense TF32 : BF16 tensor throughput
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+CASE_A = wl.CONV2D_FULL
+CASE_B = wl.CONV1D_FULL
+
+
+# ----------------------------------------------------------------------------
+# work accounting (algorithmic MACs and compulsory bytes)
+# ----------------------------------------------------------------------------
+
+def macs_conv2d(N, Cin, H, W, Cout, P):
+    """MACs of the direct method: every conv output inside a pooled window, 9*Cin each."""
+    PH, PW = (H - 2) // P, (W - 2) // P
+    return N * Cout * (PH * P) * (PW * P) * Cin * 9
+
+
+def bytes_conv2d(N, Cin, H, W, Cout, P):
+    return 4 * (N * Cin * H * W + Cout * Cin * 9 + Cout + N)
+
+
+def macs_conv1d(N, C, T, O, K, s, p):
+    To = (T + 2 * p - K) // s + 1
+    return N * C * To * K + N * O * C * To
+
+
+def macs_conv1d_pointwise(N, C, T, O, K, s, p):
+    To = (T + 2 * p - K) // s + 1
+    return N * O * C * To
+
+
+def bytes_conv1d(N, C, T, O, K, s, p, bias=True):
+    To = (T + 2 * p - K) // s + 1
+    return 4 * (N * C * T + C * K + O * C + (O if bias else 0) + N * O * To)
+
+
+def case_macs(c):
+    if c.op == "conv2d":
+        return macs_conv2d(c.N, c.Cin, c.H, c.W, c.Cout, c.P)
+    return macs_conv1d(c.N, c.C, c.T, c.O, c.K, c.stride, c.pad)
+
+
+def case_bytes(c):
+    if c.op == "conv2d":
+        return bytes_conv2d(c.N, c.Cin, c.H, c.W, c.Cout, c.P)
+    return bytes_conv1d(c.N, c.C, c.T, c.O, c.K, c.stride, c.pad, c.has_bias)
+
+
+def workload_name():
+    a, b = CASE_A, CASE_B
+    return (f"conv2d x[{a.N},{a.Cin},{a.H},{a.W}] Cout {a.Cout} 3x3 -> AvgPool2d({a.P}) -> sigmoid -> sum "
+            f"+ dwsep conv1d x[{b.N},{b.C},{b.T}] K {b.K} s {b.stride} p {b.pad} -> [{b.N},{b.O},{b.T}]")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def fma_peak_tflops(props):
+    """FP32 FMA roofline from unit counts and the maximum SM clock."""
+    return props.multi_processor_count * SPEC_FMA_LANES_PER_SM * 2 * SPEC_SM_MAX_MHZ * 1e6 / 1e12
+
+
+def roofline_time_s(macs, nbytes, peak_tflops, hbm_gbs):
+    return max(2.0 * macs / (peak_tflops * 1e12), nbytes / (hbm_gbs * 1e9))
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, RuntimeError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        return self.summary()
+
+    def summary(self):
+        sm, mx, pw = [], [], []
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                pw.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(pw)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, local, backend="nccl"):
+    if world <= 1:
+        return False
+    import torch.distributed as dist
+    kw = {"timeout": datetime.timedelta(seconds=120)}
+    if backend == "nccl":
+        kw["device_id"] = torch.device("cuda", local)
+    dist.init_process_group(backend, **kw)
+    return True
+
+
+def max_over_ranks(values, use_dist, device):
+    """Element-wise max of a list of floats over all ranks."""
+    if not use_dist:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(use_dist, device=None):
+    if use_dist:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+
+def traffic_per_launch(kernel_key):
+    """DRAM bytes per launch from the committed ncu capture, or None if the
+    kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(kernel_key)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return e["bytes_per_launch"] if h == e["source_sha256"] else None
+
+
+def run_oracle_sample(budget_s=12.0):
+    """Time the CPU oracle (as it stands) on whole batch items of both workloads."""
+    import oracle
+    xa, wa, ba = wl.conv2d_inputs(CASE_A)
+    xb, dwb, pwb, bb = wl.conv1d_inputs(CASE_B)
+    xa, wa, ba = xa.numpy(), wa.numpy(), ba.numpy()
+    xb, dwb, pwb, bb = xb.numpy(), dwb.numpy(), pwb.numpy(), bb.numpy()
+    per_a = macs_conv2d(1, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout, CASE_A.P)
+    per_b = macs_conv1d(1, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K, CASE_B.stride, CASE_B.pad)
+
+    def time_a(n):
+        t = time.perf_counter()
+        oracle.conv2d_pool_sigmoid_sum(xa[:n], wa, ba, CASE_A.P)
+        return time.perf_counter() - t
+
+    def time_b(n):
+        t = time.perf_counter()
+        oracle.dwsep_conv1d(xb[:n], dwb, pwb, bb, CASE_B.stride, CASE_B.pad)
+        return time.perf_counter() - t
+
+    ta1, tb1 = time_a(1), time_b(1)
+    na = max(1, min(CASE_A.N, int(budget_s / 2 / max(ta1, 1e-3))))
+    nb = max(1, min(CASE_B.N, int(budget_s / 2 / max(tb1, 1e-3))))
+    ta, tb = time_a(na), time_b(nb)
+    flops = 2.0 * (na * per_a + nb * per_b)
+    return {"value": flops / (ta + tb) / 1e9, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"op A batch items 0..{na - 1} of {CASE_A.N} ({ta:.2f} s) + op B batch items "
+                      f"0..{nb - 1} of {CASE_B.N} ({tb:.2f} s); double-precision OpenMP loops"}
+
+
+def run_gpu(args):
+    import direct_convolution_chip_b200 as fcv
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    use_dist = init_dist(world, local)
+    lib = fcv.load()
+    props = torch.cuda.get_device_properties(device)
+
+    # Inputs: seeded synthetic data of the pages' shapes, resident in HBM.
+    xa, wa, ba = wl.conv2d_inputs(CASE_A)
+    xb, dwb, pwb, bb = wl.conv1d_inputs(CASE_B)
+    host = [t.pin_memory() for t in (xa, wa, ba, xb, dwb, pwb, bb)]
+    xa_d, wa_d, ba_d, xb_d, dwb_d, pwb_d, bb_d = [t.to(device) for t in host]
+    out_a = torch.empty((CASE_A.N,), device=device)
+    To = (CASE_B.T + 2 * CASE_B.pad - CASE_B.K) // CASE_B.stride + 1
+    out_b = torch.empty((CASE_B.N, CASE_B.O, To), device=device)
+    stream = torch.cuda.current_stream(device)
+    sp = stream.cuda_stream
+
+    import ctypes
+    P = ctypes.c_void_p
+
+    def op_a():
+        st = lib.fcv_conv2d_pool_sigmoid_sum(P(xa_d.data_ptr()), P(wa_d.data_ptr()), P(ba_d.data_ptr()),
+                                             CASE_A.N, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout, CASE_A.P,
+                                             P(out_a.data_ptr()), P(sp))
+        if st:
+            raise fcv.FcvError(st, "fcv_conv2d_pool_sigmoid_sum")
+
+    def op_b():
+        st = lib.fcv_dwsep_conv1d(P(xb_d.data_ptr()), P(dwb_d.data_ptr()), P(pwb_d.data_ptr()),
+                                  P(bb_d.data_ptr()), CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K,
+                                  CASE_B.stride, CASE_B.pad, P(out_b.data_ptr()), P(sp))
+        if st:
+            raise fcv.FcvError(st, "fcv_dwsep_conv1d")
+
+    for _ in range(args.warmup):
+        op_a()
+        op_b()
+    torch.cuda.synchronize(device)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(use_dist, device)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    time.sleep(0.2)  # let the sampler attach before the timed region
+    t_start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        op_a()
+        ev[i][1].record(stream)
+        op_b()
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    barrier(use_dist, device)
+    total_ms = t_start.elapsed_time(t_end)
+    ta_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    tb_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
+    total_ms, ta_ms, tb_ms = max_over_ranks([total_ms, ta_ms, tb_ms], use_dist, device)
+
+    # End to end through the public API with pinned host buffers.
+    e2e_steps = max(2, min(8, K // 25))
+    xa_h, wa_h, ba_h, xb_h, dwb_h, pwb_h, bb_h = host
+    for _ in range(1):
+        fcv.conv2d_pool_sigmoid_sum(xa_h, wa_h, ba_h, CASE_A.P)
+        fcv.dwsep_conv1d(xb_h, dwb_h, pwb_h, bb_h, CASE_B.stride, CASE_B.pad)
+    barrier(use_dist, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        ra = fcv.conv2d_pool_sigmoid_sum(xa_h, wa_h, ba_h, CASE_A.P)
+        rb = fcv.dwsep_conv1d(xb_h, dwb_h, pwb_h, bb_h, CASE_B.stride, CASE_B.pad)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], use_dist, device)[0]
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = ra.numel() * 4 + rb.numel() * 4
+
+    macs_a, macs_b = case_macs(CASE_A), case_macs(CASE_B)
+    bytes_a, bytes_b = case_bytes(CASE_A), case_bytes(CASE_B)
+    step_s = total_ms / K / 1e3
+    value = 2.0 * (macs_a + macs_b) * world / step_s / 1e9
+    peaks, peak_src = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    fma_peak = fma_peak_tflops(props)
+    tf32_peak = peaks["bf16_tflops"] * TF32_OVER_BF16
+    ta_s, tb_s = ta_ms / K / 1e3, tb_ms / K / 1e3
+
+    conv1d_tc = os.environ.get("FCV_BENCH_CONV1D_PATH", "auto")
+    per_op = {
+        "conv2d": {"workload": CASE_A.name, "ms": ta_s * 1e3, "gflops": 2 * macs_a / ta_s / 1e9,
+                   "macs": macs_a, "compulsory_bytes": bytes_a,
+                   "roofline_frac_fp32_fma": roofline_time_s(macs_a, bytes_a, fma_peak, hbm) / ta_s},
+        "dwsep_conv1d": {"workload": CASE_B.name, "ms": tb_s * 1e3, "gflops": 2 * macs_b / tb_s / 1e9,
+                         "macs": macs_b, "compulsory_bytes": bytes_b,
+                         "roofline_frac_fp32_fma": roofline_time_s(macs_b, bytes_b, fma_peak, hbm) / tb_s,
+                         "roofline_frac_3xtf32": roofline_time_s(
+                             macs_conv1d_pointwise(CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K,
+                                                   CASE_B.stride, CASE_B.pad),
+                             bytes_b, tf32_peak / 3.0, hbm) / tb_s},
+    }
+    dom = "conv2d" if ta_s >= tb_s else "dwsep_conv1d"
+    if dom == "conv2d":
+        achieved = 2 * macs_a / ta_s / 1e12
+        roof = {"kernel": "conv2d_direct_kernel<4,false>", "bound": "alu", "achieved": achieved,
+                "peak": fma_peak, "unit": "TFLOP/s", "frac": achieved / fma_peak,
+                "traffic": traffic_per_launch("conv2d_direct_p4"),
+                "peak_source": "148 SMs x 128 FP32 FMA lanes x 2 FLOP x 1965 MHz (spec clocks)"}
+    else:
+        achieved = 2 * macs_b / tb_s / 1e12
+        roof = {"kernel": "dwsep_conv1d", "bound": "alu", "achieved": achieved, "peak": fma_peak,
+                "unit": "TFLOP/s", "frac": achieved / fma_peak, "traffic": traffic_per_launch("dwsep_conv1d"),
+                "peak_source": "148 SMs x 128 FP32 FMA lanes x 2 FLOP x 1965 MHz (spec clocks)"}
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": workload_name(), "l2": "inputs larger than L2 (x 604 MB and 134 MB, out 268 MB); "
+                   "no flush", "parallelism": f"replicas x{world} (independent batches, no collective)",
+                   "conv1d_path": conv1d_tc},
+        "per_op": per_op, "roofline": roof,
+        "peaks": {"hbm_gbs": hbm, "fp32_fma_tflops": fma_peak, "tf32_tflops": tf32_peak, "source": peak_src},
+        "e2e": {"value": 2.0 * (macs_a + macs_b) * world / (e2e_ms / 1e3) / 1e9, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "steps": e2e_steps},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = run_oracle_sample()
+    if use_dist:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# the reference arm: the CPU oracle on a bounded sample per step
+# ----------------------------------------------------------------------------
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    xa, wa, ba = wl.conv2d_inputs(CASE_A)
+    xb, dwb, pwb, bb = wl.conv1d_inputs(CASE_B)
+    xa, wa, ba = xa.numpy(), wa.numpy(), ba.numpy()
+    xb, dwb, pwb, bb = xb.numpy(), dwb.numpy(), pwb.numpy(), bb.numpy()
+    # Per step: one batch item of each op, restricted to the first m output
+    # channels so that warm-up + timed steps end within a few minutes.
+    budget = min(1.5, 150.0 / max(1, args.steps + args.warmup))
+
+    def step(i, ca, cb):
+        na, nb = i % CASE_A.N, i % CASE_B.N
+        oracle.conv2d_pool_sigmoid_sum(xa[na:na + 1], wa[:ca], ba[:ca], CASE_A.P)
+        oracle.dwsep_conv1d(xb[nb:nb + 1], dwb, pwb[:cb], bb[:cb], CASE_B.stride, CASE_B.pad)
+
+    t = time.perf_counter()
+    step(0, 4, 16)
+    t1 = time.perf_counter() - t
+    scale = max(1.0, budget / max(t1, 1e-4))
+    ca = int(min(CASE_A.Cout, max(1, 4 * scale)))
+    cb = int(min(CASE_B.O, max(1, 16 * scale)))
+    for i in range(args.warmup):
+        step(i, ca, cb)
+    t = time.perf_counter()
+    for i in range(args.steps):
+        step(i, ca, cb)
+    dt = time.perf_counter() - t
+    macs = (macs_conv2d(1, CASE_A.Cin, CASE_A.H, CASE_A.W, ca, CASE_A.P)
+            + macs_conv1d(1, CASE_B.C, CASE_B.T, cb, CASE_B.K, CASE_B.stride, CASE_B.pad))
+    value = 2.0 * macs * args.steps / dt / 1e9
+    sample = (f"per step: op A on 1 batch item with {ca} of {CASE_A.Cout} output channels, op B on 1 batch "
+              f"item with {cb} of {CASE_B.O} output channels")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(), "parallelism": "CPU oracle, rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["fcv", "reference"], default="fcv")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

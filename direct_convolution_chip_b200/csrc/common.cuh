@@ -1,0 +1,50 @@
+// common.cuh -- internals shared by the libfcv kernels (one translation unit).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fcv.h"
+
+namespace fcv {
+
+// Device error word of the current device.  A kernel whose bounded wait runs
+// out ORs a code in here and returns early; fcv_device_error() reads and
+// clears it.  Nothing in the library traps or faults on purpose.
+__device__ unsigned int g_device_error;
+
+constexpr unsigned int kErrTimeout = 1u;
+
+__device__ __forceinline__ void record_device_error(unsigned int code)
+{
+    atomicOr(&g_device_error, code);
+}
+
+// Sum of `v` over a thread block, valid in thread 0.  `scratch` holds one
+// float per warp.
+template <int NT>
+__device__ __forceinline__ float block_sum(float v, float* scratch)
+{
+    static_assert(NT % 32 == 0, "block size must be a multiple of 32");
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    float s = 0.f;
+    if (threadIdx.x < 32) {
+        s = (lane < NT / 32) ? scratch[lane] : 0.f;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    }
+    return s;
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline int launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? FCV_OK : FCV_ERR_CUDA;
+}
+
+}  // namespace fcv

@@ -1,0 +1,221 @@
+// conv2d_direct.cuh -- op A on FP32 FMA: conv2d 3x3 -> AvgPool2d(P) -> sigmoid -> sum.
+//
+// Method (POPCORNBENCH trace "Kimi-K2.6__l2_p65", tile-fusion design and final
+// kernel): every pooled value is the mean of the P x P conv outputs of its
+// window, and the windows do not overlap, so computing the conv only inside
+// the windows does the same work as conv-then-pool while the conv output never
+// leaves registers.  The bias is added once per pooled value (mean(conv + b) =
+// mean(conv) + b, the bias-folding step of the same trace).  Rows and columns
+// past PH*P / PW*P are never computed (floor pooling drops them).
+//
+// B200 design:
+//   * One CTA covers a TPH x (TPW*RX) tile of pooled outputs for a block of
+//     CB = CG*NCH output channels of one image.  Its input halo
+//     [ICC][P*TPH+2][P*TPW*RX+2] is staged in shared memory (zero-filled past
+//     the image) one chunk of ICC input channels at a time.
+//   * Each thread owns RX adjacent pooled positions for CG channels.  It keeps
+//     its (P+2) x (RX*P+2) input patch in registers and, per 3x3 tap, the CG
+//     weights of that tap (a broadcast shared-memory read), then issues
+//     P*P*RX*CG independent FMAs -- consecutive FMAs update different
+//     accumulators, so the FMA pipe is not stalled on a dependency chain.
+//   * Epilogue: mean + bias, sigmoid (CUDA expf), a warp-shuffle + shared
+//     memory block sum, and one atomicAdd per CTA into out[n].
+#pragma once
+
+#include "common.cuh"
+
+namespace fcv {
+
+template <int P>
+struct Conv2dTile;
+
+// (RX, CG, TPH, TPW, NCH, ICC) per pool size: register patch + accumulators
+// stay well under 128 registers; halo + weights stay under ~60 KB so several
+// CTAs share an SM.
+template <> struct Conv2dTile<1> { static constexpr int RX = 4, CG = 16, TPH = 16, TPW = 8,  NCH = 2, ICC = 8; };
+template <> struct Conv2dTile<2> { static constexpr int RX = 2, CG = 16, TPH = 8,  TPW = 8,  NCH = 4, ICC = 8; };
+template <> struct Conv2dTile<3> { static constexpr int RX = 1, CG = 16, TPH = 8,  TPW = 8,  NCH = 4, ICC = 8; };
+template <> struct Conv2dTile<4> { static constexpr int RX = 1, CG = 16, TPH = 8,  TPW = 8,  NCH = 4, ICC = 8; };
+template <> struct Conv2dTile<5> { static constexpr int RX = 1, CG = 8,  TPH = 4,  TPW = 8,  NCH = 4, ICC = 4; };
+template <> struct Conv2dTile<6> { static constexpr int RX = 1, CG = 8,  TPH = 4,  TPW = 8,  NCH = 4, ICC = 4; };
+template <> struct Conv2dTile<7> { static constexpr int RX = 1, CG = 8,  TPH = 4,  TPW = 8,  NCH = 4, ICC = 4; };
+template <> struct Conv2dTile<8> { static constexpr int RX = 1, CG = 8,  TPH = 4,  TPW = 8,  NCH = 4, ICC = 2; };
+
+template <int P>
+struct Conv2dGeom {
+    using T = Conv2dTile<P>;
+    static constexpr int RX = T::RX, CG = T::CG, TPH = T::TPH, TPW = T::TPW, NCH = T::NCH, ICC = T::ICC;
+    static constexpr int NPOS = TPH * TPW;          // threads per channel group
+    static constexpr int NT = NPOS * NCH;           // threads per CTA
+    static constexpr int CB = CG * NCH;             // output channels per CTA
+    static constexpr int TILE_PH = TPH;             // pooled rows per CTA
+    static constexpr int TILE_PW = TPW * RX;        // pooled cols per CTA
+    static constexpr int HY = P * TILE_PH + 2;      // halo rows
+    static constexpr int HX = P * TILE_PW + 2;      // halo cols
+    static constexpr int HXP = (HX + 3) & ~3;       // halo row pitch (16-byte rows)
+    static constexpr int PY = P + 2;                // register patch rows
+    static constexpr int PX = RX * P + 2;           // register patch cols
+    static constexpr int HALO_FLOATS = ICC * HY * HXP;
+    static constexpr int W_FLOATS = ICC * 9 * CB;
+    static constexpr size_t SMEM_BYTES = sizeof(float) * (HALO_FLOATS + W_FLOATS + NT / 32);
+};
+
+template <int P, bool TAP>
+__global__ void __launch_bounds__(Conv2dGeom<P>::NT, 2)
+conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
+                     const float* __restrict__ bias, int Cin, int H, int W, int Cout,
+                     int PH, int PW, int tiles_y, int tiles_x, float* __restrict__ out)
+{
+    using G = Conv2dGeom<P>;
+    constexpr int RX = G::RX, CG = G::CG, NPOS = G::NPOS, NT = G::NT, CB = G::CB;
+    constexpr int HY = G::HY, HX = G::HX, HXP = G::HXP, PY = G::PY, PX = G::PX, ICC = G::ICC;
+
+    extern __shared__ __align__(16) float smem[];
+    float* halo = smem;                      // [ICC][HY][HXP]
+    float* ws = smem + G::HALO_FLOATS;       // [ICC][9][CB]
+    float* red = ws + G::W_FLOATS;           // [NT/32]
+
+    int tile = blockIdx.x;
+    const int tx_tile = tile % tiles_x;
+    tile /= tiles_x;
+    const int ty_tile = tile % tiles_y;
+    const int n = tile / tiles_y;
+    const int c_base = blockIdx.y * CB;
+    const int ph0 = ty_tile * G::TILE_PH, pw0 = tx_tile * G::TILE_PW;
+    const int y0 = ph0 * P, x0 = pw0 * P;
+
+    const int tid = threadIdx.x;
+    const int grp = tid / NPOS, pos = tid % NPOS;
+    const int ty = pos / G::TPW, tx = pos % G::TPW;
+
+    float acc[RX][CG];
+#pragma unroll
+    for (int r = 0; r < RX; ++r)
+#pragma unroll
+        for (int c = 0; c < CG; ++c) acc[r][c] = 0.f;
+
+    const float* xn = x + (size_t)n * Cin * H * W;
+
+    for (int ic0 = 0; ic0 < Cin; ic0 += ICC) {
+        // Stage the halo of this input-channel chunk (zero past the image and past Cin).
+        for (int i = tid; i < ICC * HY * HX; i += NT) {
+            const int icl = i / (HY * HX);
+            const int rem = i - icl * (HY * HX);
+            const int r = rem / HX, s = rem - (rem / HX) * HX;
+            const int ic = ic0 + icl, yy = y0 + r, xx = x0 + s;
+            float v = 0.f;
+            if (ic < Cin && yy < H && xx < W) v = __ldg(xn + ((size_t)ic * H + yy) * W + xx);
+            halo[(icl * HY + r) * HXP + s] = v;
+        }
+        // Stage the weights as [icl][tap][c_local] so a thread's CG channels of one tap are contiguous.
+        for (int i = tid; i < ICC * 9 * CB; i += NT) {
+            const int cl = i % CB;
+            const int tap = (i / CB) % 9;
+            const int icl = i / (9 * CB);
+            const int c = c_base + cl, ic = ic0 + icl;
+            ws[i] = (c < Cout && ic < Cin) ? __ldg(w + ((size_t)c * Cin + ic) * 9 + tap) : 0.f;
+        }
+        __syncthreads();
+
+        const int nic = min(ICC, Cin - ic0);
+        for (int icl = 0; icl < nic; ++icl) {
+            float patch[PY][PX];
+            const float* hp = halo + (icl * HY + ty * P) * HXP + tx * (RX * P);
+#pragma unroll
+            for (int r = 0; r < PY; ++r)
+#pragma unroll
+                for (int s = 0; s < PX; ++s) patch[r][s] = hp[r * HXP + s];
+
+            const float* wp = ws + icl * 9 * CB + grp * CG;
+#pragma unroll
+            for (int ky = 0; ky < 3; ++ky) {
+#pragma unroll
+                for (int kx = 0; kx < 3; ++kx) {
+                    float wr[CG];
+#pragma unroll
+                    for (int c = 0; c < CG; c += 4) {
+                        const float4 v = *reinterpret_cast<const float4*>(wp + (ky * 3 + kx) * CB + c);
+                        wr[c] = v.x; wr[c + 1] = v.y; wr[c + 2] = v.z; wr[c + 3] = v.w;
+                    }
+#pragma unroll
+                    for (int rx = 0; rx < RX; ++rx)
+#pragma unroll
+                        for (int dy = 0; dy < P; ++dy)
+#pragma unroll
+                            for (int dx = 0; dx < P; ++dx) {
+                                const float pv = patch[dy + ky][rx * P + dx + kx];
+#pragma unroll
+                                for (int c = 0; c < CG; ++c) acc[rx][c] = fmaf(pv, wr[c], acc[rx][c]);
+                            }
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // Epilogue: mean of the window + bias, then sigmoid and the block sum.
+    const int ph = ph0 + ty;
+    float local = 0.f;
+#pragma unroll
+    for (int rx = 0; rx < RX; ++rx) {
+        const int pw = pw0 + tx * RX + rx;
+        const bool valid = ph < PH && pw < PW;
+#pragma unroll
+        for (int c = 0; c < CG; ++c) {
+            const int cc = c_base + grp * CG + c;
+            if (valid && cc < Cout) {
+                const float avg = acc[rx][c] / (float)(P * P) + __ldg(bias + cc);
+                if (TAP) {
+                    out[(((size_t)n * Cout + cc) * PH + ph) * PW + pw] = avg;
+                } else {
+                    local += 1.0f / (1.0f + expf(-avg));
+                }
+            }
+        }
+    }
+    if (!TAP) {
+        const float total = block_sum<NT>(local, red);
+        if (tid == 0) atomicAdd(out + n, total);
+    }
+}
+
+template <int P, bool TAP>
+int launch_conv2d_direct_p(const float* x, const float* w, const float* b, int N, int Cin, int H,
+                           int W, int Cout, int PH, int PW, float* out, cudaStream_t stream)
+{
+    using G = Conv2dGeom<P>;
+    const int tiles_y = (PH + G::TILE_PH - 1) / G::TILE_PH;
+    const int tiles_x = (PW + G::TILE_PW - 1) / G::TILE_PW;
+    const long long nblk = (long long)N * tiles_y * tiles_x;
+    const int cblk = (Cout + G::CB - 1) / G::CB;
+    if (nblk > 0x7fffffffLL || cblk > 65535) return FCV_ERR_UNSUPPORTED;
+    auto kern = conv2d_direct_kernel<P, TAP>;
+    if (G::SMEM_BYTES > 48 * 1024) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)G::SMEM_BYTES) != cudaSuccess)
+            return FCV_ERR_CUDA;
+    }
+    dim3 grid((unsigned)nblk, (unsigned)cblk);
+    kern<<<grid, G::NT, G::SMEM_BYTES, stream>>>(x, w, b, Cin, H, W, Cout, PH, PW, tiles_y, tiles_x, out);
+    return launch_status();
+}
+
+// PH, PW >= 1 here; the caller handles the empty cases.
+template <bool TAP>
+int launch_conv2d_direct(const float* x, const float* w, const float* b, int N, int Cin, int H,
+                         int W, int Cout, int P, int PH, int PW, float* out, cudaStream_t stream)
+{
+    switch (P) {
+    case 1: return launch_conv2d_direct_p<1, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
+    case 2: return launch_conv2d_direct_p<2, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
+    case 3: return launch_conv2d_direct_p<3, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
+    case 4: return launch_conv2d_direct_p<4, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
+    case 5: return launch_conv2d_direct_p<5, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
+    case 6: return launch_conv2d_direct_p<6, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
+    case 7: return launch_conv2d_direct_p<7, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
+    case 8: return launch_conv2d_direct_p<8, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
+    default: return FCV_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace fcv

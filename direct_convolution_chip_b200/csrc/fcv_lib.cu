@@ -1,0 +1,162 @@
+// fcv_lib.cu -- the extern "C" boundary of libfcv (declared in include/fcv.h).
+//
+// Host side only: argument validation (synchronous, before anything is
+// enqueued), output zeroing, algorithm dispatch and launch-status mapping.
+// Every arithmetic step of both operations runs in the kernels included below.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "conv1d_fma.cuh"
+#include "conv1d_tc.cuh"
+#include "conv2d_direct.cuh"
+
+#define FCV_VERSION_MAJOR 0
+#define FCV_VERSION_MINOR 1
+#define FCV_VERSION_PATCH 0
+
+namespace {
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// a * b * c * d without int64 overflow (all factors >= 0).
+bool mul_ok(long long a, long long b, long long c, long long d)
+{
+    const long long lim = (long long)1 << 62;
+    long long v = a;
+    for (long long f : {b, c, d}) {
+        if (f != 0 && v > lim / f) return false;
+        v *= f;
+    }
+    return true;
+}
+
+int check_conv2d(const float* x, const float* w, const float* b, int N, int Cin, int H, int W,
+                 int Cout, int pool, const float* out)
+{
+    if (!x || !w || !b || !out) return FCV_ERR_INVALID_ARG;
+    if (N < 0 || Cin < 1 || Cout < 1 || H < 3 || W < 3 || pool < 1) return FCV_ERR_INVALID_ARG;
+    if (!aligned4(x) || !aligned4(w) || !aligned4(b) || !aligned4(out)) return FCV_ERR_INVALID_ARG;
+    if (!mul_ok(N, Cin, H, W) || !mul_ok(Cout, Cin, 9, 1) || !mul_ok(N, Cout, H, W))
+        return FCV_ERR_INVALID_ARG;
+    if (pool > 8) return FCV_ERR_UNSUPPORTED;
+    return FCV_OK;
+}
+
+int check_conv1d(const float* x, const float* dw, const float* pw, const float* bias, int N, int C,
+                 int T, int O, int K, int stride, int pad, const float* out, int* To)
+{
+    if (!x || !dw || !pw || !out) return FCV_ERR_INVALID_ARG;
+    if (N < 0 || C < 1 || O < 1 || T < 1 || K < 1 || stride < 1 || pad < 0) return FCV_ERR_INVALID_ARG;
+    if (!aligned4(x) || !aligned4(dw) || !aligned4(pw) || !aligned4(out) || (bias && !aligned4(bias)))
+        return FCV_ERR_INVALID_ARG;
+    const long long span = (long long)T + 2LL * pad - K;
+    if (span < 0) return FCV_ERR_INVALID_ARG;  // To < 1
+    const long long to = span / stride + 1;
+    if (to > 0x7fffffffLL) return FCV_ERR_INVALID_ARG;
+    if (!mul_ok(N, C, T, 1) || !mul_ok(N, O, to, 1) || !mul_ok(O, C, 1, 1)) return FCV_ERR_INVALID_ARG;
+    if (K > fcv::Conv1dFmaTile::KMAX || stride > fcv::Conv1dFmaTile::SMAX || pad >= (1 << 20))
+        return FCV_ERR_UNSUPPORTED;
+    *To = (int)to;
+    return FCV_OK;
+}
+
+int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin, int H, int W,
+                  int Cout, int pool, float* out, int algo, bool tap, void* stream)
+{
+    int st = check_conv2d(x, w, b, N, Cin, H, W, Cout, pool, out);
+    if (st != FCV_OK) return st;
+    if (algo != FCV_ALGO_AUTO && algo != FCV_CONV2D_DIRECT) return FCV_ERR_INVALID_ARG;
+    if (N == 0) return FCV_OK;
+    cudaStream_t s = fcv::as_stream(stream);
+    const int PH = (H - 2) / pool, PW = (W - 2) / pool;
+    if (!tap) {
+        // The kernel accumulates one atomic add per CTA into out[n]; start from zero.
+        if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N, s) != cudaSuccess) return FCV_ERR_CUDA;
+    }
+    if (PH == 0 || PW == 0) return FCV_OK;  // empty sum: out stays 0; the tap has no elements
+    return tap ? fcv::launch_conv2d_direct<true>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
+               : fcv::launch_conv2d_direct<false>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fcv_conv2d_pool_sigmoid_sum(const float* x, const float* w, const float* b, int N, int Cin, int H,
+                                int W, int Cout, int pool, float* out, void* stream)
+{
+    return conv2d_common(x, w, b, N, Cin, H, W, Cout, pool, out, FCV_ALGO_AUTO, false, stream);
+}
+
+int fcv_conv2d_pool_sigmoid_sum_ex(const float* x, const float* w, const float* b, int N, int Cin,
+                                   int H, int W, int Cout, int pool, float* out, int algo, void* stream)
+{
+    return conv2d_common(x, w, b, N, Cin, H, W, Cout, pool, out, algo, false, stream);
+}
+
+int fcv_conv2d_pool_tap(const float* x, const float* w, const float* b, int N, int Cin, int H, int W,
+                        int Cout, int pool, float* pooled, int algo, void* stream)
+{
+    return conv2d_common(x, w, b, N, Cin, H, W, Cout, pool, pooled, algo, true, stream);
+}
+
+int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, const float* bias, int N,
+                        int C, int T, int O, int K, int stride, int pad, float* out, int algo, void* stream)
+{
+    int To = 0;
+    int st = check_conv1d(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, out, &To);
+    if (st != FCV_OK) return st;
+    if (N == 0) return FCV_OK;
+    cudaStream_t s = fcv::as_stream(stream);
+    switch (algo) {
+    case FCV_ALGO_AUTO:
+        if (fcv::conv1d_tc_supported(C, O, K, stride)) {
+            return fcv::launch_dwsep_conv1d_tc(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
+        }
+        return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
+    case FCV_CONV1D_FMA:
+        return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
+    case FCV_CONV1D_TC_3XTF32:
+        if (!fcv::conv1d_tc_supported(C, O, K, stride)) return FCV_ERR_UNSUPPORTED;
+        return fcv::launch_dwsep_conv1d_tc(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
+    default:
+        return FCV_ERR_INVALID_ARG;
+    }
+}
+
+int fcv_dwsep_conv1d(const float* x, const float* dw_w, const float* pw_w, const float* bias, int N,
+                     int C, int T, int O, int K, int stride, int pad, float* out, void* stream)
+{
+    return fcv_dwsep_conv1d_ex(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, out, FCV_ALGO_AUTO, stream);
+}
+
+const char* fcv_status_string(int status)
+{
+    switch (status) {
+    case FCV_OK: return "FCV_OK";
+    case FCV_ERR_INVALID_ARG: return "FCV_ERR_INVALID_ARG: invalid argument";
+    case FCV_ERR_UNSUPPORTED: return "FCV_ERR_UNSUPPORTED: shape outside the supported envelope";
+    case FCV_ERR_CUDA: return "FCV_ERR_CUDA: CUDA runtime error";
+    case FCV_ERR_TIMEOUT: return "FCV_ERR_TIMEOUT: a kernel's bounded wait ran out";
+    default: return "unknown fcv status";
+    }
+}
+
+int fcv_version(void)
+{
+    return FCV_VERSION_MAJOR * 10000 + FCV_VERSION_MINOR * 100 + FCV_VERSION_PATCH;
+}
+
+int fcv_device_error(void* stream)
+{
+    if (cudaStreamSynchronize(fcv::as_stream(stream)) != cudaSuccess) return FCV_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, fcv::g_device_error, sizeof(v)) != cudaSuccess) return FCV_ERR_CUDA;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(fcv::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return FCV_ERR_CUDA;
+    }
+    return (v & fcv::kErrTimeout) ? FCV_ERR_TIMEOUT : FCV_OK;
+}
+
+}  // extern "C"

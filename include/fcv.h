@@ -1,0 +1,144 @@
+/*
+ * fcv.h -- C ABI of libfcv, fused small-channel direct convolution for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Two fused operations whose intermediate never reaches device memory:
+ *
+ *   A. conv2d 3x3 (stride 1, no padding) -> AvgPool2d(P, stride P, floor)
+ *      -> sigmoid -> sum over (channels, pooled rows, pooled cols),
+ *      one fp32 scalar per batch item.
+ *      Defined on POPCORNBENCH trace "Kimi-K2.6__l2_p65" (fused Conv2d ->
+ *      AvgPool2d -> Sigmoid -> Sum), opening analysis: the conv formula
+ *      out[i,j] = sum_{c,ky,kx} in[b,c,i+ky,j+kx] * w[oc,c,ky,kx] + bias[oc],
+ *      the shapes [128,8,384,384] -> [128,64,382,382] -> [128,64,95,95] -> [128],
+ *      and the pool-semantics check (stride = kernel, floor, trailing rows and
+ *      columns dropped).
+ *
+ *   B. depthwise conv1d (kernel K, stride s, zero padding p, no bias) folded
+ *      into the pointwise 1x1 conv1d (C -> O) that consumes it, plus bias[o].
+ *      Defined on POPCORNBENCH trace "Kimi-K2.6__l2_p7" (depthwise-separable
+ *      Conv1d), opening analysis:
+ *      out[b,o,t] = sum_c ( sum_k in[b,c,t*s+k-p] * dw[c,k] ) * pw[o,c] + bias[o],
+ *      T_out = (T + 2p - K)/s + 1, input zero outside [0, T).
+ *
+ * Conventions for every compute entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; fp32,
+ *     contiguous, row-major (NCHW for op A, NCT for op B).  Inputs are read
+ *     only.  Outputs must not alias inputs.  Pointers must be 4-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Calls are asynchronous on that stream: they never synchronize
+ *     and never allocate memory.
+ *   - Argument errors are reported synchronously, before anything is
+ *     enqueued, with FCV_ERR_INVALID_ARG or FCV_ERR_UNSUPPORTED.  A launch
+ *     failure reported by the CUDA runtime returns FCV_ERR_CUDA.  Device-side
+ *     faults are never raised on purpose: a kernel whose bounded wait runs out
+ *     records FCV_ERR_TIMEOUT in a device error word (fcv_device_error) and
+ *     returns early.
+ *   - N == 0 (an empty batch) is valid and enqueues nothing.
+ *   - The library holds no per-call state; concurrent calls on different
+ *     streams with disjoint outputs are safe.
+ */
+#ifndef FCV_H
+#define FCV_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FCV_OK = 0,
+    FCV_ERR_INVALID_ARG = 1, /* null pointer, size out of domain, misaligned pointer, overflow */
+    FCV_ERR_UNSUPPORTED = 2, /* valid operation, but outside the shapes this build runs */
+    FCV_ERR_CUDA = 3,        /* the CUDA runtime reported an error at launch */
+    FCV_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (see fcv_device_error) */
+} fcv_status;
+
+/* Algorithm selectors for the *_ex entry points.  FCV_ALGO_AUTO picks the
+ * fastest path that is valid for the shape. */
+typedef enum {
+    FCV_ALGO_AUTO = 0,
+    /* op A */
+    FCV_CONV2D_DIRECT = 10,       /* direct 3x3 conv of every pooled window, FP32 FMA */
+    /* op B */
+    FCV_CONV1D_FMA = 20,          /* depthwise + pointwise on FP32 FMA */
+    FCV_CONV1D_TC_3XTF32 = 21     /* pointwise on tcgen05 tensor cores, 3xTF32 split */
+} fcv_algo;
+
+/* ---------------------------------------------------------------- op A --- */
+
+/* out[n] = sum_{c<Cout, ph<PH, pw<PW} sigmoid( avgpool_P( conv3x3(x, w) + b )[n,c,ph,pw] )
+ *
+ *   x    [N, Cin, H, W]     input
+ *   w    [Cout, Cin, 3, 3]  conv weight
+ *   b    [Cout]             conv bias (required)
+ *   out  [N]                result; fully overwritten (the library zeroes it
+ *                           on `stream` before accumulating)
+ *   pool                    AvgPool2d kernel = stride, no padding, floor mode
+ *
+ * Ho = H - 2, Wo = W - 2, PH = floor(Ho / pool), PW = floor(Wo / pool).
+ * PH == 0 or PW == 0 is valid and gives out = 0.
+ * INVALID_ARG: x, w, b or out NULL; N < 0; Cin, Cout < 1; H, W < 3; pool < 1;
+ *              element counts beyond 2^31 * 2^31; misaligned pointers.
+ * UNSUPPORTED: pool > 8.
+ * The per-batch sum is accumulated with one atomic add per thread block, so
+ * the last bits may differ between runs. */
+int fcv_conv2d_pool_sigmoid_sum(const float* x, const float* w, const float* b,
+                                int N, int Cin, int H, int W, int Cout, int pool,
+                                float* out, void* stream);
+
+int fcv_conv2d_pool_sigmoid_sum_ex(const float* x, const float* w, const float* b,
+                                   int N, int Cin, int H, int W, int Cout, int pool,
+                                   float* out, int algo, void* stream);
+
+/* The pooled pre-sigmoid values of the same kernel, for checking the conv and
+ * pool stages element by element:
+ *   pooled [N, Cout, PH, PW]  = avgpool_P( conv3x3(x, w) + b ), fully overwritten.
+ * Same arguments, errors and algorithms as fcv_conv2d_pool_sigmoid_sum_ex;
+ * nothing is summed. */
+int fcv_conv2d_pool_tap(const float* x, const float* w, const float* b,
+                        int N, int Cin, int H, int W, int Cout, int pool,
+                        float* pooled, int algo, void* stream);
+
+/* ---------------------------------------------------------------- op B --- */
+
+/* out[n,o,t] = sum_{c<C} pw_w[o,c] * ( sum_{k<K} xpad[n,c,t*stride+k-pad] * dw_w[c,k] ) + bias[o]
+ *
+ *   x     [N, C, T]   input; xpad is x with zeros outside [0, T)
+ *   dw_w  [C, K]      depthwise weight (the [C,1,K] tensor)
+ *   pw_w  [O, C]      pointwise weight (the [O,C,1] tensor)
+ *   bias  [O] or NULL (NULL: no bias)
+ *   out   [N, O, To]  To = floor((T + 2*pad - K) / stride) + 1; fully overwritten
+ *
+ * The depthwise result lives only in on-chip memory.  Every algorithm is
+ * fp32-accurate (FP32 FMA, or tensor cores through a 3xTF32 split); results
+ * are deterministic run to run.
+ * INVALID_ARG: x, dw_w, pw_w or out NULL; N < 0; C, O, T, K, stride < 1;
+ *              pad < 0; To < 1; sizes beyond the 64-bit index range;
+ *              misaligned pointers.
+ * UNSUPPORTED: K > 32, pad >= 2^20, stride > 16. */
+int fcv_dwsep_conv1d(const float* x, const float* dw_w, const float* pw_w, const float* bias,
+                     int N, int C, int T, int O, int K, int stride, int pad,
+                     float* out, void* stream);
+
+int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, const float* bias,
+                        int N, int C, int T, int O, int K, int stride, int pad,
+                        float* out, int algo, void* stream);
+
+/* -------------------------------------------------------------- utility --- */
+
+/* Human-readable name of a status code (static storage). */
+const char* fcv_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int fcv_version(void);
+
+/* Synchronizes `stream`, then returns and clears the device error word of the
+ * current device: FCV_OK, or FCV_ERR_TIMEOUT if a kernel gave up a bounded
+ * wait since the last call.  Returns FCV_ERR_CUDA if the synchronization fails. */
+int fcv_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FCV_H */

@@ -1,0 +1,106 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments synchronously before touching the
+device (these calls return before any CUDA API call)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from direct_convolution_chip_b200 import binding
+from direct_convolution_chip_b200 import build as fcv_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fcv.h")
+
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+P = ctypes.c_void_p
+FAKE = P(0x10000)     # never dereferenced: every call below returns during validation
+MISALIGNED = P(0x10002)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fcv_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fcv_build.build()
+    return binding.load()
+
+
+def test_header_declares_the_two_ops():
+    names = declared_functions()
+    assert "fcv_conv2d_pool_sigmoid_sum" in names and "fcv_dwsep_conv1d" in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.lib_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (fcv_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    assert set(binding.SIGNATURES) == set(declared_functions())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.fcv_version() >= 100
+    for st in range(5):
+        assert lib.fcv_status_string(st).decode().startswith(binding.STATUS_NAMES[st])
+    assert b"unknown" in lib.fcv_status_string(99)
+
+
+def c2d(lib, x=FAKE, w=FAKE, b=FAKE, N=2, Cin=8, H=64, W=64, Cout=16, pool=4, out=FAKE, algo=0):
+    return lib.fcv_conv2d_pool_sigmoid_sum_ex(x, w, b, N, Cin, H, W, Cout, pool, out, algo, None)
+
+
+def c1d(lib, x=FAKE, dw=FAKE, pw=FAKE, bias=FAKE, N=2, C=8, T=64, O=16, K=9, s=1, p=4, out=FAKE, algo=0):
+    return lib.fcv_dwsep_conv1d_ex(x, dw, pw, bias, N, C, T, O, K, s, p, out, algo, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(x=None), dict(w=None), dict(b=None), dict(out=None),
+    dict(N=-1), dict(Cin=0), dict(Cout=0), dict(H=2), dict(W=2), dict(pool=0),
+    dict(x=MISALIGNED), dict(out=MISALIGNED),
+    dict(N=1 << 30, Cin=1 << 30, H=1 << 20, W=1 << 20),  # element count overflows int64
+    dict(algo=999), dict(algo=21),
+])
+def test_conv2d_invalid(lib, kw):
+    assert c2d(lib, **kw) == INVALID
+
+
+def test_conv2d_unsupported_pool(lib):
+    assert c2d(lib, pool=9) == UNSUPPORTED
+
+
+def test_conv2d_empty_batch_is_a_noop(lib):
+    assert c2d(lib, N=0) == OK
+    assert lib.fcv_conv2d_pool_tap(FAKE, FAKE, FAKE, 0, 3, 9, 9, 4, 2, FAKE, 0, None) == OK
+
+
+@pytest.mark.parametrize("kw", [
+    dict(x=None), dict(dw=None), dict(pw=None), dict(out=None),
+    dict(N=-1), dict(C=0), dict(O=0), dict(T=0), dict(K=0), dict(s=0), dict(p=-1),
+    dict(T=4, K=9, p=0),  # To < 1
+    dict(x=MISALIGNED), dict(bias=MISALIGNED),
+    dict(algo=10), dict(algo=7),
+])
+def test_conv1d_invalid(lib, kw):
+    assert c1d(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("kw", [dict(K=33, p=16), dict(s=17), dict(p=1 << 20)])
+def test_conv1d_unsupported(lib, kw):
+    assert c1d(lib, **kw) == UNSUPPORTED
+
+
+def test_conv1d_empty_batch_and_null_bias(lib):
+    assert c1d(lib, N=0) == OK
+    assert c1d(lib, N=0, bias=None) == OK
+
+
+def test_binding_raises_without_library(tmp_path):
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        binding.load(str(tmp_path / "missing.so"))

@@ -1,0 +1,297 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs, element by element at allclose(atol=rtol=1e-4).
+
+Small workloads are compared in full.  The full-size workloads and the shape
+sweep are compared on whole batch items the oracle can finish in seconds and
+on sampled outputs the oracle evaluates one by one, all produced by the same
+entry points (and launch configuration) the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import direct_convolution_chip_b200 as fcv
+import oracle
+from direct_convolution_chip_b200 import workloads as wl
+from tests.parity import assert_close, requires_cuda, sample_indices
+
+pytestmark = [pytest.mark.gpu, requires_cuda]
+
+CONV2D_ALGOS = [fcv.CONV2D_DIRECT]
+CONV1D_ALGOS = [fcv.CONV1D_FMA, fcv.CONV1D_TC_3XTF32]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from direct_convolution_chip_b200 import build
+    build.build()
+    fcv.load()
+
+
+def cuda(*ts):
+    return [None if t is None else t.cuda() for t in ts]
+
+
+def conv1d_or_skip(x, dw, pw, bias, s, p, algo):
+    try:
+        return fcv.dwsep_conv1d(x, dw, pw, bias, s, p, algo=algo)
+    except fcv.FcvError as e:
+        if e.status == 2 and algo == fcv.CONV1D_TC_3XTF32:
+            pytest.skip("tensor-core path does not cover this shape")
+        raise
+
+
+# ------------------------------------------------------------------ op A ---
+
+def check_conv2d_case(case, algo, batch_items=None, n_samples=2000, x_mean=0.0, w_scale=1.0):
+    x, w, b = wl.conv2d_inputs(case, x_mean=x_mean, w_scale=w_scale)
+    xd, wd, bd = cuda(x, w, b)
+    out = fcv.conv2d_pool_sigmoid_sum(xd, wd, bd, case.P, algo=algo)
+    tap = fcv.conv2d_pool_tap(xd, wd, bd, case.P, algo=algo)
+    torch.cuda.synchronize()
+    xn, wn, bn = x.numpy(), w.numpy(), b.numpy()
+    items = range(case.N) if batch_items is None else batch_items
+    for bi in items:
+        xs = xn[bi:bi + 1]
+        assert_close(out[bi:bi + 1], oracle.conv2d_pool_sigmoid_sum(xs, wn, bn, case.P), f"{case.name} out[{bi}]")
+        assert_close(tap[bi:bi + 1], oracle.conv2d_pool_tap(xs, wn, bn, case.P), f"{case.name} tap[{bi}]")
+    if n_samples and tap.numel():
+        idx = sample_indices(tuple(tap.shape), n_samples, seed=case.seed)
+        ref = oracle.conv2d_pool_tap_at(xn, wn, bn, case.P, idx)
+        got = tap.cpu().numpy()[idx[:, 0], idx[:, 1], idx[:, 2], idx[:, 3]]
+        assert_close(got, ref, f"{case.name} tap samples")
+    return out, tap
+
+
+@pytest.mark.parametrize("algo", CONV2D_ALGOS)
+def test_conv2d_small_full(algo):
+    check_conv2d_case(wl.CONV2D_SMALL, algo, n_samples=0)
+
+
+@pytest.mark.parametrize("algo", CONV2D_ALGOS)
+def test_conv2d_full_size(algo):
+    """x[128,8,384,384], Cout 64, pool 4: items 0, 63, 127 in full, 4096 sampled pooled values."""
+    check_conv2d_case(wl.CONV2D_FULL, algo, batch_items=[0, 63, 127], n_samples=4096)
+
+
+@pytest.mark.parametrize("case", [c for c in wl.sweep_cases() if c.op == "conv2d"], ids=lambda c: c.name)
+def test_conv2d_sweep(case):
+    heavy = case.Cin * case.Cout * case.H * case.W > 16 * 128 * 200 * 200
+    check_conv2d_case(case, fcv.CONV2D_DIRECT, batch_items=[0] if heavy else [0, case.N - 1], n_samples=2000)
+
+
+EDGE_2D = [
+    # (N, Cin, H, W, Cout, P)
+    (1, 1, 3, 3, 1, 1),        # smallest image: one conv output
+    (2, 3, 9, 9, 5, 1),
+    (1, 2, 11, 13, 7, 3),      # ragged floors in both dims
+    (3, 5, 37, 29, 17, 2),     # Cout not a multiple of the channel group
+    (1, 4, 41, 70, 33, 5),
+    (2, 2, 30, 31, 3, 6),
+    (1, 3, 25, 60, 9, 7),
+    (1, 2, 44, 50, 4, 8),
+    (2, 8, 70, 90, 130, 4),    # more than one channel block
+    (1, 20, 35, 36, 6, 4),     # more than one input-channel chunk
+    (1, 3, 509, 509, 1, 4),    # single output channel, large odd image
+    (4, 1, 130, 3, 2, 1),      # one conv column
+]
+
+
+@pytest.mark.parametrize("shape", EDGE_2D, ids=lambda s: "x".join(map(str, s)))
+def test_conv2d_edges(shape):
+    N, Cin, H, W, Cout, P = shape
+    case = wl.Conv2dCase("edge", N, Cin, H, W, Cout, P, seed=sum(shape))
+    check_conv2d_case(case, fcv.CONV2D_DIRECT, n_samples=0)
+
+
+def test_conv2d_empty_pool_gives_zero():
+    """Ho = 3 < pool = 4: PH = 0, so out = 0 (the library zeroes out itself)."""
+    case = wl.Conv2dCase("empty", 3, 2, 5, 40, 4, 4, seed=9)
+    x, w, b = cuda(*wl.conv2d_inputs(case))
+    out = torch.full((3,), 7.0, device="cuda")
+    fcv.conv2d_pool_sigmoid_sum(x, w, b, 4, out=out)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+    assert fcv.conv2d_pool_tap(x, w, b, 4).numel() == 0
+
+
+@pytest.mark.parametrize("variant", [dict(w_scale=30.0), dict(x_mean=1.0), dict(x_mean=1.0, w_scale=30.0)],
+                         ids=["w_x30", "x_mean1", "both"])
+def test_conv2d_adversarial(variant):
+    """Weights x30 and/or x ~ N(1,1): the sigmoid leaves its linear range."""
+    case = wl.Conv2dCase("adv", 2, 8, 96, 80, 24, 4, seed=21)
+    check_conv2d_case(case, fcv.CONV2D_DIRECT, n_samples=0, **variant)
+
+
+def test_conv2d_output_fully_overwritten():
+    case = wl.CONV2D_SMALL
+    x, w, b = cuda(*wl.conv2d_inputs(case))
+    ref = fcv.conv2d_pool_sigmoid_sum(x, w, b, case.P).clone()
+    out = torch.full_like(ref, 1e30)
+    fcv.conv2d_pool_sigmoid_sum(x, w, b, case.P, out=out)
+    torch.cuda.synchronize()
+    assert torch.allclose(out, ref, rtol=1e-6, atol=0)
+
+
+# ------------------------------------------------------------------ op B ---
+
+def check_conv1d_case(case, algo, full_items=None, n_samples=2000, bias_none=False):
+    x, dw, pw, bias = wl.conv1d_inputs(case)
+    if bias_none:
+        bias = None
+    xd, dwd, pwd, bd = cuda(x, dw, pw, bias)
+    out = conv1d_or_skip(xd, dwd, pwd, bd, case.stride, case.pad, algo)
+    torch.cuda.synchronize()
+    xn, dwn, pwn = x.numpy(), dw.numpy(), pw.numpy()
+    bn = None if bias is None else bias.numpy()
+    items = range(case.N) if full_items is None else full_items
+    for bi in items:
+        ref = oracle.dwsep_conv1d(xn[bi:bi + 1], dwn, pwn, bn, case.stride, case.pad)
+        assert_close(out[bi:bi + 1], ref, f"{case.name} out[{bi}]")
+    if n_samples:
+        idx = sample_indices(tuple(out.shape), n_samples, seed=case.seed)
+        ref = oracle.dwsep_conv1d_at(xn, dwn, pwn, bn, case.stride, case.pad, idx)
+        got = out.cpu().numpy()[idx[:, 0], idx[:, 1], idx[:, 2]]
+        assert_close(got, ref, f"{case.name} samples")
+    return out
+
+
+@pytest.mark.parametrize("algo", CONV1D_ALGOS)
+def test_conv1d_small_full(algo):
+    check_conv1d_case(wl.CONV1D_SMALL, algo, n_samples=0)
+
+
+@pytest.mark.parametrize("algo", CONV1D_ALGOS)
+def test_conv1d_full_size(algo):
+    """x[32,256,4096] -> [32,512,4096]: items 0 and 31 in full, 4096 sampled outputs."""
+    check_conv1d_case(wl.CONV1D_FULL, algo, full_items=[0, 31], n_samples=4096)
+
+
+def test_conv1d_auto_matches_oracle():
+    check_conv1d_case(wl.CONV1D_SMALL, fcv.ALGO_AUTO, n_samples=0)
+
+
+@pytest.mark.parametrize("case", [c for c in wl.sweep_cases() if c.op == "conv1d"], ids=lambda c: c.name)
+@pytest.mark.parametrize("algo", CONV1D_ALGOS)
+def test_conv1d_sweep(case, algo):
+    full = [0] if case.T <= 1000 else []
+    check_conv1d_case(case, algo, full_items=full, n_samples=2000)
+
+
+EDGE_1D = [
+    # (N, C, T, O, K, s, p, bias)
+    (1, 1, 1, 1, 1, 1, 0, True),      # single sample, K = 1
+    (2, 3, 17, 5, 3, 1, 1, False),    # no bias
+    (1, 7, 130, 9, 9, 2, 4, True),    # stride 2, odd sizes
+    (2, 5, 300, 129, 5, 3, 0, True),  # stride 3, no padding, O just over a tile
+    (1, 17, 257, 200, 9, 1, 12, True),  # pad larger than K
+    (1, 33, 64, 16, 32, 1, 16, True),   # the largest supported K
+    (1, 16, 1000, 64, 1, 1, 0, True),   # pointwise only (K = 1)
+    (3, 40, 129, 33, 7, 16, 3, False),  # the largest supported stride
+    (1, 300, 70, 20, 4, 1, 1, True),    # C not a multiple of the channel chunk
+]
+
+
+@pytest.mark.parametrize("shape", EDGE_1D, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("algo", CONV1D_ALGOS)
+def test_conv1d_edges(shape, algo):
+    N, C, T, O, K, s, p, has_bias = shape
+    case = wl.Conv1dCase("edge", N, C, T, O, K, s, p, seed=sum(shape[:7]), has_bias=has_bias)
+    check_conv1d_case(case, algo, n_samples=0)
+
+
+# ------------------------------------------------------- both ops, hygiene ---
+
+def _guarded(n, fill=float("nan"), guard=1024):
+    buf = torch.full((n + 2 * guard,), fill, device="cuda")
+    return buf, buf[guard:guard + n]
+
+
+def test_guard_bands_untouched():
+    """Outputs inside NaN-filled guard regions: nothing outside the output is written."""
+    guard = 1024
+    case = wl.Conv2dCase("canary", 3, 5, 61, 47, 19, 4, seed=5)
+    x, w, b = cuda(*wl.conv2d_inputs(case))
+    PH, PW = fcv.conv2d_out_shape(case.H, case.W, case.P)
+    buf, out = _guarded(case.N)
+    fcv.conv2d_pool_sigmoid_sum(x, w, b, case.P, out=out)
+    tbuf, tap = _guarded(case.N * case.Cout * PH * PW)
+    fcv.conv2d_pool_tap(x, w, b, case.P, out=tap.view(case.N, case.Cout, PH, PW))
+    c1 = wl.Conv1dCase("canary", 2, 19, 333, 37, 9, 2, 4, seed=6)
+    xs, dw, pw, bias = cuda(*wl.conv1d_inputs(c1))
+    To = fcv.conv1d_out_len(c1.T, c1.K, c1.stride, c1.pad)
+    results = []
+    for algo in CONV1D_ALGOS:
+        obuf, o = _guarded(c1.N * c1.O * To)
+        try:
+            fcv.dwsep_conv1d(xs, dw, pw, bias, c1.stride, c1.pad, out=o.view(c1.N, c1.O, To), algo=algo)
+        except fcv.FcvError as e:
+            if e.status != 2:
+                raise
+            continue
+        results.append((obuf, o))
+    torch.cuda.synchronize()
+    for b_, o_ in [(buf, out), (tbuf, tap)] + results:
+        assert torch.isnan(b_[:guard]).all() and torch.isnan(b_[-guard:]).all()
+        assert torch.isfinite(o_).all()
+
+
+def test_conv1d_bitwise_repeatable():
+    case = wl.CONV1D_SMALL
+    x, dw, pw, bias = cuda(*wl.conv1d_inputs(case))
+    for algo in CONV1D_ALGOS:
+        try:
+            a = fcv.dwsep_conv1d(x, dw, pw, bias, case.stride, case.pad, algo=algo)
+        except fcv.FcvError as e:
+            if e.status == 2:
+                continue
+            raise
+        b_ = fcv.dwsep_conv1d(x, dw, pw, bias, case.stride, case.pad, algo=algo)
+        torch.cuda.synchronize()
+        assert torch.equal(a, b_)
+
+
+def test_conv2d_repeatable_within_rounding():
+    case = wl.Conv2dCase("rep", 4, 8, 128, 128, 64, 4, seed=13)
+    x, w, b = cuda(*wl.conv2d_inputs(case))
+    a = fcv.conv2d_pool_sigmoid_sum(x, w, b, case.P)
+    b_ = fcv.conv2d_pool_sigmoid_sum(x, w, b, case.P)
+    torch.cuda.synchronize()
+    assert torch.allclose(a, b_, rtol=1e-6, atol=0)
+
+
+def test_non_default_stream_and_device_error():
+    case = wl.CONV2D_SMALL
+    x, w, b = cuda(*wl.conv2d_inputs(case))
+    ref = fcv.conv2d_pool_sigmoid_sum(x, w, b, case.P)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        out = fcv.conv2d_pool_sigmoid_sum(x, w, b, case.P, stream=s)
+    s.synchronize()
+    assert torch.allclose(out, ref, rtol=1e-6, atol=0)
+    assert fcv.device_error() == 0
+
+
+def test_host_tensors_through_public_api():
+    """CPU inputs: the binding copies to the device, runs the kernel, copies back."""
+    case = wl.CONV1D_SMALL
+    x, dw, pw, bias = wl.conv1d_inputs(case)
+    out = fcv.dwsep_conv1d(x.pin_memory(), dw, pw, bias, case.stride, case.pad)
+    assert not out.is_cuda
+    assert_close(out, oracle.dwsep_conv1d(x.numpy(), dw.numpy(), pw.numpy(), bias.numpy(), 1, 4), "host conv1d")
+    c2 = wl.CONV2D_SMALL
+    x2, w2, b2 = wl.conv2d_inputs(c2)
+    out2 = fcv.conv2d_pool_sigmoid_sum(x2, w2, b2, c2.P)
+    assert not out2.is_cuda
+    assert_close(out2, oracle.conv2d_pool_sigmoid_sum(x2.numpy(), w2.numpy(), b2.numpy(), c2.P), "host conv2d")
+
+
+def test_empty_batch_through_binding():
+    x = torch.zeros((0, 3, 10, 10), device="cuda")
+    w = torch.zeros((4, 3, 3, 3), device="cuda")
+    b = torch.zeros((4,), device="cuda")
+    assert fcv.conv2d_pool_sigmoid_sum(x, w, b, 2).shape == (0,)
+    x1 = torch.zeros((0, 3, 10), device="cuda")
+    out = fcv.dwsep_conv1d(x1, torch.zeros((3, 3), device="cuda"), torch.zeros((5, 3), device="cuda"), None, 1, 1)
+    assert out.shape == (0, 5, 10)
