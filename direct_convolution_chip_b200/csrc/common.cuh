@@ -40,6 +40,21 @@ __device__ __forceinline__ float block_sum(float v, float* scratch)
     return s;
 }
 
+// 4-byte asynchronous global->shared copy; when `pred` is false nothing is
+// read and the destination is zero-filled (src-size 0).  `gsrc` must still be
+// a valid global address, so callers pass a base pointer in that case.
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc, bool pred)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(s), "l"(gsrc), "r"(pred ? 4 : 0)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 inline int launch_status()

@@ -13,16 +13,29 @@
 //     CB = CG*NCH output channels of one image.  Its input halo
 //     [ICC][P*TPH+2][P*TPW*RX+2] is staged in shared memory (zero-filled past
 //     the image) one chunk of ICC input channels at a time.
+//   * The halo and weights arrive by cp.async, every copy of a chunk in flight
+//     at once, so a CTA waits for one memory latency per chunk, not one per
+//     element.
 //   * Each thread owns RX adjacent pooled positions for CG channels.  It keeps
 //     its (P+2) x (RX*P+2) input patch in registers and, per 3x3 tap, the CG
 //     weights of that tap (a broadcast shared-memory read), then issues
 //     P*P*RX*CG independent FMAs -- consecutive FMAs update different
 //     accumulators, so the FMA pipe is not stalled on a dependency chain.
+//     For P <= 4 the FMAs are packed (fma.rn.f32x2, two channels per
+//     instruction): the FP32 pipe does the same 128 FMA/clk/SM either way, but
+//     half the issue slots go to the FMAs, leaving room for loads and
+//     addressing.
 //   * Epilogue: mean + bias, sigmoid (CUDA expf), a warp-shuffle + shared
 //     memory block sum, and one atomicAdd per CTA into out[n].
 #pragma once
 
 #include "common.cuh"
+
+// Largest pool size that uses packed fma.rn.f32x2 (its register patch holds
+// every input value twice).
+#ifndef FCV_CONV2D_PACKED_MAX_P
+#define FCV_CONV2D_PACKED_MAX_P 4
+#endif
 
 namespace fcv {
 
@@ -32,7 +45,7 @@ struct Conv2dTile;
 // (RX, CG, TPH, TPW, NCH, ICC) per pool size: register patch + accumulators
 // stay well under 128 registers; halo + weights stay under ~60 KB so several
 // CTAs share an SM.
-template <> struct Conv2dTile<1> { static constexpr int RX = 4, CG = 16, TPH = 16, TPW = 8,  NCH = 2, ICC = 8; };
+template <> struct Conv2dTile<1> { static constexpr int RX = 2, CG = 16, TPH = 16, TPW = 8,  NCH = 2, ICC = 8; };
 template <> struct Conv2dTile<2> { static constexpr int RX = 2, CG = 16, TPH = 8,  TPW = 8,  NCH = 4, ICC = 8; };
 template <> struct Conv2dTile<3> { static constexpr int RX = 1, CG = 16, TPH = 8,  TPW = 8,  NCH = 4, ICC = 8; };
 template <> struct Conv2dTile<4> { static constexpr int RX = 1, CG = 16, TPH = 8,  TPW = 8,  NCH = 4, ICC = 8; };
@@ -60,7 +73,7 @@ struct Conv2dGeom {
     static constexpr size_t SMEM_BYTES = sizeof(float) * (HALO_FLOATS + W_FLOATS + NT / 32);
 };
 
-template <int P, bool TAP>
+template <int P, bool TAP, bool PACKED = (P <= FCV_CONV2D_PACKED_MAX_P)>
 __global__ void __launch_bounds__(Conv2dGeom<P>::NT, 2)
 conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
                      const float* __restrict__ bias, int Cin, int H, int W, int Cout,
@@ -88,65 +101,107 @@ conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
     const int grp = tid / NPOS, pos = tid % NPOS;
     const int ty = pos / G::TPW, tx = pos % G::TPW;
 
-    float acc[RX][CG];
+    float2 acc2[RX][CG / 2];  // acc2[rx][c/2] holds channels c (x) and c+1 (y)
 #pragma unroll
     for (int r = 0; r < RX; ++r)
 #pragma unroll
-        for (int c = 0; c < CG; ++c) acc[r][c] = 0.f;
+        for (int c = 0; c < CG / 2; ++c) acc2[r][c] = make_float2(0.f, 0.f);
 
     const float* xn = x + (size_t)n * Cin * H * W;
 
     for (int ic0 = 0; ic0 < Cin; ic0 += ICC) {
-        // Stage the halo of this input-channel chunk (zero past the image and past Cin).
+        // Stage the halo of this input-channel chunk and its weights with
+        // asynchronous copies, all in flight at once (zero past the image and
+        // past Cin); weights as [icl][tap][c_local] so a thread's CG channels
+        // of one tap are contiguous.
         for (int i = tid; i < ICC * HY * HX; i += NT) {
             const int icl = i / (HY * HX);
             const int rem = i - icl * (HY * HX);
-            const int r = rem / HX, s = rem - (rem / HX) * HX;
-            const int ic = ic0 + icl, yy = y0 + r, xx = x0 + s;
-            float v = 0.f;
-            if (ic < Cin && yy < H && xx < W) v = __ldg(xn + ((size_t)ic * H + yy) * W + xx);
-            halo[(icl * HY + r) * HXP + s] = v;
+            const int r = rem / HX, sc = rem - (rem / HX) * HX;
+            const int ic = ic0 + icl, yy = y0 + r, xx = x0 + sc;
+            const bool in = ic < Cin && yy < H && xx < W;
+            cp_async4(halo + (icl * HY + r) * HXP + sc, in ? xn + ((size_t)ic * H + yy) * W + xx : x, in);
         }
-        // Stage the weights as [icl][tap][c_local] so a thread's CG channels of one tap are contiguous.
         for (int i = tid; i < ICC * 9 * CB; i += NT) {
             const int cl = i % CB;
             const int tap = (i / CB) % 9;
             const int icl = i / (9 * CB);
             const int c = c_base + cl, ic = ic0 + icl;
-            ws[i] = (c < Cout && ic < Cin) ? __ldg(w + ((size_t)c * Cin + ic) * 9 + tap) : 0.f;
+            const bool in = c < Cout && ic < Cin;
+            cp_async4(ws + i, in ? w + ((size_t)c * Cin + ic) * 9 + tap : w, in);
         }
+        cp_async_commit();
+        cp_async_wait<0>();
         __syncthreads();
 
         const int nic = min(ICC, Cin - ic0);
         for (int icl = 0; icl < nic; ++icl) {
-            float patch[PY][PX];
             const float* hp = halo + (icl * HY + ty * P) * HXP + tx * (RX * P);
-#pragma unroll
-            for (int r = 0; r < PY; ++r)
-#pragma unroll
-                for (int s = 0; s < PX; ++s) patch[r][s] = hp[r * HXP + s];
-
             const float* wp = ws + icl * 9 * CB + grp * CG;
+            if constexpr (PACKED) {
+                // Packed FP32 FMA: each fma.rn.f32x2 updates two adjacent
+                // output channels; the input value is duplicated into both
+                // halves of a register pair once per patch load.
+                float2 patch[PY][PX];
 #pragma unroll
-            for (int ky = 0; ky < 3; ++ky) {
+                for (int r = 0; r < PY; ++r)
 #pragma unroll
-                for (int kx = 0; kx < 3; ++kx) {
-                    float wr[CG];
-#pragma unroll
-                    for (int c = 0; c < CG; c += 4) {
-                        const float4 v = *reinterpret_cast<const float4*>(wp + (ky * 3 + kx) * CB + c);
-                        wr[c] = v.x; wr[c + 1] = v.y; wr[c + 2] = v.z; wr[c + 3] = v.w;
+                    for (int sc = 0; sc < PX; ++sc) {
+                        const float v = hp[r * HXP + sc];
+                        patch[r][sc] = make_float2(v, v);
                     }
 #pragma unroll
-                    for (int rx = 0; rx < RX; ++rx)
+                for (int ky = 0; ky < 3; ++ky) {
 #pragma unroll
-                        for (int dy = 0; dy < P; ++dy)
+                    for (int kx = 0; kx < 3; ++kx) {
+                        float2 wr[CG / 2];
 #pragma unroll
-                            for (int dx = 0; dx < P; ++dx) {
-                                const float pv = patch[dy + ky][rx * P + dx + kx];
+                        for (int c = 0; c < CG; c += 4) {
+                            const float4 v = *reinterpret_cast<const float4*>(wp + (ky * 3 + kx) * CB + c);
+                            wr[c / 2] = make_float2(v.x, v.y);
+                            wr[c / 2 + 1] = make_float2(v.z, v.w);
+                        }
 #pragma unroll
-                                for (int c = 0; c < CG; ++c) acc[rx][c] = fmaf(pv, wr[c], acc[rx][c]);
-                            }
+                        for (int rx = 0; rx < RX; ++rx)
+#pragma unroll
+                            for (int dy = 0; dy < P; ++dy)
+#pragma unroll
+                                for (int dx = 0; dx < P; ++dx) {
+                                    const float2 pv = patch[dy + ky][rx * P + dx + kx];
+#pragma unroll
+                                    for (int c = 0; c < CG / 2; ++c) acc2[rx][c] = __ffma2_rn(pv, wr[c], acc2[rx][c]);
+                                }
+                    }
+                }
+            } else {
+                float patch[PY][PX];
+#pragma unroll
+                for (int r = 0; r < PY; ++r)
+#pragma unroll
+                    for (int sc = 0; sc < PX; ++sc) patch[r][sc] = hp[r * HXP + sc];
+#pragma unroll
+                for (int ky = 0; ky < 3; ++ky) {
+#pragma unroll
+                    for (int kx = 0; kx < 3; ++kx) {
+                        float wr[CG];
+#pragma unroll
+                        for (int c = 0; c < CG; c += 4) {
+                            const float4 v = *reinterpret_cast<const float4*>(wp + (ky * 3 + kx) * CB + c);
+                            wr[c] = v.x; wr[c + 1] = v.y; wr[c + 2] = v.z; wr[c + 3] = v.w;
+                        }
+#pragma unroll
+                        for (int rx = 0; rx < RX; ++rx)
+#pragma unroll
+                            for (int dy = 0; dy < P; ++dy)
+#pragma unroll
+                                for (int dx = 0; dx < P; ++dx) {
+                                    const float pv = patch[dy + ky][rx * P + dx + kx];
+#pragma unroll
+                                    for (int c = 0; c < CG; ++c)
+                                        acc2[rx][c / 2] = (c & 1) ? make_float2(acc2[rx][c / 2].x, fmaf(pv, wr[c], acc2[rx][c / 2].y))
+                                                                  : make_float2(fmaf(pv, wr[c], acc2[rx][c / 2].x), acc2[rx][c / 2].y);
+                                }
+                    }
                 }
             }
         }
@@ -164,7 +219,8 @@ conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
         for (int c = 0; c < CG; ++c) {
             const int cc = c_base + grp * CG + c;
             if (valid && cc < Cout) {
-                const float avg = acc[rx][c] / (float)(P * P) + __ldg(bias + cc);
+                const float a = (c & 1) ? acc2[rx][c / 2].y : acc2[rx][c / 2].x;
+                const float avg = a / (float)(P * P) + __ldg(bias + cc);
                 if (TAP) {
                     out[(((size_t)n * Cout + cc) * PH + ph) * PW + pw] = avg;
                 } else {

@@ -30,13 +30,20 @@ bool mul_ok(long long a, long long b, long long c, long long d)
     return true;
 }
 
+// A pointer may be NULL exactly when the tensor behind it has no elements or
+// nothing is read or written (N == 0); otherwise it must be non-NULL and
+// 4-byte aligned.
+bool ptr_ok(const void* p, bool needed) { return needed ? (p != nullptr && aligned4(p)) : aligned4(p); }
+
 int check_conv2d(const float* x, const float* w, const float* b, int N, int Cin, int H, int W,
-                 int Cout, int pool, const float* out)
+                 int Cout, int pool, const float* out, bool tap)
 {
-    if (!x || !w || !b || !out) return FCV_ERR_INVALID_ARG;
     if (N < 0 || Cin < 1 || Cout < 1 || H < 3 || W < 3 || pool < 1) return FCV_ERR_INVALID_ARG;
-    if (!aligned4(x) || !aligned4(w) || !aligned4(b) || !aligned4(out)) return FCV_ERR_INVALID_ARG;
     if (!mul_ok(N, Cin, H, W) || !mul_ok(Cout, Cin, 9, 1) || !mul_ok(N, Cout, H, W))
+        return FCV_ERR_INVALID_ARG;
+    const bool work = N > 0;
+    const bool out_has_elems = work && (!tap || ((H - 2) / pool > 0 && (W - 2) / pool > 0));
+    if (!ptr_ok(x, work) || !ptr_ok(w, work) || !ptr_ok(b, work) || !ptr_ok(out, out_has_elems))
         return FCV_ERR_INVALID_ARG;
     if (pool > 8) return FCV_ERR_UNSUPPORTED;
     return FCV_OK;
@@ -45,9 +52,9 @@ int check_conv2d(const float* x, const float* w, const float* b, int N, int Cin,
 int check_conv1d(const float* x, const float* dw, const float* pw, const float* bias, int N, int C,
                  int T, int O, int K, int stride, int pad, const float* out, int* To)
 {
-    if (!x || !dw || !pw || !out) return FCV_ERR_INVALID_ARG;
     if (N < 0 || C < 1 || O < 1 || T < 1 || K < 1 || stride < 1 || pad < 0) return FCV_ERR_INVALID_ARG;
-    if (!aligned4(x) || !aligned4(dw) || !aligned4(pw) || !aligned4(out) || (bias && !aligned4(bias)))
+    const bool work = N > 0;
+    if (!ptr_ok(x, work) || !ptr_ok(dw, work) || !ptr_ok(pw, work) || !ptr_ok(out, work) || !aligned4(bias))
         return FCV_ERR_INVALID_ARG;
     const long long span = (long long)T + 2LL * pad - K;
     if (span < 0) return FCV_ERR_INVALID_ARG;  // To < 1
@@ -63,7 +70,7 @@ int check_conv1d(const float* x, const float* dw, const float* pw, const float* 
 int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin, int H, int W,
                   int Cout, int pool, float* out, int algo, bool tap, void* stream)
 {
-    int st = check_conv2d(x, w, b, N, Cin, H, W, Cout, pool, out);
+    int st = check_conv2d(x, w, b, N, Cin, H, W, Cout, pool, out, tap);
     if (st != FCV_OK) return st;
     if (algo != FCV_ALGO_AUTO && algo != FCV_CONV2D_DIRECT) return FCV_ERR_INVALID_ARG;
     if (N == 0) return FCV_OK;

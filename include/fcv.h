@@ -25,6 +25,8 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller; fp32,
  *     contiguous, row-major (NCHW for op A, NCT for op B).  Inputs are read
  *     only.  Outputs must not alias inputs.  Pointers must be 4-byte aligned.
+ *     A pointer may be NULL when its tensor has no elements, or when N == 0
+ *     (nothing is then read or written); otherwise NULL is INVALID_ARG.
  *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *     stream.  Calls are asynchronous on that stream: they never synchronize
  *     and never allocate memory.
@@ -77,7 +79,7 @@ typedef enum {
  *
  * Ho = H - 2, Wo = W - 2, PH = floor(Ho / pool), PW = floor(Wo / pool).
  * PH == 0 or PW == 0 is valid and gives out = 0.
- * INVALID_ARG: x, w, b or out NULL; N < 0; Cin, Cout < 1; H, W < 3; pool < 1;
+ * INVALID_ARG: x, w, b or out NULL while N > 0; N < 0; Cin, Cout < 1; H, W < 3; pool < 1;
  *              element counts beyond 2^31 * 2^31; misaligned pointers.
  * UNSUPPORTED: pool > 8.
  * The per-batch sum is accumulated with one atomic add per thread block, so
@@ -94,7 +96,7 @@ int fcv_conv2d_pool_sigmoid_sum_ex(const float* x, const float* w, const float* 
  * pool stages element by element:
  *   pooled [N, Cout, PH, PW]  = avgpool_P( conv3x3(x, w) + b ), fully overwritten.
  * Same arguments, errors and algorithms as fcv_conv2d_pool_sigmoid_sum_ex;
- * nothing is summed. */
+ * nothing is summed.  `pooled` may be NULL when PH or PW is 0. */
 int fcv_conv2d_pool_tap(const float* x, const float* w, const float* b,
                         int N, int Cin, int H, int W, int Cout, int pool,
                         float* pooled, int algo, void* stream);
@@ -112,10 +114,10 @@ int fcv_conv2d_pool_tap(const float* x, const float* w, const float* b,
  * The depthwise result lives only in on-chip memory.  Every algorithm is
  * fp32-accurate (FP32 FMA, or tensor cores through a 3xTF32 split); results
  * are deterministic run to run.
- * INVALID_ARG: x, dw_w, pw_w or out NULL; N < 0; C, O, T, K, stride < 1;
+ * INVALID_ARG: x, dw_w, pw_w or out NULL while N > 0; N < 0; C, O, T, K, stride < 1;
  *              pad < 0; To < 1; sizes beyond the 64-bit index range;
  *              misaligned pointers.
- * UNSUPPORTED: K > 32, pad >= 2^20, stride > 16. */
+ * UNSUPPORTED: K > 32, pad >= 2^20, stride > 8. */
 int fcv_dwsep_conv1d(const float* x, const float* dw_w, const float* pw_w, const float* bias,
                      int N, int C, int T, int O, int K, int stride, int pad,
                      float* out, void* stream);

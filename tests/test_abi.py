@@ -77,7 +77,14 @@ def test_conv2d_unsupported_pool(lib):
 
 def test_conv2d_empty_batch_is_a_noop(lib):
     assert c2d(lib, N=0) == OK
+    assert c2d(lib, N=0, x=None, w=None, b=None, out=None) == OK  # empty tensors may be NULL
     assert lib.fcv_conv2d_pool_tap(FAKE, FAKE, FAKE, 0, 3, 9, 9, 4, 2, FAKE, 0, None) == OK
+
+
+def test_conv2d_tap_null_when_pool_is_empty(lib):
+    # Ho = 3 < pool 4: the tap has no elements, so it may be NULL; the sum output may not.
+    assert lib.fcv_conv2d_pool_tap(FAKE, FAKE, FAKE, 2, 3, 5, 40, 4, 4, None, 0, None) == OK
+    assert c2d(lib, H=5, pool=4, out=None) == INVALID
 
 
 @pytest.mark.parametrize("kw", [
@@ -91,7 +98,7 @@ def test_conv1d_invalid(lib, kw):
     assert c1d(lib, **kw) == INVALID
 
 
-@pytest.mark.parametrize("kw", [dict(K=33, p=16), dict(s=17), dict(p=1 << 20)])
+@pytest.mark.parametrize("kw", [dict(K=33, p=16), dict(s=9), dict(p=1 << 20)])
 def test_conv1d_unsupported(lib, kw):
     assert c1d(lib, **kw) == UNSUPPORTED
 
@@ -99,6 +106,7 @@ def test_conv1d_unsupported(lib, kw):
 def test_conv1d_empty_batch_and_null_bias(lib):
     assert c1d(lib, N=0) == OK
     assert c1d(lib, N=0, bias=None) == OK
+    assert c1d(lib, N=0, x=None, dw=None, pw=None, out=None) == OK
 
 
 def test_binding_raises_without_library(tmp_path):

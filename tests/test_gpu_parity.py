@@ -187,7 +187,7 @@ EDGE_1D = [
     (1, 17, 257, 200, 9, 1, 12, True),  # pad larger than K
     (1, 33, 64, 16, 32, 1, 16, True),   # the largest supported K
     (1, 16, 1000, 64, 1, 1, 0, True),   # pointwise only (K = 1)
-    (3, 40, 129, 33, 7, 16, 3, False),  # the largest supported stride
+    (3, 40, 129, 33, 7, 8, 3, False),   # the largest supported stride
     (1, 300, 70, 20, 4, 1, 1, True),    # C not a multiple of the channel chunk
 ]
 
