@@ -17,10 +17,11 @@
 // output channels, K stepped in chunks of 32 channels = one 128-byte row):
 //   * warps 0-7 (producers): stage the input halo x[n, c0:c0+32, t0-p : ...]
 //     in shared memory, compute the depthwise tile with FP32 FMA (4 times x 4
-//     channels per thread from a 16-sample register window), split it into
-//     TF32 hi/lo and write both as K-major, 128B-swizzled UMMA operands; the
-//     pw chunk (256 x 32) is split the same way.  Global loads of the next
-//     chunk are issued before the current chunk is processed.
+//     channels per thread from a 16-sample register window; the depthwise
+//     weights of all channels stay resident), split it into TF32 hi/lo and
+//     write both as K-major, 128B-swizzled UMMA operands; the pw chunk
+//     (256 x 32) is split the same way.  The global loads of the next chunk
+//     are in flight while the current chunk is computed.
 //   * warp 8: allocates 512 TMEM columns (two 128 x 256 fp32 accumulators);
 //     one thread issues 12 tcgen05.mma (kind::tf32, M=128, N=256, K=8) per
 //     chunk and commits them to the stage's "empty" barrier and, after the
@@ -47,10 +48,10 @@ constexpr int MMA_WARP = 8;
 constexpr int NTHREADS = 13 * 32;
 constexpr int KMAXW = 13;      // largest depthwise kernel (stride 1) of the register window
 constexpr int XW_MAX = TM - 1 + KMAXW;  // 140 halo samples per channel at most
-constexpr int XR = (KC * XW_MAX + NPROD - 1) / NPROD;  // halo prefetch registers per thread
+constexpr int XU = (XW_MAX + 31) / 32;  // halo samples per lane per channel
 constexpr int XWP = 144;       // halo row pitch in floats (multiple of 8)
 constexpr int XS_FLOATS = KC * XWP + 28;  // + skew of 4 floats per group of 4 channels
-constexpr int DWP = 17;        // depthwise weight row pitch (odd: spreads banks)
+constexpr int DW_MAX = 4000;   // resident depthwise weights: C * K at most
 constexpr uint32_t TMEM_COLS = 2 * TN;
 
 constexpr uint32_t A_BYTES = TM * KC * 4;    // 16 KB
@@ -58,13 +59,13 @@ constexpr uint32_t B_BYTES = TN * KC * 4;    // 32 KB
 constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;  // A_hi | A_lo | B_hi | B_lo
 constexpr uint32_t OFF_XS = STAGES * STAGE_BYTES;
 constexpr uint32_t OFF_DWS = OFF_XS + XS_FLOATS * 4;
-constexpr uint32_t OFF_BAR = (OFF_DWS + KC * DWP * 4 + 7) & ~7u;
+constexpr uint32_t OFF_BAR = (OFF_DWS + DW_MAX * 4 + 7) & ~7u;
 constexpr uint32_t NBAR = 9;   // full[2] empty[2] afull[2] aempty[2] drain
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024 B
 
-static_assert(XR * NPROD >= KC * XW_MAX, "halo prefetch too small");
+static_assert(XU * 32 >= XW_MAX, "halo prefetch too small");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(XWP >= XW_MAX && XWP % 8 == 0, "halo pitch");
 
@@ -216,6 +217,8 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& p, int tile)
     return tc;
 }
 
+// KT: the depthwise kernel size when known at compile time, 0 for any K <= KMAXW.
+template <int KT>
 __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Params p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -260,40 +263,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
     const int nk = (p.C + KC - 1) / KC;
     const int XW = TM - 1 + p.K;  // halo samples per channel (stride 1)
 
+    // Depthwise weights of every channel stay resident: [C][K], row pitch K.
+    for (int e = threadIdx.x; e < p.C * p.K; e += NTHREADS) dws[e] = __ldg(p.dw + e);
+    __syncthreads();
+
     if (warp < 8) {
         // ------------------------------------------------------------ producers
         const int ptid = threadIdx.x;
         const int cg = lane & 7;               // depthwise: channel group of 4
         const int tq = (lane >> 3) + 4 * warp; // depthwise: times 4*tq .. 4*tq+3
-        float xr[XR];
-        float4 pr[8];
-        float dwr[2];
+        const int K = KT > 0 ? KT : p.K;
+        float xr[4][XU];   // halo of channels 4*warp .. 4*warp+3, samples lane + 32*u
+        float4 pr[8];      // pw chunk rows, 16 bytes each
 
         auto fetch = [&](int tile, int kc) {
             const TileCoord tcd = decode_tile(p, tile);
             const int c0 = kc * KC;
-            const float* xn = p.x + (size_t)tcd.n * p.C * p.T;
+            const int tb = tcd.t0 - p.pad;
 #pragma unroll
-            for (int r = 0; r < XR; ++r) {
-                const int e = ptid + NPROD * r;
-                float v = 0.f;
-                if (e < KC * XW) {
-                    const int cl = e / XW, j = e - (e / XW) * XW;
-                    const int c = c0 + cl;
-                    const int ti = tcd.t0 - p.pad + j;
-                    if (c < p.C && ti >= 0 && ti < p.T) v = __ldg(xn + (size_t)c * p.T + ti);
-                }
-                xr[r] = v;
-            }
+            for (int i = 0; i < 4; ++i) {
+                const int c = c0 + 4 * warp + i;
+                const float* xrow = p.x + ((size_t)tcd.n * p.C + (c < p.C ? c : 0)) * p.T;
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int e = ptid + NPROD * r;
-                float v = 0.f;
-                if (e < KC * p.K) {
-                    const int cl = e / p.K, k = e - (e / p.K) * p.K;
-                    if (c0 + cl < p.C) v = __ldg(p.dw + (size_t)(c0 + cl) * p.K + k);
+                for (int u = 0; u < XU; ++u) {
+                    const int ti = tb + lane + 32 * u;
+                    xr[i][u] = (c < p.C && ti >= 0 && ti < p.T) ? __ldg(xrow + ti) : 0.f;
                 }
-                dwr[r] = v;
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -329,22 +324,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
             const uint32_t a_lo = a_hi + A_BYTES;
             const uint32_t b_hi = a_lo + A_BYTES;
             const uint32_t b_lo = b_hi + B_BYTES;
+            const int c0 = kc * KC;
 
-            // Halo and depthwise weights of this chunk into shared memory.
+            // Halo of this chunk into shared memory (rows skewed by 4 floats per channel group).
 #pragma unroll
-            for (int r = 0; r < XR; ++r) {
-                const int e = ptid + NPROD * r;
-                if (e < KC * XW) {
-                    const int cl = e / XW, j = e - (e / XW) * XW;
-                    xs[cl * XWP + 4 * ((cl >> 2) & 7) + j] = xr[r];
-                }
-            }
+            for (int i = 0; i < 4; ++i) {
+                const int cl = 4 * warp + i;
+                float* dst = xs + cl * XWP + 4 * ((cl >> 2) & 7);
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int e = ptid + NPROD * r;
-                if (e < KC * p.K) {
-                    const int cl = e / p.K, k = e - (e / p.K) * p.K;
-                    dws[cl * DWP + k] = dwr[r];
+                for (int u = 0; u < XU; ++u) {
+                    const int j = lane + 32 * u;
+                    if (j < XWP) dst[j] = xr[i][u];
                 }
             }
             // pw chunk, split into TF32 hi/lo, as the K-major B operand.
@@ -357,39 +347,51 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
                 sts128(b_hi + off, hi);
                 sts128(b_lo + off, lo);
             }
-            asm volatile("bar.sync 1, 256;\n" ::: "memory");  // halo and weights visible
+            asm volatile("bar.sync 1, 256;\n" ::: "memory");  // halo visible to every producer
 
             // Issue the global loads of the next chunk now; they land while this one is computed.
-            const int cur_tile = tile;
             if (++kc == nk) {
                 kc = 0;
                 tile += gridDim.x;
             }
             if (tile < p.total_tiles) fetch(tile, kc);
-            (void)cur_tile;
 
             // Depthwise tile: 4 times x 4 channels per thread, then the TF32 split as the A operand.
             float dv[4][4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int cl = 4 * cg + i;
-                const float* xrow = xs + cl * XWP + 4 * ((cl >> 2) & 7) + 4 * tq;
-                float win[16];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
-                    win[4 * q] = v.x; win[4 * q + 1] = v.y; win[4 * q + 2] = v.z; win[4 * q + 3] = v.w;
-                }
+                const int c = c0 + cl;
                 float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
-                const float* wrow = dws + cl * DWP;
+                if (c < p.C) {
+                    const float* xrow = xs + cl * XWP + 4 * ((cl >> 2) & 7) + 4 * tq;
+                    float win[16];
 #pragma unroll
-                for (int k = 0; k < KMAXW; ++k) {
-                    if (k < p.K) {
-                        const float wk = wrow[k];
-                        d0 = fmaf(win[k], wk, d0);
-                        d1 = fmaf(win[k + 1], wk, d1);
-                        d2 = fmaf(win[k + 2], wk, d2);
-                        d3 = fmaf(win[k + 3], wk, d3);
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
+                        win[4 * q] = v.x; win[4 * q + 1] = v.y; win[4 * q + 2] = v.z; win[4 * q + 3] = v.w;
+                    }
+                    const float* wrow = dws + c * K;
+                    if constexpr (KT > 0) {
+#pragma unroll
+                        for (int k = 0; k < KT; ++k) {
+                            const float wk = wrow[k];
+                            d0 = fmaf(win[k], wk, d0);
+                            d1 = fmaf(win[k + 1], wk, d1);
+                            d2 = fmaf(win[k + 2], wk, d2);
+                            d3 = fmaf(win[k + 3], wk, d3);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < KMAXW; ++k) {
+                            if (k < K) {
+                                const float wk = wrow[k];
+                                d0 = fmaf(win[k], wk, d0);
+                                d1 = fmaf(win[k + 1], wk, d1);
+                                d2 = fmaf(win[k + 2], wk, d2);
+                                d3 = fmaf(win[k + 3], wk, d3);
+                            }
+                        }
                     }
                 }
                 dv[i][0] = d0; dv[i][1] = d1; dv[i][2] = d2; dv[i][3] = d3;
@@ -507,7 +509,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
 // fits the 16-sample register window.  Others take the FP32-FMA path.
 inline bool conv1d_tc_supported(int C, int O, int K, int stride)
 {
-    return stride == 1 && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1;
+    return stride == 1 && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1 && (long long)C * K <= tc::DW_MAX;
 }
 
 inline int launch_dwsep_conv1d_tc(const float* x, const float* dw, const float* pw, const float* bias, int N,
@@ -527,11 +529,12 @@ inline int launch_dwsep_conv1d_tc(const float* x, const float* dw, const float* 
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
-    if (cudaFuncSetAttribute(tc::dwsep_conv1d_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::SMEM_BYTES) != cudaSuccess)
+    auto kern = K == 9 ? tc::dwsep_conv1d_tc_kernel<9>
+              : K == 3 ? tc::dwsep_conv1d_tc_kernel<3> : tc::dwsep_conv1d_tc_kernel<0>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM_BYTES) != cudaSuccess)
         return FCV_ERR_CUDA;
     const int grid = (int)(total < sms ? total : sms);
-    tc::dwsep_conv1d_tc_kernel<<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(prm);
+    kern<<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(prm);
     return launch_status();
 }
 
