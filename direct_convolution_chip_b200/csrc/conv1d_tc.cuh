@@ -8,31 +8,40 @@
 // item with M = time, N = output channels, K = input channels.  The trace
 // planned mma.sync with TF32 operands and judged plain TF32 (10-bit mantissa)
 // too coarse for atol = rtol = 1e-4 (its precision discussion); here each fp32
-// operand v is split as hi = rna_tf32(v), lo = rna_tf32(v - hi), and
+// operand v is split as hi = round_tf32(v), lo = v - hi, and
 //     d * pw ~= d_hi*pw_hi + d_hi*pw_lo + d_lo*pw_hi,
 // dropping only d_lo*pw_lo (relative size ~2^-22), accumulated in fp32 in
 // tensor memory (the error-corrected TF32 scheme of Ootomo & Yokota, 2022).
+// hi is rounded to nearest (ties away from zero) with two integer operations.
 //
 // B200 design (one CTA per SM, persistent over tiles of 128 times x 256
 // output channels, K stepped in chunks of 32 channels = one 128-byte row):
-//   * warps 0-7 (producers): stage the input halo x[n, c0:c0+32, t0-p : ...]
-//     in shared memory, compute the depthwise tile with FP32 FMA (4 times x 4
-//     channels per thread from a 16-sample register window; the depthwise
-//     weights of all channels stay resident), split it into TF32 hi/lo and
-//     write both as K-major, 128B-swizzled UMMA operands; the pw chunk
-//     (256 x 32) is split the same way.  The global loads of the next chunk
-//     are in flight while the current chunk is computed.
+//   * warp 13 (TMA): as soon as a stage is free, one thread loads the raw
+//     pw chunk (256 output channels x 32 channels) with a 2-D TMA copy
+//     straight into the stage's B_hi buffer; the copy lands in the K-major,
+//     128B-swizzled layout the MMA reads.
+//   * warps 0-7 (producers): split that pw chunk in place into TF32 hi/lo
+//     (B_hi, B_lo); stage the input halo x[n, c0:c0+32, t0-p : ...] in shared
+//     memory, compute the depthwise tile with FP32 FMA (4 times x 4 channels
+//     per thread from a 16-sample register window; the depthwise weights of
+//     all channels stay resident) and write its hi/lo split as the A operand.
+//     The halo loads of the next chunk are in flight while the current chunk
+//     is computed.
 //   * warp 8: allocates 512 TMEM columns (two 128 x 256 fp32 accumulators);
 //     one thread issues 12 tcgen05.mma (kind::tf32, M=128, N=256, K=8) per
 //     chunk and commits them to the stage's "empty" barrier and, after the
 //     last chunk of a tile, to the accumulator's "full" barrier.
 //   * warps 9-12 (epilogue): drain one accumulator with tcgen05.ld while the
-//     MMAs fill the other, add the bias and store along t (each warp store
-//     covers 32 consecutive times of one output channel: 128 coalesced bytes).
+//     MMAs fill the other, add the bias, transpose 4x4 blocks inside lane
+//     quads and store 16 bytes of consecutive times per lane (one warp store
+//     covers 128 contiguous bytes in each of 4 output rows).
 //   * Every wait is bounded: a wait that runs out sets a CTA abort flag and
 //     the device error word, every role then leaves its loop, outstanding
 //     MMAs are drained (bounded) and TMEM is freed before the CTA exits.
 #pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include "common.cuh"
 
@@ -45,13 +54,14 @@ constexpr int KC = 32;         // channels per chunk: one 128-byte fp32 row
 constexpr int STAGES = 2;
 constexpr int NPROD = 256;     // producer threads, warps 0..7
 constexpr int MMA_WARP = 8;
-constexpr int NTHREADS = 13 * 32;
+constexpr int TMA_WARP = 13;
+constexpr int NTHREADS = 14 * 32;
 constexpr int KMAXW = 13;      // largest depthwise kernel (stride 1) of the register window
 constexpr int XW_MAX = TM - 1 + KMAXW;  // 140 halo samples per channel at most
 constexpr int XU = (XW_MAX + 31) / 32;  // halo samples per lane per channel
 constexpr int XWP = 144;       // halo row pitch in floats (multiple of 8)
 constexpr int XS_FLOATS = KC * XWP + 28;  // + skew of 4 floats per group of 4 channels
-constexpr int DW_MAX = 4000;   // resident depthwise weights: C * K at most
+constexpr int DW_MAX = 4000;   // resident depthwise weights: K * round_up(C, 4) at most
 constexpr uint32_t TMEM_COLS = 2 * TN;
 
 constexpr uint32_t A_BYTES = TM * KC * 4;    // 16 KB
@@ -60,7 +70,7 @@ constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;  // A_hi | A_lo | B_
 constexpr uint32_t OFF_XS = STAGES * STAGE_BYTES;
 constexpr uint32_t OFF_DWS = OFF_XS + XS_FLOATS * 4;
 constexpr uint32_t OFF_BAR = (OFF_DWS + DW_MAX * 4 + 7) & ~7u;
-constexpr uint32_t NBAR = 9;   // full[2] empty[2] afull[2] aempty[2] drain
+constexpr uint32_t NBAR = 11;  // full[2] empty[2] afull[2] aempty[2] drain tma[2]
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024 B
@@ -170,25 +180,52 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int ch)
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4));
 }
 
-__device__ __forceinline__ float tf32_rna(float v)
+// Round an fp32 value to the nearest TF32 value (10 explicit mantissa bits),
+// ties away from zero: add half of the 13 dropped bits to the magnitude bits
+// and clear them.  A mantissa carry propagates into the exponent as it should.
+// Exact for every finite input whose rounded magnitude stays finite.
+__device__ __forceinline__ float tf32_round(float v)
 {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(v));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(v) + 0x1000u) & 0xFFFFE000u);
 }
 
+// v = hi + lo with hi the TF32 rounding of v; lo = v - hi is exact in fp32 and
+// |lo| <= 2^-11 |v|, so dropping lo's bits below TF32 precision costs at most
+// 2^-21 |v|.
 __device__ __forceinline__ void split4(const float4 v, float4& hi, float4& lo)
 {
-    hi.x = tf32_rna(v.x); lo.x = tf32_rna(v.x - hi.x);
-    hi.y = tf32_rna(v.y); lo.y = tf32_rna(v.y - hi.y);
-    hi.z = tf32_rna(v.z); lo.z = tf32_rna(v.z - hi.z);
-    hi.w = tf32_rna(v.w); lo.w = tf32_rna(v.w - hi.w);
+    hi.x = tf32_round(v.x); lo.x = v.x - hi.x;
+    hi.y = tf32_round(v.y); lo.y = v.y - hi.y;
+    hi.z = tf32_round(v.z); lo.z = v.z - hi.z;
+    hi.w = tf32_round(v.w); lo.w = v.w - hi.w;
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, float4 v)
 {
     asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
                  : "memory");
+}
+
+__device__ __forceinline__ float4 lds128(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];\n" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// 2-D tiled TMA load (no multicast) completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x0, int x1, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x0), "r"(x1), "r"(bar)
+        : "memory");
 }
 
 struct Params {
@@ -199,27 +236,46 @@ struct Params {
     float* out;
     int C, T, O, K, pad, To;
     int tiles_t, tiles_o, total_tiles;
-    int pw_vec;  // pw rows 16-byte aligned (C % 4 == 0, aligned base)
+    int out_vec;  // output rows 16-byte aligned (To % 4 == 0, aligned base)
 };
 
 struct TileCoord {
     int n, t0, o0;
 };
 
+// Tiles are numbered with time fastest, then output-channel tile, then batch:
+// CTAs running at the same moment write neighbouring 512-byte segments of the
+// same output rows, and both output-channel tiles of a batch item read its
+// input while it is still in L2.
 __device__ __forceinline__ TileCoord decode_tile(const Params& p, int tile)
 {
     TileCoord tc;
-    const int o_tile = tile % p.tiles_o;
-    const int rest = tile / p.tiles_o;
-    tc.t0 = (rest % p.tiles_t) * TM;
-    tc.n = rest / p.tiles_t;
-    tc.o0 = o_tile * TN;
+    tc.t0 = (tile % p.tiles_t) * TM;
+    const int rest = tile / p.tiles_t;
+    tc.o0 = (rest % p.tiles_o) * TN;
+    tc.n = rest / p.tiles_o;
     return tc;
+}
+
+// 4x4 transpose across the 4 lanes of a quad: lane j holds row j (x0..x3) on
+// entry and column j on exit.  Two butterfly stages of xor-shuffles.
+__device__ __forceinline__ void quad_transpose(float& x0, float& x1, float& x2, float& x3, int j)
+{
+    const bool b1 = (j & 2) != 0, b0 = (j & 1) != 0;
+    float s0 = b1 ? x0 : x2, s1 = b1 ? x1 : x3;
+    float r0 = __shfl_xor_sync(0xffffffffu, s0, 2), r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
+    if (b1) { x0 = r0; x1 = r1; } else { x2 = r0; x3 = r1; }
+    s0 = b0 ? x0 : x1;
+    s1 = b0 ? x2 : x3;
+    r0 = __shfl_xor_sync(0xffffffffu, s0, 1);
+    r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+    if (b0) { x0 = r0; x2 = r1; } else { x1 = r0; x3 = r1; }
 }
 
 // KT: the depthwise kernel size when known at compile time, 0 for any K <= KMAXW.
 template <int KT>
-__global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Params p)
+__global__ void __launch_bounds__(NTHREADS, 1)
+dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_map)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -231,6 +287,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
     const uint32_t bar_afull = bar_full + 32;        // + 8 * buf
     const uint32_t bar_aempty = bar_full + 48;       // + 8 * buf
     const uint32_t bar_drain = bar_full + 64;
+    const uint32_t bar_tma = bar_full + 72;          // + 8 * stage
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
     volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 8);
@@ -245,6 +302,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
             mbar_init(bar_aempty + 8 * i, 4);  // one arrival per epilogue warp
         }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_tma, 1);       // expect_tx arrival + TMA bytes
+        mbar_init(bar_tma + 8, 1);
         *abort_flag = 0u;
         *prod_abort = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -263,8 +322,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
     const int nk = (p.C + KC - 1) / KC;
     const int XW = TM - 1 + p.K;  // halo samples per channel (stride 1)
 
-    // Depthwise weights of every channel stay resident: [C][K], row pitch K.
-    for (int e = threadIdx.x; e < p.C * p.K; e += NTHREADS) dws[e] = __ldg(p.dw + e);
+    // Depthwise weights of every channel stay resident, transposed to [K][CP]
+    // (CP = C rounded up to 4, zero-padded) so one 16-byte load serves the 4
+    // channels a thread computes.
+    const int CP = (p.C + 3) & ~3;
+    for (int e = threadIdx.x; e < p.K * CP; e += NTHREADS) {
+        const int k = e / CP, c = e - (e / CP) * CP;
+        dws[e] = c < p.C ? __ldg(p.dw + (size_t)c * p.K + k) : 0.f;
+    }
     __syncthreads();
 
     if (warp < 8) {
@@ -274,51 +339,47 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
         const int tq = (lane >> 3) + 4 * warp; // depthwise: times 4*tq .. 4*tq+3
         const int K = KT > 0 ? KT : p.K;
         float xr[4][XU];   // halo of channels 4*warp .. 4*warp+3, samples lane + 32*u
-        float4 pr[8];      // pw chunk rows, 16 bytes each
-
-        auto fetch = [&](int tile, int kc) {
-            const TileCoord tcd = decode_tile(p, tile);
+        TileCoord ft = {0, 0, 0};
+        auto fetch = [&](int kc) {
             const int c0 = kc * KC;
-            const int tb = tcd.t0 - p.pad;
+            const int tb = ft.t0 - p.pad;
+            const bool interior = tb >= 0 && tb + 32 * XU <= p.T && c0 + KC <= p.C;
+            const float* xw = p.x + ((size_t)ft.n * p.C + c0 + 4 * warp) * p.T + tb + lane;
+            if (interior) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int c = c0 + 4 * warp + i;
-                const float* xrow = p.x + ((size_t)tcd.n * p.C + (c < p.C ? c : 0)) * p.T;
+                for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int u = 0; u < XU; ++u) {
-                    const int ti = tb + lane + 32 * u;
-                    xr[i][u] = (c < p.C && ti >= 0 && ti < p.T) ? __ldg(xrow + ti) : 0.f;
-                }
-            }
+                    for (int u = 0; u < XU; ++u) xr[i][u] = __ldg(xw + (size_t)i * p.T + 32 * u);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int row = warp * 32 + i * 4 + (lane >> 3);
-                const int o = tcd.o0 + row, c = c0 + 4 * (lane & 7);
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (o < p.O) {
-                    const float* src = p.pw + (size_t)o * p.C + c;
-                    if (p.pw_vec) {
-                        if (c < p.C) v = __ldg(reinterpret_cast<const float4*>(src));
-                    } else {
-                        if (c < p.C) v.x = __ldg(src);
-                        if (c + 1 < p.C) v.y = __ldg(src + 1);
-                        if (c + 2 < p.C) v.z = __ldg(src + 2);
-                        if (c + 3 < p.C) v.w = __ldg(src + 3);
+                for (int i = 0; i < 4; ++i) {
+                    const bool cok = c0 + 4 * warp + i < p.C;
+#pragma unroll
+                    for (int u = 0; u < XU; ++u) {
+                        const int ti = tb + lane + 32 * u;
+                        xr[i][u] = (cok && ti >= 0 && ti < p.T) ? __ldg(xw + (size_t)i * p.T + 32 * u) : 0.f;
                     }
                 }
-                pr[i] = v;
             }
         };
 
         int seq = 0;
         int tile = blockIdx.x, kc = 0;
-        if (tile < p.total_tiles) fetch(tile, kc);
+        if (tile < p.total_tiles) {
+            ft = decode_tile(p, tile);
+            fetch(kc);
+        }
         while (tile < p.total_tiles) {
             const int stage = seq & 1;
-            const uint32_t parity = ((seq >> 1) & 1) ^ 1;
-            if (ptid == 0 && !wait_bounded(bar_empty + 8 * stage, parity, abort_flag)) *prod_abort = 1u;
+            const uint32_t parity = (seq >> 1) & 1;
+            // The TMA of this stage's pw chunk has landed (so the stage is free as well).
+            if (ptid == 0 && !wait_bounded(bar_tma + 8 * stage, parity, abort_flag)) *prod_abort = 1u;
             asm volatile("bar.sync 1, 256;\n" ::: "memory");
             if (*prod_abort) break;
+            // Thread 0 saw this phase complete, so this returns at once; it gives
+            // every producer its own acquire of the TMA bytes.
+            for (int spin = 0; !mbar_try_wait(bar_tma + 8 * stage, parity) && spin < (1 << 20); ++spin) {
+            }
 
             const uint32_t a_hi = sbase + stage * STAGE_BYTES;
             const uint32_t a_lo = a_hi + A_BYTES;
@@ -337,13 +398,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
                     if (j < XWP) dst[j] = xr[i][u];
                 }
             }
-            // pw chunk, split into TF32 hi/lo, as the K-major B operand.
+            // pw chunk (raw fp32, as the TMA left it in B_hi), split in place into TF32 hi/lo.
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int row = warp * 32 + i * 4 + (lane >> 3);
-                float4 hi, lo;
-                split4(pr[i], hi, lo);
                 const uint32_t off = sw128_off(row, lane & 7);
+                float4 hi, lo;
+                split4(lds128(b_hi + off), hi, lo);
                 sts128(b_hi + off, hi);
                 sts128(b_lo + off, lo);
             }
@@ -353,48 +414,46 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
             if (++kc == nk) {
                 kc = 0;
                 tile += gridDim.x;
+                if (tile < p.total_tiles) ft = decode_tile(p, tile);
             }
-            if (tile < p.total_tiles) fetch(tile, kc);
+            if (tile < p.total_tiles) fetch(kc);
 
             // Depthwise tile: 4 times x 4 channels per thread, then the TF32 split as the A operand.
             float dv[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int cl = 4 * cg + i;
-                const int c = c0 + cl;
-                float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
-                if (c < p.C) {
-                    const float* xrow = xs + cl * XWP + 4 * ((cl >> 2) & 7) + 4 * tq;
-                    float win[16];
+            for (int i = 0; i < 4; ++i) dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
+            if (c0 + 4 * cg < p.C) {  // channels past C stay zero (their weights are zero-padded too)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
-                        win[4 * q] = v.x; win[4 * q + 1] = v.y; win[4 * q + 2] = v.z; win[4 * q + 3] = v.w;
+                for (int h = 0; h < 2; ++h) {  // two channel pairs: 2 windows of 16 samples live at a time
+                    float win[2][16];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int cl = 4 * cg + 2 * h + i;
+                        const float* xrow = xs + cl * XWP + 4 * ((cl >> 2) & 7) + 4 * tq;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
+                            win[i][4 * q] = v.x; win[i][4 * q + 1] = v.y; win[i][4 * q + 2] = v.z; win[i][4 * q + 3] = v.w;
+                        }
                     }
-                    const float* wrow = dws + c * K;
+                    const float* wcol = dws + c0 + 4 * cg + 2 * h;
+                    auto tap = [&](int k) {
+                        const float2 wk = *reinterpret_cast<const float2*>(wcol + k * CP);
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            dv[2 * h][r] = fmaf(win[0][k + r], wk.x, dv[2 * h][r]);
+                            dv[2 * h + 1][r] = fmaf(win[1][k + r], wk.y, dv[2 * h + 1][r]);
+                        }
+                    };
                     if constexpr (KT > 0) {
 #pragma unroll
-                        for (int k = 0; k < KT; ++k) {
-                            const float wk = wrow[k];
-                            d0 = fmaf(win[k], wk, d0);
-                            d1 = fmaf(win[k + 1], wk, d1);
-                            d2 = fmaf(win[k + 2], wk, d2);
-                            d3 = fmaf(win[k + 3], wk, d3);
-                        }
+                        for (int k = 0; k < KT; ++k) tap(k);
                     } else {
 #pragma unroll
-                        for (int k = 0; k < KMAXW; ++k) {
-                            if (k < K) {
-                                const float wk = wrow[k];
-                                d0 = fmaf(win[k], wk, d0);
-                                d1 = fmaf(win[k + 1], wk, d1);
-                                d2 = fmaf(win[k + 2], wk, d2);
-                                d3 = fmaf(win[k + 3], wk, d3);
-                            }
-                        }
+                        for (int k = 0; k < KMAXW; ++k)
+                            if (k < K) tap(k);
                     }
                 }
-                dv[i][0] = d0; dv[i][1] = d1; dv[i][2] = d2; dv[i][3] = d3;
             }
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
@@ -457,6 +516,40 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
             }
         }
         __syncwarp();
+    } else if (warp == TMA_WARP) {
+        // -------------------------------------------------------- TMA issuer
+        if (lane == 0) {
+            int seq = 0;
+            bool pending[2] = {false, false};
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+                const TileCoord tcd = decode_tile(p, tile);
+                for (int k = 0; k < nk; ++k, ++seq) {
+                    const int stage = seq & 1;
+                    if (!wait_bounded(bar_empty + 8 * stage, ((seq >> 1) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    pending[stage] = false;  // the producers consumed its previous load before the MMA ran
+                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES);
+                    tma_load_2d(sbase + stage * STAGE_BYTES + 2 * A_BYTES, &pw_map, k * KC, tcd.o0,
+                                bar_tma + 8 * stage);
+                    pending[stage] = true;
+                }
+            }
+            // On an abort, wait (bounded) for copies still in flight before the CTA can exit.
+            if (!ok) {
+                for (int st = 0; st < 2; ++st) {
+                    if (!pending[st]) continue;
+                    const int last = seq - 1 - ((seq - 1 - st) & 1);  // latest sequence number on this stage
+                    const unsigned long long t0 = globaltimer();
+                    while (last >= 0 && !mbar_try_wait(bar_tma + 8 * st, (last >> 1) & 1)) {
+                        if (globaltimer() - t0 > kWaitLimitNs) break;
+                    }
+                }
+            }
+        }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -469,22 +562,45 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
             if (!ok) break;
             tc_fence_after();
             const TileCoord tcd = decode_tile(p, tile);
-            const int t = tcd.t0 + 32 * q + lane;
-            const bool t_ok = t < p.To;
-            float* out_nt = p.out + (size_t)tcd.n * p.O * p.To + t;
+            const int tw = tcd.t0 + 32 * q;  // first time of this warp's 32 TMEM lanes
             const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TN);
+            // Fast path: all 32 times in range and 16-byte aligned rows.  After a
+            // 4x4 transpose inside each lane quad, lane 4k+j holds times
+            // tw+4k .. tw+4k+3 of output channels 4j .. 4j+3 (of the 16 loaded), so
+            // each 16-byte store instruction covers 128 contiguous bytes of 4 rows.
+            const bool vec = tw + 32 <= p.To && p.out_vec;
+            const int kq = lane >> 2, jq = lane & 3;
 #pragma unroll 1
             for (int cb = 0; cb < TN / 16; ++cb) {
                 uint32_t r[16];
                 tmem_ld16(taddr + (uint32_t)(cb * 16), r);
                 tmem_wait_ld();
                 const int obase = tcd.o0 + cb * 16;
+                float v[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int o = obase + j;
-                    if (t_ok && o < p.O) {
-                        const float bo = p.bias ? __ldg(p.bias + o) : 0.f;
-                        out_nt[(size_t)o * p.To] = __uint_as_float(r[j]) + bo;
+                    v[j] = __uint_as_float(r[j]) + ((p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f);
+                }
+                if (vec) {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        // block m: rows = the 4 lanes' times, columns = channels m, 4+m, 8+m, 12+m
+                        float x0 = v[m], x1 = v[4 + m], x2 = v[8 + m], x3 = v[12 + m];
+                        quad_transpose(x0, x1, x2, x3, jq);
+                        const int o = obase + 4 * jq + m;
+                        if (o < p.O) {
+                            float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
+                            *reinterpret_cast<float4*>(dst) = make_float4(x0, x1, x2, x3);
+                        }
+                    }
+                } else {
+                    const int t = tw + lane;
+                    float* out_nt = p.out + (size_t)tcd.n * p.O * p.To + t;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int o = obase + j;
+                        if (t < p.To && o < p.O) out_nt[(size_t)o * p.To] = v[j];
                     }
                 }
             }
@@ -507,9 +623,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) dwsep_conv1d_tc_kernel(const Para
 
 // Shapes the tensor-core path covers: stride 1 and a depthwise kernel that
 // fits the 16-sample register window.  Others take the FP32-FMA path.
-inline bool conv1d_tc_supported(int C, int O, int K, int stride)
+inline bool conv1d_tc_supported(int C, int O, int K, int stride, const void* pw = nullptr)
 {
-    return stride == 1 && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1 && (long long)C * K <= tc::DW_MAX;
+    // C % 4 == 0 and a 16-byte aligned pw: the TMA copy of pw needs 16-byte row strides.
+    return stride == 1 && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1 && (C & 3) == 0 &&
+           (reinterpret_cast<uintptr_t>(pw) & 15) == 0 && (long long)C * K <= tc::DW_MAX;
+}
+
+// cuTensorMapEncodeTiled, resolved once through the runtime (no libcuda link).
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
 }
 
 inline int launch_dwsep_conv1d_tc(const float* x, const float* dw, const float* pw, const float* bias, int N,
@@ -525,7 +657,23 @@ inline int launch_dwsep_conv1d_tc(const float* x, const float* dw, const float* 
     const long long total = (long long)N * prm.tiles_t * prm.tiles_o;
     if (total > 0x7fffffffLL) return FCV_ERR_UNSUPPORTED;
     prm.total_tiles = (int)total;
-    prm.pw_vec = ((C & 3) == 0 && (reinterpret_cast<uintptr_t>(pw) & 15) == 0) ? 1 : 0;
+    prm.out_vec = ((To & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0) ? 1 : 0;
+
+    // pw [O][C] as a 2-D tensor: inner dim C (contiguous), outer dim O; one box
+    // is 32 channels x 256 output channels, 128B-swizzled; out-of-range rows
+    // and columns read as zero.
+    auto encode = tensor_map_encoder();
+    if (!encode) return FCV_ERR_CUDA;
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {(cuuint64_t)C, (cuuint64_t)O};
+    const cuuint64_t gstride[1] = {(cuuint64_t)C * sizeof(float)};
+    const cuuint32_t box[2] = {(cuuint32_t)tc::KC, (cuuint32_t)tc::TN};
+    const cuuint32_t estride[2] = {1, 1};
+    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pw), gdim, gstride, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return FCV_ERR_CUDA;
+
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
@@ -534,7 +682,7 @@ inline int launch_dwsep_conv1d_tc(const float* x, const float* dw, const float* 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM_BYTES) != cudaSuccess)
         return FCV_ERR_CUDA;
     const int grid = (int)(total < sms ? total : sms);
-    kern<<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(prm);
+    kern<<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(prm, map);
     return launch_status();
 }
 

@@ -117,14 +117,14 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
     cudaStream_t s = fcv::as_stream(stream);
     switch (algo) {
     case FCV_ALGO_AUTO:
-        if (fcv::conv1d_tc_supported(C, O, K, stride)) {
+        if (fcv::conv1d_tc_supported(C, O, K, stride, pw_w)) {
             return fcv::launch_dwsep_conv1d_tc(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
         }
         return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     case FCV_CONV1D_FMA:
         return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     case FCV_CONV1D_TC_3XTF32:
-        if (!fcv::conv1d_tc_supported(C, O, K, stride)) return FCV_ERR_UNSUPPORTED;
+        if (!fcv::conv1d_tc_supported(C, O, K, stride, pw_w)) return FCV_ERR_UNSUPPORTED;
         return fcv::launch_dwsep_conv1d_tc(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     default:
         return FCV_ERR_INVALID_ARG;
