@@ -242,8 +242,14 @@ def traffic_per_launch(kernel_key):
     return e["bytes_per_launch"] if h == e["source_sha256"] else None
 
 
+def job_throughput(flops_per_rank_step, world, max_step_s):
+    """Whole-job GFLOP/s: every rank's work divided by the slowest rank's step time."""
+    return flops_per_rank_step * world / max_step_s / 1e9
+
+
 def run_oracle_sample(budget_s=12.0):
-    """Time the CPU oracle (as it stands) on whole batch items of both workloads."""
+    """Time the CPU oracle (as it stands) on whole batch items of both workloads,
+    repeating full passes until about `budget_s` seconds of CPU work."""
     import oracle
     xa, wa, ba = wl.conv2d_inputs(CASE_A)
     xb, dwb, pwb, bb = wl.conv1d_inputs(CASE_B)
@@ -251,25 +257,21 @@ def run_oracle_sample(budget_s=12.0):
     xb, dwb, pwb, bb = xb.numpy(), dwb.numpy(), pwb.numpy(), bb.numpy()
     per_a = macs_conv2d(1, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout, CASE_A.P)
     per_b = macs_conv1d(1, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K, CASE_B.stride, CASE_B.pad)
-
-    def time_a(n):
+    items_a = items_b = 0
+    ta = tb = 0.0
+    while ta + tb < budget_s:
         t = time.perf_counter()
-        oracle.conv2d_pool_sigmoid_sum(xa[:n], wa, ba, CASE_A.P)
-        return time.perf_counter() - t
-
-    def time_b(n):
+        oracle.conv2d_pool_sigmoid_sum(xa, wa, ba, CASE_A.P)
+        ta += time.perf_counter() - t
+        items_a += CASE_A.N
         t = time.perf_counter()
-        oracle.dwsep_conv1d(xb[:n], dwb, pwb, bb, CASE_B.stride, CASE_B.pad)
-        return time.perf_counter() - t
-
-    ta1, tb1 = time_a(1), time_b(1)
-    na = max(1, min(CASE_A.N, int(budget_s / 2 / max(ta1, 1e-3))))
-    nb = max(1, min(CASE_B.N, int(budget_s / 2 / max(tb1, 1e-3))))
-    ta, tb = time_a(na), time_b(nb)
-    flops = 2.0 * (na * per_a + nb * per_b)
+        oracle.dwsep_conv1d(xb, dwb, pwb, bb, CASE_B.stride, CASE_B.pad)
+        tb += time.perf_counter() - t
+        items_b += CASE_B.N
+    flops = 2.0 * (items_a * per_a + items_b * per_b)
     return {"value": flops / (ta + tb) / 1e9, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"op A batch items 0..{na - 1} of {CASE_A.N} ({ta:.2f} s) + op B batch items "
-                      f"0..{nb - 1} of {CASE_B.N} ({tb:.2f} s); double-precision OpenMP loops"}
+            "sample": f"{items_a // CASE_A.N} full pass(es) of both workloads: op A {items_a} batch items "
+                      f"({ta:.2f} s), op B {items_b} batch items ({tb:.2f} s); double-precision OpenMP loops"}
 
 
 def run_gpu(args):
@@ -361,7 +363,7 @@ def run_gpu(args):
     macs_a, macs_b = case_macs(CASE_A), case_macs(CASE_B)
     bytes_a, bytes_b = case_bytes(CASE_A), case_bytes(CASE_B)
     step_s = total_ms / K / 1e3
-    value = 2.0 * (macs_a + macs_b) * world / step_s / 1e9
+    value = job_throughput(2.0 * (macs_a + macs_b), world, step_s)
     peaks, peak_src = load_peaks()
     hbm = peaks["hbm_gbs"]
     fma_peak = fma_peak_tflops(props)
@@ -403,7 +405,7 @@ def run_gpu(args):
                    "conv1d_path": conv1d_tc},
         "per_op": per_op, "roofline": roof,
         "peaks": {"hbm_gbs": hbm, "fp32_fma_tflops": fma_peak, "tf32_tflops": tf32_peak, "source": peak_src},
-        "e2e": {"value": 2.0 * (macs_a + macs_b) * world / (e2e_ms / 1e3) / 1e9, "unit": UNIT,
+        "e2e": {"value": job_throughput(2.0 * (macs_a + macs_b), world, e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": e2e_steps},
         "gpu_launches": 2 * K,
