@@ -35,6 +35,8 @@ SIGNATURES = {
     "fcv_conv2d_pool_sigmoid_sum": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "fcv_conv2d_pool_sigmoid_sum_ex": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
     "fcv_conv2d_pool_tap": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
+    "fcv_conv2d_pool_sigmoid_sum_det": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]),
+    "fcv_conv2d_workspace_bytes": (_I, [_I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
     "fcv_dwsep_conv1d": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "fcv_dwsep_conv1d_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
     "fcv_status_string": (ctypes.c_char_p, [_I]),
@@ -149,6 +151,39 @@ def conv2d_pool_sigmoid_sum(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None
     _check(lib.fcv_conv2d_pool_sigmoid_sum_ex(_ptr(xd), _ptr(wd), _ptr(bd), N, Cin, H, W, Cout, pool,
                                               _ptr(out), algo, _stream_ptr(stream)),
            "fcv_conv2d_pool_sigmoid_sum")
+    return _result(out, host, stream)
+
+
+def conv2d_workspace_bytes(N, Cin, H, W, Cout, pool) -> int:
+    """Workspace bytes the deterministic conv2d sum needs for these sizes."""
+    v = ctypes.c_size_t()
+    _check(load().fcv_conv2d_workspace_bytes(N, Cin, H, W, Cout, pool, ctypes.byref(v)),
+           "fcv_conv2d_workspace_bytes")
+    return v.value
+
+
+def conv2d_pool_sigmoid_sum_det(x, w, b, pool, out=None, workspace=None, stream=None):
+    """Bitwise-reproducible variant of conv2d_pool_sigmoid_sum.
+
+    `workspace` is a device tensor of at least conv2d_workspace_bytes(...) bytes
+    (allocated here through torch when omitted)."""
+    lib = load()
+    host = _host_mode(x, w, b)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    N, Cin, H, W = x.shape
+    Cout = w.shape[0]
+    if tuple(w.shape) != (Cout, Cin, 3, 3) or tuple(b.shape) != (Cout,):
+        raise ValueError("w must be [Cout,Cin,3,3] and b [Cout]")
+    need = conv2d_workspace_bytes(N, Cin, H, W, Cout, pool)
+    if workspace is None:
+        workspace = torch.empty(((need + 15) // 16 * 4,), dtype=torch.float32, device=dev)
+    nbytes = workspace.numel() * workspace.element_size()
+    xd, wd, bd = _dev(x, "x", dev), _dev(w, "w", dev), _dev(b, "b", dev)
+    if out is None or host:
+        out = torch.empty((N,), dtype=torch.float32, device=xd.device)
+    _check(lib.fcv_conv2d_pool_sigmoid_sum_det(_ptr(xd), _ptr(wd), _ptr(bd), N, Cin, H, W, Cout, pool, _ptr(out),
+                                               _ptr(workspace) if need else None, nbytes, _stream_ptr(stream)),
+           "fcv_conv2d_pool_sigmoid_sum_det")
     return _result(out, host, stream)
 
 

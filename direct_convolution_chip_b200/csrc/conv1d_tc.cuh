@@ -320,7 +320,6 @@ dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_ma
     const uint32_t tmem = *tmem_holder;
 
     const int nk = (p.C + KC - 1) / KC;
-    const int XW = TM - 1 + p.K;  // halo samples per channel (stride 1)
 
     // Depthwise weights of every channel stay resident, transposed to [K][CP]
     // (CP = C rounded up to 4, zero-padded) so one 16-byte load serves the 4

@@ -70,15 +70,45 @@ struct Conv2dGeom {
     static constexpr int PX = RX * P + 2;           // register patch cols
     static constexpr int HALO_FLOATS = ICC * HY * HXP;
     static constexpr int W_FLOATS = ICC * 9 * CB;
-    static constexpr size_t SMEM_BYTES = sizeof(float) * (HALO_FLOATS + W_FLOATS + NT / 32);
+    static constexpr size_t SMEM_BYTES = sizeof(float) * (HALO_FLOATS + W_FLOATS + NT / 32 + 1);
 };
 
-template <int P, bool TAP, bool PACKED = (P <= FCV_CONV2D_PACKED_MAX_P)>
+// What the kernel produces.
+enum Conv2dMode : int {
+    kSumAtomic = 0,  // out[n] += one block sum per CTA (atomicAdd; out pre-zeroed)
+    kTap = 1,        // pooled pre-sigmoid values, no sum
+    kSumDet = 2,     // block sums to a workspace; the last CTA of each image sums them in a fixed order
+};
+
+// Sum of `v` (double) over a thread block, valid in thread 0; fixed order.
+template <int NT>
+__device__ __forceinline__ double block_sum_d(double v, double* scratch)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    double s = 0.0;
+    if (threadIdx.x < 32) {
+        s = (lane < NT / 32) ? scratch[lane] : 0.0;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    }
+    return s;
+}
+
+// MODE is a Conv2dMode.  partials/counters are used by kSumDet only: the
+// workspace holds one float per CTA ([N][per_image]) and one counter per image
+// (zero at launch).
+template <int P, int MODE, bool PACKED = (P <= FCV_CONV2D_PACKED_MAX_P)>
 __global__ void __launch_bounds__(Conv2dGeom<P>::NT, 2)
 conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
                      const float* __restrict__ bias, int Cin, int H, int W, int Cout,
-                     int PH, int PW, int tiles_y, int tiles_x, float* __restrict__ out)
+                     int PH, int PW, int tiles_y, int tiles_x, float* __restrict__ out,
+                     float* __restrict__ partials, unsigned int* __restrict__ counters)
 {
+    constexpr bool TAP = MODE == kTap;
     using G = Conv2dGeom<P>;
     constexpr int RX = G::RX, CG = G::CG, NPOS = G::NPOS, NT = G::NT, CB = G::CB;
     constexpr int HY = G::HY, HX = G::HX, HXP = G::HXP, PY = G::PY, PX = G::PX, ICC = G::ICC;
@@ -229,49 +259,110 @@ conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
             }
         }
     }
-    if (!TAP) {
+    if (MODE == kSumAtomic) {
         const float total = block_sum<NT>(local, red);
         if (tid == 0) atomicAdd(out + n, total);
+    } else if (MODE == kSumDet) {
+        // Deterministic: this CTA's block sum goes to its own workspace slot; the
+        // CTA that finishes last for image n (seen through a counter, nothing
+        // waits) adds the slots in a fixed order and writes out[n].
+        const float total = block_sum<NT>(local, red);
+        const int per_image = tiles_y * tiles_x * (int)gridDim.y;
+        const int slot = ((int)(blockIdx.x % (unsigned)(tiles_y * tiles_x))) * (int)gridDim.y + (int)blockIdx.y;
+        volatile int* last = reinterpret_cast<volatile int*>(red + NT / 32);
+        if (tid == 0) {
+            partials[(size_t)n * per_image + slot] = total;
+            __threadfence();
+            const unsigned int prev = atomicAdd(counters + n, 1u);
+            *last = (prev == (unsigned int)per_image - 1u) ? 1 : 0;
+        }
+        __syncthreads();
+        if (*last) {
+            __threadfence();
+            double sacc = 0.0;
+            for (int i = tid; i < per_image; i += NT) sacc += (double)__ldcg(partials + (size_t)n * per_image + i);
+            __syncthreads();  // red is reused below
+            const double all = block_sum_d<NT>(sacc, reinterpret_cast<double*>(halo));
+            if (tid == 0) out[n] = (float)all;
+        }
     }
 }
 
-template <int P, bool TAP>
-int launch_conv2d_direct_p(const float* x, const float* w, const float* b, int N, int Cin, int H,
-                           int W, int Cout, int PH, int PW, float* out, cudaStream_t stream)
+// Grid of the direct kernel for pool size P: tiles per image and channel blocks.
+template <int P>
+void conv2d_grid_p(int PH, int PW, int Cout, int* tiles_y, int* tiles_x, int* cblocks)
 {
     using G = Conv2dGeom<P>;
-    const int tiles_y = (PH + G::TILE_PH - 1) / G::TILE_PH;
-    const int tiles_x = (PW + G::TILE_PW - 1) / G::TILE_PW;
+    *tiles_y = (PH + G::TILE_PH - 1) / G::TILE_PH;
+    *tiles_x = (PW + G::TILE_PW - 1) / G::TILE_PW;
+    *cblocks = (Cout + G::CB - 1) / G::CB;
+}
+
+inline bool conv2d_grid(int P, int PH, int PW, int Cout, int* tiles_y, int* tiles_x, int* cblocks)
+{
+    switch (P) {
+    case 1: conv2d_grid_p<1>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 2: conv2d_grid_p<2>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 3: conv2d_grid_p<3>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 4: conv2d_grid_p<4>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 5: conv2d_grid_p<5>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 6: conv2d_grid_p<6>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 7: conv2d_grid_p<7>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 8: conv2d_grid_p<8>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    default: return false;
+    }
+}
+
+template <int P, int MODE>
+int launch_conv2d_direct_p(const float* x, const float* w, const float* b, int N, int Cin, int H,
+                           int W, int Cout, int PH, int PW, float* out, float* partials,
+                           unsigned int* counters, cudaStream_t stream)
+{
+    using G = Conv2dGeom<P>;
+    int tiles_y, tiles_x, cblk;
+    conv2d_grid_p<P>(PH, PW, Cout, &tiles_y, &tiles_x, &cblk);
     const long long nblk = (long long)N * tiles_y * tiles_x;
-    const int cblk = (Cout + G::CB - 1) / G::CB;
     if (nblk > 0x7fffffffLL || cblk > 65535) return FCV_ERR_UNSUPPORTED;
-    auto kern = conv2d_direct_kernel<P, TAP>;
+    auto kern = conv2d_direct_kernel<P, MODE>;
     if (G::SMEM_BYTES > 48 * 1024) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)G::SMEM_BYTES) != cudaSuccess)
             return FCV_ERR_CUDA;
     }
     dim3 grid((unsigned)nblk, (unsigned)cblk);
-    kern<<<grid, G::NT, G::SMEM_BYTES, stream>>>(x, w, b, Cin, H, W, Cout, PH, PW, tiles_y, tiles_x, out);
+    kern<<<grid, G::NT, G::SMEM_BYTES, stream>>>(x, w, b, Cin, H, W, Cout, PH, PW, tiles_y, tiles_x, out,
+                                                  partials, counters);
     return launch_status();
 }
 
 // PH, PW >= 1 here; the caller handles the empty cases.
-template <bool TAP>
+template <int MODE>
 int launch_conv2d_direct(const float* x, const float* w, const float* b, int N, int Cin, int H,
-                         int W, int Cout, int P, int PH, int PW, float* out, cudaStream_t stream)
+                         int W, int Cout, int P, int PH, int PW, float* out, cudaStream_t stream,
+                         float* partials = nullptr, unsigned int* counters = nullptr)
 {
     switch (P) {
-    case 1: return launch_conv2d_direct_p<1, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
-    case 2: return launch_conv2d_direct_p<2, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
-    case 3: return launch_conv2d_direct_p<3, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
-    case 4: return launch_conv2d_direct_p<4, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
-    case 5: return launch_conv2d_direct_p<5, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
-    case 6: return launch_conv2d_direct_p<6, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
-    case 7: return launch_conv2d_direct_p<7, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
-    case 8: return launch_conv2d_direct_p<8, TAP>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, stream);
+    case 1: return launch_conv2d_direct_p<1, MODE>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials, counters, stream);
+    case 2: return launch_conv2d_direct_p<2, MODE>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials, counters, stream);
+    case 3: return launch_conv2d_direct_p<3, MODE>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials, counters, stream);
+    case 4: return launch_conv2d_direct_p<4, MODE>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials, counters, stream);
+    case 5: return launch_conv2d_direct_p<5, MODE>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials, counters, stream);
+    case 6: return launch_conv2d_direct_p<6, MODE>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials, counters, stream);
+    case 7: return launch_conv2d_direct_p<7, MODE>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials, counters, stream);
+    case 8: return launch_conv2d_direct_p<8, MODE>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials, counters, stream);
     default: return FCV_ERR_UNSUPPORTED;
     }
+}
+
+// Workspace of the deterministic sum: [N][per_image] floats, then N counters
+// (16-byte aligned).  0 bytes when nothing is launched (PH or PW == 0).
+inline size_t conv2d_det_workspace_bytes(int N, int Cout, int P, int PH, int PW)
+{
+    if (N <= 0 || PH <= 0 || PW <= 0) return 0;
+    int ty, tx, cb;
+    if (!conv2d_grid(P, PH, PW, Cout, &ty, &tx, &cb)) return 0;
+    const size_t part = ((size_t)N * ty * tx * cb * sizeof(float) + 15) & ~(size_t)15;
+    return part + (size_t)N * sizeof(unsigned int);
 }
 
 }  // namespace fcv

@@ -81,13 +81,45 @@ int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin
         if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N, s) != cudaSuccess) return FCV_ERR_CUDA;
     }
     if (PH == 0 || PW == 0) return FCV_OK;  // empty sum: out stays 0; the tap has no elements
-    return tap ? fcv::launch_conv2d_direct<true>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
-               : fcv::launch_conv2d_direct<false>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
+    return tap ? fcv::launch_conv2d_direct<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
+               : fcv::launch_conv2d_direct<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
 }
 
 }  // namespace
 
 extern "C" {
+
+int fcv_conv2d_workspace_bytes(int N, int Cin, int H, int W, int Cout, int pool, size_t* bytes)
+{
+    if (!bytes) return FCV_ERR_INVALID_ARG;
+    if (N < 0 || Cin < 1 || Cout < 1 || H < 3 || W < 3 || pool < 1) return FCV_ERR_INVALID_ARG;
+    if (!mul_ok(N, Cin, H, W) || !mul_ok(N, Cout, H, W)) return FCV_ERR_INVALID_ARG;
+    if (pool > 8) return FCV_ERR_UNSUPPORTED;
+    *bytes = fcv::conv2d_det_workspace_bytes(N, Cout, pool, (H - 2) / pool, (W - 2) / pool);
+    return FCV_OK;
+}
+
+int fcv_conv2d_pool_sigmoid_sum_det(const float* x, const float* w, const float* b, int N, int Cin, int H,
+                                    int W, int Cout, int pool, float* out, void* workspace,
+                                    size_t workspace_bytes, void* stream)
+{
+    int st = check_conv2d(x, w, b, N, Cin, H, W, Cout, pool, out, false);
+    if (st != FCV_OK) return st;
+    const int PH = (H - 2) / pool, PW = (W - 2) / pool;
+    const size_t need = fcv::conv2d_det_workspace_bytes(N, Cout, pool, PH, PW);
+    if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 15) != 0 || workspace_bytes < need))
+        return FCV_ERR_INVALID_ARG;
+    if (N == 0) return FCV_OK;
+    cudaStream_t s = fcv::as_stream(stream);
+    if (PH == 0 || PW == 0) {
+        return cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N, s) == cudaSuccess ? FCV_OK : FCV_ERR_CUDA;
+    }
+    unsigned char* base = static_cast<unsigned char*>(workspace);
+    unsigned int* counters = reinterpret_cast<unsigned int*>(base + need - sizeof(unsigned int) * (size_t)N);
+    if (cudaMemsetAsync(counters, 0, sizeof(unsigned int) * (size_t)N, s) != cudaSuccess) return FCV_ERR_CUDA;
+    return fcv::launch_conv2d_direct<fcv::kSumDet>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s,
+                                                   reinterpret_cast<float*>(base), counters);
+}
 
 int fcv_conv2d_pool_sigmoid_sum(const float* x, const float* w, const float* b, int N, int Cin, int H,
                                 int W, int Cout, int pool, float* out, void* stream)

@@ -43,6 +43,8 @@
 #ifndef FCV_H
 #define FCV_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -91,6 +93,31 @@ int fcv_conv2d_pool_sigmoid_sum(const float* x, const float* w, const float* b,
 int fcv_conv2d_pool_sigmoid_sum_ex(const float* x, const float* w, const float* b,
                                    int N, int Cin, int H, int W, int Cout, int pool,
                                    float* out, int algo, void* stream);
+
+/* Deterministic variant of fcv_conv2d_pool_sigmoid_sum: bitwise-identical
+ * results from run to run.  Each thread block writes its partial sum to its
+ * own slot of a caller-provided workspace; the block that finishes last for a
+ * batch item (detected with a counter; nothing waits) adds that item's slots
+ * in a fixed order and stores out[n].  Same result within rounding as the
+ * atomic variant; the alternative the l2_p65 trace weighs in its
+ * atomic-contention analysis (a per-tile workspace plus a fixed-order pass).
+ *
+ *   workspace        device memory owned by the caller, 16-byte aligned, at
+ *                    least fcv_conv2d_workspace_bytes(...) bytes; its contents
+ *                    on entry do not matter (the library clears what it needs
+ *                    on `stream`).  Calls sharing a workspace must not overlap.
+ *   workspace_bytes  its size.
+ * INVALID_ARG additionally when the workspace is NULL, misaligned or too small
+ * (a zero-byte requirement accepts NULL). */
+int fcv_conv2d_pool_sigmoid_sum_det(const float* x, const float* w, const float* b,
+                                    int N, int Cin, int H, int W, int Cout, int pool,
+                                    float* out, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/* Bytes of workspace fcv_conv2d_pool_sigmoid_sum_det needs for these sizes
+ * (0 when nothing is launched, e.g. PH or PW == 0).  Host only, no CUDA call.
+ * Same INVALID_ARG / UNSUPPORTED rules as the compute entry points. */
+int fcv_conv2d_workspace_bytes(int N, int Cin, int H, int W, int Cout, int pool, size_t* bytes);
 
 /* The pooled pre-sigmoid values of the same kernel, for checking the conv and
  * pool stages element by element:

@@ -112,3 +112,24 @@ def test_conv1d_empty_batch_and_null_bias(lib):
 def test_binding_raises_without_library(tmp_path):
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         binding.load(str(tmp_path / "missing.so"))
+
+
+def test_det_workspace_bytes(lib):
+    v = ctypes.c_size_t()
+    # x[128,8,384,384], Cout 64, pool 4: 12 x 12 tiles of 8x8 pooled outputs, one channel block
+    assert lib.fcv_conv2d_workspace_bytes(128, 8, 384, 384, 64, 4, ctypes.byref(v)) == OK
+    assert v.value == 128 * 144 * 4 + 128 * 4
+    assert lib.fcv_conv2d_workspace_bytes(2, 3, 5, 40, 4, 4, ctypes.byref(v)) == OK and v.value == 0  # PH = 0
+    assert lib.fcv_conv2d_workspace_bytes(0, 3, 9, 9, 4, 2, ctypes.byref(v)) == OK and v.value == 0
+    assert lib.fcv_conv2d_workspace_bytes(1, 3, 9, 9, 4, 9, ctypes.byref(v)) == UNSUPPORTED
+    assert lib.fcv_conv2d_workspace_bytes(1, 0, 9, 9, 4, 2, ctypes.byref(v)) == INVALID
+    assert lib.fcv_conv2d_workspace_bytes(1, 3, 9, 9, 4, 2, None) == INVALID
+
+
+def test_det_rejects_missing_or_small_workspace(lib):
+    det = lib.fcv_conv2d_pool_sigmoid_sum_det
+    args = (FAKE, FAKE, FAKE, 2, 8, 64, 64, 16, 4, FAKE)
+    assert det(*args, None, 1 << 20, None) == INVALID          # workspace needed
+    assert det(*args, P(0x10008), 1 << 20, None) == INVALID    # not 16-byte aligned
+    assert det(*args, FAKE, 8, None) == INVALID                # too small
+    assert det(FAKE, FAKE, FAKE, 0, 8, 64, 64, 16, 4, FAKE, None, 0, None) == OK  # empty batch

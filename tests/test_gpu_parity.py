@@ -295,3 +295,48 @@ def test_empty_batch_through_binding():
     x1 = torch.zeros((0, 3, 10), device="cuda")
     out = fcv.dwsep_conv1d(x1, torch.zeros((3, 3), device="cuda"), torch.zeros((5, 3), device="cuda"), None, 1, 1)
     assert out.shape == (0, 5, 10)
+
+
+# ------------------------------------------------- op A, deterministic sum ---
+
+@pytest.mark.parametrize("case", [wl.CONV2D_SMALL, wl.CONV2D_FULL,
+                                  wl.Conv2dCase("det_odd", 3, 5, 61, 47, 70, 3, seed=17),
+                                  wl.Conv2dCase("det_p2", 4, 16, 130, 130, 128, 2, seed=18)],
+                         ids=lambda c: c.name)
+def test_conv2d_det_parity_and_bitwise_repeatable(case):
+    x, w, b = wl.conv2d_inputs(case)
+    xd, wd, bd = cuda(x, w, b)
+    need = fcv.conv2d_workspace_bytes(case.N, case.Cin, case.H, case.W, case.Cout, case.P)
+    ws = torch.full(((need + 15) // 16 * 4,), float("nan"), device="cuda")  # contents on entry do not matter
+    first = fcv.conv2d_pool_sigmoid_sum_det(xd, wd, bd, case.P, workspace=ws).clone()
+    ws.fill_(123.0)
+    second = fcv.conv2d_pool_sigmoid_sum_det(xd, wd, bd, case.P, workspace=ws)
+    atomic = fcv.conv2d_pool_sigmoid_sum(xd, wd, bd, case.P)
+    torch.cuda.synchronize()
+    assert torch.equal(first, second), "deterministic mode differs between runs"
+    assert torch.allclose(first, atomic, rtol=1e-6, atol=0)
+    xn, wn, bn = x.numpy(), w.numpy(), b.numpy()
+    for bi in sorted({0, case.N - 1}):
+        assert_close(first[bi:bi + 1], oracle.conv2d_pool_sigmoid_sum(xn[bi:bi + 1], wn, bn, case.P),
+                     f"{case.name} det out[{bi}]")
+
+
+def test_conv2d_det_empty_pool_and_guard_bands():
+    case = wl.Conv2dCase("det_empty", 3, 2, 5, 40, 4, 4, seed=9)  # PH = 0: no workspace needed
+    x, w, b = cuda(*wl.conv2d_inputs(case))
+    assert fcv.conv2d_workspace_bytes(3, 2, 5, 40, 4, 4) == 0
+    out = torch.full((3,), 7.0, device="cuda")
+    fcv.conv2d_pool_sigmoid_sum_det(x, w, b, 4, out=out)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+    guard = 256
+    c2 = wl.Conv2dCase("det_guard", 5, 3, 50, 45, 20, 4, seed=10)
+    x, w, b = cuda(*wl.conv2d_inputs(c2))
+    need = fcv.conv2d_workspace_bytes(c2.N, c2.Cin, c2.H, c2.W, c2.Cout, c2.P)
+    wbuf = torch.full((need // 4 + 2 * guard,), float("nan"), device="cuda")
+    obuf = torch.full((c2.N + 2 * guard,), float("nan"), device="cuda")
+    fcv.conv2d_pool_sigmoid_sum_det(x, w, b, c2.P, out=obuf[guard:guard + c2.N], workspace=wbuf[guard:guard + need // 4])
+    torch.cuda.synchronize()
+    for buf in (wbuf, obuf):
+        assert torch.isnan(buf[:guard]).all() and torch.isnan(buf[-guard:]).all()
+    assert torch.isfinite(obuf[guard:guard + c2.N]).all()
