@@ -37,6 +37,7 @@ SIGNATURES = {
     "fcv_conv2d_pool_tap": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
     "fcv_conv2d_pool_sigmoid_sum_det": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]),
     "fcv_conv2d_workspace_bytes": (_I, [_I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "fcv_conv2d_pool_sigmoid_sum_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "fcv_dwsep_conv1d": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "fcv_dwsep_conv1d_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
     "fcv_status_string": (ctypes.c_char_p, [_I]),

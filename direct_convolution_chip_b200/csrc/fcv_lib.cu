@@ -199,3 +199,77 @@ int fcv_device_error(void* stream)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the deterministic conv2d sum.
+//
+// Some callers cannot allocate device memory at the point where they run this
+// operation: a plugin inside an inference engine or framework that owns every
+// device allocation and forbids cudaMalloc while it executes, a latency-critical
+// loop that cannot afford the implicit device synchronisation cudaMalloc and
+// cudaFree may perform, or a deployment whose device-memory budget is fixed at
+// start-up.  For them the workspace of fcv_conv2d_pool_sigmoid_sum_det lives in
+// a fixed-size array that the library places in device memory when it is
+// loaded; every GPU that loads the library keeps that array until the process
+// exits.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 256 * 1024;  // the largest workspace this variant serves
+
+// One instance per device (per CUDA context).  In host code this name is only a
+// host-side stand-in for the device array: its device address comes from
+// cudaGetSymbolAddress below, never from taking the address here.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::once_flag g_noalloc_once[kNoAllocMaxDevices];
+void* g_noalloc_ptr[kNoAllocMaxDevices];
+cudaError_t g_noalloc_status[kNoAllocMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (with that device current) and then cached.
+int noalloc_scratch(void** ptr)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return FCV_ERR_UNSUPPORTED;
+    std::call_once(g_noalloc_once[dev], [dev] {
+        g_noalloc_status[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+    });
+    if (g_noalloc_status[dev] != cudaSuccess || g_noalloc_ptr[dev] == nullptr) return FCV_ERR_CUDA;
+    *ptr = g_noalloc_ptr[dev];
+    return FCV_OK;
+}
+
+}  // namespace
+
+extern "C" int fcv_conv2d_pool_sigmoid_sum_noalloc(const float* x, const float* w, const float* b, int N,
+                                                   int Cin, int H, int W, int Cout, int pool, float* out,
+                                                   void* stream)
+{
+    int st = check_conv2d(x, w, b, N, Cin, H, W, Cout, pool, out, false);
+    if (st != FCV_OK) return st;
+    const int PH = (H - 2) / pool, PW = (W - 2) / pool;
+    const size_t need = fcv::conv2d_det_workspace_bytes(N, Cout, pool, PH, PW);
+    if (need > kNoAllocScratchBytes) return FCV_ERR_UNSUPPORTED;  // too large for the static scratch
+    if (N == 0) return FCV_OK;
+    cudaStream_t s = fcv::as_stream(stream);
+    if (PH == 0 || PW == 0) {
+        return cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N, s) == cudaSuccess ? FCV_OK : FCV_ERR_CUDA;
+    }
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != FCV_OK) return st;
+    // The array keeps whatever the previous call left: clear the per-image
+    // counters, which must start at zero (the partial-sum slots are always
+    // written before they are read).
+    unsigned char* base = static_cast<unsigned char*>(scratch);
+    unsigned int* counters = reinterpret_cast<unsigned int*>(base + need - sizeof(unsigned int) * (size_t)N);
+    if (cudaMemsetAsync(counters, 0, sizeof(unsigned int) * (size_t)N, s) != cudaSuccess) return FCV_ERR_CUDA;
+    return fcv::launch_conv2d_direct<fcv::kSumDet>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s,
+                                                   reinterpret_cast<float*>(base), counters);
+}

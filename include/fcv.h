@@ -114,6 +114,27 @@ int fcv_conv2d_pool_sigmoid_sum_det(const float* x, const float* w, const float*
                                     float* out, void* workspace, size_t workspace_bytes,
                                     void* stream);
 
+/* fcv_conv2d_pool_sigmoid_sum_det without a caller workspace and without any
+ * allocation, for callers that may not allocate device memory while they run
+ * (a plugin in an engine that owns all device memory, a loop that cannot take
+ * the implicit synchronisation of cudaMalloc/cudaFree, a fixed memory budget).
+ * The pages have no counterpart; this is a library facility.
+ *
+ * The workspace is a 256 KiB array in the library's own device memory (every
+ * GPU that loads the library holds it until the process exits).  The first
+ * call on each device looks up that array's address (cudaGetSymbolAddress) with
+ * the device current; make that first call before any stream capture.  Sizes
+ * whose workspace (fcv_conv2d_workspace_bytes) exceeds 256 KiB are rejected
+ * with FCV_ERR_UNSUPPORTED before anything is enqueued.  All calls on a device
+ * share the one array: calls that overlap on the GPU (other streams, other
+ * host threads) race and must be serialised by the caller.  The array keeps
+ * the previous call's contents; the call clears what must start at zero.
+ * Otherwise the same arguments, results and errors as
+ * fcv_conv2d_pool_sigmoid_sum_det; it calls no allocator. */
+int fcv_conv2d_pool_sigmoid_sum_noalloc(const float* x, const float* w, const float* b,
+                                        int N, int Cin, int H, int W, int Cout, int pool,
+                                        float* out, void* stream);
+
 /* Bytes of workspace fcv_conv2d_pool_sigmoid_sum_det needs for these sizes
  * (0 when nothing is launched, e.g. PH or PW == 0).  Host only, no CUDA call.
  * Same INVALID_ARG / UNSUPPORTED rules as the compute entry points. */
