@@ -412,12 +412,102 @@ def run_gpu(args):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["unfused_gpu_baselines"] = unfused_baselines(xa_d, wa_d, ba_d, xb_d, dwb_d, pwb_d, bb_d)
         result["cpu_baseline"] = run_oracle_sample()
     if use_dist:
         import torch.distributed as dist
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# unfused GPU baselines (context only; never part of the library)
+# ----------------------------------------------------------------------------
+
+def _event_ms(fn, iters, stream):
+    """Average device time of fn() over `iters` calls, CUDA events on `stream`."""
+    for _ in range(3):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(iters):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def unfused_baselines(xa, wa, ba, xb, dwb, pwb, bb, iters=5):
+    """PyTorch eager (cuDNN/cuBLAS) versions of both ops with the intermediates in
+    HBM, fp32 with TF32 disabled -- the unfused pipelines the fused kernels replace."""
+    import torch.nn.functional as F
+    stream = torch.cuda.current_stream()
+    prev = (torch.backends.cudnn.allow_tf32, torch.backends.cuda.matmul.allow_tf32)
+    torch.backends.cudnn.allow_tf32 = False
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        def op_a():
+            y = F.conv2d(xa, wa, ba)
+            return torch.sigmoid(F.avg_pool2d(y, CASE_A.P)).sum(dim=(1, 2, 3))
+
+        def op_b():
+            d = F.conv1d(xb, dwb.view(CASE_B.C, 1, CASE_B.K), stride=CASE_B.stride, padding=CASE_B.pad,
+                         groups=CASE_B.C)
+            return F.conv1d(d, pwb.view(CASE_B.O, CASE_B.C, 1), bb)
+
+        ta = _event_ms(op_a, iters, stream)
+        tb = _event_ms(op_b, iters, stream)
+    finally:
+        torch.backends.cudnn.allow_tf32, torch.backends.cuda.matmul.allow_tf32 = prev
+    return {"torch_eager_conv2d_pool_sigmoid_sum_ms": ta, "torch_eager_dwsep_conv1d_ms": tb,
+            "precision": "fp32, TF32 disabled", "note": "unfused: conv output / depthwise output in HBM"}
+
+
+def run_configs(args):
+    """One JSON line per workload (named configs and the 48-point sweep): the
+    metric per config, GFLOP/s and fraction of its roofline."""
+    import ctypes
+    import direct_convolution_chip_b200 as fcv
+    torch.cuda.set_device(0)
+    lib = fcv.load()
+    P = ctypes.c_void_p
+    props = torch.cuda.get_device_properties(0)
+    peaks, _ = load_peaks()
+    fma_peak = fma_peak_tflops(props)
+    tf32_peak = peaks["bf16_tflops"] * TF32_OVER_BF16
+    stream = torch.cuda.current_stream()
+    sp = P(stream.cuda_stream)
+    cases = list(wl.NAMED) + (wl.sweep_cases() if args.sweep else [])
+    for c in cases:
+        if c.op == "conv2d":
+            x, w, b = [t.cuda() for t in wl.conv2d_inputs(c)]
+            out = torch.empty((c.N,), device="cuda")
+            fn = lambda: lib.fcv_conv2d_pool_sigmoid_sum(P(x.data_ptr()), P(w.data_ptr()), P(b.data_ptr()), c.N,
+                                                         c.Cin, c.H, c.W, c.Cout, c.P, P(out.data_ptr()), sp)
+            pipe, peak = "fp32_fma", fma_peak
+        else:
+            x, dw, pw, b = [t.cuda() for t in wl.conv1d_inputs(c)]
+            To = (c.T + 2 * c.pad - c.K) // c.stride + 1
+            out = torch.empty((c.N, c.O, To), device="cuda")
+            fn = lambda: lib.fcv_dwsep_conv1d(P(x.data_ptr()), P(dw.data_ptr()), P(pw.data_ptr()), P(b.data_ptr()),
+                                              c.N, c.C, c.T, c.O, c.K, c.stride, c.pad, P(out.data_ptr()), sp)
+            tc = lib.fcv_dwsep_conv1d_ex(P(x.data_ptr()), P(dw.data_ptr()), P(pw.data_ptr()), P(b.data_ptr()),
+                                         c.N, c.C, c.T, c.O, c.K, c.stride, c.pad, P(out.data_ptr()),
+                                         21, sp) == 0
+            pipe, peak = ("3xtf32", tf32_peak / 3.0) if tc else ("fp32_fma", fma_peak)
+        assert fn() == 0
+        macs, nbytes = case_macs(c), case_bytes(c)
+        iters = max(3, min(200, int(0.2 / max(2.0 * macs / (peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)))))
+        ms = _event_ms(fn, iters, stream)
+        roof = roofline_time_s(macs if pipe == "fp32_fma" else
+                               (macs_conv1d_pointwise(c.N, c.C, c.T, c.O, c.K, c.stride, c.pad)),
+                               nbytes, peak, peaks["hbm_gbs"])
+        print(json.dumps({"config": c.name, "op": c.op, "ms": ms, "gflops": 2.0 * macs / (ms / 1e3) / 1e9,
+                          "macs": macs, "bytes": nbytes, "pipe": pipe, "roofline_ms": roof * 1e3,
+                          "roofline_frac": roof / (ms / 1e3), "l2": "inputs resident; no flush"}), flush=True)
+        del x, out
 
 
 # ----------------------------------------------------------------------------
@@ -476,11 +566,15 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["fcv", "reference"], default="fcv")
-    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle and unfused-baseline legs")
+    ap.add_argument("--configs", action="store_true", help="time every named workload, one JSON line each")
+    ap.add_argument("--sweep", action="store_true", help="with --configs: the 48-point shape sweep as well")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.configs:
+        run_configs(args)
     else:
         run_gpu(args)
 
