@@ -22,6 +22,7 @@ _LIB = None
 
 ALGO_AUTO = 0
 CONV2D_DIRECT = 10
+CONV2D_POOLFIRST = 11
 CONV1D_FMA = 20
 CONV1D_TC_3XTF32 = 21
 

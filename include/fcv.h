@@ -57,12 +57,17 @@ typedef enum {
     FCV_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (see fcv_device_error) */
 } fcv_status;
 
-/* Algorithm selectors for the *_ex entry points.  FCV_ALGO_AUTO picks the
- * fastest path that is valid for the shape. */
+/* Algorithm selectors for the *_ex entry points.  For op B, FCV_ALGO_AUTO
+ * picks the fastest path valid for the shape; for op A it is the direct
+ * method. */
 typedef enum {
     FCV_ALGO_AUTO = 0,
     /* op A */
     FCV_CONV2D_DIRECT = 10,       /* direct 3x3 conv of every pooled window, FP32 FMA */
+    FCV_CONV2D_POOLFIRST = 11,    /* pool the input first (exact identity, 9*Cin MACs per pooled
+                                     value instead of 9*Cin*P*P), FP32 FMA; same results within
+                                     rounding.  Never chosen by FCV_ALGO_AUTO, which keeps the
+                                     direct method. */
     /* op B */
     FCV_CONV1D_FMA = 20,          /* depthwise + pointwise on FP32 FMA */
     FCV_CONV1D_TC_3XTF32 = 21     /* pointwise on tcgen05 tensor cores, 3xTF32 split */

@@ -17,7 +17,7 @@ from tests.parity import assert_close, requires_cuda, sample_indices
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
 
-CONV2D_ALGOS = [fcv.CONV2D_DIRECT]
+CONV2D_ALGOS = [fcv.CONV2D_DIRECT, fcv.CONV2D_POOLFIRST]
 CONV1D_ALGOS = [fcv.CONV1D_FMA, fcv.CONV1D_TC_3XTF32]
 
 
@@ -75,9 +75,10 @@ def test_conv2d_full_size(algo):
 
 
 @pytest.mark.parametrize("case", [c for c in wl.sweep_cases() if c.op == "conv2d"], ids=lambda c: c.name)
-def test_conv2d_sweep(case):
+@pytest.mark.parametrize("algo", CONV2D_ALGOS)
+def test_conv2d_sweep(case, algo):
     heavy = case.Cin * case.Cout * case.H * case.W > 16 * 128 * 200 * 200
-    check_conv2d_case(case, fcv.CONV2D_DIRECT, batch_items=[0] if heavy else [0, case.N - 1], n_samples=2000)
+    check_conv2d_case(case, algo, batch_items=[0] if heavy else [0, case.N - 1], n_samples=2000)
 
 
 EDGE_2D = [
@@ -98,10 +99,11 @@ EDGE_2D = [
 
 
 @pytest.mark.parametrize("shape", EDGE_2D, ids=lambda s: "x".join(map(str, s)))
-def test_conv2d_edges(shape):
+@pytest.mark.parametrize("algo", CONV2D_ALGOS)
+def test_conv2d_edges(shape, algo):
     N, Cin, H, W, Cout, P = shape
     case = wl.Conv2dCase("edge", N, Cin, H, W, Cout, P, seed=sum(shape))
-    check_conv2d_case(case, fcv.CONV2D_DIRECT, n_samples=0)
+    check_conv2d_case(case, algo, n_samples=0)
 
 
 def test_conv2d_empty_pool_gives_zero():
@@ -117,10 +119,11 @@ def test_conv2d_empty_pool_gives_zero():
 
 @pytest.mark.parametrize("variant", [dict(w_scale=30.0), dict(x_mean=1.0), dict(x_mean=1.0, w_scale=30.0)],
                          ids=["w_x30", "x_mean1", "both"])
-def test_conv2d_adversarial(variant):
+@pytest.mark.parametrize("algo", CONV2D_ALGOS)
+def test_conv2d_adversarial(variant, algo):
     """Weights x30 and/or x ~ N(1,1): the sigmoid leaves its linear range."""
     case = wl.Conv2dCase("adv", 2, 8, 96, 80, 24, 4, seed=21)
-    check_conv2d_case(case, fcv.CONV2D_DIRECT, n_samples=0, **variant)
+    check_conv2d_case(case, algo, n_samples=0, **variant)
 
 
 def test_conv2d_output_fully_overwritten():
