@@ -44,6 +44,7 @@ SIGNATURES = {
     "fcv_status_string": (ctypes.c_char_p, [_I]),
     "fcv_version": (_I, []),
     "fcv_device_error": (_I, [_P]),
+    "fcv_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
 }
 
 

@@ -119,7 +119,8 @@ __device__ __forceinline__ unsigned long long globaltimer()
 // Wait for the phase of `bar` with parity `parity`.  Returns false (without
 // completing the wait) once the CTA abort flag is set, or after kWaitLimitNs,
 // in which case it sets the abort flag and the device error word itself.
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag)
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                             unsigned long long limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
@@ -127,13 +128,30 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort_flag = 1u;
                 record_device_error(kErrTimeout);
                 return false;
             }
         }
     }
+}
+
+// Self-test of the failure path: one thread waits, with the given limit, on an
+// mbarrier that nothing will ever complete.  The wait must give up, set the
+// device error word and return; the kernel then exits normally.
+__global__ void selftest_wait_timeout_kernel(unsigned long long limit_ns)
+{
+    __shared__ __align__(8) unsigned long long bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)wait_bounded(smem_u32(&bar), 0, &abort_flag, limit_ns);
+    __syncthreads();
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }

@@ -54,10 +54,15 @@ template <> struct Conv2dTile<6> { static constexpr int RX = 1, CG = 8,  TPH = 4
 template <> struct Conv2dTile<7> { static constexpr int RX = 1, CG = 8,  TPH = 4,  TPW = 8,  NCH = 4, ICC = 4; };
 template <> struct Conv2dTile<8> { static constexpr int RX = 1, CG = 8,  TPH = 4,  TPW = 8,  NCH = 4, ICC = 2; };
 
-template <int P>
+// NARROW (layers with Cout <= 32 at P <= 4): half the channel groups and twice
+// the pooled rows per CTA, so no thread computes channels that do not exist.
+template <int P, bool NARROW = false>
 struct Conv2dGeom {
     using T = Conv2dTile<P>;
-    static constexpr int RX = T::RX, CG = T::CG, TPH = T::TPH, TPW = T::TPW, NCH = T::NCH, ICC = T::ICC;
+    static constexpr bool NR = NARROW && P <= 4;
+    static constexpr int RX = T::RX, CG = T::CG, TPW = T::TPW, ICC = T::ICC;
+    static constexpr int TPH = NR ? 2 * T::TPH : T::TPH;
+    static constexpr int NCH = NR ? T::NCH / 2 : T::NCH;
     static constexpr int NPOS = TPH * TPW;          // threads per channel group
     static constexpr int NT = NPOS * NCH;           // threads per CTA
     static constexpr int CB = CG * NCH;             // output channels per CTA
@@ -101,15 +106,15 @@ __device__ __forceinline__ double block_sum_d(double v, double* scratch)
 // MODE is a Conv2dMode.  partials/counters are used by kSumDet only: the
 // workspace holds one float per CTA ([N][per_image]) and one counter per image
 // (zero at launch).
-template <int P, int MODE, bool PACKED = (P <= FCV_CONV2D_PACKED_MAX_P)>
-__global__ void __launch_bounds__(Conv2dGeom<P>::NT, 2)
+template <int P, int MODE, bool NARROW, bool PACKED = (P <= FCV_CONV2D_PACKED_MAX_P)>
+__global__ void __launch_bounds__(Conv2dGeom<P, NARROW>::NT, 2)
 conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
                      const float* __restrict__ bias, int Cin, int H, int W, int Cout,
                      int PH, int PW, int tiles_y, int tiles_x, float* __restrict__ out,
                      float* __restrict__ partials, unsigned int* __restrict__ counters)
 {
     constexpr bool TAP = MODE == kTap;
-    using G = Conv2dGeom<P>;
+    using G = Conv2dGeom<P, NARROW>;
     constexpr int RX = G::RX, CG = G::CG, NPOS = G::NPOS, NT = G::NT, CB = G::CB;
     constexpr int HY = G::HY, HX = G::HX, HXP = G::HXP, PY = G::PY, PX = G::PX, ICC = G::ICC;
 
@@ -288,42 +293,51 @@ conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
     }
 }
 
+inline bool conv2d_narrow(int P, int Cout) { return P <= 4 && Cout <= 32; }
+
 // Grid of the direct kernel for pool size P: tiles per image and channel blocks.
-template <int P>
+template <int P, bool NARROW>
 void conv2d_grid_p(int PH, int PW, int Cout, int* tiles_y, int* tiles_x, int* cblocks)
 {
-    using G = Conv2dGeom<P>;
+    using G = Conv2dGeom<P, NARROW>;
     *tiles_y = (PH + G::TILE_PH - 1) / G::TILE_PH;
     *tiles_x = (PW + G::TILE_PW - 1) / G::TILE_PW;
     *cblocks = (Cout + G::CB - 1) / G::CB;
 }
 
+template <int P>
+void conv2d_grid_pp(int PH, int PW, int Cout, int* tiles_y, int* tiles_x, int* cblocks)
+{
+    if (conv2d_narrow(P, Cout)) conv2d_grid_p<P, true>(PH, PW, Cout, tiles_y, tiles_x, cblocks);
+    else conv2d_grid_p<P, false>(PH, PW, Cout, tiles_y, tiles_x, cblocks);
+}
+
 inline bool conv2d_grid(int P, int PH, int PW, int Cout, int* tiles_y, int* tiles_x, int* cblocks)
 {
     switch (P) {
-    case 1: conv2d_grid_p<1>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
-    case 2: conv2d_grid_p<2>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
-    case 3: conv2d_grid_p<3>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
-    case 4: conv2d_grid_p<4>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
-    case 5: conv2d_grid_p<5>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
-    case 6: conv2d_grid_p<6>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
-    case 7: conv2d_grid_p<7>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
-    case 8: conv2d_grid_p<8>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 1: conv2d_grid_pp<1>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 2: conv2d_grid_pp<2>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 3: conv2d_grid_pp<3>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 4: conv2d_grid_pp<4>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 5: conv2d_grid_pp<5>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 6: conv2d_grid_pp<6>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 7: conv2d_grid_pp<7>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
+    case 8: conv2d_grid_pp<8>(PH, PW, Cout, tiles_y, tiles_x, cblocks); return true;
     default: return false;
     }
 }
 
-template <int P, int MODE>
-int launch_conv2d_direct_p(const float* x, const float* w, const float* b, int N, int Cin, int H,
-                           int W, int Cout, int PH, int PW, float* out, float* partials,
-                           unsigned int* counters, cudaStream_t stream)
+template <int P, int MODE, bool NARROW>
+int launch_conv2d_direct_pn(const float* x, const float* w, const float* b, int N, int Cin, int H,
+                            int W, int Cout, int PH, int PW, float* out, float* partials,
+                            unsigned int* counters, cudaStream_t stream)
 {
-    using G = Conv2dGeom<P>;
+    using G = Conv2dGeom<P, NARROW>;
     int tiles_y, tiles_x, cblk;
-    conv2d_grid_p<P>(PH, PW, Cout, &tiles_y, &tiles_x, &cblk);
+    conv2d_grid_p<P, NARROW>(PH, PW, Cout, &tiles_y, &tiles_x, &cblk);
     const long long nblk = (long long)N * tiles_y * tiles_x;
     if (nblk > 0x7fffffffLL || cblk > 65535) return FCV_ERR_UNSUPPORTED;
-    auto kern = conv2d_direct_kernel<P, MODE>;
+    auto kern = conv2d_direct_kernel<P, MODE, NARROW>;
     if (G::SMEM_BYTES > 48 * 1024) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)G::SMEM_BYTES) != cudaSuccess)
@@ -333,6 +347,18 @@ int launch_conv2d_direct_p(const float* x, const float* w, const float* b, int N
     kern<<<grid, G::NT, G::SMEM_BYTES, stream>>>(x, w, b, Cin, H, W, Cout, PH, PW, tiles_y, tiles_x, out,
                                                   partials, counters);
     return launch_status();
+}
+
+template <int P, int MODE>
+int launch_conv2d_direct_p(const float* x, const float* w, const float* b, int N, int Cin, int H,
+                           int W, int Cout, int PH, int PW, float* out, float* partials,
+                           unsigned int* counters, cudaStream_t stream)
+{
+    if (conv2d_narrow(P, Cout))
+        return launch_conv2d_direct_pn<P, MODE, true>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials,
+                                                      counters, stream);
+    return launch_conv2d_direct_pn<P, MODE, false>(x, w, b, N, Cin, H, W, Cout, PH, PW, out, partials,
+                                                   counters, stream);
 }
 
 // PH, PW >= 1 here; the caller handles the empty cases.

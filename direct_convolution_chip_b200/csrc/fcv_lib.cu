@@ -175,6 +175,13 @@ int fcv_dwsep_conv1d(const float* x, const float* dw_w, const float* pw_w, const
     return fcv_dwsep_conv1d_ex(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, out, FCV_ALGO_AUTO, stream);
 }
 
+int fcv_selftest_wait_timeout(unsigned long long limit_ns, void* stream)
+{
+    if (limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000) return FCV_ERR_INVALID_ARG;
+    fcv::tc::selftest_wait_timeout_kernel<<<1, 32, 0, fcv::as_stream(stream)>>>(limit_ns);
+    return fcv::launch_status();
+}
+
 const char* fcv_status_string(int status)
 {
     switch (status) {

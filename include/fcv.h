@@ -192,6 +192,14 @@ int fcv_version(void);
  * wait since the last call.  Returns FCV_ERR_CUDA if the synchronization fails. */
 int fcv_device_error(void* stream);
 
+/* Self-test of the failure path (no counterpart on the pages): launches one
+ * tiny kernel whose thread waits, with limit `limit_ns` (1 ns .. 10 s), on a
+ * barrier that nothing completes.  The bounded wait gives up, records
+ * FCV_ERR_TIMEOUT in the device error word and the kernel exits normally, so a
+ * following fcv_device_error(stream) returns FCV_ERR_TIMEOUT and the context
+ * stays usable.  Nothing faults, traps or hangs.  Asynchronous on `stream`. */
+int fcv_selftest_wait_timeout(unsigned long long limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -133,3 +133,8 @@ def test_det_rejects_missing_or_small_workspace(lib):
     assert det(*args, P(0x10008), 1 << 20, None) == INVALID    # not 16-byte aligned
     assert det(*args, FAKE, 8, None) == INVALID                # too small
     assert det(FAKE, FAKE, FAKE, 0, 8, 64, 64, 16, 4, FAKE, None, 0, None) == OK  # empty batch
+
+
+def test_selftest_rejects_bad_limits(lib):
+    assert lib.fcv_selftest_wait_timeout(0, None) == INVALID
+    assert lib.fcv_selftest_wait_timeout(11 * 10**9, None) == INVALID

@@ -343,3 +343,21 @@ def test_conv2d_det_empty_pool_and_guard_bands():
     for buf in (wbuf, obuf):
         assert torch.isnan(buf[:guard]).all() and torch.isnan(buf[-guard:]).all()
     assert torch.isfinite(obuf[guard:guard + c2.N]).all()
+
+
+# ---------------------------------------------------------- failure path ---
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A wait on a barrier nothing completes (2 ms limit) records FCV_ERR_TIMEOUT
+    in the device error word; the error is read once and cleared, and the
+    context keeps working."""
+    lib = fcv.load()
+    import ctypes
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.fcv_device_error(stream) == 0
+    assert lib.fcv_selftest_wait_timeout(2_000_000, stream) == 0
+    assert lib.fcv_device_error(stream) == 4   # FCV_ERR_TIMEOUT
+    assert lib.fcv_device_error(stream) == 0   # cleared by the read
+    case = wl.CONV1D_SMALL
+    check_conv1d_case(case, fcv.CONV1D_TC_3XTF32, n_samples=0)
+    assert lib.fcv_device_error(stream) == 0
