@@ -50,6 +50,15 @@ __device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc, bool
                  : "memory");
 }
 
+// 16-byte asynchronous global->shared copy of `bytes` (0..16) valid bytes; the
+// rest of the 16 destination bytes are zero-filled.  Both addresses must be
+// 16-byte aligned (for bytes == 0 pass an aligned base pointer).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, int bytes)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gsrc), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 
 template <int N>

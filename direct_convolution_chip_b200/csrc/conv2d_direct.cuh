@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(Conv2dGeom<P, NARROW>::NT, 2)
 conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
                      const float* __restrict__ bias, int Cin, int H, int W, int Cout,
                      int PH, int PW, int tiles_y, int tiles_x, float* __restrict__ out,
-                     float* __restrict__ partials, unsigned int* __restrict__ counters)
+                     float* __restrict__ partials, unsigned int* __restrict__ counters, int vec16)
 {
     constexpr bool TAP = MODE == kTap;
     using G = Conv2dGeom<P, NARROW>;
@@ -146,18 +146,33 @@ conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
 
     for (int ic0 = 0; ic0 < Cin; ic0 += ICC) {
         // Stage the halo of this input-channel chunk and its weights with
-        // asynchronous copies, all in flight at once (zero past the image and
-        // past Cin); weights as [icl][tap][c_local] so a thread's CG channels
-        // of one tap are contiguous.
-        for (int i = tid; i < ICC * HY * HX; i += NT) {
-            const int icl = i / (HY * HX);
-            const int rem = i - icl * (HY * HX);
-            const int r = rem / HX, sc = rem - (rem / HX) * HX;
-            const int ic = ic0 + icl, yy = y0 + r, xx = x0 + sc;
-            const bool in = ic < Cin && yy < H && xx < W;
-            cp_async4(halo + (icl * HY + r) * HXP + sc, in ? xn + ((size_t)ic * H + yy) * W + xx : x, in);
+        // asynchronous copies, all in flight at once (zero past the image);
+        // only the chunk's nic real channels are staged.  Weights as
+        // [icl][tap][c_local] so a thread's CG channels of one tap are contiguous.
+        const int nic = min(ICC, Cin - ic0);
+        if (vec16) {
+            // Rows are 16-byte aligned (W % 4 == 0, aligned x, x0 a multiple of 4):
+            // HXP/4 copies of 16 bytes per halo row, zero-filled past the image.
+            constexpr int CPR = HXP / 4;
+            for (int i = tid; i < nic * HY * CPR; i += NT) {
+                const int row = i / CPR, q = i - (i / CPR) * CPR;
+                const int icl = row / HY, r = row - (row / HY) * HY;
+                const int yy = y0 + r, xx = x0 + 4 * q;
+                const int bytes = yy < H ? 4 * max(0, min(4, W - xx)) : 0;
+                cp_async16(halo + (icl * HY + r) * HXP + 4 * q,
+                           bytes ? xn + ((size_t)(ic0 + icl) * H + yy) * W + xx : x, bytes);
+            }
+        } else {
+            for (int i = tid; i < nic * HY * HX; i += NT) {
+                const int icl = i / (HY * HX);
+                const int rem = i - icl * (HY * HX);
+                const int r = rem / HX, sc = rem - (rem / HX) * HX;
+                const int ic = ic0 + icl, yy = y0 + r, xx = x0 + sc;
+                const bool in = ic < Cin && yy < H && xx < W;
+                cp_async4(halo + (icl * HY + r) * HXP + sc, in ? xn + ((size_t)ic * H + yy) * W + xx : x, in);
+            }
         }
-        for (int i = tid; i < ICC * 9 * CB; i += NT) {
+        for (int i = tid; i < nic * 9 * CB; i += NT) {
             const int cl = i % CB;
             const int tap = (i / CB) % 9;
             const int icl = i / (9 * CB);
@@ -169,7 +184,6 @@ conv2d_direct_kernel(const float* __restrict__ x, const float* __restrict__ w,
         cp_async_wait<0>();
         __syncthreads();
 
-        const int nic = min(ICC, Cin - ic0);
         for (int icl = 0; icl < nic; ++icl) {
             const float* hp = halo + (icl * HY + ty * P) * HXP + tx * (RX * P);
             const float* wp = ws + icl * 9 * CB + grp * CG;
@@ -344,8 +358,9 @@ int launch_conv2d_direct_pn(const float* x, const float* w, const float* b, int 
             return FCV_ERR_CUDA;
     }
     dim3 grid((unsigned)nblk, (unsigned)cblk);
+    const int vec16 = ((W & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 && (P * G::TILE_PW) % 4 == 0) ? 1 : 0;
     kern<<<grid, G::NT, G::SMEM_BYTES, stream>>>(x, w, b, Cin, H, W, Cout, PH, PW, tiles_y, tiles_x, out,
-                                                  partials, counters);
+                                                  partials, counters, vec16);
     return launch_status();
 }
 
