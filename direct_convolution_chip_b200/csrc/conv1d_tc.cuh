@@ -60,7 +60,8 @@ constexpr int KMAXW = 13;      // largest depthwise kernel (stride 1) of the reg
 constexpr int XW_MAX = TM - 1 + KMAXW;  // 140 halo samples per channel at most
 constexpr int XU = (XW_MAX + 31) / 32;  // halo samples per lane per channel
 constexpr int XWP = 144;       // halo row pitch in floats (multiple of 8)
-constexpr int XS_FLOATS = KC * XWP + 28;  // + skew of 4 floats per group of 4 channels
+constexpr int XPP = 2 * XWP;   // pitch of an interleaved channel-pair row
+constexpr int XS_FLOATS = KC * XWP + 28;  // 16 pair rows + skew of 4 floats per group of 4 channels
 constexpr int DW_MAX = 4000;   // resident depthwise weights: K * round_up(C, 4) at most
 constexpr uint32_t TMEM_COLS = 2 * TN;
 
@@ -404,15 +405,17 @@ dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_ma
             const uint32_t b_lo = b_hi + B_BYTES;
             const int c0 = kc * KC;
 
-            // Halo of this chunk into shared memory (rows skewed by 4 floats per channel group).
+            // Halo of this chunk into shared memory, channel pairs interleaved:
+            // xs[(c/2)*XPP + skew + 2*j + (c&1)], skewed by 4 floats per group of 4
+            // channels, so the packed depthwise reads both channels of a pair at once.
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 4; i += 2) {
                 const int cl = 4 * warp + i;
-                float* dst = xs + cl * XWP + 4 * ((cl >> 2) & 7);
+                float* dst = xs + (cl >> 1) * XPP + 4 * ((cl >> 2) & 7);
 #pragma unroll
                 for (int u = 0; u < XU; ++u) {
                     const int j = lane + 32 * u;
-                    if (j < XWP) dst[j] = xr[i][u];
+                    if (j < XWP) *reinterpret_cast<float2*>(dst + 2 * j) = make_float2(xr[i][u], xr[i + 1][u]);
                 }
             }
             // pw chunk (raw fp32, as the TMA left it in B_hi), split in place into TF32 hi/lo.
@@ -436,31 +439,30 @@ dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_ma
             if (tile < p.total_tiles) fetch(kc);
 
             // Depthwise tile: 4 times x 4 channels per thread, then the TF32 split as the A operand.
-            float dv[4][4];
+            // Depthwise tile: 4 times x 4 channels per thread as two channel pairs,
+            // each tap one packed fma.rn.f32x2 per time (both channels of a pair).
+            float2 d2[2][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) d2[h][r] = make_float2(0.f, 0.f);
             if (c0 + 4 * cg < p.C) {  // channels past C stay zero (their weights are zero-padded too)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {  // two channel pairs: 2 windows of 16 samples live at a time
-                    float win[2][16];
+                for (int h = 0; h < 2; ++h) {
+                    const int pr = 2 * cg + h;  // pair row: channels 4*cg + 2*h, +1
+                    const float* xrow = xs + pr * XPP + 4 * cg + 8 * tq;
+                    float2 win[16];
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const int cl = 4 * cg + 2 * h + i;
-                        const float* xrow = xs + cl * XWP + 4 * ((cl >> 2) & 7) + 4 * tq;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
-                            win[i][4 * q] = v.x; win[i][4 * q + 1] = v.y; win[i][4 * q + 2] = v.z; win[i][4 * q + 3] = v.w;
-                        }
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
+                        win[2 * q] = make_float2(v.x, v.y);
+                        win[2 * q + 1] = make_float2(v.z, v.w);
                     }
                     const float* wcol = dws + c0 + 4 * cg + 2 * h;
                     auto tap = [&](int k) {
                         const float2 wk = *reinterpret_cast<const float2*>(wcol + k * CP);
 #pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            dv[2 * h][r] = fmaf(win[0][k + r], wk.x, dv[2 * h][r]);
-                            dv[2 * h + 1][r] = fmaf(win[1][k + r], wk.y, dv[2 * h + 1][r]);
-                        }
+                        for (int r = 0; r < 4; ++r) d2[h][r] = __ffma2_rn(win[k + r], wk, d2[h][r]);
                     };
                     if constexpr (KT > 0) {
 #pragma unroll
@@ -476,7 +478,7 @@ dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_ma
             for (int r = 0; r < 4; ++r) {
                 const int t = 4 * tq + r;
                 float4 hi, lo;
-                split4(make_float4(dv[0][r], dv[1][r], dv[2][r], dv[3][r]), hi, lo);
+                split4(make_float4(d2[0][r].x, d2[0][r].y, d2[1][r].x, d2[1][r].y), hi, lo);
                 const uint32_t off = sw128_off(t, cg);
                 sts128(a_hi + off, hi);
                 sts128(a_lo + off, lo);
@@ -587,18 +589,27 @@ dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_ma
             // each 16-byte store instruction covers 128 contiguous bytes of 4 rows.
             const bool vec = tw + 32 <= p.To && p.out_vec;
             const int kq = lane >> 2, jq = lane & 3;
+            // bias of output channels o0 + 32*i + lane, one load per lane per 32
+            // columns, fetched a step ahead and broadcast by shuffle
+            auto bias_at = [&](int i) {
+                const int o = tcd.o0 + 32 * i + lane;
+                return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f;
+            };
+            float bnext = bias_at(0), bcur = 0.f;
 #pragma unroll 1
             for (int cb = 0; cb < TN / 16; ++cb) {
+                if ((cb & 1) == 0) {
+                    bcur = bnext;
+                    if (cb + 2 < TN / 16) bnext = bias_at((cb >> 1) + 1);
+                }
                 uint32_t r[16];
                 tmem_ld16(taddr + (uint32_t)(cb * 16), r);
                 tmem_wait_ld();
                 const int obase = tcd.o0 + cb * 16;
                 float v[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int o = obase + j;
-                    v[j] = __uint_as_float(r[j]) + ((p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f);
-                }
+                for (int j = 0; j < 16; ++j)
+                    v[j] = __uint_as_float(r[j]) + __shfl_sync(0xffffffffu, bcur, (cb & 1) * 16 + j);
                 if (vec) {
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
@@ -608,7 +619,7 @@ dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_ma
                         const int o = obase + 4 * jq + m;
                         if (o < p.O) {
                             float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
-                            *reinterpret_cast<float4*>(dst) = make_float4(x0, x1, x2, x3);
+                            __stcs(reinterpret_cast<float4*>(dst), make_float4(x0, x1, x2, x3));  // streaming store
                         }
                     }
                 } else {

@@ -1,0 +1,553 @@
+// conv1d_tc2.cuh -- op B on a pair of SMs: the 2-CTA (cta_group::2) form of
+// the tensor-core separable conv1d in conv1d_tc.cuh.
+//
+// Same arithmetic as conv1d_tc.cuh (depthwise on FP32 FMA into the A operand,
+// pointwise as a 3xTF32 tcgen05 contraction, fp32 accumulation in TMEM; see
+// there for the split and its accuracy).  What changes is the tiling: two CTAs
+// of a cluster compute one 256-time x 256-output-channel tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 8).  Each CTA holds its own
+// 128 rows of A (its times) and HALF of B (128 of the 256 pw rows), so per CTA
+// the pw split work and the B stage size are halved; the freed shared memory
+// holds a 3-deep ring of input halos filled by cp.async two chunks ahead.
+//
+// Roles per CTA (448 threads): warps 0-7 produce (halo copies, in-place pw
+// split, depthwise + A split); warp 8 allocates TMEM (both CTAs) and, in the
+// leader CTA only, one thread issues the MMAs for the pair; warps 9-12 drain
+// this CTA's accumulator rows; warp 13 loads this CTA's half of the pw chunk
+// by TMA.  The leader's "full" and "aempty" barriers collect arrivals from
+// both CTAs (remote mbarrier arrives); MMA completion is committed to both
+// CTAs' "empty"/"afull" barriers with a multicast commit.  Every mbarrier
+// wait is bounded; a cluster barrier follows initialisation and precedes exit,
+// so no CTA leaves while its peer may still signal it.  No TMA multicast.
+#pragma once
+
+#include "conv1d_tc.cuh"
+
+namespace fcv {
+namespace tc2 {
+
+using tc::TileCoord;
+
+constexpr int TM = 128;          // times per CTA (pair: 256)
+constexpr int TN = 256;          // output channels per pair tile (UMMA N)
+constexpr int TNH = TN / 2;      // pw rows held by each CTA
+constexpr int KC = 32;
+constexpr int STAGES = 2;
+constexpr int XSTAGES = 3;       // input-halo ring depth
+constexpr int NPROD = 256;
+constexpr int MMA_WARP = 8, TMA_WARP = 13;
+constexpr int NTHREADS = 14 * 32;
+constexpr int KMAXW = tc::KMAXW;
+constexpr int XWP = 144;         // halo row pitch (floats)
+constexpr int XS_FLOATS = KC * XWP + 28;
+constexpr int DW_MAX = tc::DW_MAX;
+constexpr uint32_t TMEM_COLS = 2 * TN;
+
+constexpr uint32_t A_BYTES = TM * KC * 4;    // 16 KB
+constexpr uint32_t B_BYTES = TNH * KC * 4;   // 16 KB
+constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
+constexpr uint32_t OFF_XS = STAGES * STAGE_BYTES;
+constexpr uint32_t XS_BYTES = ((uint32_t)XS_FLOATS * 4 + 127) & ~127u;
+constexpr uint32_t OFF_DWS = OFF_XS + XSTAGES * XS_BYTES;
+constexpr uint32_t OFF_BAR = (OFF_DWS + DW_MAX * 4 + 7) & ~7u;
+constexpr uint32_t NBAR = 11;    // full[2] empty[2] afull[2] aempty[2] drain tma[2]
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+// D fp32, A/B tf32, K-major, N = 256, M = 256 (the pair).
+constexpr uint32_t kIdesc2 = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(TN >> 3) << 17) |
+                             ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire (barriers that the peer CTA signals).
+__device__ __forceinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag)
+{
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const unsigned long long t0 = tc::globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((i & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (tc::globaltimer() - t0 > tc::kWaitLimitNs) {
+                *abort_flag = 1u;
+                record_device_error(kErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void mma2_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc2), "r"(accumulate)
+        : "memory");
+}
+
+// Commit all prior MMAs of this thread to `bar` in both CTAs of the pair.
+__device__ __forceinline__ void commit2(uint32_t bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::"r"(bar),
+        "h"((unsigned short)3)
+        : "memory");
+}
+
+struct Params {
+    const float* x;
+    const float* dw;
+    const float* pw;
+    const float* bias;
+    float* out;
+    int C, T, O, K, pad, To;
+    int tiles_t, tiles_o, total_tiles;  // pair tiles (256 times each)
+    int out_vec;                         // output rows 16-byte aligned
+    int x_vec;                           // 16-byte halo copies possible
+};
+
+__device__ __forceinline__ TileCoord decode_pair_tile(const Params& p, int tile)
+{
+    TileCoord tc;
+    tc.t0 = (tile % p.tiles_t) * (2 * TM);
+    const int rest = tile / p.tiles_t;
+    tc.o0 = (rest % p.tiles_o) * TN;
+    tc.n = rest / p.tiles_o;
+    return tc;
+}
+
+template <int KT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_map)
+{
+    using namespace tc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    float* dws = reinterpret_cast<float*>(smem + OFF_DWS);
+    const uint32_t bar_full = sbase + OFF_BAR;   // + 8 * stage (leader's collects both CTAs)
+    const uint32_t bar_empty = bar_full + 16;    // + 8 * stage
+    const uint32_t bar_afull = bar_full + 32;    // + 8 * buf
+    const uint32_t bar_aempty = bar_full + 48;   // + 8 * buf (leader's collects both CTAs)
+    const uint32_t bar_drain = bar_full + 64;
+    const uint32_t bar_tma = bar_full + 72;      // + 8 * stage
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
+    volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_full + 8 * i, 16);   // 8 producer warps x 2 CTAs (used in the leader)
+            mbar_init(bar_empty + 8 * i, 1);   // multicast commit
+            mbar_init(bar_afull + 8 * i, 1);   // multicast commit
+            mbar_init(bar_aempty + 8 * i, 8);  // 4 epilogue warps x 2 CTAs (used in the leader)
+            mbar_init(bar_tma + 8 * i, 1);     // expect_tx arrival + TMA bytes
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0u;
+        *prod_abort = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == MMA_WARP) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_holder)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
+    }
+    const int CP = (p.C + 3) & ~3;
+    for (int e = threadIdx.x; e < p.K * CP; e += NTHREADS) {
+        const int k = e / CP, c = e - (e / CP) * CP;
+        dws[e] = c < p.C ? __ldg(p.dw + (size_t)c * p.K + k) : 0.f;
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated, weights staged
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const int nk = (p.C + KC - 1) / KC;
+
+    if (warp < 8) {
+        // ------------------------------------------------------------ producers
+        const int ptid = threadIdx.x;
+        const int cg = lane & 7;
+        const int tq = (lane >> 3) + 4 * warp;
+        const int K = KT > 0 ? KT : p.K;
+        const uint32_t full_leader = mapa(bar_full, 0);
+
+        // Halo of chunk (tile, kc) into ring slot `slot`: channel rows of XWP
+        // samples from t0 - pad (this CTA's 128 times), skewed by 4 floats per
+        // group of 4 channels; zero outside [0, T) and past C.
+        auto stage_x = [&](int tile, int kc, int slot) {
+            const TileCoord tcd = decode_pair_tile(p, tile);
+            const int c0 = kc * KC;
+            const int tb = tcd.t0 + (int)rank * TM - p.pad;
+            float* xs = reinterpret_cast<float*>(smem + OFF_XS + slot * XS_BYTES);
+            const float* xn = p.x + (size_t)tcd.n * p.C * p.T;
+            if (p.x_vec) {
+                constexpr int CPR = XWP / 4;  // 16-byte copies per channel row
+                for (int i = ptid; i < KC * CPR; i += NPROD) {
+                    const int cl = i / CPR, q = i - (i / CPR) * CPR;
+                    const int c = c0 + cl, ti = tb + 4 * q;
+                    const int bytes = (c < p.C && ti >= 0) ? 4 * max(0, min(4, p.T - ti)) : 0;
+                    cp_async16(xs + cl * XWP + 4 * ((cl >> 2) & 7) + 4 * q,
+                               bytes ? xn + (size_t)c * p.T + ti : p.x, bytes);
+                }
+            } else {
+                for (int i = ptid; i < KC * XWP; i += NPROD) {
+                    const int cl = i / XWP, j = i - (i / XWP) * XWP;
+                    const int c = c0 + cl, ti = tb + j;
+                    const bool in = c < p.C && ti >= 0 && ti < p.T;
+                    cp_async4(xs + cl * XWP + 4 * ((cl >> 2) & 7) + j, in ? xn + (size_t)c * p.T + ti : p.x, in);
+                }
+            }
+        };
+        // Sequence position `ahead` chunks after (tile, kc), or tile = -1 past the end.
+        auto advance = [&](int& tile, int& kc) {
+            if (++kc == nk) {
+                kc = 0;
+                tile += npairs;
+            }
+            if (tile >= p.total_tiles) tile = -1;
+        };
+
+        int seq = 0, tile = pair, kc = 0;
+        // Prefetch the halos of the first two chunks.
+        int ftile = tile, fkc = kc;
+        for (int a = 0; a < 2; ++a) {
+            if (ftile >= 0 && ftile < p.total_tiles) stage_x(ftile, fkc, a);
+            cp_async_commit();
+            if (ftile >= 0) advance(ftile, fkc);
+        }
+        while (tile < p.total_tiles) {
+            const int stage = seq & 1;
+            const uint32_t parity = (seq >> 1) & 1;
+            if (ptid == 0 && !wait_bounded(bar_tma + 8 * stage, parity, abort_flag)) *prod_abort = 1u;
+            asm volatile("bar.sync 1, 256;\n" ::: "memory");  // B1: also, every producer is done with slot (seq-1)%3
+            if (*prod_abort) break;
+            for (int spin = 0; !mbar_try_wait(bar_tma + 8 * stage, parity) && spin < (1 << 20); ++spin) {
+            }
+            // Halo of chunk seq+2 into the slot chunk seq-1 used.
+            if (ftile >= 0) stage_x(ftile, fkc, (seq + 2) % XSTAGES);
+            cp_async_commit();
+            if (ftile >= 0) advance(ftile, fkc);
+
+            const uint32_t a_hi = sbase + stage * STAGE_BYTES;
+            const uint32_t a_lo = a_hi + A_BYTES;
+            const uint32_t b_hi = a_lo + A_BYTES;
+            const uint32_t b_lo = b_hi + B_BYTES;
+            const int c0 = kc * KC;
+            // This CTA's half of the pw chunk (128 rows), split in place into TF32 hi/lo.
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = warp * 16 + i * 4 + (lane >> 3);
+                const uint32_t off = sw128_off(row, lane & 7);
+                float4 hi, lo;
+                split4(lds128(b_hi + off), hi, lo);
+                sts128(b_hi + off, hi);
+                sts128(b_lo + off, lo);
+            }
+            cp_async_wait<2>();                               // this thread's copies of chunk seq landed
+            asm volatile("bar.sync 1, 256;\n" ::: "memory");  // B2: everyone's copies landed
+
+            const float* xs = reinterpret_cast<const float*>(smem + OFF_XS + (seq % XSTAGES) * XS_BYTES);
+            float dv[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
+            if (c0 + 4 * cg < p.C) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float win[2][16];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int cl = 4 * cg + 2 * h + i;
+                        const float* xrow = xs + cl * XWP + 4 * ((cl >> 2) & 7) + 4 * tq;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
+                            win[i][4 * q] = v.x; win[i][4 * q + 1] = v.y; win[i][4 * q + 2] = v.z; win[i][4 * q + 3] = v.w;
+                        }
+                    }
+                    const float* wcol = dws + c0 + 4 * cg + 2 * h;
+                    auto tap = [&](int k) {
+                        const float2 wk = *reinterpret_cast<const float2*>(wcol + k * CP);
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            dv[2 * h][r] = fmaf(win[0][k + r], wk.x, dv[2 * h][r]);
+                            dv[2 * h + 1][r] = fmaf(win[1][k + r], wk.y, dv[2 * h + 1][r]);
+                        }
+                    };
+                    if constexpr (KT > 0) {
+#pragma unroll
+                        for (int k = 0; k < KT; ++k) tap(k);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < KMAXW; ++k)
+                            if (k < K) tap(k);
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int t = 4 * tq + r;
+                float4 hi, lo;
+                split4(make_float4(dv[0][r], dv[1][r], dv[2][r], dv[3][r]), hi, lo);
+                const uint32_t off = sw128_off(t, cg);
+                sts128(a_hi + off, hi);
+                sts128(a_lo + off, lo);
+            }
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(full_leader + 8 * stage);
+            ++seq;
+            advance(tile, kc);
+            if (tile < 0) break;
+        }
+        cp_async_wait<0>();  // no copy may still be landing when the CTA exits
+    } else if (warp == MMA_WARP) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0 && leader) {
+            int seq = 0, local = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < p.total_tiles; tile += npairs, ++local) {
+                const int buf = local & 1;
+                if (!wait_bounded_cluster(bar_aempty + 8 * buf, ((local >> 1) & 1) ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
+                for (int k = 0; k < nk; ++k, ++seq) {
+                    const int stage = seq & 1;
+                    if (!wait_bounded_cluster(bar_full + 8 * stage, (seq >> 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_hi = sbase + stage * STAGE_BYTES;
+                    const uint32_t a_lo = a_hi + A_BYTES;
+                    const uint32_t b_hi = a_lo + A_BYTES;
+                    const uint32_t b_lo = b_hi + B_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < KC / 8; ++kk) {
+                        const uint32_t koff = 32u * kk;
+                        const uint64_t dah = sw128_desc(a_hi + koff), dal = sw128_desc(a_lo + koff);
+                        const uint64_t dbh = sw128_desc(b_hi + koff), dbl = sw128_desc(b_lo + koff);
+                        mma2_tf32(d_tmem, dah, dbh, (k > 0 || kk > 0) ? 1u : 0u);
+                        mma2_tf32(d_tmem, dah, dbl, 1u);
+                        mma2_tf32(d_tmem, dal, dbh, 1u);
+                    }
+                    commit2(bar_empty + 8 * stage);  // both CTAs' stage free once these MMAs read it
+                }
+                if (ok) commit2(bar_afull + 8 * buf);  // both CTAs' accumulator rows complete
+            }
+            commit2(bar_drain);  // every MMA issued for the pair has completed once this fires
+        }
+        if (lane == 0) {
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait_cluster(bar_drain, 0)) {
+                if (globaltimer() - t0 > kWaitLimitNs) {
+                    *abort_flag = 1u;
+                    record_device_error(kErrTimeout);
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == TMA_WARP) {
+        // -------------------------------------------------------- TMA issuer
+        if (lane == 0) {
+            int seq = 0;
+            bool pending[2] = {false, false};
+            bool ok = true;
+            for (int tile = pair; ok && tile < p.total_tiles; tile += npairs) {
+                const TileCoord tcd = decode_pair_tile(p, tile);
+                for (int k = 0; k < nk; ++k, ++seq) {
+                    const int stage = seq & 1;
+                    if (!wait_bounded_cluster(bar_empty + 8 * stage, ((seq >> 1) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    pending[stage] = false;
+                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES);
+                    tma_load_2d(sbase + stage * STAGE_BYTES + 2 * A_BYTES, &pw_map, k * KC,
+                                tcd.o0 + (int)rank * TNH, bar_tma + 8 * stage);
+                    pending[stage] = true;
+                }
+            }
+            if (!ok) {
+                for (int st = 0; st < 2; ++st) {
+                    if (!pending[st]) continue;
+                    const int last = seq - 1 - ((seq - 1 - st) & 1);
+                    const unsigned long long t0 = globaltimer();
+                    while (last >= 0 && !mbar_try_wait(bar_tma + 8 * st, (last >> 1) & 1)) {
+                        if (globaltimer() - t0 > kWaitLimitNs) break;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const uint32_t aempty_leader = mapa(bar_aempty, 0);
+        int local = 0;
+        for (int tile = pair; tile < p.total_tiles; tile += npairs, ++local) {
+            const int buf = local & 1;
+            int ok = 1;
+            if (lane == 0) ok = wait_bounded_cluster(bar_afull + 8 * buf, (local >> 1) & 1, abort_flag) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const TileCoord tcd = decode_pair_tile(p, tile);
+            const int tw = tcd.t0 + (int)rank * TM + 32 * q;
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TN);
+            const bool vec = tw + 32 <= p.To && p.out_vec;
+            const int kq = lane >> 2, jq = lane & 3;
+            // bias of output channels o0 + 32*i + lane, one load per lane per 32
+            // columns, fetched a step ahead and broadcast by shuffle
+            auto bias_at = [&](int i) {
+                const int o = tcd.o0 + 32 * i + lane;
+                return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f;
+            };
+            float bnext = bias_at(0), bcur = 0.f;
+#pragma unroll 1
+            for (int cb = 0; cb < TN / 16; ++cb) {
+                if ((cb & 1) == 0) {
+                    bcur = bnext;
+                    if (cb + 2 < TN / 16) bnext = bias_at((cb >> 1) + 1);
+                }
+                uint32_t r[16];
+                tmem_ld16(taddr + (uint32_t)(cb * 16), r);
+                tmem_wait_ld();
+                const int obase = tcd.o0 + cb * 16;
+                float v[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    v[j] = __uint_as_float(r[j]) + __shfl_sync(0xffffffffu, bcur, (cb & 1) * 16 + j);
+                if (vec) {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        float x0 = v[m], x1 = v[4 + m], x2 = v[8 + m], x3 = v[12 + m];
+                        quad_transpose(x0, x1, x2, x3, jq);
+                        const int o = obase + 4 * jq + m;
+                        if (o < p.O) {
+                            float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
+                            __stcs(reinterpret_cast<float4*>(dst), make_float4(x0, x1, x2, x3));  // streaming store
+                        }
+                    }
+                } else {
+                    const int t = tw + lane;
+                    float* out_nt = p.out + (size_t)tcd.n * p.O * p.To + t;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int o = obase + j;
+                        if (t < p.To && o < p.O) out_nt[(size_t)o * p.To] = v[j];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(aempty_leader + 8 * buf);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the peer no longer signals this CTA's barriers
+    tc_fence_after();
+    if (warp == MMA_WARP) {
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace tc2
+
+// The 2-SM path covers the same shapes as the 1-SM tensor-core path and needs
+// at least one full pair of SMs worth of work to pay off; the halo copies
+// are 16 bytes wide when rows and the padding keep them aligned.
+inline bool conv1d_tc2_supported(int N, int C, int O, int K, int stride, int To, const void* pw)
+{
+    (void)N; (void)To;
+    return conv1d_tc_supported(C, O, K, stride, pw);
+}
+
+inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float* pw, const float* bias, int N,
+                                   int C, int T, int O, int K, int pad, int To, float* out, cudaStream_t stream)
+{
+    tc2::Params prm;
+    prm.x = x; prm.dw = dw; prm.pw = pw; prm.bias = bias; prm.out = out;
+    prm.C = C; prm.T = T; prm.O = O; prm.K = K; prm.pad = pad; prm.To = To;
+    prm.tiles_t = (To + 2 * tc2::TM - 1) / (2 * tc2::TM);
+    prm.tiles_o = (O + tc2::TN - 1) / tc2::TN;
+    const long long total = (long long)N * prm.tiles_t * prm.tiles_o;
+    if (total > 0x7fffffffLL) return FCV_ERR_UNSUPPORTED;
+    prm.total_tiles = (int)total;
+    prm.out_vec = ((To & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0) ? 1 : 0;
+    prm.x_vec = ((T & 3) == 0 && (pad & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) ? 1 : 0;
+
+    auto encode = tensor_map_encoder();
+    if (!encode) return FCV_ERR_CUDA;
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {(cuuint64_t)C, (cuuint64_t)O};
+    const cuuint64_t gstride[1] = {(cuuint64_t)C * sizeof(float)};
+    const cuuint32_t box[2] = {(cuuint32_t)tc2::KC, (cuuint32_t)tc2::TNH};
+    const cuuint32_t estride[2] = {1, 1};
+    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pw), gdim, gstride, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return FCV_ERR_CUDA;
+
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
+    auto kern = K == 9 ? tc2::dwsep_conv1d_tc2_kernel<9>
+              : K == 3 ? tc2::dwsep_conv1d_tc2_kernel<3> : tc2::dwsep_conv1d_tc2_kernel<0>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc2::SMEM_BYTES) != cudaSuccess)
+        return FCV_ERR_CUDA;
+    const long long pairs = total < sms / 2 ? total : sms / 2;
+    dim3 grid((unsigned)(2 * pairs));
+    kern<<<grid, tc2::NTHREADS, tc2::SMEM_BYTES, stream>>>(prm, map);
+    return launch_status();
+}
+
+}  // namespace fcv

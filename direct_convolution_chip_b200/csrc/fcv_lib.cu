@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "conv1d_fma.cuh"
 #include "conv1d_tc.cuh"
+#include "conv1d_tc2.cuh"
 #include "conv2d_direct.cuh"
 #include "conv2d_poolfirst.cuh"
 
@@ -159,6 +160,9 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
             return fcv::launch_dwsep_conv1d_tc(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
         }
         return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
+    case FCV_CONV1D_TC2_3XTF32:
+        if (!fcv::conv1d_tc2_supported(N, C, O, K, stride, To, pw_w)) return FCV_ERR_UNSUPPORTED;
+        return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, s);
     case FCV_CONV1D_FMA:
         return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     case FCV_CONV1D_TC_3XTF32:

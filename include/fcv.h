@@ -70,7 +70,8 @@ typedef enum {
                                      direct method. */
     /* op B */
     FCV_CONV1D_FMA = 20,          /* depthwise + pointwise on FP32 FMA */
-    FCV_CONV1D_TC_3XTF32 = 21     /* pointwise on tcgen05 tensor cores, 3xTF32 split */
+    FCV_CONV1D_TC_3XTF32 = 21,    /* pointwise on tcgen05 tensor cores, 3xTF32 split, one SM per tile */
+    FCV_CONV1D_TC2_3XTF32 = 22    /* the same on SM pairs (tcgen05 cta_group::2, 256x256 tiles) */
 } fcv_algo;
 
 /* ---------------------------------------------------------------- op A --- */
