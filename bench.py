@@ -420,23 +420,30 @@ def run_gpu(args):
             if st:
                 raise fcv.FcvError(st, "pool-first conv2d")
 
-        def alt_b():
-            st = lib.fcv_dwsep_conv1d_ex(P(xb_d.data_ptr()), P(dwb_d.data_ptr()), P(pwb_d.data_ptr()),
-                                         P(bb_d.data_ptr()), CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K,
-                                         CASE_B.stride, CASE_B.pad, P(out_b.data_ptr()), fcv.CONV1D_TC2_3XTF32, P(sp))
-            if st:
-                raise fcv.FcvError(st, "2-SM conv1d")
+        def alt_b(algo):
+            def fn():
+                st = lib.fcv_dwsep_conv1d_ex(P(xb_d.data_ptr()), P(dwb_d.data_ptr()), P(pwb_d.data_ptr()),
+                                             P(bb_d.data_ptr()), CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K,
+                                             CASE_B.stride, CASE_B.pad, P(out_b.data_ptr()), algo, P(sp))
+                if st:
+                    raise fcv.FcvError(st, f"conv1d algorithm {algo}")
+            return fn
 
         ta2 = _event_ms(alt_a, 10, stream)
-        tb2 = _event_ms(alt_b, 10, stream)
+        tb = {name: _event_ms(alt_b(algo), 10, stream)
+              for name, algo in (("dwsep_conv1d_fma", fcv.CONV1D_FMA),
+                                 ("dwsep_conv1d_tc_register_halo", fcv.CONV1D_TC_3XTF32),
+                                 ("dwsep_conv1d_tc_tma_halo", fcv.CONV1D_TC_TMA_3XTF32),
+                                 ("dwsep_conv1d_2sm", fcv.CONV1D_TC2_3XTF32))}
         pf_macs = CASE_A.N * ((CASE_A.H - 2) // CASE_A.P) * ((CASE_A.W - 2) // CASE_A.P) * CASE_A.Cout * CASE_A.Cin * 9
         result["variants"] = {
             "conv2d_poolfirst": {"ms": ta2, "executed_macs": pf_macs,
                                  "executed_gflops": 2.0 * pf_macs / (ta2 / 1e3) / 1e9,
                                  "speedup_vs_direct": ta_s * 1e3 / ta2,
                                  "note": "pools the input first (exact identity): 9*Cin MACs per pooled value"},
-            "dwsep_conv1d_2sm": {"ms": tb2, "gflops": 2.0 * macs_b / (tb2 / 1e3) / 1e9},
         }
+        for name, ms in tb.items():
+            result["variants"][name] = {"ms": ms, "gflops": 2.0 * macs_b / (ms / 1e3) / 1e9}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["unfused_gpu_baselines"] = unfused_baselines(xa_d, wa_d, ba_d, xb_d, dwb_d, pwb_d, bb_d)
         result["cpu_baseline"] = run_oracle_sample()

@@ -26,6 +26,7 @@ CONV2D_POOLFIRST = 11
 CONV1D_FMA = 20
 CONV1D_TC_3XTF32 = 21
 CONV1D_TC2_3XTF32 = 22
+CONV1D_TC_TMA_3XTF32 = 23
 
 STATUS_NAMES = {0: "FCV_OK", 1: "FCV_ERR_INVALID_ARG", 2: "FCV_ERR_UNSUPPORTED",
                 3: "FCV_ERR_CUDA", 4: "FCV_ERR_TIMEOUT"}

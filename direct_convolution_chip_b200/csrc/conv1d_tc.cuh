@@ -291,6 +291,131 @@ __device__ __forceinline__ void quad_transpose(float& x0, float& x1, float& x2, 
     if (b0) { x0 = r0; x2 = r1; } else { x1 = r0; x3 = r1; }
 }
 
+// Single-thread MMA issuer: for every tile, wait until its accumulator buffer
+// is drained; for every chunk, wait until the producers filled the stage, issue
+// the 12 MMAs of the 3xTF32 split (K = 8 each) and commit them to the stage's
+// "empty" barrier; after the last chunk commit to the accumulator's "full"
+// barrier.  Finally drain every MMA issued (bounded) so TMEM can be freed.
+__device__ __forceinline__ void mma_issuer(const Params& p, uint32_t tmem, uint32_t sbase, uint32_t bar_full,
+                                           uint32_t bar_empty, uint32_t bar_afull, uint32_t bar_aempty,
+                                           uint32_t bar_drain, volatile uint32_t* abort_flag, int nk)
+{
+    int seq = 0, local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++local) {
+        const int buf = local & 1;
+        if (!wait_bounded(bar_aempty + 8 * buf, ((local >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
+        for (int k = 0; k < nk; ++k, ++seq) {
+            const int stage = seq & 1;
+            if (!wait_bounded(bar_full + 8 * stage, (seq >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a_hi = sbase + stage * STAGE_BYTES;
+            const uint32_t a_lo = a_hi + A_BYTES;
+            const uint32_t b_hi = a_lo + A_BYTES;
+            const uint32_t b_lo = b_hi + B_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < KC / 8; ++kk) {
+                const uint32_t koff = 32u * kk;
+                const uint64_t dah = sw128_desc(a_hi + koff), dal = sw128_desc(a_lo + koff);
+                const uint64_t dbh = sw128_desc(b_hi + koff), dbl = sw128_desc(b_lo + koff);
+                tc_mma_tf32(d_tmem, dah, dbh, (k > 0 || kk > 0) ? 1u : 0u);
+                tc_mma_tf32(d_tmem, dah, dbl, 1u);
+                tc_mma_tf32(d_tmem, dal, dbh, 1u);
+            }
+            tc_commit(bar_empty + 8 * stage);  // stage free once these MMAs have read it
+        }
+        if (ok) tc_commit(bar_afull + 8 * buf);  // accumulator complete
+    }
+    // Drain: every MMA this thread issued has completed before TMEM is freed.
+    tc_commit(bar_drain);
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(bar_drain, 0)) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1u;
+            record_device_error(kErrTimeout);
+            break;
+        }
+    }
+}
+
+// One epilogue warp: drains its 32 TMEM lanes of each finished accumulator,
+// adds the bias and stores the tile's outputs, then frees the buffer.
+__device__ __forceinline__ void epilogue_warp(const Params& p, uint32_t tmem, uint32_t bar_afull,
+                                              uint32_t bar_aempty, volatile uint32_t* abort_flag, int warp,
+                                              int lane)
+{
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int local = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
+        const int buf = local & 1;
+        int ok = 1;
+        if (lane == 0) ok = wait_bounded(bar_afull + 8 * buf, (local >> 1) & 1, abort_flag) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        const TileCoord tcd = decode_tile(p, tile);
+        const int tw = tcd.t0 + 32 * q;  // first time of this warp's 32 TMEM lanes
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TN);
+        // Fast path: all 32 times in range and 16-byte aligned rows.  After a
+        // 4x4 transpose inside each lane quad, lane 4k+j holds times
+        // tw+4k .. tw+4k+3 of output channels 4j .. 4j+3 (of the 16 loaded), so
+        // each 16-byte store instruction covers 128 contiguous bytes of 4 rows.
+        const bool vec = tw + 32 <= p.To && p.out_vec;
+        const int kq = lane >> 2, jq = lane & 3;
+        // bias of output channels o0 + 32*i + lane, one load per lane per 32
+        // columns, fetched a step ahead and broadcast by shuffle
+        auto bias_at = [&](int i) {
+            const int o = tcd.o0 + 32 * i + lane;
+            return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f;
+        };
+        float bnext = bias_at(0), bcur = 0.f;
+#pragma unroll 1
+        for (int cb = 0; cb < TN / 16; ++cb) {
+            if ((cb & 1) == 0) {
+                bcur = bnext;
+                if (cb + 2 < TN / 16) bnext = bias_at((cb >> 1) + 1);
+            }
+            uint32_t r[16];
+            tmem_ld16(taddr + (uint32_t)(cb * 16), r);
+            tmem_wait_ld();
+            const int obase = tcd.o0 + cb * 16;
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                v[j] = __uint_as_float(r[j]) + __shfl_sync(0xffffffffu, bcur, (cb & 1) * 16 + j);
+            if (vec) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    // block m: rows = the 4 lanes' times, columns = channels m, 4+m, 8+m, 12+m
+                    float x0 = v[m], x1 = v[4 + m], x2 = v[8 + m], x3 = v[12 + m];
+                    quad_transpose(x0, x1, x2, x3, jq);
+                    const int o = obase + 4 * jq + m;
+                    if (o < p.O) {
+                        float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
+                        __stcs(reinterpret_cast<float4*>(dst), make_float4(x0, x1, x2, x3));  // streaming store
+                    }
+                }
+            } else {
+                const int t = tw + lane;
+                float* out_nt = p.out + (size_t)tcd.n * p.O * p.To + t;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int o = obase + j;
+                    if (t < p.To && o < p.O) out_nt[(size_t)o * p.To] = v[j];
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_aempty + 8 * buf);
+    }
+}
+
 // KT: the depthwise kernel size when known at compile time, 0 for any K <= KMAXW.
 template <int KT>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -491,49 +616,8 @@ dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_ma
         }
     } else if (warp == MMA_WARP) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            int seq = 0, local = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++local) {
-                const int buf = local & 1;
-                if (!wait_bounded(bar_aempty + 8 * buf, ((local >> 1) & 1) ^ 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
-                for (int k = 0; k < nk; ++k, ++seq) {
-                    const int stage = seq & 1;
-                    if (!wait_bounded(bar_full + 8 * stage, (seq >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a_hi = sbase + stage * STAGE_BYTES;
-                    const uint32_t a_lo = a_hi + A_BYTES;
-                    const uint32_t b_hi = a_lo + A_BYTES;
-                    const uint32_t b_lo = b_hi + B_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < KC / 8; ++kk) {
-                        const uint32_t koff = 32u * kk;
-                        const uint64_t dah = sw128_desc(a_hi + koff), dal = sw128_desc(a_lo + koff);
-                        const uint64_t dbh = sw128_desc(b_hi + koff), dbl = sw128_desc(b_lo + koff);
-                        tc_mma_tf32(d_tmem, dah, dbh, (k > 0 || kk > 0) ? 1u : 0u);
-                        tc_mma_tf32(d_tmem, dah, dbl, 1u);
-                        tc_mma_tf32(d_tmem, dal, dbh, 1u);
-                    }
-                    tc_commit(bar_empty + 8 * stage);  // stage free once these MMAs have read it
-                }
-                if (ok) tc_commit(bar_afull + 8 * buf);  // accumulator complete
-            }
-            // Drain: every MMA this thread issued has completed before TMEM is freed.
-            tc_commit(bar_drain);
-            const unsigned long long t0 = globaltimer();
-            while (!mbar_try_wait(bar_drain, 0)) {
-                if (globaltimer() - t0 > kWaitLimitNs) {
-                    *abort_flag = 1u;
-                    record_device_error(kErrTimeout);
-                    break;
-                }
-            }
-        }
+        if (lane == 0)
+            mma_issuer(p, tmem, sbase, bar_full, bar_empty, bar_afull, bar_aempty, bar_drain, abort_flag, nk);
         __syncwarp();
     } else if (warp == TMA_WARP) {
         // -------------------------------------------------------- TMA issuer
@@ -571,71 +655,7 @@ dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_ma
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
-        int local = 0;
-        for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
-            const int buf = local & 1;
-            int ok = 1;
-            if (lane == 0) ok = wait_bounded(bar_afull + 8 * buf, (local >> 1) & 1, abort_flag) ? 1 : 0;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            tc_fence_after();
-            const TileCoord tcd = decode_tile(p, tile);
-            const int tw = tcd.t0 + 32 * q;  // first time of this warp's 32 TMEM lanes
-            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TN);
-            // Fast path: all 32 times in range and 16-byte aligned rows.  After a
-            // 4x4 transpose inside each lane quad, lane 4k+j holds times
-            // tw+4k .. tw+4k+3 of output channels 4j .. 4j+3 (of the 16 loaded), so
-            // each 16-byte store instruction covers 128 contiguous bytes of 4 rows.
-            const bool vec = tw + 32 <= p.To && p.out_vec;
-            const int kq = lane >> 2, jq = lane & 3;
-            // bias of output channels o0 + 32*i + lane, one load per lane per 32
-            // columns, fetched a step ahead and broadcast by shuffle
-            auto bias_at = [&](int i) {
-                const int o = tcd.o0 + 32 * i + lane;
-                return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f;
-            };
-            float bnext = bias_at(0), bcur = 0.f;
-#pragma unroll 1
-            for (int cb = 0; cb < TN / 16; ++cb) {
-                if ((cb & 1) == 0) {
-                    bcur = bnext;
-                    if (cb + 2 < TN / 16) bnext = bias_at((cb >> 1) + 1);
-                }
-                uint32_t r[16];
-                tmem_ld16(taddr + (uint32_t)(cb * 16), r);
-                tmem_wait_ld();
-                const int obase = tcd.o0 + cb * 16;
-                float v[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    v[j] = __uint_as_float(r[j]) + __shfl_sync(0xffffffffu, bcur, (cb & 1) * 16 + j);
-                if (vec) {
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        // block m: rows = the 4 lanes' times, columns = channels m, 4+m, 8+m, 12+m
-                        float x0 = v[m], x1 = v[4 + m], x2 = v[8 + m], x3 = v[12 + m];
-                        quad_transpose(x0, x1, x2, x3, jq);
-                        const int o = obase + 4 * jq + m;
-                        if (o < p.O) {
-                            float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
-                            __stcs(reinterpret_cast<float4*>(dst), make_float4(x0, x1, x2, x3));  // streaming store
-                        }
-                    }
-                } else {
-                    const int t = tw + lane;
-                    float* out_nt = p.out + (size_t)tcd.n * p.O * p.To + t;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int o = obase + j;
-                        if (t < p.To && o < p.O) out_nt[(size_t)o * p.To] = v[j];
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_aempty + 8 * buf);
-        }
+        epilogue_warp(p, tmem, bar_afull, bar_aempty, abort_flag, warp, lane);
     }
 
     tc_fence_before();

@@ -1,0 +1,362 @@
+// conv1d_tcx.cuh -- op B on tcgen05 tensor cores with the input halo staged by TMA.
+//
+// Same contraction, tiling, 3xTF32 split, MMA issuer and epilogue as the
+// kernel in conv1d_tc.cuh (POPCORNBENCH trace "Kimi-K2.6__l2_p7", tile-GEMM
+// formulation: depthwise tile on chip, pointwise contraction as a GEMM with
+// M = time, N = output channels, K = input channels).  What changes is how the
+// producers feed the A operand, because that kernel is bound by the shared
+// memory pipe, not by the tensor cores: per 32-channel chunk its producers
+// spent ~2,000 shared-memory wavefronts (halo stores, 4-fold redundant window
+// reads) next to the 1,152 the MMAs themselves read.
+//
+//   * The TMA warp loads, next to the pw chunk, the input halo of the chunk
+//     x[n, c0:c0+32, t0-pad-r : +148] as one 3-D box (time x channel x batch)
+//     into the stage's A region, which the producers overwrite with the A
+//     operand only after reading it.  Out-of-range times (the zero padding)
+//     and channels read as zero, so there is no edge code at all.
+//   * Producer thread = one channel (lane) x 16 consecutive times (warp): it
+//     reads its window once (16 + K - 1 samples as 16-byte loads; the 148-float
+//     row pitch makes a quarter-warp's loads hit distinct banks), runs the K
+//     taps with packed FMA over time pairs, and writes its 16 A values as
+//     32-bit stores that fill one 128-byte row per warp instruction.
+//   * The pw operand's hi part is the raw fp32 chunk itself (the tensor core
+//     ignores the 13 low mantissa bits); only lo = v - truncate(v) is written.
+//   * r = (t0 - pad) mod 4 (the same for every tile) keeps the box's first
+//     time on a 16-byte boundary, as TMA requires; it is a template parameter
+//     so the window indexing stays in registers.
+//
+// Requirements beyond the register-staged kernel: T % 4 == 0 and a 16-byte
+// aligned x (the TMA map's row strides are T*4 and C*T*4 bytes).
+#pragma once
+
+#include "conv1d_tc.cuh"
+
+namespace fcv {
+namespace tcx {
+
+using namespace tc;
+
+constexpr int XW = 148;                                     // halo box width = smem row pitch (floats)
+constexpr uint32_t X_BYTES = (uint32_t)XW * KC * 4;         // 18,944 B per chunk
+constexpr int DWX_MAX = 8192;                               // resident depthwise weights, [K][32*nk]
+constexpr uint32_t OFF_DWS = STAGES * STAGE_BYTES;
+constexpr uint32_t OFF_BAR = OFF_DWS + DWX_MAX * 4;
+constexpr uint32_t NBAR = 11;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr uint32_t SMEM_USED = OFF_MISC + 16;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;           // slack to align the base to 1024 B
+
+static_assert(X_BYTES <= 2 * A_BYTES, "the halo box must fit the stage's A region");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert((XW * 4) % 16 == 0, "TMA box inner extent must be a multiple of 16 bytes");
+
+// 3-D tiled TMA load (no multicast) completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x0, int x1, int x2,
+                                            uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x0), "r"(x1), "r"(x2), "r"(bar)
+        : "memory");
+}
+
+// Prefetch of one 3-D box into L2 (a hint: nothing waits for it).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x0, int x1, int x2)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x0), "r"(x1), "r"(x2)
+                 : "memory");
+}
+
+// v - truncate_tf32(v) per component: the part of v below the TF32 mantissa, exact in fp32.
+__device__ __forceinline__ float4 tf32_trunc_rest4(const float4 v)
+{
+    auto rest = [](float a) { return a - __uint_as_float(__float_as_uint(a) & 0xFFFFE000u); };
+    return make_float4(rest(v.x), rest(v.y), rest(v.z), rest(v.w));
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, float v)
+{
+    asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(addr), "f"(v) : "memory");
+}
+
+// KT: depthwise kernel size when fixed at compile time (0: any K <= KMAXW).
+// R: (t0 - pad) mod 4, the offset of the first needed sample inside the box.
+template <int KT, int R>
+__global__ void __launch_bounds__(NTHREADS, 1)
+dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_map,
+                        const __grid_constant__ CUtensorMap x_map)
+{
+    constexpr int KW = KT > 0 ? KT : KMAXW;            // taps the window must cover
+    constexpr int NV = (R + 15 + KW + 3) / 4;          // 16-byte window loads per thread
+    static_assert(16 * 7 + 4 * NV <= XW, "window inside the halo box");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    float* dws = reinterpret_cast<float*>(smem + OFF_DWS);
+    const uint32_t bar_full = sbase + OFF_BAR;       // + 8 * stage
+    const uint32_t bar_empty = bar_full + 16;        // + 8 * stage
+    const uint32_t bar_afull = bar_full + 32;        // + 8 * buf
+    const uint32_t bar_aempty = bar_full + 48;       // + 8 * buf
+    const uint32_t bar_drain = bar_full + 64;
+    const uint32_t bar_tma = bar_full + 72;          // + 8 * stage
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
+    volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_full + 8 * i, 8);    // one arrival per producer warp
+            mbar_init(bar_empty + 8 * i, 1);   // tcgen05.commit
+            mbar_init(bar_afull + 8 * i, 1);   // tcgen05.commit
+            mbar_init(bar_aempty + 8 * i, 4);  // one arrival per epilogue warp
+        }
+        mbar_init(bar_drain, 1);
+        mbar_init(bar_tma, 1);       // expect_tx arrival + TMA bytes
+        mbar_init(bar_tma + 8, 1);
+        *abort_flag = 0u;
+        *prod_abort = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == MMA_WARP) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_holder)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+
+    const int nk = (p.C + KC - 1) / KC;
+    // Depthwise weights of every channel stay resident, transposed to [K][CW]
+    // with CW = 32 * nk (zero beyond C), so lane c of chunk kc reads its tap k
+    // at dws[k * CW + 32 * kc + c]: 32 consecutive floats per warp load.
+    const int CW = KC * nk;
+    for (int e = threadIdx.x; e < p.K * CW; e += NTHREADS) {
+        const int k = e / CW, c = e - (e / CW) * CW;
+        dws[e] = c < p.C ? __ldg(p.dw + (size_t)c * p.K + k) : 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp < 8) {
+        // ------------------------------------------------------------ producers
+        const int ptid = threadIdx.x;
+        const int K = KT > 0 ? KT : p.K;
+        int seq = 0;
+        bool run = true;
+        for (int tile = blockIdx.x; run && tile < p.total_tiles; tile += gridDim.x) {
+            for (int kc = 0; kc < nk; ++kc, ++seq) {
+                const int stage = seq & 1;
+                const uint32_t parity = (seq >> 1) & 1;
+                // The TMA copies of this stage (pw chunk and halo) have landed.
+                if (ptid == 0 && !wait_bounded(bar_tma + 8 * stage, parity, abort_flag)) *prod_abort = 1u;
+                asm volatile("bar.sync 1, 256;\n" ::: "memory");
+                if (*prod_abort) {
+                    run = false;
+                    break;
+                }
+                // Thread 0 saw this phase complete, so this returns at once; it gives
+                // every producer its own acquire of the TMA bytes.
+                for (int spin = 0; !mbar_try_wait(bar_tma + 8 * stage, parity) && spin < (1 << 20); ++spin) {
+                }
+
+                const uint32_t a_hi = sbase + stage * STAGE_BYTES;
+                const uint32_t a_lo = a_hi + A_BYTES;
+                const uint32_t b_hi = a_lo + A_BYTES;
+                const uint32_t b_lo = b_hi + B_BYTES;
+
+                // pw chunk: B_hi stays the raw fp32 the TMA wrote, because the MMA
+                // reads only the TF32 bits of an fp32 operand (the 13 low mantissa
+                // bits are ignored, i.e. hi = truncate(v)); B_lo = v - truncate(v)
+                // is exact and |B_lo| < 2^-10 |v|.  This saves the in-place rewrite.
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int row = warp * 32 + i * 4 + (lane >> 3);
+                    const uint32_t off = sw128_off(row, lane & 7);
+                    sts128(b_lo + off, tf32_trunc_rest4(lds128(b_hi + off)));
+                }
+
+                // Depthwise: channel lane, times 16*warp .. 16*warp+15 of the tile.
+                // Sample j of the halo row is x[t0 - pad - R + j]; output time
+                // 16*warp + i takes samples 16*warp + R + i + k, k < K.
+                const float* xrow = reinterpret_cast<const float*>(smem + stage * STAGE_BYTES) + lane * XW + 16 * warp;
+                float win[4 * NV];
+#pragma unroll
+                for (int q = 0; q < NV; ++q) {
+                    const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
+                    win[4 * q] = v.x;
+                    win[4 * q + 1] = v.y;
+                    win[4 * q + 2] = v.z;
+                    win[4 * q + 3] = v.w;
+                }
+                float2 d2[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) d2[j] = make_float2(0.f, 0.f);
+                const float* wcol = dws + KC * kc + lane;
+#pragma unroll
+                for (int k = 0; k < KW; ++k) {
+                    if (KT > 0 || k < K) {
+                        const float w = wcol[k * CW];
+                        const float2 w2 = make_float2(w, w);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            d2[j] = __ffma2_rn(make_float2(win[R + 2 * j + k], win[R + 2 * j + k + 1]), w2, d2[j]);
+                    }
+                }
+                // Every producer has read its halo window before the A operand overwrites it.
+                asm volatile("bar.sync 1, 256;\n" ::: "memory");
+
+                // A operand: row t = 16*warp + i, column = channel lane; one warp
+                // store fills one 128-byte swizzled row.
+                const uint32_t col = ((uint32_t)(lane & 3) << 2);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float v = (i & 1) ? d2[i >> 1].y : d2[i >> 1].x;
+                    const float hi = tf32_round(v);
+                    const uint32_t off = sw128_off(16 * warp + i, lane >> 2) + col;
+                    sts32(a_hi + off, hi);
+                    sts32(a_lo + off, v - hi);
+                }
+                // Make the generic-proxy writes visible to the tensor core, then signal the stage full.
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_full + 8 * stage);
+            }
+        }
+    } else if (warp == MMA_WARP) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0)
+            mma_issuer(p, tmem, sbase, bar_full, bar_empty, bar_afull, bar_aempty, bar_drain, abort_flag, nk);
+        __syncwarp();
+    } else if (warp == TMA_WARP) {
+        // -------------------------------------------------------- TMA issuer
+        if (lane == 0) {
+            int seq = 0;
+            bool pending[2] = {false, false};
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+                const TileCoord tcd = decode_tile(p, tile);
+                const int x0 = tcd.t0 - p.pad - R;  // a multiple of 4: 16-byte aligned time coordinate
+                // Pull the next tile's halo boxes into L2 now, so its TMA loads
+                // wait on L2 rather than on DRAM latency.
+                if (tile + (int)gridDim.x < p.total_tiles) {
+                    const TileCoord nx = decode_tile(p, tile + gridDim.x);
+                    for (int k = 0; k < nk; ++k) tma_prefetch_3d(&x_map, nx.t0 - p.pad - R, k * KC, nx.n);
+                }
+                for (int k = 0; k < nk; ++k, ++seq) {
+                    const int stage = seq & 1;
+                    if (!wait_bounded(bar_empty + 8 * stage, ((seq >> 1) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    pending[stage] = false;  // the producers consumed its previous loads before the MMA ran
+                    const uint32_t st = sbase + stage * STAGE_BYTES;
+                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES + X_BYTES);
+                    tma_load_2d(st + 2 * A_BYTES, &pw_map, k * KC, tcd.o0, bar_tma + 8 * stage);
+                    tma_load_3d(st, &x_map, x0, k * KC, tcd.n, bar_tma + 8 * stage);
+                    pending[stage] = true;
+                }
+            }
+            // On an abort, wait (bounded) for copies still in flight before the CTA can exit.
+            if (!ok) {
+                for (int st = 0; st < 2; ++st) {
+                    if (!pending[st]) continue;
+                    const int last = seq - 1 - ((seq - 1 - st) & 1);  // latest sequence number on this stage
+                    const unsigned long long t0 = globaltimer();
+                    while (last >= 0 && !mbar_try_wait(bar_tma + 8 * st, (last >> 1) & 1)) {
+                        if (globaltimer() - t0 > kWaitLimitNs) break;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        epilogue_warp(p, tmem, bar_afull, bar_aempty, abort_flag, warp, lane);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == MMA_WARP) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace tcx
+
+// Shapes the TMA-halo tensor-core kernel covers.
+inline bool conv1d_tcx_supported(int C, int T, int O, int K, int stride, const void* x, const void* pw)
+{
+    const long long cw = (long long)tc::KC * ((C + tc::KC - 1) / tc::KC);
+    return stride == 1 && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1 && T >= 1 && (C & 3) == 0 &&
+           (T & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(pw) & 15) == 0 && cw * K <= tcx::DWX_MAX;
+}
+
+inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float* pw, const float* bias, int N,
+                                   int C, int T, int O, int K, int pad, int To, float* out, cudaStream_t stream)
+{
+    tc::Params prm;
+    prm.x = x; prm.dw = dw; prm.pw = pw; prm.bias = bias; prm.out = out;
+    prm.C = C; prm.T = T; prm.O = O; prm.K = K; prm.pad = pad; prm.To = To;
+    prm.tiles_t = (To + tc::TM - 1) / tc::TM;
+    prm.tiles_o = (O + tc::TN - 1) / tc::TN;
+    const long long total = (long long)N * prm.tiles_t * prm.tiles_o;
+    if (total > 0x7fffffffLL) return FCV_ERR_UNSUPPORTED;
+    prm.total_tiles = (int)total;
+    prm.out_vec = ((To & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0) ? 1 : 0;
+
+    auto encode = tensor_map_encoder();
+    if (!encode) return FCV_ERR_CUDA;
+    // pw [O][C]: 32 channels x 256 output channels per box, 128B-swizzled.
+    CUtensorMap pw_map, x_map;
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)C, (cuuint64_t)O};
+        const cuuint64_t gstride[1] = {(cuuint64_t)C * sizeof(float)};
+        const cuuint32_t box[2] = {(cuuint32_t)tc::KC, (cuuint32_t)tc::TN};
+        const cuuint32_t estride[2] = {1, 1};
+        if (encode(&pw_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pw), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return FCV_ERR_CUDA;
+    }
+    // x [N][C][T]: 148 times x 32 channels x 1 batch item per box, rows packed
+    // (no swizzle); times and channels outside the tensor read as zero.
+    {
+        const cuuint64_t gdim[3] = {(cuuint64_t)T, (cuuint64_t)C, (cuuint64_t)N};
+        const cuuint64_t gstride[2] = {(cuuint64_t)T * sizeof(float), (cuuint64_t)C * T * sizeof(float)};
+        const cuuint32_t box[3] = {(cuuint32_t)tcx::XW, (cuuint32_t)tc::KC, 1};
+        const cuuint32_t estride[3] = {1, 1, 1};
+        if (encode(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(x), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return FCV_ERR_CUDA;
+    }
+
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
+    const int r = (-pad) & 3;  // (t0 - pad) mod 4 with t0 a multiple of 128
+    decltype(&tcx::dwsep_conv1d_tcx_kernel<0, 0>) kern;
+    if (K == 9 && r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<9, 0>;
+    else if (K == 3 && r == 3) kern = tcx::dwsep_conv1d_tcx_kernel<3, 3>;
+    else if (r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<0, 0>;
+    else if (r == 1) kern = tcx::dwsep_conv1d_tcx_kernel<0, 1>;
+    else if (r == 2) kern = tcx::dwsep_conv1d_tcx_kernel<0, 2>;
+    else kern = tcx::dwsep_conv1d_tcx_kernel<0, 3>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcx::SMEM_BYTES) != cudaSuccess)
+        return FCV_ERR_CUDA;
+    const int grid = (int)(total < sms ? total : sms);
+    kern<<<grid, tc::NTHREADS, tcx::SMEM_BYTES, stream>>>(prm, pw_map, x_map);
+    return launch_status();
+}
+
+}  // namespace fcv

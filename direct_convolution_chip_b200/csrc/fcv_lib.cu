@@ -9,6 +9,7 @@
 #include "conv1d_fma.cuh"
 #include "conv1d_tc.cuh"
 #include "conv1d_tc2.cuh"
+#include "conv1d_tcx.cuh"
 #include "conv2d_direct.cuh"
 #include "conv2d_poolfirst.cuh"
 
@@ -156,6 +157,8 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
     cudaStream_t s = fcv::as_stream(stream);
     switch (algo) {
     case FCV_ALGO_AUTO:
+        if (fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w))
+            return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, s);
         if (fcv::conv1d_tc_supported(C, O, K, stride, pw_w)) {
             return fcv::launch_dwsep_conv1d_tc(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
         }
@@ -168,6 +171,9 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
     case FCV_CONV1D_TC_3XTF32:
         if (!fcv::conv1d_tc_supported(C, O, K, stride, pw_w)) return FCV_ERR_UNSUPPORTED;
         return fcv::launch_dwsep_conv1d_tc(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
+    case FCV_CONV1D_TC_TMA_3XTF32:
+        if (!fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w)) return FCV_ERR_UNSUPPORTED;
+        return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, s);
     default:
         return FCV_ERR_INVALID_ARG;
     }

@@ -18,7 +18,7 @@ from tests.parity import assert_close, requires_cuda, sample_indices
 pytestmark = [pytest.mark.gpu, requires_cuda]
 
 CONV2D_ALGOS = [fcv.CONV2D_DIRECT, fcv.CONV2D_POOLFIRST]
-CONV1D_ALGOS = [fcv.CONV1D_FMA, fcv.CONV1D_TC_3XTF32, fcv.CONV1D_TC2_3XTF32]
+CONV1D_ALGOS = [fcv.CONV1D_FMA, fcv.CONV1D_TC_3XTF32, fcv.CONV1D_TC2_3XTF32, fcv.CONV1D_TC_TMA_3XTF32]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -36,7 +36,7 @@ def conv1d_or_skip(x, dw, pw, bias, s, p, algo):
     try:
         return fcv.dwsep_conv1d(x, dw, pw, bias, s, p, algo=algo)
     except fcv.FcvError as e:
-        if e.status == 2 and algo in (fcv.CONV1D_TC_3XTF32, fcv.CONV1D_TC2_3XTF32):
+        if e.status == 2 and algo in (fcv.CONV1D_TC_3XTF32, fcv.CONV1D_TC2_3XTF32, fcv.CONV1D_TC_TMA_3XTF32):
             pytest.skip("tensor-core path does not cover this shape")
         raise
 
