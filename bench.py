@@ -429,7 +429,15 @@ def run_gpu(args):
                     raise fcv.FcvError(st, f"conv1d algorithm {algo}")
             return fn
 
+        def alt_a_tc():
+            st = lib.fcv_conv2d_pool_sigmoid_sum_ex(P(xa_d.data_ptr()), P(wa_d.data_ptr()), P(ba_d.data_ptr()),
+                                                    CASE_A.N, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout, CASE_A.P,
+                                                    P(out_a.data_ptr()), fcv.CONV2D_TC_3XTF32, P(sp))
+            if st:
+                raise fcv.FcvError(st, "tensor-core conv2d")
+
         ta2 = _event_ms(alt_a, 10, stream)
+        ta3 = _event_ms(alt_a_tc, 10, stream)
         tb = {name: _event_ms(alt_b(algo), 10, stream)
               for name, algo in (("dwsep_conv1d_fma", fcv.CONV1D_FMA),
                                  ("dwsep_conv1d_tc_register_halo", fcv.CONV1D_TC_3XTF32),
@@ -441,6 +449,8 @@ def run_gpu(args):
                                  "executed_gflops": 2.0 * pf_macs / (ta2 / 1e3) / 1e9,
                                  "speedup_vs_direct": ta_s * 1e3 / ta2,
                                  "note": "pools the input first (exact identity): 9*Cin MACs per pooled value"},
+            "conv2d_tc_3xtf32": {"ms": ta3, "gflops": 2.0 * macs_a / (ta3 / 1e3) / 1e9,
+                                 "frac_of_3xtf32_peak": 2.0 * macs_a / (ta3 / 1e3) / 1e12 / (tf32_peak / 3.0)},
         }
         for name, ms in tb.items():
             result["variants"][name] = {"ms": ms, "gflops": 2.0 * macs_b / (ms / 1e3) / 1e9}

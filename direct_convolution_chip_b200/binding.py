@@ -23,6 +23,7 @@ _LIB = None
 ALGO_AUTO = 0
 CONV2D_DIRECT = 10
 CONV2D_POOLFIRST = 11
+CONV2D_TC_3XTF32 = 12
 CONV1D_FMA = 20
 CONV1D_TC_3XTF32 = 21
 CONV1D_TC2_3XTF32 = 22

@@ -27,12 +27,13 @@ def sources():
 
 
 def build_probes(force: bool = False) -> str:
-    """Compile libfcv_probes.so (the FP32-FMA peak probe) if missing or stale."""
-    src = os.path.join(CSRC, "probes", "fma_peak.cu")
-    if not force and os.path.exists(PROBE_LIB) and os.path.getmtime(PROBE_LIB) >= os.path.getmtime(src):
+    """Compile libfcv_probes.so (the FP32-FMA and tcgen05 TF32 peak probes) if missing or stale."""
+    srcs = [os.path.join(CSRC, "probes", f) for f in ("fma_peak.cu", "tf32_mma_rate.cu")]
+    if not force and os.path.exists(PROBE_LIB) and all(
+            os.path.getmtime(PROBE_LIB) >= os.path.getmtime(s) for s in srcs):
         return PROBE_LIB
     tmp = PROBE_LIB + ".tmp"
-    subprocess.run([nvcc()] + NVCC_FLAGS + ["-o", tmp, src], check=True)
+    subprocess.run([nvcc()] + NVCC_FLAGS + ["-o", tmp] + srcs, check=True)
     os.replace(tmp, PROBE_LIB)
     return PROBE_LIB
 

@@ -1,0 +1,592 @@
+// conv2d_tc.cuh -- op A on tcgen05 tensor cores: the direct 3x3 convolution of
+// every pooled window as an implicit GEMM, fp32-accurate through a 3xTF32 split.
+//
+// What it computes (POPCORNBENCH trace of the fused Conv2d -> AvgPool -> Sigmoid
+// -> Sum kernel; the trace notes cuDNN would run this convolution on TF32
+// tensor cores): every conv output y[n, co, r, c] = b[co] + sum over (ci, ky, kx)
+// of w[co, ci, ky, kx] * x[n, ci, r+ky, c+kx], averaged over P x P windows,
+// passed through the sigmoid and summed per image.  Written as a GEMM per
+// tile, D[m, co] = sum_k A[m, k] * B[co, k] with
+//     m = one of 128 conv positions (P conv rows x 128/P conv columns),
+//     k = (ci, ky, kx), chunks of 8 input channels = 72 K elements,
+//     A = the im2col rows of x, B = w.
+// Every conv output is computed (the same multiply-adds as the FMA kernel),
+// only on the tensor cores; the P x P pooling is a sum over accumulator rows
+// done in the epilogue.
+//
+// B200 design (one CTA per SM, persistent over tiles, 9 warps):
+//   * warps 0-3 (producers, one per TMEM lane quarter): stage the input halo
+//     of the next (tile, chunk) with cp.async while building the current one:
+//     each thread owns one conv position (= one TMEM lane), reads its 72
+//     im2col values from the halo, splits them into TF32 hi/lo and writes them
+//     straight into tensor memory with tcgen05.st (the A operand of the MMA is
+//     read from TMEM, so A costs no shared-memory bandwidth).
+//   * warp 4: allocates TMEM (two accumulators of Cout' columns, two A stages
+//     of 144 columns); one thread issues 27 tcgen05.mma (kind::tf32, M = 128,
+//     N = Cout', K = 8, A from TMEM, B from shared memory) per chunk:
+//     A_hi*B_hi + A_hi*B_lo + A_lo*B_hi.
+//   * The weights, split into TF32 hi/lo once per CTA, stay in shared memory
+//     in the K-major 128-byte-swizzled layout for the whole kernel.
+//   * warps 5-8 (epilogue): drain an accumulator with tcgen05.ld into a
+//     transposed shared buffer, release it to the MMA, then each thread sums
+//     the P x P conv outputs of its (window, channel) values, adds the bias,
+//     applies the sigmoid and accumulates; one atomic add per warp and image.
+//   * Every wait is bounded, as in the conv1d kernels.
+#pragma once
+
+#include "conv1d_tc.cuh"
+#include "conv2d_direct.cuh"
+
+#include <type_traits>
+
+namespace fcv {
+namespace c2tc {
+
+using tc::globaltimer;
+using tc::kWaitLimitNs;
+using tc::mbar_arrive;
+using tc::mbar_init;
+using tc::mbar_try_wait;
+using tc::smem_u32;
+using tc::sw128_desc;
+using tc::sw128_off;
+using tc::tc_commit;
+using tc::tc_fence_after;
+using tc::tc_fence_before;
+using tc::tf32_round;
+using tc::tmem_ld16;
+using tc::tmem_wait_ld;
+using tc::wait_bounded;
+
+constexpr int MT = 128;           // conv positions per tile (UMMA M)
+constexpr int CCH = 8;            // input channels per K chunk
+constexpr int KCH = 9 * CCH;      // 72 K elements per chunk
+constexpr int KST = KCH / 8;      // 9 MMA K-steps per chunk
+constexpr int A_COLS = 2 * KCH;   // one A stage in TMEM: hi (72 columns) | lo (72 columns)
+constexpr int NP_MAX = 112;       // padded Cout: 2 * NP + 2 * A_COLS <= 512 TMEM columns
+constexpr int NPROD = 256;        // producer threads: warps 0-7, two per TMEM lane quarter
+constexpr int MMA_WARP = 8;
+constexpr int EPI_WARP0 = 9;      // epilogue: warps 9-16, two per TMEM lane quarter
+constexpr int NEPI = 256;
+constexpr int NTHREADS = 17 * 32;
+constexpr int TP = 132;           // pitch of the transposed accumulator buffer (floats)
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int SMEM_LIMIT = 227 * 1024;
+
+template <int P>
+struct Geo {
+    static constexpr int WC = MT / P;                                // conv columns per tile
+    static constexpr int WPT = WC / P;                               // pooled windows per tile
+    static constexpr int HR = P + 2;                                 // halo rows
+    static constexpr int HW = WC + 2;                                // halo columns
+    static constexpr int HP = P == 8 ? 48 : ((HW + 3) & ~3);         // halo row pitch (floats)
+    static constexpr int CHS = HR * HP;                              // halo channel stride
+    static constexpr int HALO = CCH * CHS;                           // floats per halo buffer
+    static_assert(WC * P == MT && WPT * P == WC, "tile shape");
+    static_assert(HP >= HW, "halo pitch");
+};
+
+struct Params {
+    const float* x;
+    const float* w;
+    const float* b;
+    float* out;       // sum mode: out[N]; tap mode: pooled[N, Cout, PH, PW]
+    int Cin, H, W, Cout, PH, PW;
+    int NP;           // Cout rounded up to 16 (MMA N)
+    int nchunks;      // ceil(Cin / 8)
+    int natoms;       // 128-byte-wide K blocks of the weight operand
+    int tiles_x;      // tiles per pooled row
+    int tiles_img;    // tiles per image
+    int total_tiles;
+    int use_tma;      // halo by one 4-D TMA box (W % 4 == 0, aligned x), else by cp.async
+};
+
+// Shared-memory layout (bytes, from a 1024-aligned base).
+struct Layout {
+    uint32_t b_hi, b_lo, halo, tbuf, bias, bar, misc, total;
+};
+
+template <int P>
+__host__ __device__ inline Layout make_layout(int NP, int natoms)
+{
+    Layout L;
+    const uint32_t atoms_bytes = (uint32_t)natoms * (uint32_t)NP * 128u;
+    L.b_hi = 0;
+    L.b_lo = atoms_bytes;
+    L.halo = 2 * atoms_bytes;
+    L.tbuf = L.halo + 2u * Geo<P>::HALO * 4u;
+    L.bias = L.tbuf + (uint32_t)NP * TP * 4u;
+    L.bar = (L.bias + (uint32_t)NP * 4u + 7u) & ~7u;
+    L.misc = L.bar + 11u * 8u;
+    L.total = L.misc + 16u;
+    return L;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::tf32, A read from tensor memory.
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 8 consecutive 32-bit TMEM columns of the warp's 32 lanes (one register each).
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]));
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// 4-D tiled TMA load (no multicast) completing on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+        : "memory");
+}
+
+struct TileCoord {
+    int n, py, tx;  // image, pooled row, tile column
+};
+
+__device__ __forceinline__ TileCoord decode(const Params& p, int tile)
+{
+    TileCoord t;
+    t.n = tile / p.tiles_img;
+    const int r = tile - t.n * p.tiles_img;
+    t.py = r / p.tiles_x;
+    t.tx = r - t.py * p.tiles_x;
+    return t;
+}
+
+template <int P, int MODE>
+__global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap x_map)
+{
+    using G = Geo<P>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    const Layout L = make_layout<P>(p.NP, p.natoms);
+    float* halo = reinterpret_cast<float*>(smem + L.halo);
+    float* tbuf = reinterpret_cast<float*>(smem + L.tbuf);
+    float* bias_s = reinterpret_cast<float*>(smem + L.bias);
+    const uint32_t bar_afull = sbase + L.bar;         // + 8 * stage, 4 producer-warp arrivals
+    const uint32_t bar_aempty = bar_afull + 16;       // + 8 * stage, tcgen05.commit
+    const uint32_t bar_accfull = bar_afull + 32;      // + 8 * buf, tcgen05.commit
+    const uint32_t bar_accempty = bar_afull + 48;     // + 8 * buf, 4 epilogue-warp arrivals
+    const uint32_t bar_drain = bar_afull + 64;
+    const uint32_t bar_hfull = bar_afull + 72;        // + 8 * buf, TMA halo landed
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.misc);
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 4);
+    volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 8);
+    volatile uint32_t* epi_abort = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 12);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NP = p.NP;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_afull + 8 * i, 8);
+            mbar_init(bar_aempty + 8 * i, 1);
+            mbar_init(bar_accfull + 8 * i, 1);
+            mbar_init(bar_accempty + 8 * i, 8);
+        }
+        mbar_init(bar_drain, 1);
+        mbar_init(bar_hfull, 1);
+        mbar_init(bar_hfull + 8, 1);
+        *abort_flag = 0u;
+        *prod_abort = 0u;
+        *epi_abort = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == MMA_WARP) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_holder)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+
+    // Weights as the B operand, split into TF32 hi/lo: element (co, k) with
+    // k = 72 * chunk + 9 * (ci mod 8) + 3 * ky + kx sits in 128-byte K block
+    // k / 32 (blocks of NP rows), row co, swizzled 16-byte chunk (k mod 32) / 4.
+    const int ktot = KCH * p.nchunks;
+    for (int idx = threadIdx.x; idx < NP * ktot; idx += NTHREADS) {
+        const int co = idx / ktot, k = idx - co * ktot;
+        const int ch = k / KCH, e = k - ch * KCH;
+        const int ci = ch * CCH + e / 9, t = e % 9;
+        const float v = (co < p.Cout && ci < p.Cin) ? __ldg(p.w + ((size_t)co * p.Cin + ci) * 9 + t) : 0.f;
+        const float hi = tf32_round(v);
+        const int a = k >> 5, kin = k & 31;
+        const uint32_t off = (uint32_t)a * NP * 128u + sw128_off(co, kin >> 2) + (uint32_t)(kin & 3) * 4u;
+        *reinterpret_cast<float*>(smem + L.b_hi + off) = hi;
+        *reinterpret_cast<float*>(smem + L.b_lo + off) = v - hi;
+    }
+    for (int i = threadIdx.x; i < NP; i += NTHREADS) bias_s[i] = i < p.Cout ? __ldg(p.b + i) : 0.f;
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // weights visible to the tensor core
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t a_col0 = 2u * (uint32_t)NP;  // first A-stage column
+
+    if (warp < 8) {
+        // ------------------------------------------------------------ producers
+        const int tid = threadIdx.x;               // 0..255
+        const int m = 32 * (warp & 3) + lane;      // conv position = TMEM lane
+        const int half = warp >> 2;                // K groups 0-4 or 5-8 of the chunk
+        const int r = m / G::WC, c = m - (m / G::WC) * G::WC;
+        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        int pseq_tile = blockIdx.x, pseq_ch = 0;  // the (tile, chunk) whose halo is being fetched
+
+        bool hpending[2] = {false, false};
+        auto fetch = [&](int tile, int ch, int buf) {
+            const TileCoord tcd = decode(p, tile);
+            const int y0 = tcd.py * P, x0 = tcd.tx * G::WC, c0 = ch * CCH;
+            if (p.use_tma) {
+                // One box [8 channels][P + 2 rows][HP columns] lands with the
+                // halo layout itself; rows, columns and channels outside x read 0.
+                if (tid == 0) {
+                    tc::mbar_arrive_expect_tx(bar_hfull + 8 * buf, (uint32_t)G::HALO * 4u);
+                    tma_load_4d(smem_u32(halo + buf * G::HALO), &x_map, x0, y0, c0, tcd.n, bar_hfull + 8 * buf);
+                }
+                hpending[buf] = true;
+                return;
+            }
+            float* dst = halo + buf * G::HALO;
+            const float* src = p.x + ((size_t)tcd.n * p.Cin) * p.H * p.W;
+            for (int i = tid; i < CCH * G::HR * G::HW; i += NPROD) {
+                const int ci = i / (G::HR * G::HW);
+                const int rem = i - ci * (G::HR * G::HW);
+                const int hr = rem / G::HW, hc = rem - (rem / G::HW) * G::HW;
+                const int gy = y0 + hr, gx = x0 + hc, gc = c0 + ci;
+                const bool ok = gc < p.Cin && gy < p.H && gx < p.W;
+                const float* s = ok ? src + ((size_t)gc * p.H + gy) * p.W + gx : p.x;
+                cp_async4(dst + ci * G::CHS + hr * G::HP + hc, s, ok);
+            }
+            cp_async_commit();
+        };
+
+        if (pseq_tile < p.total_tiles) fetch(pseq_tile, 0, 0);
+        int seq = 0, tile = blockIdx.x, ch = 0;
+        for (; tile < p.total_tiles; ++seq) {
+            const int stage = seq & 1;
+            // The MMAs that read this A stage two chunks ago have completed.  One
+            // thread waits (bounded) before the barrier, so the abort decision
+            // read after it is the same for every producer.
+            if (tid == 0 && !wait_bounded(bar_aempty + 8 * stage, ((seq >> 1) & 1) ^ 1, abort_flag)) *prod_abort = 1u;
+            if (p.use_tma) {
+                if (tid == 0 && !wait_bounded(bar_hfull + 8 * stage, (seq >> 1) & 1, abort_flag)) *prod_abort = 1u;
+            } else {
+                cp_async_wait<0>();
+            }
+            asm volatile("bar.sync 1, 256;\n" ::: "memory");  // halo landed, stage free
+            if (*prod_abort) break;
+            if (p.use_tma) {
+                hpending[stage] = false;
+                for (int spin = 0; !mbar_try_wait(bar_hfull + 8 * stage, (seq >> 1) & 1) && spin < (1 << 20); ++spin) {
+                }
+            }
+            for (int spin = 0; !mbar_try_wait(bar_aempty + 8 * stage, ((seq >> 1) & 1) ^ 1) && spin < (1 << 20);
+                 ++spin) {
+            }
+            tc_fence_after();
+            // Fetch the next (tile, chunk) halo into the other buffer.
+            if (++pseq_ch == p.nchunks) {
+                pseq_ch = 0;
+                pseq_tile += gridDim.x;
+            }
+            if (pseq_tile < p.total_tiles) fetch(pseq_tile, pseq_ch, stage ^ 1);
+
+            // im2col row of position (r, c): 72 values, 8 per TMEM store; the two
+            // warps of a lane quarter take K groups 0-4 and 5-8.
+            const float* hb = halo + stage * G::HALO + r * G::HP + c;
+            const uint32_t a_hi = tmem + lane_base + a_col0 + (uint32_t)(stage * A_COLS);
+            auto build = [&](auto g0c, auto g1c) {
+                constexpr int g0 = decltype(g0c)::value, g1 = decltype(g1c)::value;
+#pragma unroll
+            for (int g = g0; g < g1; ++g) {
+                uint32_t hi[8], lo[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int e = 8 * g + q;
+                    const int ci = e / 9, t = e % 9;
+                    const float v = hb[ci * G::CHS + (t / 3) * G::HP + (t % 3)];
+                    const float h = tf32_round(v);
+                    hi[q] = __float_as_uint(h);
+                    lo[q] = __float_as_uint(v - h);
+                }
+                tmem_st8(a_hi + (uint32_t)(8 * g), hi);
+                tmem_st8(a_hi + (uint32_t)(KCH + 8 * g), lo);
+            }
+            };
+            if (half == 0) build(std::integral_constant<int, 0>{}, std::integral_constant<int, 5>{});
+            else build(std::integral_constant<int, 5>{}, std::integral_constant<int, KST>{});
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_afull + 8 * stage);
+            if (++ch == p.nchunks) {
+                ch = 0;
+                tile += gridDim.x;
+            }
+        }
+        cp_async_wait<0>();  // no copy may land after the CTA has left
+        if (tid == 0) {
+            // After an abort a TMA box may still be in flight: wait for it (bounded).
+            for (int b = 0; b < 2; ++b) {
+                if (!hpending[b]) continue;
+                const int sq = ((seq & 1) == b) ? seq : seq + 1;  // the sequence number that box belongs to
+                const unsigned long long t0 = globaltimer();
+                while (!mbar_try_wait(bar_hfull + 8 * b, (sq >> 1) & 1)) {
+                    if (globaltimer() - t0 > kWaitLimitNs) break;
+                }
+            }
+        }
+    } else if (warp == MMA_WARP) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NP >> 3) << 17) |
+                                   ((uint32_t)(MT >> 4) << 24);
+            int seq = 0, local = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++local) {
+                const int buf = local & 1;
+                if (!wait_bounded(bar_accempty + 8 * buf, ((local >> 1) & 1) ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(buf * NP);
+                for (int ch = 0; ch < p.nchunks; ++ch, ++seq) {
+                    const int stage = seq & 1;
+                    if (!wait_bounded(bar_afull + 8 * stage, (seq >> 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_hi = tmem + a_col0 + (uint32_t)(stage * A_COLS);
+#pragma unroll
+                    for (int kk = 0; kk < KST; ++kk) {
+                        const int gk = ch * KST + kk;  // global K-step
+                        const uint32_t boff = (uint32_t)(gk >> 2) * NP * 128u + 32u * (uint32_t)(gk & 3);
+                        const uint64_t bh = sw128_desc(sbase + L.b_hi + boff), bl = sw128_desc(sbase + L.b_lo + boff);
+                        const uint32_t ah = a_hi + 8u * kk, al = a_hi + (uint32_t)KCH + 8u * kk;
+                        mma_tf32_ts(d_tmem, ah, bh, idesc, (ch > 0 || kk > 0) ? 1u : 0u);
+                        mma_tf32_ts(d_tmem, ah, bl, idesc, 1u);
+                        mma_tf32_ts(d_tmem, al, bh, idesc, 1u);
+                    }
+                    tc_commit(bar_aempty + 8 * stage);  // A stage free once these MMAs are done
+                }
+                if (ok) tc_commit(bar_accfull + 8 * buf);
+            }
+            tc_commit(bar_drain);
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait(bar_drain, 0)) {
+                if (globaltimer() - t0 > kWaitLimitNs) {
+                    *abort_flag = 1u;
+                    record_device_error(kErrTimeout);
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                         // TMEM lane quarter of this warp
+        const int ehalf = (warp - EPI_WARP0) >> 2;      // even or odd 16-column blocks
+        const int etid = threadIdx.x - 32 * EPI_WARP0;  // 0..255
+        const float inv_area = 1.f / (float)(P * P);
+        const float inv_cout = 1.f / (float)p.Cout;
+        float acc = 0.f;
+        int cur = -1;
+        auto flush = [&]() {
+            float s = acc;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if (lane == 0 && cur >= 0) atomicAdd(p.out + cur, s);
+            acc = 0.f;
+        };
+        int local = 0;
+        for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
+            const int buf = local & 1;
+            // One thread waits (bounded) before the barrier; the abort decision
+            // after it is the same for all four epilogue warps.
+            if (etid == 0 && !wait_bounded(bar_accfull + 8 * buf, (local >> 1) & 1, abort_flag)) *epi_abort = 1u;
+            asm volatile("bar.sync 2, 256;\n" ::: "memory");
+            if (*epi_abort) break;
+            for (int spin = 0; !mbar_try_wait(bar_accfull + 8 * buf, (local >> 1) & 1) && spin < (1 << 20); ++spin) {
+            }
+            tc_fence_after();
+            const TileCoord tcd = decode(p, tile);
+            {
+                const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * NP);
+                const int mrow = 32 * q + lane;
+                // Blocks ehalf, ehalf + 2, ... of 16 columns, two TMEM loads per wait.
+                for (int cb = ehalf; cb < NP / 16; cb += 4) {
+                    uint32_t v[16], u[16];
+                    const bool two = cb + 2 < NP / 16;
+                    tmem_ld16(taddr + (uint32_t)(16 * cb), v);
+                    if (two) tmem_ld16(taddr + (uint32_t)(16 * (cb + 2)), u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) tbuf[(16 * cb + j) * TP + mrow] = __uint_as_float(v[j]);
+                    if (two) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) tbuf[(16 * (cb + 2) + j) * TP + mrow] = __uint_as_float(u[j]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_accempty + 8 * buf);  // accumulator free for the MMA
+            }
+            asm volatile("bar.sync 2, 256;\n" ::: "memory");  // the whole accumulator is in tbuf
+            if (MODE != kTap && tcd.n != cur) {
+                flush();
+                cur = tcd.n;
+            }
+            const int nval = G::WPT * p.Cout;
+#pragma unroll 2
+            for (int v = etid; v < nval; v += NEPI) {
+                // j = v / Cout exactly: (v + 1/2) / Cout is at least 1/(2 Cout) away
+                // from an integer and v < 2^14, far inside fp32 precision.
+                const int j = (int)(((float)v + 0.5f) * inv_cout), co = v - j * p.Cout;
+                const int px = tcd.tx * G::WPT + j;
+                if (px >= p.PW) continue;
+                const float* tb = tbuf + co * TP + j * P;
+                float s = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < P; ++rr) {
+                    if constexpr (P % 4 == 0) {
+#pragma unroll
+                        for (int dc = 0; dc < P; dc += 4) {
+                            const float4 f = *reinterpret_cast<const float4*>(tb + rr * G::WC + dc);
+                            s += (f.x + f.y) + (f.z + f.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int dc = 0; dc < P; ++dc) s += tb[rr * G::WC + dc];
+                    }
+                }
+                const float pooled = s * inv_area + bias_s[co];
+                if (MODE == kTap) {
+                    p.out[(((size_t)tcd.n * p.Cout + co) * p.PH + tcd.py) * p.PW + px] = pooled;
+                } else {
+                    acc += __fdividef(1.f, 1.f + __expf(-pooled));  // sigmoid; 0 once exp overflows
+                }
+            }
+            // No barrier here: the next tile's first barrier also orders these
+            // reads of tbuf before its overwrite.
+        }
+        if (MODE != kTap) flush();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == MMA_WARP) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace c2tc
+
+inline bool conv2d_tc_pool_ok(int P) { return P == 1 || P == 2 || P == 4 || P == 8; }
+
+template <int P>
+inline uint32_t conv2d_tc_smem(int Cin, int Cout)
+{
+    const int NP = (Cout + 15) & ~15;
+    const int nchunks = (Cin + c2tc::CCH - 1) / c2tc::CCH;
+    const int natoms = (c2tc::KST * nchunks + 3) / 4;
+    return c2tc::make_layout<P>(NP, natoms).total + 1024u;
+}
+
+// Shapes the tensor-core conv2d covers: pool 1, 2, 4 or 8, Cout <= 112 and a
+// weight operand that fits shared memory next to the buffers.
+inline bool conv2d_tc_supported(int Cin, int Cout, int P)
+{
+    if (!conv2d_tc_pool_ok(P) || Cout < 1 || Cout > c2tc::NP_MAX || Cin < 1) return false;
+    uint32_t s = 0;
+    switch (P) {
+    case 1: s = conv2d_tc_smem<1>(Cin, Cout); break;
+    case 2: s = conv2d_tc_smem<2>(Cin, Cout); break;
+    case 4: s = conv2d_tc_smem<4>(Cin, Cout); break;
+    default: s = conv2d_tc_smem<8>(Cin, Cout); break;
+    }
+    return s <= (uint32_t)c2tc::SMEM_LIMIT;
+}
+
+template <int P, int MODE>
+inline int launch_conv2d_tc_p(c2tc::Params prm, int N, int grid, cudaStream_t stream)
+{
+    // x [N][Cin][H][W] as a 4-D tensor; one box is the halo of one (tile,
+    // chunk): HP columns x (P + 2) rows x 8 channels x 1 image.  Needs 16-byte
+    // row strides (W % 4 == 0) and an aligned x; otherwise cp.async stages it.
+    CUtensorMap map;
+    memset(&map, 0, sizeof(map));
+    prm.use_tma = 0;
+    if ((prm.W & 3) == 0 && (reinterpret_cast<uintptr_t>(prm.x) & 15) == 0) {
+        auto encode = tensor_map_encoder();
+        if (!encode) return FCV_ERR_CUDA;
+        using G = c2tc::Geo<P>;
+        const cuuint64_t gdim[4] = {(cuuint64_t)prm.W, (cuuint64_t)prm.H, (cuuint64_t)prm.Cin, (cuuint64_t)N};
+        const cuuint64_t gstride[3] = {(cuuint64_t)prm.W * 4, (cuuint64_t)prm.H * prm.W * 4,
+                                       (cuuint64_t)prm.Cin * prm.H * prm.W * 4};
+        const cuuint32_t box[4] = {(cuuint32_t)G::HP, (cuuint32_t)G::HR, (cuuint32_t)c2tc::CCH, 1};
+        const cuuint32_t estride[4] = {1, 1, 1, 1};
+        if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(prm.x), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return FCV_ERR_CUDA;
+        prm.use_tma = 1;
+    }
+    // At least 120 KB, so that two CTAs never share an SM: each allocates all
+    // 512 TMEM columns.
+    uint32_t smem = conv2d_tc_smem<P>(prm.Cin, prm.Cout);
+    if (smem < 120u * 1024u) smem = 120u * 1024u;
+    auto kern = c2tc::conv2d_tc_kernel<P, MODE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return FCV_ERR_CUDA;
+    kern<<<grid, c2tc::NTHREADS, smem, stream>>>(prm, map);
+    return launch_status();
+}
+
+// MODE: kSumAtomic (out[N], zeroed by the caller) or kTap (pooled values).
+template <int MODE>
+inline int launch_conv2d_tc(const float* x, const float* w, const float* b, int N, int Cin, int H, int W, int Cout,
+                            int P, int PH, int PW, float* out, cudaStream_t stream)
+{
+    if (!conv2d_tc_supported(Cin, Cout, P)) return FCV_ERR_UNSUPPORTED;
+    c2tc::Params prm;
+    prm.x = x; prm.w = w; prm.b = b; prm.out = out;
+    prm.Cin = Cin; prm.H = H; prm.W = W; prm.Cout = Cout; prm.PH = PH; prm.PW = PW;
+    prm.NP = (Cout + 15) & ~15;
+    prm.nchunks = (Cin + c2tc::CCH - 1) / c2tc::CCH;
+    prm.natoms = (c2tc::KST * prm.nchunks + 3) / 4;
+    const int wpt = c2tc::MT / (P * P);
+    prm.tiles_x = (PW + wpt - 1) / wpt;
+    const long long per_img = (long long)PH * prm.tiles_x;
+    const long long total = per_img * N;
+    if (total > 0x7fffffffLL) return FCV_ERR_UNSUPPORTED;
+    prm.tiles_img = (int)per_img;
+    prm.total_tiles = (int)total;
+    prm.use_tma = 0;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
+    const int grid = (int)(total < sms ? total : sms);
+    switch (P) {
+    case 1: return launch_conv2d_tc_p<1, MODE>(prm, N, grid, stream);
+    case 2: return launch_conv2d_tc_p<2, MODE>(prm, N, grid, stream);
+    case 4: return launch_conv2d_tc_p<4, MODE>(prm, N, grid, stream);
+    default: return launch_conv2d_tc_p<8, MODE>(prm, N, grid, stream);
+    }
+}
+
+}  // namespace fcv

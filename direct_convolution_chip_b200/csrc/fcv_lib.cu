@@ -12,6 +12,7 @@
 #include "conv1d_tcx.cuh"
 #include "conv2d_direct.cuh"
 #include "conv2d_poolfirst.cuh"
+#include "conv2d_tc.cuh"
 
 #define FCV_VERSION_MAJOR 0
 #define FCV_VERSION_MINOR 1
@@ -75,8 +76,10 @@ int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin
 {
     int st = check_conv2d(x, w, b, N, Cin, H, W, Cout, pool, out, tap);
     if (st != FCV_OK) return st;
-    if (algo != FCV_ALGO_AUTO && algo != FCV_CONV2D_DIRECT && algo != FCV_CONV2D_POOLFIRST)
+    if (algo != FCV_ALGO_AUTO && algo != FCV_CONV2D_DIRECT && algo != FCV_CONV2D_POOLFIRST &&
+        algo != FCV_CONV2D_TC_3XTF32)
         return FCV_ERR_INVALID_ARG;
+    if (algo == FCV_CONV2D_TC_3XTF32 && !fcv::conv2d_tc_supported(Cin, Cout, pool)) return FCV_ERR_UNSUPPORTED;
     if (N == 0) return FCV_OK;
     cudaStream_t s = fcv::as_stream(stream);
     const int PH = (H - 2) / pool, PW = (W - 2) / pool;
@@ -85,6 +88,10 @@ int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin
         if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N, s) != cudaSuccess) return FCV_ERR_CUDA;
     }
     if (PH == 0 || PW == 0) return FCV_OK;  // empty sum: out stays 0; the tap has no elements
+    if (algo == FCV_CONV2D_TC_3XTF32) {
+        return tap ? fcv::launch_conv2d_tc<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
+                   : fcv::launch_conv2d_tc<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
+    }
     if (algo == FCV_CONV2D_POOLFIRST) {
         return tap ? fcv::launch_conv2d_poolfirst<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
                    : fcv::launch_conv2d_poolfirst<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);

@@ -68,6 +68,10 @@ typedef enum {
                                      value instead of 9*Cin*P*P), FP32 FMA; same results within
                                      rounding.  Never chosen by FCV_ALGO_AUTO, which keeps the
                                      direct method. */
+    FCV_CONV2D_TC_3XTF32 = 12,    /* the direct method as an implicit GEMM on tcgen05 tensor
+                                     cores (K = 9*Cin, N = Cout), fp32-accurate through a
+                                     3xTF32 split; pool 1, 2, 4 or 8 and Cout <= 112 only,
+                                     UNSUPPORTED otherwise */
     /* op B */
     FCV_CONV1D_FMA = 20,          /* depthwise + pointwise on FP32 FMA */
     FCV_CONV1D_TC_3XTF32 = 21,    /* pointwise on tcgen05 tensor cores, 3xTF32 split, one SM per tile */

@@ -65,7 +65,7 @@ def c1d(lib, x=FAKE, dw=FAKE, pw=FAKE, bias=FAKE, N=2, C=8, T=64, O=16, K=9, s=1
     dict(N=-1), dict(Cin=0), dict(Cout=0), dict(H=2), dict(W=2), dict(pool=0),
     dict(x=MISALIGNED), dict(out=MISALIGNED),
     dict(N=1 << 30, Cin=1 << 30, H=1 << 20, W=1 << 20),  # element count overflows int64
-    dict(algo=999), dict(algo=21), dict(algo=12),
+    dict(algo=999), dict(algo=21), dict(algo=13),
 ])
 def test_conv2d_invalid(lib, kw):
     assert c2d(lib, **kw) == INVALID

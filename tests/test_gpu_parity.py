@@ -17,7 +17,7 @@ from tests.parity import assert_close, requires_cuda, sample_indices
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
 
-CONV2D_ALGOS = [fcv.CONV2D_DIRECT, fcv.CONV2D_POOLFIRST]
+CONV2D_ALGOS = [fcv.CONV2D_DIRECT, fcv.CONV2D_POOLFIRST, fcv.CONV2D_TC_3XTF32]
 CONV1D_ALGOS = [fcv.CONV1D_FMA, fcv.CONV1D_TC_3XTF32, fcv.CONV1D_TC2_3XTF32, fcv.CONV1D_TC_TMA_3XTF32]
 
 
@@ -43,11 +43,20 @@ def conv1d_or_skip(x, dw, pw, bias, s, p, algo):
 
 # ------------------------------------------------------------------ op A ---
 
+def conv2d_or_skip(fn, x, w, b, pool, algo):
+    try:
+        return fn(x, w, b, pool, algo=algo)
+    except fcv.FcvError as e:
+        if e.status == 2 and algo == fcv.CONV2D_TC_3XTF32:
+            pytest.skip("tensor-core conv2d does not cover this shape")
+        raise
+
+
 def check_conv2d_case(case, algo, batch_items=None, n_samples=2000, x_mean=0.0, w_scale=1.0):
     x, w, b = wl.conv2d_inputs(case, x_mean=x_mean, w_scale=w_scale)
     xd, wd, bd = cuda(x, w, b)
-    out = fcv.conv2d_pool_sigmoid_sum(xd, wd, bd, case.P, algo=algo)
-    tap = fcv.conv2d_pool_tap(xd, wd, bd, case.P, algo=algo)
+    out = conv2d_or_skip(fcv.conv2d_pool_sigmoid_sum, xd, wd, bd, case.P, algo)
+    tap = conv2d_or_skip(fcv.conv2d_pool_tap, xd, wd, bd, case.P, algo)
     torch.cuda.synchronize()
     xn, wn, bn = x.numpy(), w.numpy(), b.numpy()
     items = range(case.N) if batch_items is None else batch_items
