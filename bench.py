@@ -37,6 +37,9 @@ UNIT = "GFLOP/s"
 SPEC_FMA_LANES_PER_SM = 128       # FP32 FMA units per SM
 SPEC_SM_MAX_MHZ = 1965.0          # clocks.max.sm
 TF32_OVER_BF16 = 1.1 / 2.25       # nominal dense TF32 : BF16 tensor throughput
+ALGO_NAMES = {10: "conv2d_direct_fma", 11: "conv2d_poolfirst_fma", 12: "conv2d_tc_3xtf32",
+              20: "dwsep_conv1d_fma", 21: "dwsep_conv1d_tc_register_halo", 22: "dwsep_conv1d_tc_2sm",
+              23: "dwsep_conv1d_tc_tma_halo"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 CASE_A = wl.CONV2D_FULL
@@ -370,31 +373,46 @@ def run_gpu(args):
     tf32_peak = peaks["bf16_tflops"] * TF32_OVER_BF16
     ta_s, tb_s = ta_ms / K / 1e3, tb_ms / K / 1e3
 
-    conv1d_tc = os.environ.get("FCV_BENCH_CONV1D_PATH", "auto")
+    # The algorithms AUTO runs here (the library reports its own choice).
+    algo_a = fcv.conv2d_auto_algo(CASE_A.N, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout, CASE_A.P)
+    algo_b = fcv.dwsep_conv1d_auto_algo(xb_d, dwb_d, pwb_d, CASE_B.stride, CASE_B.pad)
+    tc_a = algo_a == fcv.CONV2D_TC_3XTF32
+    tc_b = algo_b in (fcv.CONV1D_TC_3XTF32, fcv.CONV1D_TC_TMA_3XTF32, fcv.CONV1D_TC2_3XTF32)
+    pw_macs_b = macs_conv1d_pointwise(CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K, CASE_B.stride, CASE_B.pad)
     per_op = {
-        "conv2d": {"workload": CASE_A.name, "ms": ta_s * 1e3, "gflops": 2 * macs_a / ta_s / 1e9,
-                   "macs": macs_a, "compulsory_bytes": bytes_a,
-                   "roofline_frac_fp32_fma": roofline_time_s(macs_a, bytes_a, fma_peak, hbm) / ta_s},
-        "dwsep_conv1d": {"workload": CASE_B.name, "ms": tb_s * 1e3, "gflops": 2 * macs_b / tb_s / 1e9,
-                         "macs": macs_b, "compulsory_bytes": bytes_b,
+        "conv2d": {"workload": CASE_A.name, "algo": ALGO_NAMES.get(algo_a, algo_a), "ms": ta_s * 1e3,
+                   "gflops": 2 * macs_a / ta_s / 1e9, "macs": macs_a, "compulsory_bytes": bytes_a,
+                   "roofline_frac_fp32_fma": roofline_time_s(macs_a, bytes_a, fma_peak, hbm) / ta_s,
+                   "roofline_frac_3xtf32": roofline_time_s(macs_a, bytes_a, tf32_peak / 3.0, hbm) / ta_s},
+        "dwsep_conv1d": {"workload": CASE_B.name, "algo": ALGO_NAMES.get(algo_b, algo_b), "ms": tb_s * 1e3,
+                         "gflops": 2 * macs_b / tb_s / 1e9, "macs": macs_b, "compulsory_bytes": bytes_b,
                          "roofline_frac_fp32_fma": roofline_time_s(macs_b, bytes_b, fma_peak, hbm) / tb_s,
-                         "roofline_frac_3xtf32": roofline_time_s(
-                             macs_conv1d_pointwise(CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K,
-                                                   CASE_B.stride, CASE_B.pad),
-                             bytes_b, tf32_peak / 3.0, hbm) / tb_s},
+                         "roofline_frac_3xtf32": roofline_time_s(pw_macs_b, bytes_b, tf32_peak / 3.0, hbm) / tb_s},
     }
+    fma_src = "148 SMs x 128 FP32 FMA lanes x 2 FLOP x 1965 MHz (spec clocks)"
+    tc_src = ("measured bf16 GEMM x nominal TF32/BF16 (1.1/2.25), / 3 for the three TF32 products of the "
+              "3xTF32 split; FLOPs are the fp32 method's (2 per MAC)")
     dom = "conv2d" if ta_s >= tb_s else "dwsep_conv1d"
     if dom == "conv2d":
         achieved = 2 * macs_a / ta_s / 1e12
-        roof = {"kernel": "conv2d_direct_kernel<4,false>", "bound": "alu", "achieved": achieved,
-                "peak": fma_peak, "unit": "TFLOP/s", "frac": achieved / fma_peak,
-                "traffic": traffic_per_launch("conv2d_direct_p4"),
-                "peak_source": "148 SMs x 128 FP32 FMA lanes x 2 FLOP x 1965 MHz (spec clocks)"}
+        if tc_a:
+            roof = {"kernel": "c2tc::conv2d_tc_kernel<4, sum>", "bound": "tensor", "achieved": achieved,
+                    "peak": tf32_peak / 3.0, "unit": "TFLOP/s", "frac": achieved / (tf32_peak / 3.0),
+                    "traffic": traffic_per_launch("conv2d_tc_p4"), "peak_source": tc_src}
+        else:
+            roof = {"kernel": "conv2d_direct_kernel<4, sum>", "bound": "alu", "achieved": achieved,
+                    "peak": fma_peak, "unit": "TFLOP/s", "frac": achieved / fma_peak,
+                    "traffic": traffic_per_launch("conv2d_direct_p4"), "peak_source": fma_src}
     else:
-        achieved = 2 * macs_b / tb_s / 1e12
-        roof = {"kernel": "dwsep_conv1d", "bound": "alu", "achieved": achieved, "peak": fma_peak,
-                "unit": "TFLOP/s", "frac": achieved / fma_peak, "traffic": traffic_per_launch("dwsep_conv1d"),
-                "peak_source": "148 SMs x 128 FP32 FMA lanes x 2 FLOP x 1965 MHz (spec clocks)"}
+        if tc_b:
+            achieved = 2 * pw_macs_b / tb_s / 1e12
+            roof = {"kernel": "dwsep_conv1d (tensor-core)", "bound": "tensor", "achieved": achieved,
+                    "peak": tf32_peak / 3.0, "unit": "TFLOP/s", "frac": achieved / (tf32_peak / 3.0),
+                    "traffic": traffic_per_launch("dwsep_conv1d"), "peak_source": tc_src}
+        else:
+            achieved = 2 * macs_b / tb_s / 1e12
+            roof = {"kernel": "dwsep_conv1d_fma_kernel", "bound": "alu", "achieved": achieved, "peak": fma_peak,
+                    "unit": "TFLOP/s", "frac": achieved / fma_peak, "traffic": None, "peak_source": fma_src}
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -402,7 +420,8 @@ def run_gpu(args):
         "dtype": "f32", "data": "synthetic",
         "config": {"workload": workload_name(), "l2": "inputs larger than L2 (x 604 MB and 134 MB, out 268 MB); "
                    "no flush", "parallelism": f"replicas x{world} (independent batches, no collective)",
-                   "conv1d_path": conv1d_tc},
+                   "algos": {"conv2d": ALGO_NAMES.get(algo_a, algo_a),
+                             "dwsep_conv1d": ALGO_NAMES.get(algo_b, algo_b)}},
         "per_op": per_op, "roofline": roof,
         "peaks": {"hbm_gbs": hbm, "fp32_fma_tflops": fma_peak, "tf32_tflops": tf32_peak, "source": peak_src},
         "e2e": {"value": job_throughput(2.0 * (macs_a + macs_b), world, e2e_ms / 1e3), "unit": UNIT,
@@ -429,15 +448,15 @@ def run_gpu(args):
                     raise fcv.FcvError(st, f"conv1d algorithm {algo}")
             return fn
 
-        def alt_a_tc():
+        def alt_a_fma():
             st = lib.fcv_conv2d_pool_sigmoid_sum_ex(P(xa_d.data_ptr()), P(wa_d.data_ptr()), P(ba_d.data_ptr()),
                                                     CASE_A.N, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout, CASE_A.P,
-                                                    P(out_a.data_ptr()), fcv.CONV2D_TC_3XTF32, P(sp))
+                                                    P(out_a.data_ptr()), fcv.CONV2D_DIRECT, P(sp))
             if st:
-                raise fcv.FcvError(st, "tensor-core conv2d")
+                raise fcv.FcvError(st, "FMA direct conv2d")
 
         ta2 = _event_ms(alt_a, 10, stream)
-        ta3 = _event_ms(alt_a_tc, 10, stream)
+        ta3 = _event_ms(alt_a_fma, 10, stream)
         tb = {name: _event_ms(alt_b(algo), 10, stream)
               for name, algo in (("dwsep_conv1d_fma", fcv.CONV1D_FMA),
                                  ("dwsep_conv1d_tc_register_halo", fcv.CONV1D_TC_3XTF32),
@@ -449,8 +468,8 @@ def run_gpu(args):
                                  "executed_gflops": 2.0 * pf_macs / (ta2 / 1e3) / 1e9,
                                  "speedup_vs_direct": ta_s * 1e3 / ta2,
                                  "note": "pools the input first (exact identity): 9*Cin MACs per pooled value"},
-            "conv2d_tc_3xtf32": {"ms": ta3, "gflops": 2.0 * macs_a / (ta3 / 1e3) / 1e9,
-                                 "frac_of_3xtf32_peak": 2.0 * macs_a / (ta3 / 1e3) / 1e12 / (tf32_peak / 3.0)},
+            "conv2d_direct_fma": {"ms": ta3, "gflops": 2.0 * macs_a / (ta3 / 1e3) / 1e9,
+                                  "frac_of_fp32_fma_peak": 2.0 * macs_a / (ta3 / 1e3) / 1e12 / fma_peak},
         }
         for name, ms in tb.items():
             result["variants"][name] = {"ms": ms, "gflops": 2.0 * macs_b / (ms / 1e3) / 1e9}

@@ -44,6 +44,8 @@ SIGNATURES = {
     "fcv_conv2d_pool_sigmoid_sum_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "fcv_dwsep_conv1d": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "fcv_dwsep_conv1d_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
+    "fcv_conv2d_auto_algo": (_I, [_I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
+    "fcv_dwsep_conv1d_auto_algo": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
     "fcv_status_string": (ctypes.c_char_p, [_I]),
     "fcv_version": (_I, []),
     "fcv_device_error": (_I, [_P]),
@@ -234,6 +236,24 @@ def dwsep_conv1d(x, dw, pw, bias, stride, pad, out=None, algo=ALGO_AUTO, stream=
     _check(lib.fcv_dwsep_conv1d_ex(_ptr(xd), _ptr(dwd), _ptr(pwd), _ptr(bd), N, C, T, O, K, stride, pad,
                                    _ptr(out), algo, _stream_ptr(stream)), "fcv_dwsep_conv1d")
     return _result(out, host, stream)
+
+
+def conv2d_auto_algo(N, Cin, H, W, Cout, pool) -> int:
+    """The algorithm FCV_ALGO_AUTO runs for these op A sizes (no GPU needed)."""
+    a = ctypes.c_int()
+    _check(load().fcv_conv2d_auto_algo(N, Cin, H, W, Cout, pool, ctypes.byref(a)), "fcv_conv2d_auto_algo")
+    return a.value
+
+
+def dwsep_conv1d_auto_algo(x, dw, pw, stride, pad) -> int:
+    """The algorithm FCV_ALGO_AUTO runs for these op B tensors (only their shapes
+    and the 16-byte alignment of x and pw matter; no data is read)."""
+    N, C, T = x.shape
+    O, K = pw.shape[0], dw.shape[-1]
+    a = ctypes.c_int()
+    _check(load().fcv_dwsep_conv1d_auto_algo(_ptr(x), _ptr(pw), N, C, T, O, K, stride, pad, ctypes.byref(a)),
+           "fcv_dwsep_conv1d_auto_algo")
+    return a.value
 
 
 def device_error(stream=None) -> int:

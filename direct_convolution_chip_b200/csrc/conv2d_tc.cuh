@@ -14,23 +14,31 @@
 // only on the tensor cores; the P x P pooling is a sum over accumulator rows
 // done in the epilogue.
 //
-// B200 design (one CTA per SM, persistent over tiles, 9 warps):
-//   * warps 0-3 (producers, one per TMEM lane quarter): stage the input halo
-//     of the next (tile, chunk) with cp.async while building the current one:
-//     each thread owns one conv position (= one TMEM lane), reads its 72
-//     im2col values from the halo, splits them into TF32 hi/lo and writes them
-//     straight into tensor memory with tcgen05.st (the A operand of the MMA is
-//     read from TMEM, so A costs no shared-memory bandwidth).
-//   * warp 4: allocates TMEM (two accumulators of Cout' columns, two A stages
-//     of 144 columns); one thread issues 27 tcgen05.mma (kind::tf32, M = 128,
-//     N = Cout', K = 8, A from TMEM, B from shared memory) per chunk:
-//     A_hi*B_hi + A_hi*B_lo + A_lo*B_hi.
+// B200 design (one CTA per SM, persistent over tiles, 19 warps):
+//   * warp 17 (TMA): one 4-D box per (tile, chunk) brings the input halo
+//     [8 channels][P + 2 rows][128/P + 2 columns] into one of two shared
+//     buffers (cp.async by the producers instead when rows are not 16-byte
+//     aligned).
+//   * warps 0-7 (producers, two per TMEM lane quarter): each thread owns one
+//     conv position (= one TMEM lane) and half of its 72 im2col values: reads
+//     them from the halo, splits them into TF32 hi/lo and writes them straight
+//     into tensor memory with tcgen05.st (the A operand of the MMA is read from
+//     TMEM, so A costs no shared-memory bandwidth).  Before a tile's first chunk
+//     they also see its accumulator drained, so the MMA issuers wait on one
+//     barrier per chunk.
+//   * warps 8 and 18 (MMA issuers, even and odd tiles): one thread each issues
+//     27 tcgen05.mma (kind::tf32, M = 128, N = Cout', K = 8, A from TMEM, B
+//     from shared memory) per chunk: A_hi*B_hi + A_hi*B_lo + A_lo*B_hi, from
+//     descriptors computed once.  Each owns one of the two A stages; while one
+//     waits on a barrier the other keeps the tensor core busy.
+//   * TMEM: 2 or 3 accumulators of Cout' columns, two A stages of 144.
 //   * The weights, split into TF32 hi/lo once per CTA, stay in shared memory
 //     in the K-major 128-byte-swizzled layout for the whole kernel.
-//   * warps 5-8 (epilogue): drain an accumulator with tcgen05.ld into a
-//     transposed shared buffer, release it to the MMA, then each thread sums
-//     the P x P conv outputs of its (window, channel) values, adds the bias,
-//     applies the sigmoid and accumulates; one atomic add per warp and image.
+//   * warps 9-16 (epilogue, two per lane quarter): drain an accumulator with
+//     tcgen05.ld into a transposed shared buffer, release it, then each thread
+//     sums the P x P conv outputs of its (window, channel) values, adds the
+//     bias, applies the sigmoid and accumulates; one atomic add per warp and
+//     image.
 //   * Every wait is bounded, as in the conv1d kernels.
 #pragma once
 
@@ -68,7 +76,9 @@ constexpr int NPROD = 256;        // producer threads: warps 0-7, two per TMEM l
 constexpr int MMA_WARP = 8;
 constexpr int EPI_WARP0 = 9;      // epilogue: warps 9-16, two per TMEM lane quarter
 constexpr int NEPI = 256;
-constexpr int NTHREADS = 17 * 32;
+constexpr int TMA_WARP = 17;
+constexpr int MMA_WARP2 = 18;     // second MMA issuer (odd tiles)
+constexpr int NTHREADS = 19 * 32;
 constexpr int TP = 132;           // pitch of the transposed accumulator buffer (floats)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_LIMIT = 227 * 1024;
@@ -94,11 +104,12 @@ struct Params {
     int Cin, H, W, Cout, PH, PW;
     int NP;           // Cout rounded up to 16 (MMA N)
     int nchunks;      // ceil(Cin / 8)
-    int natoms;       // 128-byte-wide K blocks of the weight operand
+    int natoms;       // 128-byte-wide K blocks of the weight operand (3 per chunk)
     int tiles_x;      // tiles per pooled row
     int tiles_img;    // tiles per image
     int total_tiles;
     int use_tma;      // halo by one 4-D TMA box (W % 4 == 0, aligned x), else by cp.async
+    int nacc;         // accumulator buffers in TMEM: 3 when 3 * NP + 2 * A_COLS <= 512, else 2
 };
 
 // Shared-memory layout (bytes, from a 1024-aligned base).
@@ -117,7 +128,7 @@ __host__ __device__ inline Layout make_layout(int NP, int natoms)
     L.tbuf = L.halo + 2u * Geo<P>::HALO * 4u;
     L.bias = L.tbuf + (uint32_t)NP * TP * 4u;
     L.bar = (L.bias + (uint32_t)NP * 4u + 7u) & ~7u;
-    L.misc = L.bar + 11u * 8u;
+    L.misc = L.bar + 16u * 8u;
     L.total = L.misc + 16u;
     return L;
 }
@@ -131,6 +142,14 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         " tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// The same, always accumulating.
+__device__ __forceinline__ void mma_tf32_ts_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc)
+{
+    asm volatile("tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, 1;\n" ::"r"(d_tmem), "r"(a_tmem),
+                 "l"(bdesc), "r"(idesc)
+                 : "memory");
 }
 
 // 8 consecutive 32-bit TMEM columns of the warp's 32 lanes (one register each).
@@ -178,12 +197,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
     float* halo = reinterpret_cast<float*>(smem + L.halo);
     float* tbuf = reinterpret_cast<float*>(smem + L.tbuf);
     float* bias_s = reinterpret_cast<float*>(smem + L.bias);
-    const uint32_t bar_afull = sbase + L.bar;         // + 8 * stage, 4 producer-warp arrivals
+    const uint32_t bar_afull = sbase + L.bar;         // + 8 * stage, 8 producer-warp arrivals
     const uint32_t bar_aempty = bar_afull + 16;       // + 8 * stage, tcgen05.commit
-    const uint32_t bar_accfull = bar_afull + 32;      // + 8 * buf, tcgen05.commit
-    const uint32_t bar_accempty = bar_afull + 48;     // + 8 * buf, 4 epilogue-warp arrivals
-    const uint32_t bar_drain = bar_afull + 64;
-    const uint32_t bar_hfull = bar_afull + 72;        // + 8 * buf, TMA halo landed
+    const uint32_t bar_accfull = bar_afull + 32;      // + 8 * buf (up to 3), tcgen05.commit
+    const uint32_t bar_accempty = bar_afull + 56;     // + 8 * buf (up to 3), 8 epilogue-warp arrivals
+    const uint32_t bar_drain = bar_afull + 80;
+    const uint32_t bar_hfull = bar_afull + 88;        // + 8 * buf, TMA halo landed
+    const uint32_t bar_hempty = bar_afull + 104;      // + 8 * buf, 8 producer-warp arrivals
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.misc);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 4);
     volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 8);
@@ -196,12 +216,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_afull + 8 * i, 8);
             mbar_init(bar_aempty + 8 * i, 1);
+        }
+        for (int i = 0; i < 3; ++i) {
             mbar_init(bar_accfull + 8 * i, 1);
             mbar_init(bar_accempty + 8 * i, 8);
         }
-        mbar_init(bar_drain, 1);
+        mbar_init(bar_drain, 2);  // one commit per MMA issuer
         mbar_init(bar_hfull, 1);
         mbar_init(bar_hfull + 8, 1);
+        mbar_init(bar_hempty, 8);
+        mbar_init(bar_hempty + 8, 8);
         *abort_flag = 0u;
         *prod_abort = 0u;
         *epi_abort = 0u;
@@ -215,8 +239,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
     }
 
     // Weights as the B operand, split into TF32 hi/lo: element (co, k) with
-    // k = 72 * chunk + 9 * (ci mod 8) + 3 * ky + kx sits in 128-byte K block
-    // k / 32 (blocks of NP rows), row co, swizzled 16-byte chunk (k mod 32) / 4.
+    // k = 72 * chunk + e, e = 9 * (ci mod 8) + 3 * ky + kx, sits in 128-byte K
+    // block 3 * chunk + e / 32 (blocks of NP rows), row co, swizzled 16-byte
+    // chunk (e mod 32) / 4.  Every chunk starts a K block, so the descriptors of
+    // chunk c are those of chunk 0 moved by c * 3 blocks.
     const int ktot = KCH * p.nchunks;
     for (int idx = threadIdx.x; idx < NP * ktot; idx += NTHREADS) {
         const int co = idx / ktot, k = idx - co * ktot;
@@ -224,7 +250,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
         const int ci = ch * CCH + e / 9, t = e % 9;
         const float v = (co < p.Cout && ci < p.Cin) ? __ldg(p.w + ((size_t)co * p.Cin + ci) * 9 + t) : 0.f;
         const float hi = tf32_round(v);
-        const int a = k >> 5, kin = k & 31;
+        const int a = 3 * ch + (e >> 5), kin = e & 31;
         const uint32_t off = (uint32_t)a * NP * 128u + sw128_off(co, kin >> 2) + (uint32_t)(kin & 3) * 4u;
         *reinterpret_cast<float*>(smem + L.b_hi + off) = hi;
         *reinterpret_cast<float*>(smem + L.b_lo + off) = v - hi;
@@ -235,7 +261,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const uint32_t a_col0 = 2u * (uint32_t)NP;  // first A-stage column
+    // Accumulators: p.nacc buffers of NP columns (3 when they fit next to the two
+    // A stages, else 2), used round robin: buffer abuf, phase aphase.
+    const uint32_t a_col0 = (uint32_t)(p.nacc * NP);  // first A-stage column
 
     if (warp < 8) {
         // ------------------------------------------------------------ producers
@@ -244,22 +272,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
         const int half = warp >> 2;                // K groups 0-4 or 5-8 of the chunk
         const int r = m / G::WC, c = m - (m / G::WC) * G::WC;
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-        int pseq_tile = blockIdx.x, pseq_ch = 0;  // the (tile, chunk) whose halo is being fetched
+        int pseq_tile = blockIdx.x, pseq_ch = 0;  // cp.async path: the (tile, chunk) being fetched
 
-        bool hpending[2] = {false, false};
+        // Halo of (tile, chunk) into buffer buf by cp.async, for rows that are
+        // not 16-byte aligned (the TMA warp loads it otherwise).
         auto fetch = [&](int tile, int ch, int buf) {
             const TileCoord tcd = decode(p, tile);
             const int y0 = tcd.py * P, x0 = tcd.tx * G::WC, c0 = ch * CCH;
-            if (p.use_tma) {
-                // One box [8 channels][P + 2 rows][HP columns] lands with the
-                // halo layout itself; rows, columns and channels outside x read 0.
-                if (tid == 0) {
-                    tc::mbar_arrive_expect_tx(bar_hfull + 8 * buf, (uint32_t)G::HALO * 4u);
-                    tma_load_4d(smem_u32(halo + buf * G::HALO), &x_map, x0, y0, c0, tcd.n, bar_hfull + 8 * buf);
-                }
-                hpending[buf] = true;
-                return;
-            }
             float* dst = halo + buf * G::HALO;
             const float* src = p.x + ((size_t)tcd.n * p.Cin) * p.H * p.W;
             for (int i = tid; i < CCH * G::HR * G::HW; i += NPROD) {
@@ -274,61 +293,75 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
             cp_async_commit();
         };
 
-        if (pseq_tile < p.total_tiles) fetch(pseq_tile, 0, 0);
-        int seq = 0, tile = blockIdx.x, ch = 0;
+        if (!p.use_tma && pseq_tile < p.total_tiles) fetch(pseq_tile, 0, 0);
+        int seq = 0, tile = blockIdx.x, ch = 0, abuf = 0, t = 0;
+        uint32_t aphase = 0;
         for (; tile < p.total_tiles; ++seq) {
-            const int stage = seq & 1;
-            // The MMAs that read this A stage two chunks ago have completed.  One
-            // thread waits (bounded) before the barrier, so the abort decision
-            // read after it is the same for every producer.
-            if (tid == 0 && !wait_bounded(bar_aempty + 8 * stage, ((seq >> 1) & 1) ^ 1, abort_flag)) *prod_abort = 1u;
+            // A stage = tile parity (each MMA issuer owns one stage); its use
+            // number u counts the chunks written into it so far.  Halo buffers
+            // alternate per chunk.
+            const int stage = t & 1;
+            const uint32_t upar = (uint32_t)(((t >> 1) * p.nchunks + ch) & 1);
+            const int hbuf = seq & 1;
+            const uint32_t par = (seq >> 1) & 1;
+            // The MMAs that read this A stage last have completed, the halo has
+            // landed and, for a tile's first chunk, the epilogue has drained the
+            // accumulator this tile will use: the MMA issuers then wait on
+            // "A full" alone.  One thread waits (bounded) before the barrier, so
+            // the abort decision after it is the same for all.
+            if (tid == 0 && !wait_bounded(bar_aempty + 8 * stage, upar ^ 1, abort_flag)) *prod_abort = 1u;
+            if (tid == 0 && ch == 0 && !wait_bounded(bar_accempty + 8 * abuf, aphase ^ 1, abort_flag))
+                *prod_abort = 1u;
             if (p.use_tma) {
-                if (tid == 0 && !wait_bounded(bar_hfull + 8 * stage, (seq >> 1) & 1, abort_flag)) *prod_abort = 1u;
+                if (tid == 0 && !wait_bounded(bar_hfull + 8 * hbuf, par, abort_flag)) *prod_abort = 1u;
             } else {
                 cp_async_wait<0>();
             }
             asm volatile("bar.sync 1, 256;\n" ::: "memory");  // halo landed, stage free
             if (*prod_abort) break;
             if (p.use_tma) {
-                hpending[stage] = false;
-                for (int spin = 0; !mbar_try_wait(bar_hfull + 8 * stage, (seq >> 1) & 1) && spin < (1 << 20); ++spin) {
+                for (int spin = 0; !mbar_try_wait(bar_hfull + 8 * hbuf, par) && spin < (1 << 20); ++spin) {
                 }
             }
-            for (int spin = 0; !mbar_try_wait(bar_aempty + 8 * stage, ((seq >> 1) & 1) ^ 1) && spin < (1 << 20);
-                 ++spin) {
-            }
+            // tcgen05.fence::after_thread_sync behind the barrier orders this
+            // thread's TMEM writes after the MMAs thread 0 saw complete.
             tc_fence_after();
-            // Fetch the next (tile, chunk) halo into the other buffer.
-            if (++pseq_ch == p.nchunks) {
-                pseq_ch = 0;
-                pseq_tile += gridDim.x;
+            if (!p.use_tma) {
+                // Fetch the next (tile, chunk) halo into the other buffer.
+                if (++pseq_ch == p.nchunks) {
+                    pseq_ch = 0;
+                    pseq_tile += gridDim.x;
+                }
+                if (pseq_tile < p.total_tiles) fetch(pseq_tile, pseq_ch, hbuf ^ 1);
             }
-            if (pseq_tile < p.total_tiles) fetch(pseq_tile, pseq_ch, stage ^ 1);
 
             // im2col row of position (r, c): 72 values, 8 per TMEM store; the two
-            // warps of a lane quarter take K groups 0-4 and 5-8.
-            const float* hb = halo + stage * G::HALO + r * G::HP + c;
+            // warps of a lane quarter take K groups 0-4 and 5-8.  A_hi is the raw
+            // fp32 value (the MMA reads only its TF32 bits, i.e. truncates it);
+            // A_lo = v - truncate(v) is exact.
+            const float* hb = halo + hbuf * G::HALO + r * G::HP + c;
             const uint32_t a_hi = tmem + lane_base + a_col0 + (uint32_t)(stage * A_COLS);
             auto build = [&](auto g0c, auto g1c) {
                 constexpr int g0 = decltype(g0c)::value, g1 = decltype(g1c)::value;
 #pragma unroll
-            for (int g = g0; g < g1; ++g) {
-                uint32_t hi[8], lo[8];
+                for (int g = g0; g < g1; ++g) {
+                    uint32_t hi[8], lo[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int e = 8 * g + q;
-                    const int ci = e / 9, t = e % 9;
-                    const float v = hb[ci * G::CHS + (t / 3) * G::HP + (t % 3)];
-                    const float h = tf32_round(v);
-                    hi[q] = __float_as_uint(h);
-                    lo[q] = __float_as_uint(v - h);
+                    for (int q = 0; q < 8; ++q) {
+                        const int e = 8 * g + q;
+                        const int ci = e / 9, t = e % 9;
+                        const float v = hb[ci * G::CHS + (t / 3) * G::HP + (t % 3)];
+                        hi[q] = __float_as_uint(v);
+                        lo[q] = __float_as_uint(v - __uint_as_float(hi[q] & 0xFFFFE000u));
+                    }
+                    tmem_st8(a_hi + (uint32_t)(8 * g), hi);
+                    tmem_st8(a_hi + (uint32_t)(KCH + 8 * g), lo);
                 }
-                tmem_st8(a_hi + (uint32_t)(8 * g), hi);
-                tmem_st8(a_hi + (uint32_t)(KCH + 8 * g), lo);
-            }
             };
             if (half == 0) build(std::integral_constant<int, 0>{}, std::integral_constant<int, 5>{});
             else build(std::integral_constant<int, 5>{}, std::integral_constant<int, KST>{});
+            __syncwarp();
+            if (p.use_tma && lane == 0) mbar_arrive(bar_hempty + 8 * hbuf);  // this warp is done with the halo
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -336,49 +369,97 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
             if (++ch == p.nchunks) {
                 ch = 0;
                 tile += gridDim.x;
-            }
-        }
-        cp_async_wait<0>();  // no copy may land after the CTA has left
-        if (tid == 0) {
-            // After an abort a TMA box may still be in flight: wait for it (bounded).
-            for (int b = 0; b < 2; ++b) {
-                if (!hpending[b]) continue;
-                const int sq = ((seq & 1) == b) ? seq : seq + 1;  // the sequence number that box belongs to
-                const unsigned long long t0 = globaltimer();
-                while (!mbar_try_wait(bar_hfull + 8 * b, (sq >> 1) & 1)) {
-                    if (globaltimer() - t0 > kWaitLimitNs) break;
+                ++t;
+                if (++abuf == p.nacc) {
+                    abuf = 0;
+                    aphase ^= 1u;
                 }
             }
         }
-    } else if (warp == MMA_WARP) {
-        // ---------------------------------------------------------- MMA issuer
+        cp_async_wait<0>();  // no copy may land after the CTA has left
+    } else if (warp == TMA_WARP) {
+        // -------------------------------------------------------- TMA issuer
+        // One box [8 channels][P + 2 rows][HP columns] per (tile, chunk) lands
+        // in the halo layout itself; rows, columns and channels outside x read 0.
+        if (p.use_tma && lane == 0) {
+            int seq = 0;
+            bool pending[2] = {false, false};
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+                const TileCoord tcd = decode(p, tile);
+                for (int ch = 0; ch < p.nchunks; ++ch, ++seq) {
+                    const int b = seq & 1;
+                    if (!wait_bounded(bar_hempty + 8 * b, ((seq >> 1) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    pending[b] = false;  // the producers consumed its previous box
+                    tc::mbar_arrive_expect_tx(bar_hfull + 8 * b, (uint32_t)G::HALO * 4u);
+                    tma_load_4d(smem_u32(halo + b * G::HALO), &x_map, tcd.tx * G::WC, tcd.py * P, ch * CCH, tcd.n,
+                                bar_hfull + 8 * b);
+                    pending[b] = true;
+                }
+            }
+            if (!ok) {
+                // After an abort, wait (bounded) for boxes still in flight.
+                for (int b = 0; b < 2; ++b) {
+                    if (!pending[b]) continue;
+                    const int last = seq - 1 - ((seq - 1 - b) & 1);  // latest sequence number on buffer b
+                    const unsigned long long t0 = globaltimer();
+                    while (last >= 0 && !mbar_try_wait(bar_hfull + 8 * b, (last >> 1) & 1)) {
+                        if (globaltimer() - t0 > kWaitLimitNs) break;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP || warp == MMA_WARP2) {
+        // --------------------------------------------------------- MMA issuers
+        // Two issuing threads, one for the even and one for the odd tiles of this
+        // CTA: while one waits on a barrier the other keeps the tensor core fed.
+        // Each commit tracks the issuing thread's own MMAs, which is what every
+        // barrier here needs (a stage or accumulator is used by one tile).
         if (lane == 0) {
+            const int par = warp == MMA_WARP ? 0 : 1;
             const uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NP >> 3) << 17) |
                                    ((uint32_t)(MT >> 4) << 24);
-            int seq = 0, local = 0;
+            // B descriptors of chunk 0's nine K-steps, computed once: the issue
+            // loop then spends a few instructions per MMA, so the tensor core,
+            // not this thread, sets the pace.
+            uint64_t bh0[KST], bl0[KST];
+#pragma unroll
+            for (int kk = 0; kk < KST; ++kk) {
+                const uint32_t boff = (uint32_t)(kk >> 2) * NP * 128u + 32u * (uint32_t)(kk & 3);
+                bh0[kk] = sw128_desc(sbase + L.b_hi + boff);
+                bl0[kk] = sw128_desc(sbase + L.b_lo + boff);
+            }
+            const uint64_t chunk_step = (uint64_t)(3u * NP * 128u) >> 4;  // descriptor address units
+            int abuf = par % p.nacc;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++local) {
-                const int buf = local & 1;
-                if (!wait_bounded(bar_accempty + 8 * buf, ((local >> 1) & 1) ^ 1, abort_flag)) break;
-                tc_fence_after();
+            for (int t = par, tile = blockIdx.x + par * gridDim.x; ok && tile < p.total_tiles;
+                 t += 2, tile += 2 * gridDim.x) {
+                const int buf = abuf;  // drained: the producers saw it before "A full"
+                abuf = (abuf + 2) % p.nacc;
                 const uint32_t d_tmem = tmem + (uint32_t)(buf * NP);
+                int seq = t * p.nchunks;
+                const int stage = par;  // = t & 1
                 for (int ch = 0; ch < p.nchunks; ++ch, ++seq) {
-                    const int stage = seq & 1;
-                    if (!wait_bounded(bar_afull + 8 * stage, (seq >> 1) & 1, abort_flag)) {
+                    const uint32_t upar = (uint32_t)(((t >> 1) * p.nchunks + ch) & 1);
+                    if (!wait_bounded(bar_afull + 8 * stage, upar, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_hi = tmem + a_col0 + (uint32_t)(stage * A_COLS);
+                    const uint32_t ah = tmem + a_col0 + (uint32_t)(stage * A_COLS), al = ah + (uint32_t)KCH;
+                    const uint64_t cofs = chunk_step * (uint64_t)ch;
+                    mma_tf32_ts(d_tmem, ah, bh0[0] + cofs, idesc, ch > 0 ? 1u : 0u);
+                    mma_tf32_ts_acc(d_tmem, ah, bl0[0] + cofs, idesc);
+                    mma_tf32_ts_acc(d_tmem, al, bh0[0] + cofs, idesc);
 #pragma unroll
-                    for (int kk = 0; kk < KST; ++kk) {
-                        const int gk = ch * KST + kk;  // global K-step
-                        const uint32_t boff = (uint32_t)(gk >> 2) * NP * 128u + 32u * (uint32_t)(gk & 3);
-                        const uint64_t bh = sw128_desc(sbase + L.b_hi + boff), bl = sw128_desc(sbase + L.b_lo + boff);
-                        const uint32_t ah = a_hi + 8u * kk, al = a_hi + (uint32_t)KCH + 8u * kk;
-                        mma_tf32_ts(d_tmem, ah, bh, idesc, (ch > 0 || kk > 0) ? 1u : 0u);
-                        mma_tf32_ts(d_tmem, ah, bl, idesc, 1u);
-                        mma_tf32_ts(d_tmem, al, bh, idesc, 1u);
+                    for (int kk = 1; kk < KST; ++kk) {
+                        mma_tf32_ts_acc(d_tmem, ah + 8u * kk, bh0[kk] + cofs, idesc);
+                        mma_tf32_ts_acc(d_tmem, ah + 8u * kk, bl0[kk] + cofs, idesc);
+                        mma_tf32_ts_acc(d_tmem, al + 8u * kk, bh0[kk] + cofs, idesc);
                     }
                     tc_commit(bar_aempty + 8 * stage);  // A stage free once these MMAs are done
                 }
@@ -411,17 +492,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
             if (lane == 0 && cur >= 0) atomicAdd(p.out + cur, s);
             acc = 0.f;
         };
-        int local = 0;
+        int abuf = 0, local = 0;
+        uint32_t aphase = 0;
         for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
-            const int buf = local & 1;
+            const int buf = abuf;
+            const uint32_t bphase = aphase;
+            if (++abuf == p.nacc) {
+                abuf = 0;
+                aphase ^= 1u;
+            }
             // One thread waits (bounded) before the barrier; the abort decision
             // after it is the same for all four epilogue warps.
-            if (etid == 0 && !wait_bounded(bar_accfull + 8 * buf, (local >> 1) & 1, abort_flag)) *epi_abort = 1u;
+            if (etid == 0 && !wait_bounded(bar_accfull + 8 * buf, bphase, abort_flag)) *epi_abort = 1u;
             asm volatile("bar.sync 2, 256;\n" ::: "memory");
             if (*epi_abort) break;
-            for (int spin = 0; !mbar_try_wait(bar_accfull + 8 * buf, (local >> 1) & 1) && spin < (1 << 20); ++spin) {
-            }
-            tc_fence_after();
+            tc_fence_after();  // behind the barrier: TMEM loads after the MMAs thread 0 saw complete
             const TileCoord tcd = decode(p, tile);
             {
                 const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * NP);
@@ -503,7 +588,7 @@ inline uint32_t conv2d_tc_smem(int Cin, int Cout)
 {
     const int NP = (Cout + 15) & ~15;
     const int nchunks = (Cin + c2tc::CCH - 1) / c2tc::CCH;
-    const int natoms = (c2tc::KST * nchunks + 3) / 4;
+    const int natoms = 3 * nchunks;
     return c2tc::make_layout<P>(NP, natoms).total + 1024u;
 }
 
@@ -568,7 +653,7 @@ inline int launch_conv2d_tc(const float* x, const float* w, const float* b, int 
     prm.Cin = Cin; prm.H = H; prm.W = W; prm.Cout = Cout; prm.PH = PH; prm.PW = PW;
     prm.NP = (Cout + 15) & ~15;
     prm.nchunks = (Cin + c2tc::CCH - 1) / c2tc::CCH;
-    prm.natoms = (c2tc::KST * prm.nchunks + 3) / 4;
+    prm.natoms = 3 * prm.nchunks;
     const int wpt = c2tc::MT / (P * P);
     prm.tiles_x = (PW + wpt - 1) / wpt;
     const long long per_img = (long long)PH * prm.tiles_x;
@@ -577,6 +662,7 @@ inline int launch_conv2d_tc(const float* x, const float* w, const float* b, int 
     prm.tiles_img = (int)per_img;
     prm.total_tiles = (int)total;
     prm.use_tma = 0;
+    prm.nacc = (3 * prm.NP + 2 * c2tc::A_COLS <= (int)c2tc::TMEM_COLS) ? 3 : 2;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;

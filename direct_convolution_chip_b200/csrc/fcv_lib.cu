@@ -96,6 +96,10 @@ int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin
         return tap ? fcv::launch_conv2d_poolfirst<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
                    : fcv::launch_conv2d_poolfirst<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
     }
+    if (algo == FCV_ALGO_AUTO && fcv::conv2d_tc_supported(Cin, Cout, pool)) {
+        return tap ? fcv::launch_conv2d_tc<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
+                   : fcv::launch_conv2d_tc<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
+    }
     return tap ? fcv::launch_conv2d_direct<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
                : fcv::launch_conv2d_direct<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
 }
@@ -197,6 +201,34 @@ int fcv_selftest_wait_timeout(unsigned long long limit_ns, void* stream)
     if (limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000) return FCV_ERR_INVALID_ARG;
     fcv::tc::selftest_wait_timeout_kernel<<<1, 32, 0, fcv::as_stream(stream)>>>(limit_ns);
     return fcv::launch_status();
+}
+
+int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* algo)
+{
+    if (!algo) return FCV_ERR_INVALID_ARG;
+    if (N < 0 || Cin < 1 || Cout < 1 || H < 3 || W < 3 || pool < 1) return FCV_ERR_INVALID_ARG;
+    if (!mul_ok(N, Cin, H, W) || !mul_ok(N, Cout, H, W)) return FCV_ERR_INVALID_ARG;
+    if (pool > 8) return FCV_ERR_UNSUPPORTED;
+    *algo = fcv::conv2d_tc_supported(Cin, Cout, pool) ? FCV_CONV2D_TC_3XTF32 : FCV_CONV2D_DIRECT;
+    return FCV_OK;
+}
+
+int fcv_dwsep_conv1d_auto_algo(const float* x, const float* pw_w, int N, int C, int T, int O, int K, int stride,
+                               int pad, int* algo)
+{
+    if (!algo) return FCV_ERR_INVALID_ARG;
+    int To = 0;
+    // Validation without reading any data: the pointers stand in for the
+    // tensors only through their alignment.
+    const float* dummy = reinterpret_cast<const float*>(16);
+    float* odummy = reinterpret_cast<float*>(16);
+    const int st = check_conv1d(N > 0 && !x ? dummy : x, dummy, N > 0 && !pw_w ? dummy : pw_w, nullptr, N, C, T, O,
+                                K, stride, pad, odummy, &To);
+    if (st != FCV_OK) return st;
+    if (fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w)) *algo = FCV_CONV1D_TC_TMA_3XTF32;
+    else if (fcv::conv1d_tc_supported(C, O, K, stride, pw_w)) *algo = FCV_CONV1D_TC_3XTF32;
+    else *algo = FCV_CONV1D_FMA;
+    return FCV_OK;
 }
 
 const char* fcv_status_string(int status)

@@ -57,9 +57,12 @@ typedef enum {
     FCV_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (see fcv_device_error) */
 } fcv_status;
 
-/* Algorithm selectors for the *_ex entry points.  For op B, FCV_ALGO_AUTO
- * picks the fastest path valid for the shape; for op A it is the direct
- * method. */
+/* Algorithm selectors for the *_ex entry points.  FCV_ALGO_AUTO picks the
+ * fastest path valid for the shape and pointers (fcv_conv2d_auto_algo and
+ * fcv_dwsep_conv1d_auto_algo report which).  For op A it is always the direct
+ * method (every conv output is computed): on tensor cores where
+ * FCV_CONV2D_TC_3XTF32 covers the shape, else on FP32 FMA; the pool-first
+ * identity is never chosen automatically. */
 typedef enum {
     FCV_ALGO_AUTO = 0,
     /* op A */
@@ -96,8 +99,9 @@ typedef enum {
  * INVALID_ARG: x, w, b or out NULL while N > 0; N < 0; Cin, Cout < 1; H, W < 3; pool < 1;
  *              element counts beyond 2^31 * 2^31; misaligned pointers.
  * UNSUPPORTED: pool > 8.
- * The per-batch sum is accumulated with one atomic add per thread block, so
- * the last bits may differ between runs. */
+ * The per-batch sum is accumulated with atomic adds (one per thread block on
+ * the FMA path, one per warp and image on the tensor-core path), so the last
+ * bits may differ between runs. */
 int fcv_conv2d_pool_sigmoid_sum(const float* x, const float* w, const float* b,
                                 int N, int Cin, int H, int W, int Cout, int pool,
                                 float* out, void* stream);
@@ -192,6 +196,16 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
                         float* out, int algo, void* stream);
 
 /* -------------------------------------------------------------- utility --- */
+
+/* The algorithm FCV_ALGO_AUTO runs for these sizes, written to *algo; no CUDA
+ * call is made.  Returns the status the compute call would return for invalid
+ * or unsupported sizes (INVALID_ARG also when algo is NULL). */
+int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* algo);
+
+/* The same for op B; x and pw_w matter only through their 16-byte alignment
+ * (they are not read). */
+int fcv_dwsep_conv1d_auto_algo(const float* x, const float* pw_w, int N, int C, int T, int O, int K,
+                               int stride, int pad, int* algo);
 
 /* Human-readable name of a status code (static storage). */
 const char* fcv_status_string(int status);

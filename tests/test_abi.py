@@ -138,3 +138,33 @@ def test_det_rejects_missing_or_small_workspace(lib):
 def test_selftest_rejects_bad_limits(lib):
     assert lib.fcv_selftest_wait_timeout(0, None) == INVALID
     assert lib.fcv_selftest_wait_timeout(11 * 10**9, None) == INVALID
+
+
+def test_auto_algo_conv2d(lib):
+    """AUTO runs the tensor-core direct conv where it covers the shape, else the FMA kernel."""
+    a = ctypes.c_int()
+    q = lib.fcv_conv2d_auto_algo
+    assert q(128, 8, 384, 384, 64, 4, ctypes.byref(a)) == OK and a.value == 12  # the full-size workload
+    for pool in (1, 2, 8):
+        assert q(2, 3, 40, 40, 16, pool, ctypes.byref(a)) == OK and a.value == 12
+    assert q(2, 3, 40, 40, 16, 3, ctypes.byref(a)) == OK and a.value == 10      # pool 3: FMA path
+    assert q(2, 3, 40, 40, 128, 4, ctypes.byref(a)) == OK and a.value == 10     # Cout > 112: FMA path
+    assert q(2, 3, 40, 40, 16, 9, ctypes.byref(a)) == UNSUPPORTED
+    assert q(2, 0, 40, 40, 16, 4, ctypes.byref(a)) == INVALID
+    assert q(2, 3, 40, 40, 16, 4, None) == INVALID
+
+
+def test_auto_algo_conv1d(lib):
+    """AUTO: TMA-halo tensor cores for aligned x/pw and T % 4 == 0, then the
+    register-halo tensor-core kernel, then FMA (stride > 1)."""
+    a = ctypes.c_int()
+    q = lib.fcv_dwsep_conv1d_auto_algo
+    X, PW = P(0x10000), P(0x20000)
+    assert q(X, PW, 32, 256, 4096, 512, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 23  # full-size workload
+    assert q(X, PW, 2, 64, 1001, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21    # T % 4 != 0
+    assert q(P(0x10004), PW, 2, 64, 1000, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21  # x not 16-B aligned
+    assert q(X, PW, 2, 64, 1000, 128, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 20    # stride 2
+    assert q(X, PW, 2, 62, 1000, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 20    # C % 4 != 0
+    assert q(X, PW, 2, 64, 1000, 128, 33, 1, 4, ctypes.byref(a)) == UNSUPPORTED           # K > 32
+    assert q(X, PW, 2, 64, 1000, 128, 9, 1, -1, ctypes.byref(a)) == INVALID
+    assert q(X, PW, 2, 64, 1000, 128, 9, 1, 4, None) == INVALID
