@@ -527,6 +527,32 @@ def unfused_baselines(xa, wa, ba, xb, dwb, pwb, bb, iters=5):
             "precision": "fp32, TF32 disabled", "note": "unfused: conv output / depthwise output in HBM"}
 
 
+def run_probes():
+    """Peak probes of libfcv_probes.so on this GPU: FP32 FMA (scalar and packed)
+    and the tcgen05 TF32 MMA rate by N, A source and accumulator chains."""
+    import ctypes
+    from direct_convolution_chip_b200 import build as fcv_build
+    torch.cuda.set_device(0)
+    lib = ctypes.CDLL(fcv_build.build_probes())
+    D = ctypes.c_double
+    for packed in (0, 1):
+        f, ms = D(), D()
+        st = lib.fcvprobe_fma_rate(packed, 2, 20000, ctypes.byref(f), ctypes.byref(ms))
+        print(json.dumps({"probe": "fp32_fma", "packed": packed, "status": st, "tflops": f.value / 1e12,
+                          "ms": ms.value}), flush=True)
+    for n in (64, 128, 256):
+        for a_tmem in (0, 1):
+            for chains in (1, 2, 4):
+                if chains * n > 448:
+                    continue
+                f, ms, cyc = D(), D(), D()
+                st = lib.fcvprobe_tf32_mma_rate(n, a_tmem, chains, 24000, ctypes.byref(f), ctypes.byref(ms),
+                                                ctypes.byref(cyc))
+                print(json.dumps({"probe": "tcgen05_tf32_mma", "n": n, "a_tmem": a_tmem, "chains": chains,
+                                  "status": st, "tflops": f.value / 1e12, "ms": ms.value,
+                                  "cycles_per_mma": cyc.value}), flush=True)
+
+
 def run_configs(args):
     """One JSON line per workload (named configs and the 48-point sweep): the
     metric per config, GFLOP/s and fraction of its roofline."""
@@ -631,10 +657,14 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle and unfused-baseline legs")
     ap.add_argument("--configs", action="store_true", help="time every named workload, one JSON line each")
     ap.add_argument("--sweep", action="store_true", help="with --configs: the 48-point shape sweep as well")
+    ap.add_argument("--probe", action="store_true",
+                    help="run the FP32-FMA and tcgen05 TF32 peak probes, one JSON line each")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.probe:
+        run_probes()
     elif args.configs:
         run_configs(args)
     else:
