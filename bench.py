@@ -574,25 +574,26 @@ def run_configs(args):
             out = torch.empty((c.N,), device="cuda")
             fn = lambda: lib.fcv_conv2d_pool_sigmoid_sum(P(x.data_ptr()), P(w.data_ptr()), P(b.data_ptr()), c.N,
                                                          c.Cin, c.H, c.W, c.Cout, c.P, P(out.data_ptr()), sp)
-            pipe, peak = "fp32_fma", fma_peak
+            algo = fcv.conv2d_auto_algo(c.N, c.Cin, c.H, c.W, c.Cout, c.P)
+            pipe, peak = ("3xtf32", tf32_peak / 3.0) if algo == fcv.CONV2D_TC_3XTF32 else ("fp32_fma", fma_peak)
         else:
             x, dw, pw, b = [t.cuda() for t in wl.conv1d_inputs(c)]
             To = (c.T + 2 * c.pad - c.K) // c.stride + 1
             out = torch.empty((c.N, c.O, To), device="cuda")
             fn = lambda: lib.fcv_dwsep_conv1d(P(x.data_ptr()), P(dw.data_ptr()), P(pw.data_ptr()), P(b.data_ptr()),
                                               c.N, c.C, c.T, c.O, c.K, c.stride, c.pad, P(out.data_ptr()), sp)
-            tc = lib.fcv_dwsep_conv1d_ex(P(x.data_ptr()), P(dw.data_ptr()), P(pw.data_ptr()), P(b.data_ptr()),
-                                         c.N, c.C, c.T, c.O, c.K, c.stride, c.pad, P(out.data_ptr()),
-                                         21, sp) == 0
+            algo = fcv.dwsep_conv1d_auto_algo(x, dw, pw, c.stride, c.pad)
+            tc = algo != fcv.CONV1D_FMA
             pipe, peak = ("3xtf32", tf32_peak / 3.0) if tc else ("fp32_fma", fma_peak)
         assert fn() == 0
         macs, nbytes = case_macs(c), case_bytes(c)
         iters = max(3, min(200, int(0.2 / max(2.0 * macs / (peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)))))
         ms = _event_ms(fn, iters, stream)
-        roof = roofline_time_s(macs if pipe == "fp32_fma" else
+        roof = roofline_time_s(macs if (pipe == "fp32_fma" or c.op == "conv2d") else
                                (macs_conv1d_pointwise(c.N, c.C, c.T, c.O, c.K, c.stride, c.pad)),
                                nbytes, peak, peaks["hbm_gbs"])
-        print(json.dumps({"config": c.name, "op": c.op, "ms": ms, "gflops": 2.0 * macs / (ms / 1e3) / 1e9,
+        print(json.dumps({"config": c.name, "op": c.op, "algo": ALGO_NAMES.get(algo, algo), "ms": ms,
+                          "gflops": 2.0 * macs / (ms / 1e3) / 1e9,
                           "macs": macs, "bytes": nbytes, "pipe": pipe, "roofline_ms": roof * 1e3,
                           "roofline_frac": roof / (ms / 1e3), "l2": "inputs resident; no flush"}), flush=True)
         del x, out

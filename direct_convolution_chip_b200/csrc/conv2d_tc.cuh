@@ -14,8 +14,8 @@
 // only on the tensor cores; the P x P pooling is a sum over accumulator rows
 // done in the epilogue.
 //
-// B200 design (one CTA per SM, persistent over tiles, 19 warps):
-//   * warp 17 (TMA): one 4-D box per (tile, chunk) brings the input halo
+// B200 design (one CTA per SM, persistent over tiles, 23 warps):
+//   * warp 21 (TMA): one 4-D box per (tile, chunk) brings the input halo
 //     [8 channels][P + 2 rows][128/P + 2 columns] into one of two shared
 //     buffers (cp.async by the producers instead when rows are not 16-byte
 //     aligned).
@@ -26,7 +26,7 @@
 //     TMEM, so A costs no shared-memory bandwidth).  Before a tile's first chunk
 //     they also see its accumulator drained, so the MMA issuers wait on one
 //     barrier per chunk.
-//   * warps 8 and 18 (MMA issuers, even and odd tiles): one thread each issues
+//   * warps 8 and 22 (MMA issuers, even and odd tiles): one thread each issues
 //     27 tcgen05.mma (kind::tf32, M = 128, N = Cout', K = 8, A from TMEM, B
 //     from shared memory) per chunk: A_hi*B_hi + A_hi*B_lo + A_lo*B_hi, from
 //     descriptors computed once.  Each owns one of the two A stages; while one
@@ -34,11 +34,13 @@
 //   * TMEM: 2 or 3 accumulators of Cout' columns, two A stages of 144.
 //   * The weights, split into TF32 hi/lo once per CTA, stay in shared memory
 //     in the K-major 128-byte-swizzled layout for the whole kernel.
-//   * warps 9-16 (epilogue, two per lane quarter): drain an accumulator with
-//     tcgen05.ld into a transposed shared buffer, release it, then each thread
-//     sums the P x P conv outputs of its (window, channel) values, adds the
-//     bias, applies the sigmoid and accumulates; one atomic add per warp and
-//     image.
+//   * warps 9-12 (drain, one per lane quarter): copy a finished accumulator
+//     with tcgen05.ld into one of two transposed shared buffers and release
+//     it at once.
+//   * warps 13-20 (pool): each thread sums the P x P conv outputs of its
+//     (window, channel) values, adds the bias, applies the sigmoid and
+//     accumulates; one atomic add per warp and image.  Pooling of one tile
+//     overlaps the drain of the next.
 //   * Every wait is bounded, as in the conv1d kernels.
 #pragma once
 
@@ -74,11 +76,12 @@ constexpr int A_COLS = 2 * KCH;   // one A stage in TMEM: hi (72 columns) | lo (
 constexpr int NP_MAX = 112;       // padded Cout: 2 * NP + 2 * A_COLS <= 512 TMEM columns
 constexpr int NPROD = 256;        // producer threads: warps 0-7, two per TMEM lane quarter
 constexpr int MMA_WARP = 8;
-constexpr int EPI_WARP0 = 9;      // epilogue: warps 9-16, two per TMEM lane quarter
-constexpr int NEPI = 256;
-constexpr int TMA_WARP = 17;
-constexpr int MMA_WARP2 = 18;     // second MMA issuer (odd tiles)
-constexpr int NTHREADS = 19 * 32;
+constexpr int DRAIN_WARP0 = 9;    // epilogue drain: warps 9-12, one per TMEM lane quarter
+constexpr int POOL_WARP0 = 13;    // epilogue pooling: warps 13-20
+constexpr int NPOOL = 256;
+constexpr int TMA_WARP = 21;
+constexpr int MMA_WARP2 = 22;     // second MMA issuer (odd tiles)
+constexpr int NTHREADS = 23 * 32;
 constexpr int TP = 132;           // pitch of the transposed accumulator buffer (floats)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_LIMIT = 227 * 1024;
@@ -126,9 +129,9 @@ __host__ __device__ inline Layout make_layout(int NP, int natoms)
     L.b_lo = atoms_bytes;
     L.halo = 2 * atoms_bytes;
     L.tbuf = L.halo + 2u * Geo<P>::HALO * 4u;
-    L.bias = L.tbuf + (uint32_t)NP * TP * 4u;
+    L.bias = L.tbuf + 2u * (uint32_t)NP * TP * 4u;  // two transposed accumulator buffers
     L.bar = (L.bias + (uint32_t)NP * 4u + 7u) & ~7u;
-    L.misc = L.bar + 16u * 8u;
+    L.misc = L.bar + 20u * 8u;
     L.total = L.misc + 16u;
     return L;
 }
@@ -200,14 +203,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
     const uint32_t bar_afull = sbase + L.bar;         // + 8 * stage, 8 producer-warp arrivals
     const uint32_t bar_aempty = bar_afull + 16;       // + 8 * stage, tcgen05.commit
     const uint32_t bar_accfull = bar_afull + 32;      // + 8 * buf (up to 3), tcgen05.commit
-    const uint32_t bar_accempty = bar_afull + 56;     // + 8 * buf (up to 3), 8 epilogue-warp arrivals
+    const uint32_t bar_accempty = bar_afull + 56;     // + 8 * buf (up to 3), 4 drain-warp arrivals
     const uint32_t bar_drain = bar_afull + 80;
     const uint32_t bar_hfull = bar_afull + 88;        // + 8 * buf, TMA halo landed
     const uint32_t bar_hempty = bar_afull + 104;      // + 8 * buf, 8 producer-warp arrivals
+    const uint32_t bar_tfull = bar_afull + 120;       // + 8 * buf, 4 drain-warp arrivals
+    const uint32_t bar_tempty = bar_afull + 136;      // + 8 * buf, 8 pool-warp arrivals
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.misc);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 4);
     volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 8);
-    volatile uint32_t* epi_abort = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 12);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NP = p.NP;
@@ -219,16 +223,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
         }
         for (int i = 0; i < 3; ++i) {
             mbar_init(bar_accfull + 8 * i, 1);
-            mbar_init(bar_accempty + 8 * i, 8);
+            mbar_init(bar_accempty + 8 * i, 4);
         }
         mbar_init(bar_drain, 2);  // one commit per MMA issuer
         mbar_init(bar_hfull, 1);
         mbar_init(bar_hfull + 8, 1);
         mbar_init(bar_hempty, 8);
         mbar_init(bar_hempty + 8, 8);
+        mbar_init(bar_tfull, 4);
+        mbar_init(bar_tfull + 8, 4);
+        mbar_init(bar_tempty, 8);
+        mbar_init(bar_tempty + 8, 8);
         *abort_flag = 0u;
         *prod_abort = 0u;
-        *epi_abort = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     if (warp == MMA_WARP) {
@@ -478,96 +485,118 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;                         // TMEM lane quarter of this warp
-        const int ehalf = (warp - EPI_WARP0) >> 2;      // even or odd 16-column blocks
-        const int etid = threadIdx.x - 32 * EPI_WARP0;  // 0..255
-        const float inv_area = 1.f / (float)(P * P);
-        const float inv_cout = 1.f / (float)p.Cout;
-        float acc = 0.f;
-        int cur = -1;
-        auto flush = [&]() {
-            float s = acc;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            if (lane == 0 && cur >= 0) atomicAdd(p.out + cur, s);
-            acc = 0.f;
-        };
+        // Drain warps (one per TMEM lane quarter) copy a finished accumulator
+        // into one of two transposed buffers and release it at once; pool warps
+        // then reduce that buffer.  Pooling of one tile overlaps the drain of
+        // the next, so the epilogue's rate is the slower of the two halves.
         int abuf = 0, local = 0;
         uint32_t aphase = 0;
-        for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
-            const int buf = abuf;
-            const uint32_t bphase = aphase;
-            if (++abuf == p.nacc) {
-                abuf = 0;
-                aphase ^= 1u;
-            }
-            // One thread waits (bounded) before the barrier; the abort decision
-            // after it is the same for all four epilogue warps.
-            if (etid == 0 && !wait_bounded(bar_accfull + 8 * buf, bphase, abort_flag)) *epi_abort = 1u;
-            asm volatile("bar.sync 2, 256;\n" ::: "memory");
-            if (*epi_abort) break;
-            tc_fence_after();  // behind the barrier: TMEM loads after the MMAs thread 0 saw complete
-            const TileCoord tcd = decode(p, tile);
-            {
+        if (warp >= DRAIN_WARP0 && warp < DRAIN_WARP0 + 4) {
+            const int q = warp & 3;  // TMEM lane quarter of this warp
+            const int mrow = 32 * q + lane;
+            for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
+                const int buf = abuf;
+                const uint32_t bphase = aphase;
+                if (++abuf == p.nacc) {
+                    abuf = 0;
+                    aphase ^= 1u;
+                }
+                const int tb = local & 1;
+                const uint32_t tphase = (local >> 1) & 1;
+                int ok = 1;
+                if (lane == 0) {
+                    ok = wait_bounded(bar_accfull + 8 * buf, bphase, abort_flag) &&
+                         wait_bounded(bar_tempty + 8 * tb, tphase ^ 1, abort_flag);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                tc_fence_after();  // TMEM loads after the MMAs lane 0 saw complete
+                float* tbw = tbuf + tb * NP * TP;
                 const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * NP);
-                const int mrow = 32 * q + lane;
-                // Blocks ehalf, ehalf + 2, ... of 16 columns, two TMEM loads per wait.
-                for (int cb = ehalf; cb < NP / 16; cb += 4) {
+                for (int cb = 0; cb < NP / 16; cb += 2) {  // two TMEM loads per wait
                     uint32_t v[16], u[16];
-                    const bool two = cb + 2 < NP / 16;
+                    const bool two = cb + 1 < NP / 16;
                     tmem_ld16(taddr + (uint32_t)(16 * cb), v);
-                    if (two) tmem_ld16(taddr + (uint32_t)(16 * (cb + 2)), u);
+                    if (two) tmem_ld16(taddr + (uint32_t)(16 * (cb + 1)), u);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) tbuf[(16 * cb + j) * TP + mrow] = __uint_as_float(v[j]);
+                    for (int j = 0; j < 16; ++j) tbw[(16 * cb + j) * TP + mrow] = __uint_as_float(v[j]);
                     if (two) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) tbuf[(16 * (cb + 2) + j) * TP + mrow] = __uint_as_float(u[j]);
+                        for (int j = 0; j < 16; ++j) tbw[(16 * (cb + 1) + j) * TP + mrow] = __uint_as_float(u[j]);
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_accempty + 8 * buf);  // accumulator free for the MMA
+                if (lane == 0) {
+                    mbar_arrive(bar_accempty + 8 * buf);  // accumulator free for the MMA
+                    mbar_arrive(bar_tfull + 8 * tb);      // this quarter of the buffer is written
+                }
             }
-            asm volatile("bar.sync 2, 256;\n" ::: "memory");  // the whole accumulator is in tbuf
-            if (MODE != kTap && tcd.n != cur) {
-                flush();
-                cur = tcd.n;
-            }
-            const int nval = G::WPT * p.Cout;
+        } else {
+            const int ptid = threadIdx.x - 32 * POOL_WARP0;  // 0..255
+            const float inv_area = 1.f / (float)(P * P);
+            const float inv_cout = 1.f / (float)p.Cout;
+            float acc = 0.f;
+            int cur = -1;
+            auto flush = [&]() {
+                float s = acc;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (lane == 0 && cur >= 0) atomicAdd(p.out + cur, s);
+                acc = 0.f;
+            };
+            for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
+                const int tb = local & 1;
+                const uint32_t tphase = (local >> 1) & 1;
+                int ok = 1;
+                if (lane == 0) ok = wait_bounded(bar_tfull + 8 * tb, tphase, abort_flag) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                // every lane acquires the drain warps' stores (returns at once)
+                for (int spin = 0; !mbar_try_wait(bar_tfull + 8 * tb, tphase) && spin < (1 << 20); ++spin) {
+                }
+                const TileCoord tcd = decode(p, tile);
+                if (MODE != kTap && tcd.n != cur) {
+                    flush();
+                    cur = tcd.n;
+                }
+                const float* tbr = tbuf + tb * NP * TP;
+                const int nval = G::WPT * p.Cout;
 #pragma unroll 2
-            for (int v = etid; v < nval; v += NEPI) {
-                // j = v / Cout exactly: (v + 1/2) / Cout is at least 1/(2 Cout) away
-                // from an integer and v < 2^14, far inside fp32 precision.
-                const int j = (int)(((float)v + 0.5f) * inv_cout), co = v - j * p.Cout;
-                const int px = tcd.tx * G::WPT + j;
-                if (px >= p.PW) continue;
-                const float* tb = tbuf + co * TP + j * P;
-                float s = 0.f;
+                for (int v = ptid; v < nval; v += NPOOL) {
+                    // j = v / Cout exactly: (v + 1/2) / Cout is at least 1/(2 Cout) away
+                    // from an integer and v < 2^14, far inside fp32 precision.
+                    const int j = (int)(((float)v + 0.5f) * inv_cout), co = v - j * p.Cout;
+                    const int px = tcd.tx * G::WPT + j;
+                    if (px >= p.PW) continue;
+                    const float* tb4 = tbr + co * TP + j * P;
+                    float s = 0.f;
 #pragma unroll
-                for (int rr = 0; rr < P; ++rr) {
-                    if constexpr (P % 4 == 0) {
+                    for (int rr = 0; rr < P; ++rr) {
+                        if constexpr (P % 4 == 0) {
 #pragma unroll
-                        for (int dc = 0; dc < P; dc += 4) {
-                            const float4 f = *reinterpret_cast<const float4*>(tb + rr * G::WC + dc);
-                            s += (f.x + f.y) + (f.z + f.w);
+                            for (int dc = 0; dc < P; dc += 4) {
+                                const float4 f = *reinterpret_cast<const float4*>(tb4 + rr * G::WC + dc);
+                                s += (f.x + f.y) + (f.z + f.w);
+                            }
+                        } else {
+#pragma unroll
+                            for (int dc = 0; dc < P; ++dc) s += tb4[rr * G::WC + dc];
                         }
+                    }
+                    const float pooled = s * inv_area + bias_s[co];
+                    if (MODE == kTap) {
+                        p.out[(((size_t)tcd.n * p.Cout + co) * p.PH + tcd.py) * p.PW + px] = pooled;
                     } else {
-#pragma unroll
-                        for (int dc = 0; dc < P; ++dc) s += tb[rr * G::WC + dc];
+                        acc += __fdividef(1.f, 1.f + __expf(-pooled));  // sigmoid; 0 once exp overflows
                     }
                 }
-                const float pooled = s * inv_area + bias_s[co];
-                if (MODE == kTap) {
-                    p.out[(((size_t)tcd.n * p.Cout + co) * p.PH + tcd.py) * p.PW + px] = pooled;
-                } else {
-                    acc += __fdividef(1.f, 1.f + __expf(-pooled));  // sigmoid; 0 once exp overflows
-                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_tempty + 8 * tb);  // this warp is done with the buffer
             }
-            // No barrier here: the next tile's first barrier also orders these
-            // reads of tbuf before its overwrite.
+            if (MODE != kTap) flush();
         }
-        if (MODE != kTap) flush();
     }
 
     tc_fence_before();
