@@ -636,6 +636,15 @@ inline bool conv2d_tc_supported(int Cin, int Cout, int P)
     return s <= (uint32_t)c2tc::SMEM_LIMIT;
 }
 
+// What AUTO prefers: the tensor-core kernel wherever it applies, except for
+// very narrow layers (Cin < 4 and Cout <= 32), where the K chunk of 8 input
+// channels is mostly padding and the FMA kernel measured faster (e.g. 383 vs
+// 438 us for x[16,3,509,509], Cout 32, pool 4).
+inline bool conv2d_tc_preferred(int Cin, int Cout, int P)
+{
+    return conv2d_tc_supported(Cin, Cout, P) && !(Cin < 4 && Cout <= 32);
+}
+
 template <int P, int MODE>
 inline int launch_conv2d_tc_p(c2tc::Params prm, int N, int grid, cudaStream_t stream)
 {

@@ -96,7 +96,7 @@ int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin
         return tap ? fcv::launch_conv2d_poolfirst<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
                    : fcv::launch_conv2d_poolfirst<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
     }
-    if (algo == FCV_ALGO_AUTO && fcv::conv2d_tc_supported(Cin, Cout, pool)) {
+    if (algo == FCV_ALGO_AUTO && fcv::conv2d_tc_preferred(Cin, Cout, pool)) {
         return tap ? fcv::launch_conv2d_tc<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
                    : fcv::launch_conv2d_tc<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
     }
@@ -209,7 +209,7 @@ int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* 
     if (N < 0 || Cin < 1 || Cout < 1 || H < 3 || W < 3 || pool < 1) return FCV_ERR_INVALID_ARG;
     if (!mul_ok(N, Cin, H, W) || !mul_ok(N, Cout, H, W)) return FCV_ERR_INVALID_ARG;
     if (pool > 8) return FCV_ERR_UNSUPPORTED;
-    *algo = fcv::conv2d_tc_supported(Cin, Cout, pool) ? FCV_CONV2D_TC_3XTF32 : FCV_CONV2D_DIRECT;
+    *algo = fcv::conv2d_tc_preferred(Cin, Cout, pool) ? FCV_CONV2D_TC_3XTF32 : FCV_CONV2D_DIRECT;
     return FCV_OK;
 }
 
