@@ -104,6 +104,10 @@ EDGE_2D = [
     (1, 20, 35, 36, 6, 4),     # more than one input-channel chunk
     (1, 3, 509, 509, 1, 4),    # single output channel, large odd image
     (4, 1, 130, 3, 2, 1),      # one conv column
+    # tensor-core conv2d envelope
+    (2, 8, 50, 52, 112, 2),    # the widest Cout (two accumulators), TMA halo
+    (1, 24, 40, 44, 48, 4),    # three input-channel chunks, three accumulators
+    (3, 5, 66, 64, 20, 1),     # pool 1, Cout padded to 32
 ]
 
 
@@ -201,6 +205,11 @@ EDGE_1D = [
     (1, 16, 1000, 64, 1, 1, 0, True),   # pointwise only (K = 1)
     (3, 40, 129, 33, 7, 8, 3, False),   # the largest supported stride
     (1, 300, 70, 20, 4, 1, 1, True),    # C not a multiple of the channel chunk
+    # TMA-halo tensor-core kernel (T % 4 == 0): every halo offset r = (-pad) mod 4
+    (2, 32, 1000, 64, 5, 1, 2, True),   # r = 2
+    (2, 36, 512, 48, 7, 1, 3, True),    # r = 1, a partial second channel chunk
+    (1, 64, 256, 300, 13, 1, 5, False), # r = 3 with the largest tensor-core K, partial output tile
+    (1, 8, 4, 8, 3, 1, 1, True),        # T = 4: one partial time tile
 ]
 
 
