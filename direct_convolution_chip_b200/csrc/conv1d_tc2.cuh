@@ -1,27 +1,29 @@
 // conv1d_tc2.cuh -- op B on a pair of SMs: the 2-CTA (cta_group::2) form of
-// the tensor-core separable conv1d in conv1d_tc.cuh.
+// the tensor-core separable conv1d with the input halo staged by TMA.
 //
-// Same arithmetic as conv1d_tc.cuh (depthwise on FP32 FMA into the A operand,
-// pointwise as a 3xTF32 tcgen05 contraction, fp32 accumulation in TMEM; see
-// there for the split and its accuracy).  What changes is the tiling: two CTAs
-// of a cluster compute one 256-time x 256-output-channel tile with
+// Same arithmetic as conv1d_tcx.cuh (depthwise on FP32 FMA into the A operand,
+// pointwise as a 3xTF32 tcgen05 contraction with the pw hi part read raw,
+// fp32 accumulation in TMEM).  What changes is the tiling: the two CTAs of a
+// cluster compute one 256-time x 256-output-channel tile with
 // tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 8).  Each CTA holds its own
 // 128 rows of A (its times) and HALF of B (128 of the 256 pw rows), so per CTA
-// the pw split work and the B stage size are halved; the freed shared memory
-// holds a 3-deep ring of input halos filled by cp.async two chunks ahead.
+// the pw split work, the B stage and the MMA's shared-memory reads are halved,
+// and three 64 KB stages fit where the single-SM kernel has two of 96 KB: the
+// extra stage hides the TMA latency that bounds the single-SM pipeline.
 //
-// Roles per CTA (448 threads): warps 0-7 produce (halo copies, in-place pw
-// split, depthwise + A split); warp 8 allocates TMEM (both CTAs) and, in the
-// leader CTA only, one thread issues the MMAs for the pair; warps 9-12 drain
-// this CTA's accumulator rows; warp 13 loads this CTA's half of the pw chunk
-// by TMA.  The leader's "full" and "aempty" barriers collect arrivals from
-// both CTAs (remote mbarrier arrives); MMA completion is committed to both
-// CTAs' "empty"/"afull" barriers with a multicast commit.  Every mbarrier
-// wait is bounded; a cluster barrier follows initialisation and precedes exit,
-// so no CTA leaves while its peer may still signal it.  No TMA multicast.
+// Roles per CTA (448 threads): warps 0-7 produce (pw split of this CTA's half,
+// depthwise from the TMA-staged halo, A split); warp 8 allocates TMEM (both
+// CTAs) and, in the leader CTA only, one thread issues the MMAs for the pair;
+// warps 9-12 drain this CTA's accumulator rows; warp 13 loads, per chunk, this
+// CTA's half of the pw chunk and its input halo by TMA.  The leader's "full"
+// and "aempty" barriers collect arrivals from both CTAs (remote mbarrier
+// arrives); MMA completion is committed to both CTAs' "empty"/"afull" barriers
+// with a multicast commit.  Every mbarrier wait is bounded; a cluster barrier
+// follows initialisation and precedes exit, so no CTA leaves while its peer
+// may still signal it.  No TMA multicast.
 #pragma once
 
-#include "conv1d_tc.cuh"
+#include "conv1d_tcx.cuh"
 
 namespace fcv {
 namespace tc2 {
@@ -32,28 +34,26 @@ constexpr int TM = 128;          // times per CTA (pair: 256)
 constexpr int TN = 256;          // output channels per pair tile (UMMA N)
 constexpr int TNH = TN / 2;      // pw rows held by each CTA
 constexpr int KC = 32;
-constexpr int STAGES = 2;
-constexpr int XSTAGES = 3;       // input-halo ring depth
+constexpr int STAGES = 3;
 constexpr int NPROD = 256;
 constexpr int MMA_WARP = 8, TMA_WARP = 13;
 constexpr int NTHREADS = 14 * 32;
 constexpr int KMAXW = tc::KMAXW;
-constexpr int XWP = 144;         // halo row pitch (floats)
-constexpr int XS_FLOATS = KC * XWP + 28;
-constexpr int DW_MAX = tc::DW_MAX;
+constexpr int XW = 148;          // halo box width = smem row pitch (floats)
+constexpr uint32_t X_BYTES = (uint32_t)XW * KC * 4;
+constexpr int DWX_MAX = 8192;    // resident depthwise weights, [K][32*nk]
 constexpr uint32_t TMEM_COLS = 2 * TN;
 
 constexpr uint32_t A_BYTES = TM * KC * 4;    // 16 KB
 constexpr uint32_t B_BYTES = TNH * KC * 4;   // 16 KB
 constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
-constexpr uint32_t OFF_XS = STAGES * STAGE_BYTES;
-constexpr uint32_t XS_BYTES = ((uint32_t)XS_FLOATS * 4 + 127) & ~127u;
-constexpr uint32_t OFF_DWS = OFF_XS + XSTAGES * XS_BYTES;
-constexpr uint32_t OFF_BAR = (OFF_DWS + DW_MAX * 4 + 7) & ~7u;
-constexpr uint32_t NBAR = 11;    // full[2] empty[2] afull[2] aempty[2] drain tma[2]
-constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr uint32_t OFF_DWS = STAGES * STAGE_BYTES;
+constexpr uint32_t OFF_BAR = OFF_DWS + DWX_MAX * 4;
+constexpr uint32_t NBAR = 14;    // full[3] empty[3] afull[2] aempty[2] drain tma[3]
+constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(X_BYTES <= 2 * A_BYTES, "the halo box must fit the stage's A region");
 
 // D fp32, A/B tf32, K-major, N = 256, M = 256 (the pair).
 constexpr uint32_t kIdesc2 = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(TN >> 3) << 17) |
@@ -141,7 +141,6 @@ struct Params {
     int C, T, O, K, pad, To;
     int tiles_t, tiles_o, total_tiles;  // pair tiles (256 times each)
     int out_vec;                         // output rows 16-byte aligned
-    int x_vec;                           // 16-byte halo copies possible
 };
 
 __device__ __forceinline__ TileCoord decode_pair_tile(const Params& p, int tile)
@@ -154,21 +153,27 @@ __device__ __forceinline__ TileCoord decode_pair_tile(const Params& p, int tile)
     return tc;
 }
 
-template <int KT>
+// KT: depthwise kernel size when fixed at compile time (0: any K <= KMAXW).
+// R: (t0 - pad) mod 4, the offset of the first needed sample inside the box.
+template <int KT, int R>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
-dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_map)
+dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_map,
+                        const __grid_constant__ CUtensorMap x_map)
 {
     using namespace tc;
+    constexpr int KW = KT > 0 ? KT : KMAXW;            // taps the window must cover
+    constexpr int NV = (R + 15 + KW + 3) / 4;          // 16-byte window loads per thread
+    static_assert(16 * 7 + 4 * NV <= XW, "window inside the halo box");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
     float* dws = reinterpret_cast<float*>(smem + OFF_DWS);
     const uint32_t bar_full = sbase + OFF_BAR;   // + 8 * stage (leader's collects both CTAs)
-    const uint32_t bar_empty = bar_full + 16;    // + 8 * stage
-    const uint32_t bar_afull = bar_full + 32;    // + 8 * buf
-    const uint32_t bar_aempty = bar_full + 48;   // + 8 * buf (leader's collects both CTAs)
-    const uint32_t bar_drain = bar_full + 64;
-    const uint32_t bar_tma = bar_full + 72;      // + 8 * stage
+    const uint32_t bar_empty = bar_full + 24;    // + 8 * stage
+    const uint32_t bar_afull = bar_full + 48;    // + 8 * buf
+    const uint32_t bar_aempty = bar_full + 64;   // + 8 * buf (leader's collects both CTAs)
+    const uint32_t bar_drain = bar_full + 80;
+    const uint32_t bar_tma = bar_full + 88;      // + 8 * stage
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
     volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 8);
@@ -179,12 +184,14 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < STAGES; ++i) {
             mbar_init(bar_full + 8 * i, 16);   // 8 producer warps x 2 CTAs (used in the leader)
             mbar_init(bar_empty + 8 * i, 1);   // multicast commit
+            mbar_init(bar_tma + 8 * i, 1);     // expect_tx arrival + TMA bytes
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(bar_afull + 8 * i, 1);   // multicast commit
             mbar_init(bar_aempty + 8 * i, 8);  // 4 epilogue warps x 2 CTAs (used in the leader)
-            mbar_init(bar_tma + 8 * i, 1);     // expect_tx arrival + TMA bytes
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0u;
@@ -197,167 +204,109 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
     }
-    const int CP = (p.C + 3) & ~3;
-    for (int e = threadIdx.x; e < p.K * CP; e += NTHREADS) {
-        const int k = e / CP, c = e - (e / CP) * CP;
+    const int nk = (p.C + KC - 1) / KC;
+    // Depthwise weights resident as [K][CW], CW = 32 * nk, zero beyond C.
+    const int CW = KC * nk;
+    for (int e = threadIdx.x; e < p.K * CW; e += NTHREADS) {
+        const int k = e / CW, c = e - (e / CW) * CW;
         dws[e] = c < p.C ? __ldg(p.dw + (size_t)c * p.K + k) : 0.f;
     }
     tc_fence_before();
     cluster_sync();  // barriers of both CTAs initialised, TMEM allocated, weights staged
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const int nk = (p.C + KC - 1) / KC;
 
     if (warp < 8) {
         // ------------------------------------------------------------ producers
         const int ptid = threadIdx.x;
-        const int cg = lane & 7;
-        const int tq = (lane >> 3) + 4 * warp;
         const int K = KT > 0 ? KT : p.K;
         const uint32_t full_leader = mapa(bar_full, 0);
-
-        // Halo of chunk (tile, kc) into ring slot `slot`: channel rows of XWP
-        // samples from t0 - pad (this CTA's 128 times), skewed by 4 floats per
-        // group of 4 channels; zero outside [0, T) and past C.
-        auto stage_x = [&](int tile, int kc, int slot) {
-            const TileCoord tcd = decode_pair_tile(p, tile);
-            const int c0 = kc * KC;
-            const int tb = tcd.t0 + (int)rank * TM - p.pad;
-            float* xs = reinterpret_cast<float*>(smem + OFF_XS + slot * XS_BYTES);
-            const float* xn = p.x + (size_t)tcd.n * p.C * p.T;
-            if (p.x_vec) {
-                constexpr int CPR = XWP / 4;  // 16-byte copies per channel row
-                for (int i = ptid; i < KC * CPR; i += NPROD) {
-                    const int cl = i / CPR, q = i - (i / CPR) * CPR;
-                    const int c = c0 + cl, ti = tb + 4 * q;
-                    const int bytes = (c < p.C && ti >= 0) ? 4 * max(0, min(4, p.T - ti)) : 0;
-                    cp_async16(xs + cl * XWP + 4 * ((cl >> 2) & 7) + 4 * q,
-                               bytes ? xn + (size_t)c * p.T + ti : p.x, bytes);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool run = true;
+        for (int tile = pair; run && tile < p.total_tiles; tile += npairs) {
+            for (int kc = 0; kc < nk; ++kc) {
+                // The TMA copies of this stage (pw half and halo) have landed.
+                if (ptid == 0 && !wait_bounded(bar_tma + 8 * stage, phase, abort_flag)) *prod_abort = 1u;
+                asm volatile("bar.sync 1, 256;\n" ::: "memory");
+                if (*prod_abort) {
+                    run = false;
+                    break;
                 }
-            } else {
-                for (int i = ptid; i < KC * XWP; i += NPROD) {
-                    const int cl = i / XWP, j = i - (i / XWP) * XWP;
-                    const int c = c0 + cl, ti = tb + j;
-                    const bool in = c < p.C && ti >= 0 && ti < p.T;
-                    cp_async4(xs + cl * XWP + 4 * ((cl >> 2) & 7) + j, in ? xn + (size_t)c * p.T + ti : p.x, in);
+                for (int spin = 0; !mbar_try_wait(bar_tma + 8 * stage, phase) && spin < (1 << 20); ++spin) {
                 }
-            }
-        };
-        // Sequence position `ahead` chunks after (tile, kc), or tile = -1 past the end.
-        auto advance = [&](int& tile, int& kc) {
-            if (++kc == nk) {
-                kc = 0;
-                tile += npairs;
-            }
-            if (tile >= p.total_tiles) tile = -1;
-        };
+                const uint32_t a_hi = sbase + stage * STAGE_BYTES;
+                const uint32_t a_lo = a_hi + A_BYTES;
+                const uint32_t b_hi = a_lo + A_BYTES;
+                const uint32_t b_lo = b_hi + B_BYTES;
 
-        int seq = 0, tile = pair, kc = 0;
-        // Prefetch the halos of the first two chunks.
-        int ftile = tile, fkc = kc;
-        for (int a = 0; a < 2; ++a) {
-            if (ftile >= 0 && ftile < p.total_tiles) stage_x(ftile, fkc, a);
-            cp_async_commit();
-            if (ftile >= 0) advance(ftile, fkc);
-        }
-        while (tile < p.total_tiles) {
-            const int stage = seq & 1;
-            const uint32_t parity = (seq >> 1) & 1;
-            if (ptid == 0 && !wait_bounded(bar_tma + 8 * stage, parity, abort_flag)) *prod_abort = 1u;
-            asm volatile("bar.sync 1, 256;\n" ::: "memory");  // B1: also, every producer is done with slot (seq-1)%3
-            if (*prod_abort) break;
-            for (int spin = 0; !mbar_try_wait(bar_tma + 8 * stage, parity) && spin < (1 << 20); ++spin) {
-            }
-            // Halo of chunk seq+2 into the slot chunk seq-1 used.
-            if (ftile >= 0) stage_x(ftile, fkc, (seq + 2) % XSTAGES);
-            cp_async_commit();
-            if (ftile >= 0) advance(ftile, fkc);
+                // This CTA's half of the pw chunk: B_hi stays raw (the MMA reads
+                // its TF32 bits); B_lo = v - truncate(v).
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t off = sw128_off(warp * 16 + i * 4 + (lane >> 3), lane & 7);
+                    sts128(b_lo + off, tcx::tf32_trunc_rest4(lds128(b_hi + off)));
+                }
 
-            const uint32_t a_hi = sbase + stage * STAGE_BYTES;
-            const uint32_t a_lo = a_hi + A_BYTES;
-            const uint32_t b_hi = a_lo + A_BYTES;
-            const uint32_t b_lo = b_hi + B_BYTES;
-            const int c0 = kc * KC;
-            // This CTA's half of the pw chunk (128 rows), split in place into TF32 hi/lo.
+                // Depthwise: channel lane, this CTA's times 16*warp .. +15; halo
+                // sample j is x[t0 + 128*rank - pad - R + j].
+                const float* xrow = reinterpret_cast<const float*>(smem + stage * STAGE_BYTES) + lane * XW + 16 * warp;
+                float win[4 * NV];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int row = warp * 16 + i * 4 + (lane >> 3);
-                const uint32_t off = sw128_off(row, lane & 7);
-                float4 hi, lo;
-                split4(lds128(b_hi + off), hi, lo);
-                sts128(b_hi + off, hi);
-                sts128(b_lo + off, lo);
-            }
-            cp_async_wait<2>();                               // this thread's copies of chunk seq landed
-            asm volatile("bar.sync 1, 256;\n" ::: "memory");  // B2: everyone's copies landed
-
-            const float* xs = reinterpret_cast<const float*>(smem + OFF_XS + (seq % XSTAGES) * XS_BYTES);
-            float dv[4][4];
+                for (int q = 0; q < NV; ++q) {
+                    const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
+                    win[4 * q] = v.x;
+                    win[4 * q + 1] = v.y;
+                    win[4 * q + 2] = v.z;
+                    win[4 * q + 3] = v.w;
+                }
+                float2 d2[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
-            if (c0 + 4 * cg < p.C) {
+                for (int j = 0; j < 8; ++j) d2[j] = make_float2(0.f, 0.f);
+                const float* wcol = dws + KC * kc + lane;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    float win[2][16];
+                for (int k = 0; k < KW; ++k) {
+                    if (KT > 0 || k < K) {
+                        const float w = wcol[k * CW];
+                        const float2 w2 = make_float2(w, w);
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const int cl = 4 * cg + 2 * h + i;
-                        const float* xrow = xs + cl * XWP + 4 * ((cl >> 2) & 7) + 4 * tq;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
-                            win[i][4 * q] = v.x; win[i][4 * q + 1] = v.y; win[i][4 * q + 2] = v.z; win[i][4 * q + 3] = v.w;
-                        }
-                    }
-                    const float* wcol = dws + c0 + 4 * cg + 2 * h;
-                    auto tap = [&](int k) {
-                        const float2 wk = *reinterpret_cast<const float2*>(wcol + k * CP);
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            dv[2 * h][r] = fmaf(win[0][k + r], wk.x, dv[2 * h][r]);
-                            dv[2 * h + 1][r] = fmaf(win[1][k + r], wk.y, dv[2 * h + 1][r]);
-                        }
-                    };
-                    if constexpr (KT > 0) {
-#pragma unroll
-                        for (int k = 0; k < KT; ++k) tap(k);
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < KMAXW; ++k)
-                            if (k < K) tap(k);
+                        for (int j = 0; j < 8; ++j)
+                            d2[j] = __ffma2_rn(make_float2(win[R + 2 * j + k], win[R + 2 * j + k + 1]), w2, d2[j]);
                     }
                 }
-            }
+                // Every producer has read its halo window before the A operand overwrites it.
+                asm volatile("bar.sync 1, 256;\n" ::: "memory");
+                const uint32_t col = ((uint32_t)(lane & 3) << 2);
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int t = 4 * tq + r;
-                float4 hi, lo;
-                split4(make_float4(dv[0][r], dv[1][r], dv[2][r], dv[3][r]), hi, lo);
-                const uint32_t off = sw128_off(t, cg);
-                sts128(a_hi + off, hi);
-                sts128(a_lo + off, lo);
+                for (int i = 0; i < 16; ++i) {
+                    const float v = (i & 1) ? d2[i >> 1].y : d2[i >> 1].x;
+                    const float hi = tf32_round(v);
+                    const uint32_t off = sw128_off(16 * warp + i, lane >> 2) + col;
+                    tcx::sts32(a_hi + off, hi);
+                    tcx::sts32(a_lo + off, v - hi);
+                }
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(full_leader + 8 * stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
-            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(full_leader + 8 * stage);
-            ++seq;
-            advance(tile, kc);
-            if (tile < 0) break;
         }
-        cp_async_wait<0>();  // no copy may still be landing when the CTA exits
     } else if (warp == MMA_WARP) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0 && leader) {
-            int seq = 0, local = 0;
+            int local = 0, stage = 0;
+            uint32_t phase = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < p.total_tiles; tile += npairs, ++local) {
                 const int buf = local & 1;
                 if (!wait_bounded_cluster(bar_aempty + 8 * buf, ((local >> 1) & 1) ^ 1, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
-                for (int k = 0; k < nk; ++k, ++seq) {
-                    const int stage = seq & 1;
-                    if (!wait_bounded_cluster(bar_full + 8 * stage, (seq >> 1) & 1, abort_flag)) {
+                for (int k = 0; k < nk; ++k) {
+                    if (!wait_bounded_cluster(bar_full + 8 * stage, phase, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -376,6 +325,10 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                         mma2_tf32(d_tmem, dal, dbh, 1u);
                     }
                     commit2(bar_empty + 8 * stage);  // both CTAs' stage free once these MMAs read it
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
                 if (ok) commit2(bar_afull + 8 * buf);  // both CTAs' accumulator rows complete
             }
@@ -394,31 +347,43 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         __syncwarp();
     } else if (warp == TMA_WARP) {
         // -------------------------------------------------------- TMA issuer
+        // Per chunk: this CTA's half of the pw chunk into B_hi and its input
+        // halo [32 channels][148 times] into the A region, once the MMAs that
+        // last read the stage (in both CTAs) have completed.
         if (lane == 0) {
-            int seq = 0;
-            bool pending[2] = {false, false};
+            int stage = 0, issued = 0;
+            uint32_t phase = 0;
+            bool pending[STAGES] = {false, false, false};
             bool ok = true;
             for (int tile = pair; ok && tile < p.total_tiles; tile += npairs) {
                 const TileCoord tcd = decode_pair_tile(p, tile);
-                for (int k = 0; k < nk; ++k, ++seq) {
-                    const int stage = seq & 1;
-                    if (!wait_bounded_cluster(bar_empty + 8 * stage, ((seq >> 1) & 1) ^ 1, abort_flag)) {
+                const int x0 = tcd.t0 + (int)rank * TM - p.pad - R;  // a multiple of 4
+                for (int k = 0; k < nk; ++k) {
+                    if (!wait_bounded_cluster(bar_empty + 8 * stage, phase ^ 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                     pending[stage] = false;
-                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES);
-                    tma_load_2d(sbase + stage * STAGE_BYTES + 2 * A_BYTES, &pw_map, k * KC,
-                                tcd.o0 + (int)rank * TNH, bar_tma + 8 * stage);
+                    const uint32_t st = sbase + stage * STAGE_BYTES;
+                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES + X_BYTES);
+                    tma_load_2d(st + 2 * A_BYTES, &pw_map, k * KC, tcd.o0 + (int)rank * TNH, bar_tma + 8 * stage);
+                    tcx::tma_load_3d(st, &x_map, x0, k * KC, tcd.n, bar_tma + 8 * stage);
                     pending[stage] = true;
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
             if (!ok) {
-                for (int st = 0; st < 2; ++st) {
+                // After an abort, wait (bounded) for copies still in flight: the
+                // latest use of stage s is number u = issued-1-((issued-1-s) mod 3).
+                for (int st = 0; st < STAGES; ++st) {
                     if (!pending[st]) continue;
-                    const int last = seq - 1 - ((seq - 1 - st) & 1);
+                    const int u = issued - 1 - ((issued - 1 - st) % STAGES);
                     const unsigned long long t0 = globaltimer();
-                    while (last >= 0 && !mbar_try_wait(bar_tma + 8 * st, (last >> 1) & 1)) {
+                    while (u >= 0 && !mbar_try_wait(bar_tma + 8 * st, (uint32_t)((u / STAGES) & 1))) {
                         if (globaltimer() - t0 > kWaitLimitNs) break;
                     }
                 }
@@ -502,13 +467,13 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
 
 }  // namespace tc2
 
-// The 2-SM path covers the same shapes as the 1-SM tensor-core path and needs
-// at least one full pair of SMs worth of work to pay off; the halo copies
-// are 16 bytes wide when rows and the padding keep them aligned.
-inline bool conv1d_tc2_supported(int N, int C, int O, int K, int stride, int To, const void* pw)
+// The 2-SM path covers the shapes of the single-SM TMA-halo kernel.
+inline bool conv1d_tc2_supported(int C, int T, int O, int K, int stride, const void* x, const void* pw)
 {
-    (void)N; (void)To;
-    return conv1d_tc_supported(C, O, K, stride, pw);
+    const long long cw = (long long)tc2::KC * ((C + tc2::KC - 1) / tc2::KC);
+    return stride == 1 && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1 && T >= 1 && (C & 3) == 0 &&
+           (T & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(pw) & 15) == 0 && cw * K <= tc2::DWX_MAX;
 }
 
 inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float* pw, const float* bias, int N,
@@ -523,30 +488,47 @@ inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float*
     if (total > 0x7fffffffLL) return FCV_ERR_UNSUPPORTED;
     prm.total_tiles = (int)total;
     prm.out_vec = ((To & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0) ? 1 : 0;
-    prm.x_vec = ((T & 3) == 0 && (pad & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) ? 1 : 0;
 
     auto encode = tensor_map_encoder();
     if (!encode) return FCV_ERR_CUDA;
-    CUtensorMap map;
-    const cuuint64_t gdim[2] = {(cuuint64_t)C, (cuuint64_t)O};
-    const cuuint64_t gstride[1] = {(cuuint64_t)C * sizeof(float)};
-    const cuuint32_t box[2] = {(cuuint32_t)tc2::KC, (cuuint32_t)tc2::TNH};
-    const cuuint32_t estride[2] = {1, 1};
-    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pw), gdim, gstride, box, estride,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return FCV_ERR_CUDA;
+    CUtensorMap pw_map, x_map;
+    {   // pw [O][C]: 32 channels x 128 output channels per box (this CTA's half), 128B-swizzled
+        const cuuint64_t gdim[2] = {(cuuint64_t)C, (cuuint64_t)O};
+        const cuuint64_t gstride[1] = {(cuuint64_t)C * sizeof(float)};
+        const cuuint32_t box[2] = {(cuuint32_t)tc2::KC, (cuuint32_t)tc2::TNH};
+        const cuuint32_t estride[2] = {1, 1};
+        if (encode(&pw_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pw), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return FCV_ERR_CUDA;
+    }
+    {   // x [N][C][T]: 148 times x 32 channels x 1 batch item per box; outside reads 0
+        const cuuint64_t gdim[3] = {(cuuint64_t)T, (cuuint64_t)C, (cuuint64_t)N};
+        const cuuint64_t gstride[2] = {(cuuint64_t)T * sizeof(float), (cuuint64_t)C * T * sizeof(float)};
+        const cuuint32_t box[3] = {(cuuint32_t)tc2::XW, (cuuint32_t)tc2::KC, 1};
+        const cuuint32_t estride[3] = {1, 1, 1};
+        if (encode(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(x), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return FCV_ERR_CUDA;
+    }
 
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
-    auto kern = K == 9 ? tc2::dwsep_conv1d_tc2_kernel<9>
-              : K == 3 ? tc2::dwsep_conv1d_tc2_kernel<3> : tc2::dwsep_conv1d_tc2_kernel<0>;
+    const int r = (-pad) & 3;  // (t0 - pad) mod 4 with t0 a multiple of 128
+    decltype(&tc2::dwsep_conv1d_tc2_kernel<0, 0>) kern;
+    if (K == 9 && r == 0) kern = tc2::dwsep_conv1d_tc2_kernel<9, 0>;
+    else if (K == 3 && r == 3) kern = tc2::dwsep_conv1d_tc2_kernel<3, 3>;
+    else if (r == 0) kern = tc2::dwsep_conv1d_tc2_kernel<0, 0>;
+    else if (r == 1) kern = tc2::dwsep_conv1d_tc2_kernel<0, 1>;
+    else if (r == 2) kern = tc2::dwsep_conv1d_tc2_kernel<0, 2>;
+    else kern = tc2::dwsep_conv1d_tc2_kernel<0, 3>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc2::SMEM_BYTES) != cudaSuccess)
         return FCV_ERR_CUDA;
     const long long pairs = total < sms / 2 ? total : sms / 2;
     dim3 grid((unsigned)(2 * pairs));
-    kern<<<grid, tc2::NTHREADS, tc2::SMEM_BYTES, stream>>>(prm, map);
+    kern<<<grid, tc2::NTHREADS, tc2::SMEM_BYTES, stream>>>(prm, pw_map, x_map);
     return launch_status();
 }
 

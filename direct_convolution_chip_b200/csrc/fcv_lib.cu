@@ -175,7 +175,7 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
         }
         return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     case FCV_CONV1D_TC2_3XTF32:
-        if (!fcv::conv1d_tc2_supported(N, C, O, K, stride, To, pw_w)) return FCV_ERR_UNSUPPORTED;
+        if (!fcv::conv1d_tc2_supported(C, T, O, K, stride, x, pw_w)) return FCV_ERR_UNSUPPORTED;
         return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, s);
     case FCV_CONV1D_FMA:
         return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
