@@ -540,17 +540,18 @@ def run_probes():
         st = lib.fcvprobe_fma_rate(packed, 2, 20000, ctypes.byref(f), ctypes.byref(ms))
         print(json.dumps({"probe": "fp32_fma", "packed": packed, "status": st, "tflops": f.value / 1e12,
                           "ms": ms.value}), flush=True)
-    for n in (64, 128, 256):
+    for n in (32, 64, 128, 256):
         for a_tmem in (0, 1):
             for chains in (1, 2, 4):
-                if chains * n > 448:
-                    continue
-                f, ms, cyc = D(), D(), D()
-                st = lib.fcvprobe_tf32_mma_rate(n, a_tmem, chains, 24000, ctypes.byref(f), ctypes.byref(ms),
-                                                ctypes.byref(cyc))
-                print(json.dumps({"probe": "tcgen05_tf32_mma", "n": n, "a_tmem": a_tmem, "chains": chains,
-                                  "status": st, "tflops": f.value / 1e12, "ms": ms.value,
-                                  "cycles_per_mma": cyc.value}), flush=True)
+                for issuers in (1, 2):
+                    if issuers * chains * n > 448:
+                        continue
+                    f, ms, cyc = D(), D(), D()
+                    st = lib.fcvprobe_tf32_mma_rate(n, a_tmem, chains, issuers, 24000, ctypes.byref(f),
+                                                    ctypes.byref(ms), ctypes.byref(cyc))
+                    print(json.dumps({"probe": "tcgen05_tf32_mma", "n": n, "a_tmem": a_tmem, "chains": chains,
+                                      "issuers": issuers, "status": st, "tflops": f.value / 1e12, "ms": ms.value,
+                                      "cycles_per_mma": cyc.value}), flush=True)
 
 
 def run_configs(args):

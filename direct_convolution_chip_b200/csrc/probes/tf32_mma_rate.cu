@@ -44,7 +44,7 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint3
 // accumulator s mod CHAINS.  Descriptors are computed once, so the issuing
 // thread spends a few instructions per MMA and the tensor core sets the rate.
 template <int N, bool A_TMEM, int CHAINS>
-__global__ void __launch_bounds__(128, 1) mma_rate_kernel(int outer, unsigned long long* cycles,
+__global__ void __launch_bounds__(128, 1) mma_rate_kernel(int outer, int issuers, unsigned long long* cycles,
                                                           unsigned int* timeouts)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int outer, unsigned lo
     const uint32_t b_lo_s = b_hi_s + 256 * 128;
     const uint32_t bar = b_lo_s + 256 * 128;
     __shared__ uint32_t tmem_holder;
-    const int ncommits = (outer + 7) / 8;
+    const int ncommits = issuers * ((outer + 7) / 8);
 
     if (threadIdx.x == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(ncommits) : "memory");
@@ -71,8 +71,11 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int outer, unsigned lo
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
     const uint32_t tmem = tmem_holder;
 
-    if (threadIdx.x == 0) {
+    // Issuer i (lane 0 of warp i) drives accumulator columns [i * CHAINS * N, ...).
+    const int issuer = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0 && issuer < issuers) {
         const uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+        const uint32_t dbase = tmem + (uint32_t)(issuer * CHAINS * N);
         uint64_t bh[4], bl[4], ah[4], al[4];
         uint32_t th[4], tl[4];
 #pragma unroll
@@ -88,7 +91,7 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int outer, unsigned lo
         for (int it = 0; it < outer; ++it) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const uint32_t d = tmem + (uint32_t)((k % CHAINS) * N);
+                const uint32_t d = dbase + (uint32_t)((k % CHAINS) * N);
                 if (A_TMEM) {
                     mma_ts(d, th[k], bh[k], idesc);
                     mma_ts(d, th[k], bl[k], idesc);
@@ -117,7 +120,7 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int outer, unsigned lo
                 break;
             }
         }
-        cycles[blockIdx.x] = clock64() - c0;
+        if (issuer == 0) cycles[blockIdx.x] = clock64() - c0;
     }
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
     __syncthreads();
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int outer, unsigned lo
 }
 
 template <int N, bool A_TMEM, int CHAINS>
-int run(int blocks, int outer, unsigned long long* cycles, unsigned int* timeouts, float* ms)
+int run(int blocks, int outer, int issuers, unsigned long long* cycles, unsigned int* timeouts, float* ms)
 {
     // Operand buffers take 97 KB; 160 KB keeps one CTA per SM (each allocates
     // all 512 TMEM columns).
@@ -139,7 +142,7 @@ int run(int blocks, int outer, unsigned long long* cycles, unsigned int* timeout
     cudaEventCreate(&e1);
     for (int rep = 0; rep < 2; ++rep) {  // warm-up, then the timed launch
         cudaEventRecord(e0);
-        k<<<blocks, 128, smem>>>(outer, cycles, timeouts);
+        k<<<blocks, 128, smem>>>(outer, issuers, cycles, timeouts);
         cudaEventRecord(e1);
     }
     const int st = (cudaEventSynchronize(e1) == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : 3;
@@ -150,11 +153,12 @@ int run(int blocks, int outer, unsigned long long* cycles, unsigned int* timeout
 }
 
 template <int N, bool A_TMEM>
-int run_chains(int chains, int blocks, int outer, unsigned long long* cycles, unsigned int* timeouts, float* ms)
+int run_chains(int chains, int blocks, int outer, int issuers, unsigned long long* cycles, unsigned int* timeouts,
+               float* ms)
 {
-    if (chains == 1) return run<N, A_TMEM, 1>(blocks, outer, cycles, timeouts, ms);
-    if (chains == 2) return run<N, A_TMEM, 2>(blocks, outer, cycles, timeouts, ms);
-    return run<N, A_TMEM, 4>(blocks, outer, cycles, timeouts, ms);
+    if (chains == 1) return run<N, A_TMEM, 1>(blocks, outer, issuers, cycles, timeouts, ms);
+    if (chains == 2) return run<N, A_TMEM, 2>(blocks, outer, issuers, cycles, timeouts, ms);
+    return run<N, A_TMEM, 4>(blocks, outer, issuers, cycles, timeouts, ms);
 }
 
 }  // namespace
@@ -163,16 +167,18 @@ extern "C" {
 
 // Runs the probe on every SM and reports the TF32 rate in FLOP/s (2 per MAC)
 // over the whole device, the elapsed time, and the average SM cycles per MMA
-// instruction.  n: 64, 128 or 256; a_tmem: 0 (A in shared memory) or 1 (A in
-// tensor memory); chains: 1, 2 or 4 independent accumulators with
-// chains * n <= 448; iters: MMAs per SM, a multiple of 12.  Synchronizes the
+// instruction.  n: 32, 64, 128 or 256; a_tmem: 0 (A in shared memory) or 1 (A in
+// tensor memory); chains: 1, 2 or 4 independent accumulators per issuing
+// thread; issuers: 1 or 2 threads (in different warps) issuing at once, with
+// issuers * chains * n <= 448; iters: MMAs per issuer, a multiple of 12.  Synchronizes the
 // device.  Returns 0 on success, 1 on bad arguments, 3 on a CUDA error, 4 if a
 // wait timed out (the result is then meaningless).
-int fcvprobe_tf32_mma_rate(int n, int a_tmem, int chains, int iters, double* flops, double* ms,
+int fcvprobe_tf32_mma_rate(int n, int a_tmem, int chains, int issuers, int iters, double* flops, double* ms,
                            double* cycles_per_mma)
 {
-    if ((n != 64 && n != 128 && n != 256) || (chains != 1 && chains != 2 && chains != 4) || chains * n > 448 ||
-        iters < 12 || iters % 12 != 0 || iters / 96 > (1 << 19) || !flops || !ms || !cycles_per_mma)
+    if ((n != 32 && n != 64 && n != 128 && n != 256) || (chains != 1 && chains != 2 && chains != 4) ||
+        (issuers != 1 && issuers != 2) || issuers * chains * n > 448 || iters < 12 || iters % 12 != 0 ||
+        iters / 96 > (1 << 18) || !flops || !ms || !cycles_per_mma)
         return 1;
     const int outer = iters / 12;
     int dev = 0, sms = 0;
@@ -188,12 +194,14 @@ int fcvprobe_tf32_mma_rate(int n, int a_tmem, int chains, int iters, double* flo
     cudaMemset(timeouts, 0, sizeof(unsigned int));
     float t = 0.f;
     int st;
-    if (n == 64) st = a_tmem ? run_chains<64, true>(chains, sms, outer, cycles, timeouts, &t)
-                             : run_chains<64, false>(chains, sms, outer, cycles, timeouts, &t);
-    else if (n == 128) st = a_tmem ? run_chains<128, true>(chains, sms, outer, cycles, timeouts, &t)
-                                   : run_chains<128, false>(chains, sms, outer, cycles, timeouts, &t);
-    else st = a_tmem ? run_chains<256, true>(chains, sms, outer, cycles, timeouts, &t)
-                     : run_chains<256, false>(chains, sms, outer, cycles, timeouts, &t);
+    if (n == 32) st = a_tmem ? run_chains<32, true>(chains, sms, outer, issuers, cycles, timeouts, &t)
+                             : run_chains<32, false>(chains, sms, outer, issuers, cycles, timeouts, &t);
+    else if (n == 64) st = a_tmem ? run_chains<64, true>(chains, sms, outer, issuers, cycles, timeouts, &t)
+                             : run_chains<64, false>(chains, sms, outer, issuers, cycles, timeouts, &t);
+    else if (n == 128) st = a_tmem ? run_chains<128, true>(chains, sms, outer, issuers, cycles, timeouts, &t)
+                                   : run_chains<128, false>(chains, sms, outer, issuers, cycles, timeouts, &t);
+    else st = a_tmem ? run_chains<256, true>(chains, sms, outer, issuers, cycles, timeouts, &t)
+                     : run_chains<256, false>(chains, sms, outer, issuers, cycles, timeouts, &t);
     unsigned long long* hc = new unsigned long long[sms];
     unsigned int to = 0;
     if (st == 0 && (cudaMemcpy(hc, cycles, sizeof(unsigned long long) * sms, cudaMemcpyDeviceToHost) != cudaSuccess ||
@@ -202,9 +210,9 @@ int fcvprobe_tf32_mma_rate(int n, int a_tmem, int chains, int iters, double* flo
     if (st == 0) {
         double c = 0.0;
         for (int i = 0; i < sms; ++i) c += (double)hc[i];
-        *cycles_per_mma = c / sms / iters;
+        *cycles_per_mma = c / sms / ((double)iters * issuers);
         *ms = t;
-        *flops = 2.0 * 128.0 * n * 8.0 * (double)iters * sms / (t * 1e-3);
+        *flops = 2.0 * 128.0 * n * 8.0 * (double)iters * issuers * sms / (t * 1e-3);
         if (to) st = 4;
     }
     delete[] hc;
