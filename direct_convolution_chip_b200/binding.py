@@ -8,8 +8,9 @@ kernels; there is no CPU or PyTorch fallback, and a missing library raises.
 PyTorch supplies device memory and streams.  Tensors already on the GPU are
 used in place (they must be fp32 and contiguous).  CPU tensors are accepted
 too: they are copied to the current device (asynchronously when pinned), the
-kernel runs, and the result is copied back into a pinned CPU tensor -- the path
-an application with host-resident data takes.
+kernel runs, and the result is copied back into `out` when a CPU tensor is
+given (pinned for an asynchronous copy), else into a new pinned CPU tensor --
+the path an application with host-resident data takes.
 """
 import ctypes
 import os
@@ -129,10 +130,18 @@ def _host_mode(*ts):
     return True
 
 
-def _result(out_dev, host, stream):
+def _result(out_dev, host, stream, out_host=None):
+    """Host mode: copy the device result into `out_host` (a caller's CPU tensor,
+    best pinned) or into a new pinned tensor, and wait for the copy."""
     if not host:
         return out_dev
-    res = torch.empty(out_dev.shape, dtype=out_dev.dtype, pin_memory=True)
+    if out_host is not None:
+        if tuple(out_host.shape) != tuple(out_dev.shape) or out_host.dtype != out_dev.dtype or \
+                not out_host.is_contiguous():
+            raise ValueError(f"out must be a contiguous {out_dev.dtype} tensor of shape {tuple(out_dev.shape)}")
+        res = out_host
+    else:
+        res = torch.empty(out_dev.shape, dtype=out_dev.dtype, pin_memory=True)
     with torch.cuda.stream(stream or torch.cuda.current_stream()):
         res.copy_(out_dev, non_blocking=True)
     (stream or torch.cuda.current_stream()).synchronize()
@@ -154,12 +163,13 @@ def conv2d_pool_sigmoid_sum(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None
     if tuple(w.shape) != (Cout, Cin, 3, 3) or tuple(b.shape) != (Cout,):
         raise ValueError(f"w must be [Cout,{Cin},3,3] and b [Cout]; got {tuple(w.shape)}, {tuple(b.shape)}")
     xd, wd, bd = _dev(x, "x", dev), _dev(w, "w", dev), _dev(b, "b", dev)
+    out_host = out if host else None
     if out is None or host:
         out = torch.empty((N,), dtype=torch.float32, device=xd.device)
     _check(lib.fcv_conv2d_pool_sigmoid_sum_ex(_ptr(xd), _ptr(wd), _ptr(bd), N, Cin, H, W, Cout, pool,
                                               _ptr(out), algo, _stream_ptr(stream)),
            "fcv_conv2d_pool_sigmoid_sum")
-    return _result(out, host, stream)
+    return _result(out, host, stream, out_host)
 
 
 def conv2d_workspace_bytes(N, Cin, H, W, Cout, pool) -> int:
@@ -187,12 +197,13 @@ def conv2d_pool_sigmoid_sum_det(x, w, b, pool, out=None, workspace=None, stream=
         workspace = torch.empty(((need + 15) // 16 * 4,), dtype=torch.float32, device=dev)
     nbytes = workspace.numel() * workspace.element_size()
     xd, wd, bd = _dev(x, "x", dev), _dev(w, "w", dev), _dev(b, "b", dev)
+    out_host = out if host else None
     if out is None or host:
         out = torch.empty((N,), dtype=torch.float32, device=xd.device)
     _check(lib.fcv_conv2d_pool_sigmoid_sum_det(_ptr(xd), _ptr(wd), _ptr(bd), N, Cin, H, W, Cout, pool, _ptr(out),
                                                _ptr(workspace) if need else None, nbytes, _stream_ptr(stream)),
            "fcv_conv2d_pool_sigmoid_sum_det")
-    return _result(out, host, stream)
+    return _result(out, host, stream, out_host)
 
 
 def conv2d_pool_tap(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None):
@@ -206,11 +217,12 @@ def conv2d_pool_tap(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None):
         raise ValueError("w must be [Cout,Cin,3,3] and b [Cout]")
     PH, PW = conv2d_out_shape(H, W, pool)
     xd, wd, bd = _dev(x, "x", dev), _dev(w, "w", dev), _dev(b, "b", dev)
+    out_host = out if host else None
     if out is None or host:
         out = torch.empty((N, Cout, max(PH, 0), max(PW, 0)), dtype=torch.float32, device=xd.device)
     _check(lib.fcv_conv2d_pool_tap(_ptr(xd), _ptr(wd), _ptr(bd), N, Cin, H, W, Cout, pool,
                                    _ptr(out), algo, _stream_ptr(stream)), "fcv_conv2d_pool_tap")
-    return _result(out, host, stream)
+    return _result(out, host, stream, out_host)
 
 
 def conv1d_out_len(T, K, stride, pad):
@@ -231,11 +243,12 @@ def dwsep_conv1d(x, dw, pw, bias, stride, pad, out=None, algo=ALGO_AUTO, stream=
     To = conv1d_out_len(T, K, stride, pad)
     xd, dwd, pwd = _dev(x, "x", dev), _dev(dw, "dw", dev), _dev(pw, "pw", dev)
     bd = _dev(bias, "bias", dev)
+    out_host = out if host else None
     if out is None or host:
         out = torch.empty((N, O, max(To, 0)), dtype=torch.float32, device=xd.device)
     _check(lib.fcv_dwsep_conv1d_ex(_ptr(xd), _ptr(dwd), _ptr(pwd), _ptr(bd), N, C, T, O, K, stride, pad,
                                    _ptr(out), algo, _stream_ptr(stream)), "fcv_dwsep_conv1d")
-    return _result(out, host, stream)
+    return _result(out, host, stream, out_host)
 
 
 def conv2d_auto_algo(N, Cin, H, W, Cout, pool) -> int:

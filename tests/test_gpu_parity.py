@@ -306,6 +306,12 @@ def test_host_tensors_through_public_api():
     out2 = fcv.conv2d_pool_sigmoid_sum(x2, w2, b2, c2.P)
     assert not out2.is_cuda
     assert_close(out2, oracle.conv2d_pool_sigmoid_sum(x2.numpy(), w2.numpy(), b2.numpy(), c2.P), "host conv2d")
+    # a caller-provided pinned output is filled in place
+    dst = torch.full(tuple(out.shape), float("nan"), pin_memory=True)
+    got = fcv.dwsep_conv1d(x.pin_memory(), dw, pw, bias, case.stride, case.pad, out=dst)
+    assert got.data_ptr() == dst.data_ptr() and torch.equal(dst, out)
+    with pytest.raises(ValueError):
+        fcv.dwsep_conv1d(x, dw, pw, bias, case.stride, case.pad, out=torch.empty((1,)))
 
 
 def test_empty_batch_through_binding():
