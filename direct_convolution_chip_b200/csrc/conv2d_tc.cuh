@@ -82,6 +82,10 @@ constexpr int NPOOL = 256;
 constexpr int TMA_WARP = 21;
 constexpr int MMA_WARP2 = 22;     // second MMA issuer (odd tiles)
 constexpr int NTHREADS = 23 * 32;
+constexpr int SUB0 = 5;           // sub-chunk kernel: K-steps 0-4 | 5-8 of a chunk
+constexpr int SUB_LO = 8 * SUB0;  // lo half of a sub-chunk A stage (columns)
+constexpr int SUB_COLS = 2 * SUB_LO;  // one sub-chunk A stage: hi (40) | lo (40); four of them
+constexpr int NP_MAX_SUB = 96;    // sub-chunk kernel: 2 * NP + 4 * SUB_COLS <= 512
 constexpr int TP = 132;           // pitch of the transposed accumulator buffer (floats)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_LIMIT = 227 * 1024;
@@ -131,7 +135,7 @@ __host__ __device__ inline Layout make_layout(int NP, int natoms)
     L.tbuf = L.halo + 2u * Geo<P>::HALO * 4u;
     L.bias = L.tbuf + 2u * (uint32_t)NP * TP * 4u;  // two transposed accumulator buffers
     L.bar = (L.bias + (uint32_t)NP * 4u + 7u) & ~7u;
-    L.misc = L.bar + 20u * 8u;
+    L.misc = L.bar + 24u * 8u;
     L.total = L.misc + 16u;
     return L;
 }
@@ -608,6 +612,408 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
     }
 }
 
+template <int P, int MODE>
+__global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc4_kernel(const Params p, const __grid_constant__ CUtensorMap x_map)
+{
+    using G = Geo<P>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    const Layout L = make_layout<P>(p.NP, p.natoms);
+    float* halo = reinterpret_cast<float*>(smem + L.halo);
+    float* tbuf = reinterpret_cast<float*>(smem + L.tbuf);
+    float* bias_s = reinterpret_cast<float*>(smem + L.bias);
+    const uint32_t bar_afull = sbase + L.bar;         // + 8 * stage (4), 4 producer-warp arrivals
+    const uint32_t bar_aempty = bar_afull + 32;       // + 8 * stage (4), tcgen05.commit
+    const uint32_t bar_accfull = bar_afull + 64;      // + 8 * buf (3), tcgen05.commit
+    const uint32_t bar_accempty = bar_afull + 88;     // + 8 * buf (3), 4 drain-warp arrivals
+    const uint32_t bar_drain = bar_afull + 112;
+    const uint32_t bar_hfull = bar_afull + 120;       // + 8 * buf, TMA halo landed
+    const uint32_t bar_hempty = bar_afull + 136;      // + 8 * buf, 8 producer-warp arrivals
+    const uint32_t bar_tfull = bar_afull + 152;       // + 8 * buf, 4 drain-warp arrivals
+    const uint32_t bar_tempty = bar_afull + 168;      // + 8 * buf, 8 pool-warp arrivals
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.misc);
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 4);
+    volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + L.misc + 8);  // [2], one per group
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NP = p.NP;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar_afull + 8 * i, 4);
+            mbar_init(bar_aempty + 8 * i, 1);
+        }
+        for (int i = 0; i < 3; ++i) {
+            mbar_init(bar_accfull + 8 * i, 1);
+            mbar_init(bar_accempty + 8 * i, 4);
+        }
+        mbar_init(bar_drain, 2);  // one commit per MMA issuer
+        mbar_init(bar_hfull, 1);
+        mbar_init(bar_hfull + 8, 1);
+        mbar_init(bar_hempty, 8);
+        mbar_init(bar_hempty + 8, 8);
+        mbar_init(bar_tfull, 4);
+        mbar_init(bar_tfull + 8, 4);
+        mbar_init(bar_tempty, 8);
+        mbar_init(bar_tempty + 8, 8);
+        *abort_flag = 0u;
+        prod_abort[0] = 0u;
+        prod_abort[1] = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == MMA_WARP) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_holder)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+
+    // Weights as the B operand, split into TF32 hi/lo: element (co, k) with
+    // k = 72 * chunk + e, e = 9 * (ci mod 8) + 3 * ky + kx, sits in 128-byte K
+    // block 3 * chunk + e / 32 (blocks of NP rows), row co, swizzled 16-byte
+    // chunk (e mod 32) / 4.  Every chunk starts a K block, so the descriptors of
+    // chunk c are those of chunk 0 moved by c * 3 blocks.
+    const int ktot = KCH * p.nchunks;
+    for (int idx = threadIdx.x; idx < NP * ktot; idx += NTHREADS) {
+        const int co = idx / ktot, k = idx - co * ktot;
+        const int ch = k / KCH, e = k - ch * KCH;
+        const int ci = ch * CCH + e / 9, t = e % 9;
+        const float v = (co < p.Cout && ci < p.Cin) ? __ldg(p.w + ((size_t)co * p.Cin + ci) * 9 + t) : 0.f;
+        const float hi = tf32_round(v);
+        const int a = 3 * ch + (e >> 5), kin = e & 31;
+        const uint32_t off = (uint32_t)a * NP * 128u + sw128_off(co, kin >> 2) + (uint32_t)(kin & 3) * 4u;
+        *reinterpret_cast<float*>(smem + L.b_hi + off) = hi;
+        *reinterpret_cast<float*>(smem + L.b_lo + off) = v - hi;
+    }
+    for (int i = threadIdx.x; i < NP; i += NTHREADS) bias_s[i] = i < p.Cout ? __ldg(p.b + i) : 0.f;
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // weights visible to the tensor core
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    // Accumulators: p.nacc buffers of NP columns (3 when they fit next to the two
+    // A stages, else 2), used round robin: buffer abuf, phase aphase.
+    const uint32_t a_col0 = (uint32_t)(p.nacc * NP);  // first A-stage column (4 stages of SUB_COLS)
+
+    if (warp < 8) {
+        // ------------------------------------------------------------ producers
+        // Two independent groups of four warps, one per K sub-chunk (K-steps
+        // 0-4 and 5-8 of every chunk); warp w of a group owns TMEM lane quarter
+        // w & 3.  Sub-chunk s of a tile with parity q goes to A stage 2q + s, so a
+        // group rebuilds its sub-stage as soon as the MMAs that read it are done,
+        // whatever the other group is doing.
+        const int grp = warp >> 2;                 // sub-chunk of this group
+        const int gtid = threadIdx.x - 128 * grp;  // 0..127
+        const int m = 32 * (warp & 3) + lane;      // conv position = TMEM lane
+        const int r = m / G::WC, c = m - (m / G::WC) * G::WC;
+        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        int seq = 0, tile = blockIdx.x, ch = 0, abuf = 0, t = 0;
+        uint32_t aphase = 0;
+        for (; tile < p.total_tiles; ++seq) {
+            const int stage = 2 * (t & 1) + grp;
+            const uint32_t upar = (uint32_t)(((t >> 1) * p.nchunks + ch) & 1);
+            const int hbuf = seq & 1;
+            const uint32_t hpar = (seq >> 1) & 1;
+            // This sub-stage's last MMAs are done, the halo has landed and, for
+            // sub-chunk 0 of a tile's first chunk, the accumulator the tile will
+            // reset is drained.  The group's first thread waits (bounded) before
+            // the group barrier, so the abort decision after it is the group's.
+            if (gtid == 0) {
+                if (!wait_bounded(bar_aempty + 8 * stage, upar ^ 1, abort_flag)) prod_abort[grp] = 1u;
+                else if (!wait_bounded(bar_hfull + 8 * hbuf, hpar, abort_flag)) prod_abort[grp] = 1u;
+                else if (grp == 0 && ch == 0 && !wait_bounded(bar_accempty + 8 * abuf, aphase ^ 1, abort_flag))
+                    prod_abort[grp] = 1u;
+            }
+            if (grp == 0) asm volatile("bar.sync 1, 128;\n" ::: "memory");
+            else asm volatile("bar.sync 3, 128;\n" ::: "memory");
+            if (prod_abort[grp]) break;
+            for (int spin = 0; !mbar_try_wait(bar_hfull + 8 * hbuf, hpar) && spin < (1 << 20); ++spin) {
+            }
+            tc_fence_after();
+            // im2col values of position (r, c) for this sub-chunk's K groups, 8 per
+            // TMEM store; A_hi is the raw fp32 value (the MMA reads its TF32
+            // bits), A_lo = v - truncate(v) is exact.
+            const float* hb = halo + hbuf * G::HALO + r * G::HP + c;
+            const uint32_t a_st = tmem + lane_base + a_col0 + (uint32_t)(stage * SUB_COLS);
+            auto build = [&](auto g0c, auto g1c) {
+                constexpr int g0 = decltype(g0c)::value, g1 = decltype(g1c)::value;
+#pragma unroll
+                for (int g = g0; g < g1; ++g) {
+                    uint32_t hi[8], lo[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int e = 8 * g + q;
+                        const int ci = e / 9, tt = e % 9;
+                        const float v = hb[ci * G::CHS + (tt / 3) * G::HP + (tt % 3)];
+                        hi[q] = __float_as_uint(v);
+                        lo[q] = __float_as_uint(v - __uint_as_float(hi[q] & 0xFFFFE000u));
+                    }
+                    tmem_st8(a_st + (uint32_t)(8 * (g - g0)), hi);
+                    tmem_st8(a_st + (uint32_t)(SUB_LO + 8 * (g - g0)), lo);
+                }
+            };
+            if (grp == 0) build(std::integral_constant<int, 0>{}, std::integral_constant<int, SUB0>{});
+            else build(std::integral_constant<int, SUB0>{}, std::integral_constant<int, KST>{});
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_hempty + 8 * hbuf);  // this warp is done with the halo
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_afull + 8 * stage);
+            if (++ch == p.nchunks) {
+                ch = 0;
+                tile += gridDim.x;
+                ++t;
+                if (++abuf == p.nacc) {
+                    abuf = 0;
+                    aphase ^= 1u;
+                }
+            }
+        }
+    } else if (warp == TMA_WARP) {
+        // -------------------------------------------------------- TMA issuer
+        // One box [8 channels][P + 2 rows][HP columns] per (tile, chunk) lands
+        // in the halo layout itself; rows, columns and channels outside x read 0.
+        if (p.use_tma && lane == 0) {
+            int seq = 0;
+            bool pending[2] = {false, false};
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+                const TileCoord tcd = decode(p, tile);
+                for (int ch = 0; ch < p.nchunks; ++ch, ++seq) {
+                    const int b = seq & 1;
+                    if (!wait_bounded(bar_hempty + 8 * b, ((seq >> 1) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    pending[b] = false;  // the producers consumed its previous box
+                    tc::mbar_arrive_expect_tx(bar_hfull + 8 * b, (uint32_t)G::HALO * 4u);
+                    tma_load_4d(smem_u32(halo + b * G::HALO), &x_map, tcd.tx * G::WC, tcd.py * P, ch * CCH, tcd.n,
+                                bar_hfull + 8 * b);
+                    pending[b] = true;
+                }
+            }
+            if (!ok) {
+                // After an abort, wait (bounded) for boxes still in flight.
+                for (int b = 0; b < 2; ++b) {
+                    if (!pending[b]) continue;
+                    const int last = seq - 1 - ((seq - 1 - b) & 1);  // latest sequence number on buffer b
+                    const unsigned long long t0 = globaltimer();
+                    while (last >= 0 && !mbar_try_wait(bar_hfull + 8 * b, (last >> 1) & 1)) {
+                        if (globaltimer() - t0 > kWaitLimitNs) break;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP || warp == MMA_WARP2) {
+        // --------------------------------------------------------- MMA issuers
+        // Two issuing threads, one for the even and one for the odd tiles of this
+        // CTA: while one waits on a barrier the other keeps the tensor core fed.
+        // Each commit tracks the issuing thread's own MMAs, which is what every
+        // barrier here needs (a stage or accumulator is used by one tile).
+        if (lane == 0) {
+            const int par = warp == MMA_WARP ? 0 : 1;
+            const uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NP >> 3) << 17) |
+                                   ((uint32_t)(MT >> 4) << 24);
+            // B descriptors of chunk 0's nine K-steps, computed once: the issue
+            // loop then spends a few instructions per MMA, so the tensor core,
+            // not this thread, sets the pace.
+            uint64_t bh0[KST], bl0[KST];
+#pragma unroll
+            for (int kk = 0; kk < KST; ++kk) {
+                const uint32_t boff = (uint32_t)(kk >> 2) * NP * 128u + 32u * (uint32_t)(kk & 3);
+                bh0[kk] = sw128_desc(sbase + L.b_hi + boff);
+                bl0[kk] = sw128_desc(sbase + L.b_lo + boff);
+            }
+            const uint64_t chunk_step = (uint64_t)(3u * NP * 128u) >> 4;  // descriptor address units
+            int abuf = par % p.nacc;
+            bool ok = true;
+            for (int t = par, tile = blockIdx.x + par * gridDim.x; ok && tile < p.total_tiles;
+                 t += 2, tile += 2 * gridDim.x) {
+                const int buf = abuf;  // drained: the producers saw it before "A full"
+                abuf = (abuf + 2) % p.nacc;
+                const uint32_t d_tmem = tmem + (uint32_t)(buf * NP);
+                for (int ch = 0; ch < p.nchunks && ok; ++ch) {
+                    const uint32_t upar = (uint32_t)(((t >> 1) * p.nchunks + ch) & 1);
+                    const uint64_t cofs = chunk_step * (uint64_t)ch;
+                    // sub-chunk 0: K-steps 0 .. SUB0-1, in A stage 2 * par
+                    {
+                        const int stage = 2 * par;
+                        if (!wait_bounded(bar_afull + 8 * stage, upar, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t ah = tmem + a_col0 + (uint32_t)(stage * SUB_COLS), al = ah + (uint32_t)SUB_LO;
+                        mma_tf32_ts(d_tmem, ah, bh0[0] + cofs, idesc, ch > 0 ? 1u : 0u);
+                        mma_tf32_ts_acc(d_tmem, ah, bl0[0] + cofs, idesc);
+                        mma_tf32_ts_acc(d_tmem, al, bh0[0] + cofs, idesc);
+#pragma unroll
+                        for (int j = 1; j < SUB0; ++j) {
+                            mma_tf32_ts_acc(d_tmem, ah + 8u * j, bh0[j] + cofs, idesc);
+                            mma_tf32_ts_acc(d_tmem, ah + 8u * j, bl0[j] + cofs, idesc);
+                            mma_tf32_ts_acc(d_tmem, al + 8u * j, bh0[j] + cofs, idesc);
+                        }
+                        tc_commit(bar_aempty + 8 * stage);
+                    }
+                    // sub-chunk 1: K-steps SUB0 .. 8, in A stage 2 * par + 1
+                    {
+                        const int stage = 2 * par + 1;
+                        if (!wait_bounded(bar_afull + 8 * stage, upar, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t ah = tmem + a_col0 + (uint32_t)(stage * SUB_COLS), al = ah + (uint32_t)SUB_LO;
+#pragma unroll
+                        for (int j = 0; j < KST - SUB0; ++j) {
+                            mma_tf32_ts_acc(d_tmem, ah + 8u * j, bh0[SUB0 + j] + cofs, idesc);
+                            mma_tf32_ts_acc(d_tmem, ah + 8u * j, bl0[SUB0 + j] + cofs, idesc);
+                            mma_tf32_ts_acc(d_tmem, al + 8u * j, bh0[SUB0 + j] + cofs, idesc);
+                        }
+                        tc_commit(bar_aempty + 8 * stage);
+                    }
+                }
+                if (ok) tc_commit(bar_accfull + 8 * buf);
+            }
+            tc_commit(bar_drain);
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait(bar_drain, 0)) {
+                if (globaltimer() - t0 > kWaitLimitNs) {
+                    *abort_flag = 1u;
+                    record_device_error(kErrTimeout);
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        // Drain warps (one per TMEM lane quarter) copy a finished accumulator
+        // into one of two transposed buffers and release it at once; pool warps
+        // then reduce that buffer.  Pooling of one tile overlaps the drain of
+        // the next, so the epilogue's rate is the slower of the two halves.
+        int abuf = 0, local = 0;
+        uint32_t aphase = 0;
+        if (warp >= DRAIN_WARP0 && warp < DRAIN_WARP0 + 4) {
+            const int q = warp & 3;  // TMEM lane quarter of this warp
+            const int mrow = 32 * q + lane;
+            for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
+                const int buf = abuf;
+                const uint32_t bphase = aphase;
+                if (++abuf == p.nacc) {
+                    abuf = 0;
+                    aphase ^= 1u;
+                }
+                const int tb = local & 1;
+                const uint32_t tphase = (local >> 1) & 1;
+                int ok = 1;
+                if (lane == 0) {
+                    ok = wait_bounded(bar_accfull + 8 * buf, bphase, abort_flag) &&
+                         wait_bounded(bar_tempty + 8 * tb, tphase ^ 1, abort_flag);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                tc_fence_after();  // TMEM loads after the MMAs lane 0 saw complete
+                float* tbw = tbuf + tb * NP * TP;
+                const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * NP);
+                for (int cb = 0; cb < NP / 16; cb += 2) {  // two TMEM loads per wait
+                    uint32_t v[16], u[16];
+                    const bool two = cb + 1 < NP / 16;
+                    tmem_ld16(taddr + (uint32_t)(16 * cb), v);
+                    if (two) tmem_ld16(taddr + (uint32_t)(16 * (cb + 1)), u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) tbw[(16 * cb + j) * TP + mrow] = __uint_as_float(v[j]);
+                    if (two) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) tbw[(16 * (cb + 1) + j) * TP + mrow] = __uint_as_float(u[j]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bar_accempty + 8 * buf);  // accumulator free for the MMA
+                    mbar_arrive(bar_tfull + 8 * tb);      // this quarter of the buffer is written
+                }
+            }
+        } else {
+            const int ptid = threadIdx.x - 32 * POOL_WARP0;  // 0..255
+            const float inv_area = 1.f / (float)(P * P);
+            const float inv_cout = 1.f / (float)p.Cout;
+            float acc = 0.f;
+            int cur = -1;
+            auto flush = [&]() {
+                float s = acc;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (lane == 0 && cur >= 0) atomicAdd(p.out + cur, s);
+                acc = 0.f;
+            };
+            for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
+                const int tb = local & 1;
+                const uint32_t tphase = (local >> 1) & 1;
+                int ok = 1;
+                if (lane == 0) ok = wait_bounded(bar_tfull + 8 * tb, tphase, abort_flag) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                // every lane acquires the drain warps' stores (returns at once)
+                for (int spin = 0; !mbar_try_wait(bar_tfull + 8 * tb, tphase) && spin < (1 << 20); ++spin) {
+                }
+                const TileCoord tcd = decode(p, tile);
+                if (MODE != kTap && tcd.n != cur) {
+                    flush();
+                    cur = tcd.n;
+                }
+                const float* tbr = tbuf + tb * NP * TP;
+                const int nval = G::WPT * p.Cout;
+#pragma unroll 2
+                for (int v = ptid; v < nval; v += NPOOL) {
+                    // j = v / Cout exactly: (v + 1/2) / Cout is at least 1/(2 Cout) away
+                    // from an integer and v < 2^14, far inside fp32 precision.
+                    const int j = (int)(((float)v + 0.5f) * inv_cout), co = v - j * p.Cout;
+                    const int px = tcd.tx * G::WPT + j;
+                    if (px >= p.PW) continue;
+                    const float* tb4 = tbr + co * TP + j * P;
+                    float s = 0.f;
+#pragma unroll
+                    for (int rr = 0; rr < P; ++rr) {
+                        if constexpr (P % 4 == 0) {
+#pragma unroll
+                            for (int dc = 0; dc < P; dc += 4) {
+                                const float4 f = *reinterpret_cast<const float4*>(tb4 + rr * G::WC + dc);
+                                s += (f.x + f.y) + (f.z + f.w);
+                            }
+                        } else {
+#pragma unroll
+                            for (int dc = 0; dc < P; ++dc) s += tb4[rr * G::WC + dc];
+                        }
+                    }
+                    const float pooled = s * inv_area + bias_s[co];
+                    if (MODE == kTap) {
+                        p.out[(((size_t)tcd.n * p.Cout + co) * p.PH + tcd.py) * p.PW + px] = pooled;
+                    } else {
+                        acc += __fdividef(1.f, 1.f + __expf(-pooled));  // sigmoid; 0 once exp overflows
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_tempty + 8 * tb);  // this warp is done with the buffer
+            }
+            if (MODE != kTap) flush();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == MMA_WARP) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
 }  // namespace c2tc
 
 inline bool conv2d_tc_pool_ok(int P) { return P == 1 || P == 2 || P == 4 || P == 8; }
@@ -673,7 +1079,12 @@ inline int launch_conv2d_tc_p(c2tc::Params prm, int N, int grid, cudaStream_t st
     // 512 TMEM columns.
     uint32_t smem = conv2d_tc_smem<P>(prm.Cin, prm.Cout);
     if (smem < 120u * 1024u) smem = 120u * 1024u;
-    auto kern = c2tc::conv2d_tc_kernel<P, MODE>;
+    // With the halo by TMA and Cout <= 96, the sub-chunk kernel: four smaller A
+    // stages let a producer group refill half a chunk while the MMAs of the
+    // other half run.
+    const bool sub = prm.use_tma && prm.NP <= c2tc::NP_MAX_SUB;
+    if (sub) prm.nacc = (3 * prm.NP + 4 * c2tc::SUB_COLS <= (int)c2tc::TMEM_COLS) ? 3 : 2;
+    auto kern = sub ? c2tc::conv2d_tc4_kernel<P, MODE> : c2tc::conv2d_tc_kernel<P, MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return FCV_ERR_CUDA;
     kern<<<grid, c2tc::NTHREADS, smem, stream>>>(prm, map);
