@@ -399,7 +399,9 @@ def run_gpu(args):
     if dom == "conv2d":
         achieved = 2 * macs_a / ta_s / 1e12
         if tc_a:
-            roof = {"kernel": "c2tc::conv2d_tc_kernel<4, sum>", "bound": "tensor", "achieved": achieved,
+            kname = ("c2tc::conv2d_tc4_kernel<4, sum>" if CASE_A.Cout <= 96 and CASE_A.W % 4 == 0
+                     else "c2tc::conv2d_tc_kernel<4, sum>")
+            roof = {"kernel": kname, "bound": "tensor", "achieved": achieved,
                     "peak": tf32_peak / 3.0, "unit": "TFLOP/s", "frac": achieved / (tf32_peak / 3.0),
                     "traffic": traffic_per_launch("conv2d_tc_p4"), "peak_source": tc_src}
         else:

@@ -42,6 +42,15 @@
 //     accumulates; one atomic add per warp and image.  Pooling of one tile
 //     overlaps the drain of the next.
 //   * Every wait is bounded, as in the conv1d kernels.
+//
+// Sub-chunk variant (conv2d_tc4_kernel; used when the halo comes by TMA and
+// Cout' <= 96): each chunk's nine K-steps are split into K-steps 0-4 and 5-8,
+// TMEM holds four A stages of 80 columns (sub-chunk s of a tile with parity q
+// in stage 2q + s), and the producers form two independent groups of four
+// warps, one per sub-chunk, so a group refills its half of the next tile while
+// the MMAs of the other half run.  Each MMA issuer commits a sub-chunk's stage
+// as soon as its MMAs are issued.  With three accumulators of 64 columns that
+// is exactly the 512 TMEM columns.
 #pragma once
 
 #include "conv1d_tc.cuh"
@@ -193,6 +202,199 @@ __device__ __forceinline__ TileCoord decode(const Params& p, int tile)
     return t;
 }
 
+// Weights as the B operand, split into TF32 hi/lo, and the padded bias, into
+// shared memory (all threads of the CTA; the caller fences and synchronises).
+template <int P>
+__device__ __forceinline__ void stage_weights(const Params& p, uint8_t* smem, const Layout& L, float* bias_s)
+{
+    const int NP = p.NP;
+    // Element (co, k) with
+    // k = 72 * chunk + e, e = 9 * (ci mod 8) + 3 * ky + kx, sits in 128-byte K
+    // block 3 * chunk + e / 32 (blocks of NP rows), row co, swizzled 16-byte
+    // chunk (e mod 32) / 4.  Every chunk starts a K block, so the descriptors of
+    // chunk c are those of chunk 0 moved by c * 3 blocks.
+    const int ktot = KCH * p.nchunks;
+    for (int idx = threadIdx.x; idx < NP * ktot; idx += NTHREADS) {
+        const int co = idx / ktot, k = idx - co * ktot;
+        const int ch = k / KCH, e = k - ch * KCH;
+        const int ci = ch * CCH + e / 9, t = e % 9;
+        const float v = (co < p.Cout && ci < p.Cin) ? __ldg(p.w + ((size_t)co * p.Cin + ci) * 9 + t) : 0.f;
+        const float hi = tf32_round(v);
+        const int a = 3 * ch + (e >> 5), kin = e & 31;
+        const uint32_t off = (uint32_t)a * NP * 128u + sw128_off(co, kin >> 2) + (uint32_t)(kin & 3) * 4u;
+        *reinterpret_cast<float*>(smem + L.b_hi + off) = hi;
+        *reinterpret_cast<float*>(smem + L.b_lo + off) = v - hi;
+    }
+    for (int i = threadIdx.x; i < NP; i += NTHREADS) bias_s[i] = i < p.Cout ? __ldg(p.b + i) : 0.f;
+}
+
+// TMA warp: one box [8 channels][P + 2 rows][HP columns] per (tile, chunk)
+// into the two halo buffers, in the order the producers consume them.
+template <int P>
+__device__ __forceinline__ void tma_halo_warp(const Params& p, const CUtensorMap& x_map, float* halo,
+                                              uint32_t bar_hfull, uint32_t bar_hempty,
+                                              volatile uint32_t* abort_flag, int lane)
+{
+    using G = Geo<P>;
+    // The box lands in the halo layout itself; rows, columns and channels
+    // outside x read 0.
+    if (p.use_tma && lane == 0) {
+        int seq = 0;
+        bool pending[2] = {false, false};
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+            const TileCoord tcd = decode(p, tile);
+            for (int ch = 0; ch < p.nchunks; ++ch, ++seq) {
+                const int b = seq & 1;
+                if (!wait_bounded(bar_hempty + 8 * b, ((seq >> 1) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                pending[b] = false;  // the producers consumed its previous box
+                tc::mbar_arrive_expect_tx(bar_hfull + 8 * b, (uint32_t)G::HALO * 4u);
+                tma_load_4d(smem_u32(halo + b * G::HALO), &x_map, tcd.tx * G::WC, tcd.py * P, ch * CCH, tcd.n,
+                            bar_hfull + 8 * b);
+                pending[b] = true;
+            }
+        }
+        if (!ok) {
+            // After an abort, wait (bounded) for boxes still in flight.
+            for (int b = 0; b < 2; ++b) {
+                if (!pending[b]) continue;
+                const int last = seq - 1 - ((seq - 1 - b) & 1);  // latest sequence number on buffer b
+                const unsigned long long t0 = globaltimer();
+                while (last >= 0 && !mbar_try_wait(bar_hfull + 8 * b, (last >> 1) & 1)) {
+                    if (globaltimer() - t0 > kWaitLimitNs) break;
+                }
+            }
+        }
+    }
+    __syncwarp();
+}
+
+// Epilogue warps 9-20: drain (9-12) and pool (13-20), as described above.
+template <int P, int MODE>
+__device__ __forceinline__ void epilogue_warps(const Params& p, float* tbuf, const float* bias_s, uint32_t tmem,
+                                               uint32_t bar_accfull, uint32_t bar_accempty, uint32_t bar_tfull,
+                                               uint32_t bar_tempty, volatile uint32_t* abort_flag, int warp,
+                                               int lane)
+{
+    using G = Geo<P>;
+    const int NP = p.NP;
+    // Drain warps (one per TMEM lane quarter) copy a finished accumulator
+    // into one of two transposed buffers and release it at once; pool warps
+    // then reduce that buffer.  Pooling of one tile overlaps the drain of
+    // the next, so the epilogue's rate is the slower of the two halves.
+    int abuf = 0, local = 0;
+    uint32_t aphase = 0;
+    if (warp >= DRAIN_WARP0 && warp < DRAIN_WARP0 + 4) {
+        const int q = warp & 3;  // TMEM lane quarter of this warp
+        const int mrow = 32 * q + lane;
+        for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
+            const int buf = abuf;
+            const uint32_t bphase = aphase;
+            if (++abuf == p.nacc) {
+                abuf = 0;
+                aphase ^= 1u;
+            }
+            const int tb = local & 1;
+            const uint32_t tphase = (local >> 1) & 1;
+            int ok = 1;
+            if (lane == 0) {
+                ok = wait_bounded(bar_accfull + 8 * buf, bphase, abort_flag) &&
+                     wait_bounded(bar_tempty + 8 * tb, tphase ^ 1, abort_flag);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();  // TMEM loads after the MMAs lane 0 saw complete
+            float* tbw = tbuf + tb * NP * TP;
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * NP);
+            for (int cb = 0; cb < NP / 16; cb += 2) {  // two TMEM loads per wait
+                uint32_t v[16], u[16];
+                const bool two = cb + 1 < NP / 16;
+                tmem_ld16(taddr + (uint32_t)(16 * cb), v);
+                if (two) tmem_ld16(taddr + (uint32_t)(16 * (cb + 1)), u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) tbw[(16 * cb + j) * TP + mrow] = __uint_as_float(v[j]);
+                if (two) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) tbw[(16 * (cb + 1) + j) * TP + mrow] = __uint_as_float(u[j]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar_accempty + 8 * buf);  // accumulator free for the MMA
+                mbar_arrive(bar_tfull + 8 * tb);      // this quarter of the buffer is written
+            }
+        }
+    } else {
+        const int ptid = threadIdx.x - 32 * POOL_WARP0;  // 0..255
+        const float inv_area = 1.f / (float)(P * P);
+        const float inv_cout = 1.f / (float)p.Cout;
+        float acc = 0.f;
+        int cur = -1;
+        auto flush = [&]() {
+            float s = acc;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if (lane == 0 && cur >= 0) atomicAdd(p.out + cur, s);
+            acc = 0.f;
+        };
+        for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
+            const int tb = local & 1;
+            const uint32_t tphase = (local >> 1) & 1;
+            int ok = 1;
+            if (lane == 0) ok = wait_bounded(bar_tfull + 8 * tb, tphase, abort_flag) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            // every lane acquires the drain warps' stores (returns at once)
+            for (int spin = 0; !mbar_try_wait(bar_tfull + 8 * tb, tphase) && spin < (1 << 20); ++spin) {
+            }
+            const TileCoord tcd = decode(p, tile);
+            if (MODE != kTap && tcd.n != cur) {
+                flush();
+                cur = tcd.n;
+            }
+            const float* tbr = tbuf + tb * NP * TP;
+            const int nval = G::WPT * p.Cout;
+#pragma unroll 2
+            for (int v = ptid; v < nval; v += NPOOL) {
+                // j = v / Cout exactly: (v + 1/2) / Cout is at least 1/(2 Cout) away
+                // from an integer and v < 2^14, far inside fp32 precision.
+                const int j = (int)(((float)v + 0.5f) * inv_cout), co = v - j * p.Cout;
+                const int px = tcd.tx * G::WPT + j;
+                if (px >= p.PW) continue;
+                const float* tb4 = tbr + co * TP + j * P;
+                float s = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < P; ++rr) {
+                    if constexpr (P % 4 == 0) {
+#pragma unroll
+                        for (int dc = 0; dc < P; dc += 4) {
+                            const float4 f = *reinterpret_cast<const float4*>(tb4 + rr * G::WC + dc);
+                            s += (f.x + f.y) + (f.z + f.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int dc = 0; dc < P; ++dc) s += tb4[rr * G::WC + dc];
+                    }
+                }
+                const float pooled = s * inv_area + bias_s[co];
+                if (MODE == kTap) {
+                    p.out[(((size_t)tcd.n * p.Cout + co) * p.PH + tcd.py) * p.PW + px] = pooled;
+                } else {
+                    acc += __fdividef(1.f, 1.f + __expf(-pooled));  // sigmoid; 0 once exp overflows
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty + 8 * tb);  // this warp is done with the buffer
+        }
+        if (MODE != kTap) flush();
+    }
+}
+
 template <int P, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap x_map)
 {
@@ -249,24 +451,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
 
-    // Weights as the B operand, split into TF32 hi/lo: element (co, k) with
-    // k = 72 * chunk + e, e = 9 * (ci mod 8) + 3 * ky + kx, sits in 128-byte K
-    // block 3 * chunk + e / 32 (blocks of NP rows), row co, swizzled 16-byte
-    // chunk (e mod 32) / 4.  Every chunk starts a K block, so the descriptors of
-    // chunk c are those of chunk 0 moved by c * 3 blocks.
-    const int ktot = KCH * p.nchunks;
-    for (int idx = threadIdx.x; idx < NP * ktot; idx += NTHREADS) {
-        const int co = idx / ktot, k = idx - co * ktot;
-        const int ch = k / KCH, e = k - ch * KCH;
-        const int ci = ch * CCH + e / 9, t = e % 9;
-        const float v = (co < p.Cout && ci < p.Cin) ? __ldg(p.w + ((size_t)co * p.Cin + ci) * 9 + t) : 0.f;
-        const float hi = tf32_round(v);
-        const int a = 3 * ch + (e >> 5), kin = e & 31;
-        const uint32_t off = (uint32_t)a * NP * 128u + sw128_off(co, kin >> 2) + (uint32_t)(kin & 3) * 4u;
-        *reinterpret_cast<float*>(smem + L.b_hi + off) = hi;
-        *reinterpret_cast<float*>(smem + L.b_lo + off) = v - hi;
-    }
-    for (int i = threadIdx.x; i < NP; i += NTHREADS) bias_s[i] = i < p.Cout ? __ldg(p.b + i) : 0.f;
+    stage_weights<P>(p, smem, L, bias_s);
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // weights visible to the tensor core
     tc_fence_before();
     __syncthreads();
@@ -389,41 +574,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
         }
         cp_async_wait<0>();  // no copy may land after the CTA has left
     } else if (warp == TMA_WARP) {
-        // -------------------------------------------------------- TMA issuer
-        // One box [8 channels][P + 2 rows][HP columns] per (tile, chunk) lands
-        // in the halo layout itself; rows, columns and channels outside x read 0.
-        if (p.use_tma && lane == 0) {
-            int seq = 0;
-            bool pending[2] = {false, false};
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
-                const TileCoord tcd = decode(p, tile);
-                for (int ch = 0; ch < p.nchunks; ++ch, ++seq) {
-                    const int b = seq & 1;
-                    if (!wait_bounded(bar_hempty + 8 * b, ((seq >> 1) & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    pending[b] = false;  // the producers consumed its previous box
-                    tc::mbar_arrive_expect_tx(bar_hfull + 8 * b, (uint32_t)G::HALO * 4u);
-                    tma_load_4d(smem_u32(halo + b * G::HALO), &x_map, tcd.tx * G::WC, tcd.py * P, ch * CCH, tcd.n,
-                                bar_hfull + 8 * b);
-                    pending[b] = true;
-                }
-            }
-            if (!ok) {
-                // After an abort, wait (bounded) for boxes still in flight.
-                for (int b = 0; b < 2; ++b) {
-                    if (!pending[b]) continue;
-                    const int last = seq - 1 - ((seq - 1 - b) & 1);  // latest sequence number on buffer b
-                    const unsigned long long t0 = globaltimer();
-                    while (last >= 0 && !mbar_try_wait(bar_hfull + 8 * b, (last >> 1) & 1)) {
-                        if (globaltimer() - t0 > kWaitLimitNs) break;
-                    }
-                }
-            }
-        }
-        __syncwarp();
+        tma_halo_warp<P>(p, x_map, halo, bar_hfull, bar_hempty, abort_flag, lane);
     } else if (warp == MMA_WARP || warp == MMA_WARP2) {
         // --------------------------------------------------------- MMA issuers
         // Two issuing threads, one for the even and one for the odd tiles of this
@@ -488,119 +639,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc_kernel(const Params p, 
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ epilogue
-        // Drain warps (one per TMEM lane quarter) copy a finished accumulator
-        // into one of two transposed buffers and release it at once; pool warps
-        // then reduce that buffer.  Pooling of one tile overlaps the drain of
-        // the next, so the epilogue's rate is the slower of the two halves.
-        int abuf = 0, local = 0;
-        uint32_t aphase = 0;
-        if (warp >= DRAIN_WARP0 && warp < DRAIN_WARP0 + 4) {
-            const int q = warp & 3;  // TMEM lane quarter of this warp
-            const int mrow = 32 * q + lane;
-            for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
-                const int buf = abuf;
-                const uint32_t bphase = aphase;
-                if (++abuf == p.nacc) {
-                    abuf = 0;
-                    aphase ^= 1u;
-                }
-                const int tb = local & 1;
-                const uint32_t tphase = (local >> 1) & 1;
-                int ok = 1;
-                if (lane == 0) {
-                    ok = wait_bounded(bar_accfull + 8 * buf, bphase, abort_flag) &&
-                         wait_bounded(bar_tempty + 8 * tb, tphase ^ 1, abort_flag);
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                tc_fence_after();  // TMEM loads after the MMAs lane 0 saw complete
-                float* tbw = tbuf + tb * NP * TP;
-                const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * NP);
-                for (int cb = 0; cb < NP / 16; cb += 2) {  // two TMEM loads per wait
-                    uint32_t v[16], u[16];
-                    const bool two = cb + 1 < NP / 16;
-                    tmem_ld16(taddr + (uint32_t)(16 * cb), v);
-                    if (two) tmem_ld16(taddr + (uint32_t)(16 * (cb + 1)), u);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) tbw[(16 * cb + j) * TP + mrow] = __uint_as_float(v[j]);
-                    if (two) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) tbw[(16 * (cb + 1) + j) * TP + mrow] = __uint_as_float(u[j]);
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(bar_accempty + 8 * buf);  // accumulator free for the MMA
-                    mbar_arrive(bar_tfull + 8 * tb);      // this quarter of the buffer is written
-                }
-            }
-        } else {
-            const int ptid = threadIdx.x - 32 * POOL_WARP0;  // 0..255
-            const float inv_area = 1.f / (float)(P * P);
-            const float inv_cout = 1.f / (float)p.Cout;
-            float acc = 0.f;
-            int cur = -1;
-            auto flush = [&]() {
-                float s = acc;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                if (lane == 0 && cur >= 0) atomicAdd(p.out + cur, s);
-                acc = 0.f;
-            };
-            for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
-                const int tb = local & 1;
-                const uint32_t tphase = (local >> 1) & 1;
-                int ok = 1;
-                if (lane == 0) ok = wait_bounded(bar_tfull + 8 * tb, tphase, abort_flag) ? 1 : 0;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                // every lane acquires the drain warps' stores (returns at once)
-                for (int spin = 0; !mbar_try_wait(bar_tfull + 8 * tb, tphase) && spin < (1 << 20); ++spin) {
-                }
-                const TileCoord tcd = decode(p, tile);
-                if (MODE != kTap && tcd.n != cur) {
-                    flush();
-                    cur = tcd.n;
-                }
-                const float* tbr = tbuf + tb * NP * TP;
-                const int nval = G::WPT * p.Cout;
-#pragma unroll 2
-                for (int v = ptid; v < nval; v += NPOOL) {
-                    // j = v / Cout exactly: (v + 1/2) / Cout is at least 1/(2 Cout) away
-                    // from an integer and v < 2^14, far inside fp32 precision.
-                    const int j = (int)(((float)v + 0.5f) * inv_cout), co = v - j * p.Cout;
-                    const int px = tcd.tx * G::WPT + j;
-                    if (px >= p.PW) continue;
-                    const float* tb4 = tbr + co * TP + j * P;
-                    float s = 0.f;
-#pragma unroll
-                    for (int rr = 0; rr < P; ++rr) {
-                        if constexpr (P % 4 == 0) {
-#pragma unroll
-                            for (int dc = 0; dc < P; dc += 4) {
-                                const float4 f = *reinterpret_cast<const float4*>(tb4 + rr * G::WC + dc);
-                                s += (f.x + f.y) + (f.z + f.w);
-                            }
-                        } else {
-#pragma unroll
-                            for (int dc = 0; dc < P; ++dc) s += tb4[rr * G::WC + dc];
-                        }
-                    }
-                    const float pooled = s * inv_area + bias_s[co];
-                    if (MODE == kTap) {
-                        p.out[(((size_t)tcd.n * p.Cout + co) * p.PH + tcd.py) * p.PW + px] = pooled;
-                    } else {
-                        acc += __fdividef(1.f, 1.f + __expf(-pooled));  // sigmoid; 0 once exp overflows
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_tempty + 8 * tb);  // this warp is done with the buffer
-            }
-            if (MODE != kTap) flush();
-        }
+        epilogue_warps<P, MODE>(p, tbuf, bias_s, tmem, bar_accfull, bar_accempty, bar_tfull, bar_tempty, abort_flag,
+                                warp, lane);
     }
 
     tc_fence_before();
@@ -669,24 +709,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc4_kernel(const Params p,
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
 
-    // Weights as the B operand, split into TF32 hi/lo: element (co, k) with
-    // k = 72 * chunk + e, e = 9 * (ci mod 8) + 3 * ky + kx, sits in 128-byte K
-    // block 3 * chunk + e / 32 (blocks of NP rows), row co, swizzled 16-byte
-    // chunk (e mod 32) / 4.  Every chunk starts a K block, so the descriptors of
-    // chunk c are those of chunk 0 moved by c * 3 blocks.
-    const int ktot = KCH * p.nchunks;
-    for (int idx = threadIdx.x; idx < NP * ktot; idx += NTHREADS) {
-        const int co = idx / ktot, k = idx - co * ktot;
-        const int ch = k / KCH, e = k - ch * KCH;
-        const int ci = ch * CCH + e / 9, t = e % 9;
-        const float v = (co < p.Cout && ci < p.Cin) ? __ldg(p.w + ((size_t)co * p.Cin + ci) * 9 + t) : 0.f;
-        const float hi = tf32_round(v);
-        const int a = 3 * ch + (e >> 5), kin = e & 31;
-        const uint32_t off = (uint32_t)a * NP * 128u + sw128_off(co, kin >> 2) + (uint32_t)(kin & 3) * 4u;
-        *reinterpret_cast<float*>(smem + L.b_hi + off) = hi;
-        *reinterpret_cast<float*>(smem + L.b_lo + off) = v - hi;
-    }
-    for (int i = threadIdx.x; i < NP; i += NTHREADS) bias_s[i] = i < p.Cout ? __ldg(p.b + i) : 0.f;
+    stage_weights<P>(p, smem, L, bias_s);
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // weights visible to the tensor core
     tc_fence_before();
     __syncthreads();
@@ -772,41 +795,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc4_kernel(const Params p,
             }
         }
     } else if (warp == TMA_WARP) {
-        // -------------------------------------------------------- TMA issuer
-        // One box [8 channels][P + 2 rows][HP columns] per (tile, chunk) lands
-        // in the halo layout itself; rows, columns and channels outside x read 0.
-        if (p.use_tma && lane == 0) {
-            int seq = 0;
-            bool pending[2] = {false, false};
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
-                const TileCoord tcd = decode(p, tile);
-                for (int ch = 0; ch < p.nchunks; ++ch, ++seq) {
-                    const int b = seq & 1;
-                    if (!wait_bounded(bar_hempty + 8 * b, ((seq >> 1) & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    pending[b] = false;  // the producers consumed its previous box
-                    tc::mbar_arrive_expect_tx(bar_hfull + 8 * b, (uint32_t)G::HALO * 4u);
-                    tma_load_4d(smem_u32(halo + b * G::HALO), &x_map, tcd.tx * G::WC, tcd.py * P, ch * CCH, tcd.n,
-                                bar_hfull + 8 * b);
-                    pending[b] = true;
-                }
-            }
-            if (!ok) {
-                // After an abort, wait (bounded) for boxes still in flight.
-                for (int b = 0; b < 2; ++b) {
-                    if (!pending[b]) continue;
-                    const int last = seq - 1 - ((seq - 1 - b) & 1);  // latest sequence number on buffer b
-                    const unsigned long long t0 = globaltimer();
-                    while (last >= 0 && !mbar_try_wait(bar_hfull + 8 * b, (last >> 1) & 1)) {
-                        if (globaltimer() - t0 > kWaitLimitNs) break;
-                    }
-                }
-            }
-        }
-        __syncwarp();
+        tma_halo_warp<P>(p, x_map, halo, bar_hfull, bar_hempty, abort_flag, lane);
     } else if (warp == MMA_WARP || warp == MMA_WARP2) {
         // --------------------------------------------------------- MMA issuers
         // Two issuing threads, one for the even and one for the odd tiles of this
@@ -890,119 +879,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc4_kernel(const Params p,
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ epilogue
-        // Drain warps (one per TMEM lane quarter) copy a finished accumulator
-        // into one of two transposed buffers and release it at once; pool warps
-        // then reduce that buffer.  Pooling of one tile overlaps the drain of
-        // the next, so the epilogue's rate is the slower of the two halves.
-        int abuf = 0, local = 0;
-        uint32_t aphase = 0;
-        if (warp >= DRAIN_WARP0 && warp < DRAIN_WARP0 + 4) {
-            const int q = warp & 3;  // TMEM lane quarter of this warp
-            const int mrow = 32 * q + lane;
-            for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
-                const int buf = abuf;
-                const uint32_t bphase = aphase;
-                if (++abuf == p.nacc) {
-                    abuf = 0;
-                    aphase ^= 1u;
-                }
-                const int tb = local & 1;
-                const uint32_t tphase = (local >> 1) & 1;
-                int ok = 1;
-                if (lane == 0) {
-                    ok = wait_bounded(bar_accfull + 8 * buf, bphase, abort_flag) &&
-                         wait_bounded(bar_tempty + 8 * tb, tphase ^ 1, abort_flag);
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                tc_fence_after();  // TMEM loads after the MMAs lane 0 saw complete
-                float* tbw = tbuf + tb * NP * TP;
-                const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * NP);
-                for (int cb = 0; cb < NP / 16; cb += 2) {  // two TMEM loads per wait
-                    uint32_t v[16], u[16];
-                    const bool two = cb + 1 < NP / 16;
-                    tmem_ld16(taddr + (uint32_t)(16 * cb), v);
-                    if (two) tmem_ld16(taddr + (uint32_t)(16 * (cb + 1)), u);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) tbw[(16 * cb + j) * TP + mrow] = __uint_as_float(v[j]);
-                    if (two) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) tbw[(16 * (cb + 1) + j) * TP + mrow] = __uint_as_float(u[j]);
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(bar_accempty + 8 * buf);  // accumulator free for the MMA
-                    mbar_arrive(bar_tfull + 8 * tb);      // this quarter of the buffer is written
-                }
-            }
-        } else {
-            const int ptid = threadIdx.x - 32 * POOL_WARP0;  // 0..255
-            const float inv_area = 1.f / (float)(P * P);
-            const float inv_cout = 1.f / (float)p.Cout;
-            float acc = 0.f;
-            int cur = -1;
-            auto flush = [&]() {
-                float s = acc;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                if (lane == 0 && cur >= 0) atomicAdd(p.out + cur, s);
-                acc = 0.f;
-            };
-            for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
-                const int tb = local & 1;
-                const uint32_t tphase = (local >> 1) & 1;
-                int ok = 1;
-                if (lane == 0) ok = wait_bounded(bar_tfull + 8 * tb, tphase, abort_flag) ? 1 : 0;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                // every lane acquires the drain warps' stores (returns at once)
-                for (int spin = 0; !mbar_try_wait(bar_tfull + 8 * tb, tphase) && spin < (1 << 20); ++spin) {
-                }
-                const TileCoord tcd = decode(p, tile);
-                if (MODE != kTap && tcd.n != cur) {
-                    flush();
-                    cur = tcd.n;
-                }
-                const float* tbr = tbuf + tb * NP * TP;
-                const int nval = G::WPT * p.Cout;
-#pragma unroll 2
-                for (int v = ptid; v < nval; v += NPOOL) {
-                    // j = v / Cout exactly: (v + 1/2) / Cout is at least 1/(2 Cout) away
-                    // from an integer and v < 2^14, far inside fp32 precision.
-                    const int j = (int)(((float)v + 0.5f) * inv_cout), co = v - j * p.Cout;
-                    const int px = tcd.tx * G::WPT + j;
-                    if (px >= p.PW) continue;
-                    const float* tb4 = tbr + co * TP + j * P;
-                    float s = 0.f;
-#pragma unroll
-                    for (int rr = 0; rr < P; ++rr) {
-                        if constexpr (P % 4 == 0) {
-#pragma unroll
-                            for (int dc = 0; dc < P; dc += 4) {
-                                const float4 f = *reinterpret_cast<const float4*>(tb4 + rr * G::WC + dc);
-                                s += (f.x + f.y) + (f.z + f.w);
-                            }
-                        } else {
-#pragma unroll
-                            for (int dc = 0; dc < P; ++dc) s += tb4[rr * G::WC + dc];
-                        }
-                    }
-                    const float pooled = s * inv_area + bias_s[co];
-                    if (MODE == kTap) {
-                        p.out[(((size_t)tcd.n * p.Cout + co) * p.PH + tcd.py) * p.PW + px] = pooled;
-                    } else {
-                        acc += __fdividef(1.f, 1.f + __expf(-pooled));  // sigmoid; 0 once exp overflows
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_tempty + 8 * tb);  // this warp is done with the buffer
-            }
-            if (MODE != kTap) flush();
-        }
+        epilogue_warps<P, MODE>(p, tbuf, bias_s, tmem, bar_accfull, bar_accempty, bar_tfull, bar_tempty, abort_flag,
+                                warp, lane);
     }
 
     tc_fence_before();
