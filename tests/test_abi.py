@@ -146,9 +146,11 @@ def test_auto_algo_conv2d(lib):
     q = lib.fcv_conv2d_auto_algo
     assert q(128, 8, 384, 384, 64, 4, ctypes.byref(a)) == OK and a.value == 12  # the full-size workload
     for pool in (1, 2, 8):
-        assert q(2, 8, 40, 40, 16, pool, ctypes.byref(a)) == OK and a.value == 12
-    assert q(2, 3, 40, 40, 32, 4, ctypes.byref(a)) == OK and a.value == 10      # Cin < 4, Cout <= 32: FMA
-    assert q(2, 3, 40, 40, 48, 4, ctypes.byref(a)) == OK and a.value == 12
+        assert q(2, 8, 40, 40, 48, pool, ctypes.byref(a)) == OK and a.value == 12
+    assert q(2, 3, 40, 40, 32, 4, ctypes.byref(a)) == OK and a.value == 10      # Cin < 4: FMA
+    assert q(2, 3, 40, 40, 48, 4, ctypes.byref(a)) == OK and a.value == 10
+    assert q(2, 16, 40, 40, 32, 4, ctypes.byref(a)) == OK and a.value == 10     # Cout <= 32: FMA
+    assert q(2, 4, 40, 40, 33, 4, ctypes.byref(a)) == OK and a.value == 12      # smallest tensor-core layer
     assert q(2, 8, 40, 40, 16, 3, ctypes.byref(a)) == OK and a.value == 10      # pool 3: FMA path
     assert q(2, 8, 40, 40, 128, 4, ctypes.byref(a)) == OK and a.value == 10     # Cout > 112: FMA path
     assert q(2, 3, 40, 40, 16, 9, ctypes.byref(a)) == UNSUPPORTED
