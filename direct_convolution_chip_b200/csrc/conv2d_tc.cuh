@@ -920,18 +920,6 @@ inline bool conv2d_tc_supported(int Cin, int Cout, int P)
     return s <= (uint32_t)c2tc::SMEM_LIMIT;
 }
 
-// What AUTO prefers: the tensor-core kernel where it applies, Cin >= 4 and
-// Cout > 32.  Below that the FMA kernel measured faster on x[16,Cin,509,509],
-// pool 2 and 4: every tile costs the tensor-core kernel the same 27 MMAs and
-// A-operand build whatever Cout is, while the FMA kernel's time scales with
-// Cin * Cout (Cout 32: 880 vs 1,069 us at Cin 16, 1,709 vs 2,280 us at Cin 32;
-// Cin 3: 338 vs 451 us at Cout 48; Cout 48 at Cin 8: 489 vs 830 us the other
-// way).
-inline bool conv2d_tc_preferred(int Cin, int Cout, int P)
-{
-    return conv2d_tc_supported(Cin, Cout, P) && Cin >= 4 && Cout > 32;
-}
-
 template <int P, int MODE>
 inline int launch_conv2d_tc_p(c2tc::Params prm, int N, int grid, cudaStream_t stream)
 {

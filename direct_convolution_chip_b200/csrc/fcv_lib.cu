@@ -71,6 +71,28 @@ int check_conv1d(const float* x, const float* dw, const float* pw, const float* 
     return FCV_OK;
 }
 
+// Smallest FMA-kernel grid (CTAs) at which AUTO lets it take a narrow layer:
+// one CTA per SM of a B200.
+constexpr long long kConv2dFmaMinCtas = 148;
+
+// What AUTO runs for op A: the tensor-core kernel where it applies, unless
+// the layer is narrow (Cin < 4 or Cout <= 32) and the FMA kernel's grid fills
+// at least one wave.  Every tile costs the tensor-core kernel the same 27 MMAs
+// and A-operand build whatever Cout is, while the FMA kernel's time scales
+// with Cin * Cout: on x[16,Cin,509,509], pool 4, FMA measured 880 vs 1,069 us
+// at Cin 16, Cout 32, 1,709 vs 2,280 at Cin 32, Cout 32 and 338 vs 451 at
+// Cin 3, Cout 48, and the other way 830 vs 489 at Cin 8, Cout 48.  Below one
+// wave the FMA kernel leaves most SMs idle: x[2,8,64,64], Cout 16, pool 4 runs
+// 34.8 us on its 8 CTAs against 10.3 us on the tensor cores.
+bool conv2d_auto_tc(int N, int Cin, int Cout, int pool, int PH, int PW)
+{
+    if (!fcv::conv2d_tc_supported(Cin, Cout, pool)) return false;
+    if (Cin >= 4 && Cout > 32) return true;
+    int ty = 0, tx = 0, cb = 0;
+    if (!fcv::conv2d_grid(pool, PH, PW, Cout, &ty, &tx, &cb)) return true;
+    return (long long)N * ty * tx * cb < kConv2dFmaMinCtas;
+}
+
 int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin, int H, int W,
                   int Cout, int pool, float* out, int algo, bool tap, void* stream)
 {
@@ -96,7 +118,7 @@ int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin
         return tap ? fcv::launch_conv2d_poolfirst<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
                    : fcv::launch_conv2d_poolfirst<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
     }
-    if (algo == FCV_ALGO_AUTO && fcv::conv2d_tc_preferred(Cin, Cout, pool)) {
+    if (algo == FCV_ALGO_AUTO && conv2d_auto_tc(N, Cin, Cout, pool, PH, PW)) {
         return tap ? fcv::launch_conv2d_tc<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
                    : fcv::launch_conv2d_tc<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
     }
@@ -209,7 +231,8 @@ int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* 
     if (N < 0 || Cin < 1 || Cout < 1 || H < 3 || W < 3 || pool < 1) return FCV_ERR_INVALID_ARG;
     if (!mul_ok(N, Cin, H, W) || !mul_ok(N, Cout, H, W)) return FCV_ERR_INVALID_ARG;
     if (pool > 8) return FCV_ERR_UNSUPPORTED;
-    *algo = fcv::conv2d_tc_preferred(Cin, Cout, pool) ? FCV_CONV2D_TC_3XTF32 : FCV_CONV2D_DIRECT;
+    const int PH = (H - 2) / pool, PW = (W - 2) / pool;
+    *algo = conv2d_auto_tc(N, Cin, Cout, pool, PH, PW) ? FCV_CONV2D_TC_3XTF32 : FCV_CONV2D_DIRECT;
     return FCV_OK;
 }
 

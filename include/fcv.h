@@ -61,9 +61,10 @@ typedef enum {
  * fastest path valid for the shape and pointers (fcv_conv2d_auto_algo and
  * fcv_dwsep_conv1d_auto_algo report which).  For op A it is always the direct
  * method (every conv output is computed): on tensor cores where
- * FCV_CONV2D_TC_3XTF32 covers the shape and Cin >= 4 and Cout > 32 (narrower
- * layers measured faster on FP32 FMA), else on FP32 FMA; the pool-first
- * identity is never chosen automatically. */
+ * FCV_CONV2D_TC_3XTF32 covers the shape, except narrow layers (Cin < 4 or
+ * Cout <= 32) whose FP32-FMA grid fills at least one wave of 148 CTAs (there
+ * FP32 FMA measured faster), else on FP32 FMA; the pool-first identity is
+ * never chosen automatically. */
 typedef enum {
     FCV_ALGO_AUTO = 0,
     /* op A */

@@ -147,10 +147,13 @@ def test_auto_algo_conv2d(lib):
     assert q(128, 8, 384, 384, 64, 4, ctypes.byref(a)) == OK and a.value == 12  # the full-size workload
     for pool in (1, 2, 8):
         assert q(2, 8, 40, 40, 48, pool, ctypes.byref(a)) == OK and a.value == 12
-    assert q(2, 3, 40, 40, 32, 4, ctypes.byref(a)) == OK and a.value == 10      # Cin < 4: FMA
-    assert q(2, 3, 40, 40, 48, 4, ctypes.byref(a)) == OK and a.value == 10
-    assert q(2, 16, 40, 40, 32, 4, ctypes.byref(a)) == OK and a.value == 10     # Cout <= 32: FMA
-    assert q(2, 4, 40, 40, 33, 4, ctypes.byref(a)) == OK and a.value == 12      # smallest tensor-core layer
+    # narrow layers (Cin < 4 or Cout <= 32): FMA once its grid fills a wave of 148 CTAs
+    assert q(16, 3, 509, 509, 32, 4, ctypes.byref(a)) == OK and a.value == 10
+    assert q(16, 3, 509, 509, 48, 4, ctypes.byref(a)) == OK and a.value == 10
+    assert q(16, 16, 509, 509, 32, 4, ctypes.byref(a)) == OK and a.value == 10
+    assert q(2, 3, 40, 40, 32, 4, ctypes.byref(a)) == OK and a.value == 12      # 8 FMA CTAs: tensor cores
+    assert q(2, 8, 64, 64, 16, 4, ctypes.byref(a)) == OK and a.value == 12      # the small workload
+    assert q(2, 4, 40, 40, 33, 4, ctypes.byref(a)) == OK and a.value == 12      # Cin >= 4, Cout > 32
     assert q(2, 8, 40, 40, 16, 3, ctypes.byref(a)) == OK and a.value == 10      # pool 3: FMA path
     assert q(2, 8, 40, 40, 128, 4, ctypes.byref(a)) == OK and a.value == 10     # Cout > 112: FMA path
     assert q(2, 3, 40, 40, 16, 9, ctypes.byref(a)) == UNSUPPORTED
