@@ -71,19 +71,21 @@ int check_conv1d(const float* x, const float* dw, const float* pw, const float* 
     return FCV_OK;
 }
 
-// Smallest FMA-kernel grid (CTAs) at which AUTO lets it take a narrow layer:
-// one CTA per SM of a B200.
-constexpr long long kConv2dFmaMinCtas = 148;
+// Smallest FMA-kernel grid (CTAs) at which AUTO lets it take a narrow layer.
+// Measured on x[16,Cin,130,130], Cout 32, pool 4 (128 FMA CTAs): FMA 20.5 vs
+// 40.9 us at Cin 3 and 73.8 vs 78.0 us at Cin 16; below that the tensor-core
+// kernel, which spreads any grid over every SM, wins.
+constexpr long long kConv2dFmaMinCtas = 128;
 
 // What AUTO runs for op A: the tensor-core kernel where it applies, unless
 // the layer is narrow (Cin < 4 or Cout <= 32) and the FMA kernel's grid fills
-// at least one wave.  Every tile costs the tensor-core kernel the same 27 MMAs
+// at least kConv2dFmaMinCtas CTAs.  Every tile costs the tensor-core kernel the same 27 MMAs
 // and A-operand build whatever Cout is, while the FMA kernel's time scales
 // with Cin * Cout: on x[16,Cin,509,509], pool 4, FMA measured 880 vs 1,069 us
 // at Cin 16, Cout 32, 1,709 vs 2,280 at Cin 32, Cout 32 and 338 vs 451 at
-// Cin 3, Cout 48, and the other way 830 vs 489 at Cin 8, Cout 48.  Below one
-// wave the FMA kernel leaves most SMs idle: x[2,8,64,64], Cout 16, pool 4 runs
-// 34.8 us on its 8 CTAs against 10.3 us on the tensor cores.
+// Cin 3, Cout 48, and the other way 830 vs 489 at Cin 8, Cout 48.  On a small
+// grid the FMA kernel leaves most SMs idle: x[2,8,64,64], Cout 16, pool 4 runs
+// 34.8 us on its 4 CTAs against 10.3 us on the tensor cores.
 bool conv2d_auto_tc(int N, int Cin, int Cout, int pool, int PH, int PW)
 {
     if (!fcv::conv2d_tc_supported(Cin, Cout, pool)) return false;

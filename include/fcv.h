@@ -62,9 +62,9 @@ typedef enum {
  * fcv_dwsep_conv1d_auto_algo report which).  For op A it is always the direct
  * method (every conv output is computed): on tensor cores where
  * FCV_CONV2D_TC_3XTF32 covers the shape, except narrow layers (Cin < 4 or
- * Cout <= 32) whose FP32-FMA grid fills at least one wave of 148 CTAs (there
- * FP32 FMA measured faster), else on FP32 FMA; the pool-first identity is
- * never chosen automatically. */
+ * Cout <= 32) whose FP32-FMA grid has at least 128 CTAs (there FP32 FMA
+ * measured faster), else on FP32 FMA; the pool-first identity is never chosen
+ * automatically. */
 typedef enum {
     FCV_ALGO_AUTO = 0,
     /* op A */

@@ -147,7 +147,9 @@ def test_auto_algo_conv2d(lib):
     assert q(128, 8, 384, 384, 64, 4, ctypes.byref(a)) == OK and a.value == 12  # the full-size workload
     for pool in (1, 2, 8):
         assert q(2, 8, 40, 40, 48, pool, ctypes.byref(a)) == OK and a.value == 12
-    # narrow layers (Cin < 4 or Cout <= 32): FMA once its grid fills a wave of 148 CTAs
+    # narrow layers (Cin < 4 or Cout <= 32): FMA once its grid has 128 CTAs
+    assert q(16, 3, 130, 130, 32, 4, ctypes.byref(a)) == OK and a.value == 10   # exactly 128
+    assert q(15, 3, 130, 130, 32, 4, ctypes.byref(a)) == OK and a.value == 12   # 120
     assert q(16, 3, 509, 509, 32, 4, ctypes.byref(a)) == OK and a.value == 10
     assert q(16, 3, 509, 509, 48, 4, ctypes.byref(a)) == OK and a.value == 10
     assert q(16, 16, 509, 509, 32, 4, ctypes.byref(a)) == OK and a.value == 10
