@@ -715,8 +715,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) conv2d_tc4_kernel(const Params p,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    // Accumulators: p.nacc buffers of NP columns (3 when they fit next to the two
-    // A stages, else 2), used round robin: buffer abuf, phase aphase.
+    // Accumulators: p.nacc buffers of NP columns (3 when they fit next to the
+    // four sub-chunk A stages, else 2), used round robin: buffer abuf, phase aphase.
     const uint32_t a_col0 = (uint32_t)(p.nacc * NP);  // first A-stage column (4 stages of SUB_COLS)
 
     if (warp < 8) {
