@@ -10,9 +10,12 @@ used in place (they must be fp32 and contiguous).  CPU tensors are accepted
 too: they are copied to the current device (asynchronously when pinned), the
 kernel runs, and the result is copied back into `out` when a CPU tensor is
 given (pinned for an asynchronous copy), else into a new pinned CPU tensor --
-the path an application with host-resident data takes.
+the path an application with host-resident data takes.  A `stream` argument
+orders all of it (copies, allocations, kernel) on that stream.
 """
 import ctypes
+import functools
+import inspect
 import os
 
 import torch
@@ -94,6 +97,24 @@ def version() -> int:
     return load().fcv_version()
 
 
+def _on_stream(fn):
+    """Run a binding call with its `stream` argument (when given) as torch's
+    current stream, so that everything the call enqueues -- the copies of CPU
+    inputs to the device, the buffers it allocates (the caching allocator ties
+    them to that stream) and the kernel -- is ordered on that one stream."""
+    pos = list(inspect.signature(fn).parameters).index("stream")
+
+    @functools.wraps(fn)
+    def call(*args, **kw):
+        stream = kw.get("stream", args[pos] if len(args) > pos else None)
+        if stream is None:
+            return fn(*args, **kw)
+        with torch.cuda.stream(stream):
+            return fn(*args, **kw)
+
+    return call
+
+
 def _stream_ptr(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
@@ -153,6 +174,7 @@ def conv2d_out_shape(H, W, pool):
     return (H - 2) // pool, (W - 2) // pool
 
 
+@_on_stream
 def conv2d_pool_sigmoid_sum(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None):
     """out[N] = sum over (C, PH, PW) of sigmoid(avgpool_pool(conv3x3(x, w) + b))."""
     lib = load()
@@ -180,6 +202,7 @@ def conv2d_workspace_bytes(N, Cin, H, W, Cout, pool) -> int:
     return v.value
 
 
+@_on_stream
 def conv2d_pool_sigmoid_sum_det(x, w, b, pool, out=None, workspace=None, stream=None):
     """Bitwise-reproducible variant of conv2d_pool_sigmoid_sum.
 
@@ -206,6 +229,7 @@ def conv2d_pool_sigmoid_sum_det(x, w, b, pool, out=None, workspace=None, stream=
     return _result(out, host, stream, out_host)
 
 
+@_on_stream
 def conv2d_pool_tap(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None):
     """Pooled pre-sigmoid values [N, Cout, PH, PW] of the same fused kernel."""
     lib = load()
@@ -230,6 +254,7 @@ def conv1d_out_len(T, K, stride, pad):
     return (T + 2 * pad - K) // stride + 1
 
 
+@_on_stream
 def dwsep_conv1d(x, dw, pw, bias, stride, pad, out=None, algo=ALGO_AUTO, stream=None):
     """out[N, O, To] = pointwise(depthwise(x)) + bias; bias may be None."""
     lib = load()

@@ -177,3 +177,31 @@ def test_auto_algo_conv1d(lib):
     assert q(X, PW, 2, 64, 1000, 128, 33, 1, 4, ctypes.byref(a)) == UNSUPPORTED           # K > 32
     assert q(X, PW, 2, 64, 1000, 128, 9, 1, -1, ctypes.byref(a)) == INVALID
     assert q(X, PW, 2, 64, 1000, 128, 9, 1, 4, None) == INVALID
+
+
+def test_binding_calls_run_on_their_stream_argument(monkeypatch):
+    """The binding enters torch's stream context for a given `stream` (passed by
+    keyword or position), so host copies, allocations and the kernel share it;
+    without one it calls straight through."""
+    seen = []
+
+    class FakeStreamContext:
+        def __init__(self, stream):
+            self.stream = stream
+
+        def __enter__(self):
+            seen.append(self.stream)
+
+        def __exit__(self, *exc):
+            return False
+
+    monkeypatch.setattr(binding.torch.cuda, "stream", FakeStreamContext)
+
+    @binding._on_stream
+    def call(a, b=1, stream=None):
+        return a, b, stream
+
+    assert call(1) == (1, 1, None) and seen == []
+    assert call(1, 2, "s1") == (1, 2, "s1") and seen == ["s1"]
+    assert call(1, stream="s2") == (1, 1, "s2") and seen == ["s1", "s2"]
+    assert call(1, 3) == (1, 3, None) and seen == ["s1", "s2"]

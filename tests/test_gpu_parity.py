@@ -317,6 +317,22 @@ def test_host_tensors_through_public_api():
         fcv.dwsep_conv1d(x, dw, pw, bias, case.stride, case.pad, out=torch.empty((1,)))
 
 
+def test_host_tensors_on_a_side_stream():
+    """CPU inputs with stream=s and no stream context: the input copies, the
+    buffers the binding allocates and the kernel are all ordered on s."""
+    s = torch.cuda.Stream()
+    c2 = wl.CONV2D_SMALL
+    x2, w2, b2 = wl.conv2d_inputs(c2)
+    ref2 = oracle.conv2d_pool_sigmoid_sum(x2.numpy(), w2.numpy(), b2.numpy(), c2.P)
+    for _ in range(3):
+        out2 = fcv.conv2d_pool_sigmoid_sum(x2.pin_memory(), w2, b2, c2.P, stream=s)
+        assert_close(out2, ref2, "side-stream conv2d")
+    case = wl.CONV1D_SMALL
+    x, dw, pw, bias = wl.conv1d_inputs(case)
+    out = fcv.dwsep_conv1d(x.pin_memory(), dw, pw, bias, case.stride, case.pad, stream=s)
+    assert_close(out, oracle.dwsep_conv1d(x.numpy(), dw.numpy(), pw.numpy(), bias.numpy(), 1, 4), "side-stream conv1d")
+
+
 def test_empty_batch_through_binding():
     x = torch.zeros((0, 3, 10, 10), device="cuda")
     w = torch.zeros((4, 3, 3, 3), device="cuda")
