@@ -1,0 +1,240 @@
+"""CPU model of the mbarrier protocol of the tensor-core conv2d kernels.
+
+Every role of one CTA (TMA warp, producer warps, MMA issuers, the tensor core
+completing what they issued, drain and pool warps) is an agent that waits on
+and arrives at mbarriers with the parities and counts the kernels in
+csrc/conv2d_tc.cuh use.  The agents run in many random interleavings; for each
+shape of the work (tiles per CTA, input-channel chunks, accumulator buffers)
+the model checks:
+
+* no deadlock: some agent can always move until all have finished;
+* no stale wait: a parity wait only passes once the phase the agent needs has
+  really completed (an mbarrier answers from the parity of its current phase,
+  so a waiter two phases behind would pass on an old phase);
+* no early arrival: every arrival lands in the phase it belongs to;
+* no overwrite in use: a buffer (halo, A stage, accumulator, transposed
+  buffer) is written only after the readers of its previous contents have
+  released it.
+
+A tcgen05.commit arrives when the MMAs before it complete, which the model
+lets happen at any time after their issue, in issue order per issuing thread.
+"""
+import random
+
+import pytest
+
+
+class Barrier:
+    def __init__(self, name, count):
+        self.name, self.count = name, count
+        self.phase = 0       # index of the current (incomplete) phase
+        self.pending = 0
+
+    def passes(self, parity):
+        # mbarrier.try_wait.parity: true once the phase with this parity is the
+        # last completed one, i.e. the current phase has the other parity
+        return (self.phase & 1) != parity
+
+    def arrive(self, use, who):
+        assert use == self.phase, f"{who}: arrival for use {use} of {self.name} in phase {self.phase}"
+        self.pending += 1
+        if self.pending == self.count:
+            self.pending = 0
+            self.phase += 1
+
+
+class Sim:
+    """Barriers plus agents; an agent is a list of steps run in order:
+    ("wait", barrier, parity, phases that must be done, who),
+    ("arrive", barrier, use, arrivals, who),
+    ("issue", counter), ("issued", counter, k)  -- ordering of a commit after its issue,
+    ("owns", barrier, phases done, who)  -- a write that needs the buffer released."""
+
+    def __init__(self):
+        self.bars, self.agents, self.counters = {}, [], {}
+
+    def bar(self, name, count):
+        self.bars[name] = Barrier(name, count)
+
+    def can_run(self, st):
+        if st[0] == "wait":
+            _, name, parity, need, who = st
+            bar = self.bars[name]
+            if not bar.passes(parity):
+                return False
+            assert bar.phase >= need, (f"{who}: wait on {name} parity {parity} passed in phase "
+                                       f"{bar.phase}, needs {need} phases done")
+            return True
+        if st[0] == "issued":
+            return self.counters.get(st[1], 0) > st[2]
+        return True
+
+    def step(self, st):
+        if st[0] == "arrive":
+            _, name, use, n, who = st
+            for _ in range(n):
+                self.bars[name].arrive(use, who)
+        elif st[0] == "issue":
+            self.counters[st[1]] = self.counters.get(st[1], 0) + 1
+        elif st[0] == "owns":
+            _, name, need, who = st
+            assert self.bars[name].phase >= need, (f"{who}: writes the buffer of {name} with "
+                                                   f"{self.bars[name].phase} of {need} releases done")
+
+    def run(self, seed):
+        rng = random.Random(seed)
+        pcs = [0] * len(self.agents)
+        while True:
+            ready = [i for i, a in enumerate(self.agents) if pcs[i] < len(a) and self.can_run(a[pcs[i]])]
+            if not ready:
+                left = [a[pcs[i]] for i, a in enumerate(self.agents) if pcs[i] < len(a)]
+                assert not left, f"deadlock at {left}"
+                break
+            i = rng.choice(ready)
+            self.step(self.agents[i][pcs[i]])
+            pcs[i] += 1
+        for bar in self.bars.values():
+            assert bar.pending == 0, f"{bar.name}: {bar.pending} arrivals left over"
+
+
+def add_tma_and_epilogue(sim, T, C, A, hempty_count):
+    """TMA warp (halo ring of 2), drain warps (4) and pool warps (8), shared by both kernels."""
+    for h in range(2):
+        sim.bar(f"hfull{h}", 1)
+        sim.bar(f"hempty{h}", hempty_count)
+        sim.bar(f"tfull{h}", 4)
+        sim.bar(f"tempty{h}", 8)
+    for a in range(A):
+        sim.bar(f"accfull{a}", 1)
+        sim.bar(f"accempty{a}", 4)
+    tma = []
+    for seq in range(T * C):
+        b, k = seq & 1, seq >> 1
+        tma += [("wait", f"hempty{b}", (k & 1) ^ 1, k, "tma"), ("owns", f"hempty{b}", k, "tma"),
+                ("arrive", f"hfull{b}", k, 1, "tma")]
+    drain, pool = [], []
+    for t in range(T):
+        buf, rnd = t % A, t // A
+        tb, tk = t & 1, t >> 1
+        drain += [("wait", f"accfull{buf}", rnd & 1, rnd + 1, "drain"),
+                  ("wait", f"tempty{tb}", (tk & 1) ^ 1, tk, "drain"),
+                  ("owns", f"tempty{tb}", tk, "drain"),
+                  ("arrive", f"accempty{buf}", rnd, 4, "drain"),
+                  ("arrive", f"tfull{tb}", tk, 4, "drain")]
+        pool += [("wait", f"tfull{tb}", tk & 1, tk + 1, "pool"), ("arrive", f"tempty{tb}", tk, 8, "pool")]
+    sim.agents += [tma, drain, pool]
+
+
+def add_issuers(sim, T, C, A, subs, stage_of):
+    """Two MMA issuers (even / odd tiles); each waits "A full" of every
+    sub-chunk of every chunk, and its commits (stage free per sub-chunk,
+    accumulator full per tile) complete later, in order."""
+    for par in range(2):
+        issue, complete = [], []
+        n = 0
+        for t in range(par, T, 2):
+            for ch in range(C):
+                use = (t >> 1) * C + ch
+                for sub in range(subs):
+                    stage = stage_of(t, sub)
+                    issue.append(("wait", f"afull{stage}", use & 1, use + 1, f"issuer{par}"))
+                    if ch == 0 and sub == 0:
+                        issue.append(("owns", f"accempty{t % A}", t // A, f"issuer{par}"))
+                    issue.append(("issue", par))
+                    complete += [("issued", par, n), ("arrive", f"aempty{stage}", use, 1, f"mma{par}")]
+                    n += 1
+            complete.append(("arrive", f"accfull{t % A}", t // A, 1, f"mma{par}"))
+        sim.agents += [issue, complete]
+
+
+def sub_chunk_kernel(T, C, A, stage_of=lambda t, g: 2 * (t & 1) + g):
+    """conv2d_tc4_kernel: two producer groups of 4 warps, one per K sub-chunk;
+    A stage 2 * (tile parity) + sub-chunk; group 0 also waits for the
+    accumulator before a tile's first chunk."""
+    sim = Sim()
+    for s in range(4):
+        sim.bar(f"afull{s}", 4)
+        sim.bar(f"aempty{s}", 1)
+    add_tma_and_epilogue(sim, T, C, A, hempty_count=8)
+    for g in range(2):
+        st = []
+        for seq in range(T * C):
+            t, ch = divmod(seq, C)
+            stage, use = stage_of(t, g), (t >> 1) * C + ch
+            b, k = seq & 1, seq >> 1
+            st += [("wait", f"aempty{stage}", (use & 1) ^ 1, use, f"group{g}"),
+                   ("wait", f"hfull{b}", k & 1, k + 1, f"group{g}")]
+            if g == 0 and ch == 0:
+                st.append(("wait", f"accempty{t % A}", ((t // A) & 1) ^ 1, t // A, f"group{g}"))
+            st += [("owns", f"aempty{stage}", use, f"group{g}"),
+                   ("arrive", f"hempty{b}", k, 4, f"group{g}"), ("arrive", f"afull{stage}", use, 4, f"group{g}")]
+        sim.agents.append(st)
+    add_issuers(sim, T, C, A, 2, stage_of)
+    return sim
+
+
+def full_chunk_kernel(T, C, A):
+    """conv2d_tc_kernel: 8 producer warps (thread 0 waits for all) build a
+    whole chunk into A stage (tile parity); before a tile's first chunk they
+    also wait for its accumulator."""
+    sim = Sim()
+    for s in range(2):
+        sim.bar(f"afull{s}", 8)
+        sim.bar(f"aempty{s}", 1)
+    add_tma_and_epilogue(sim, T, C, A, hempty_count=8)
+    st = []
+    for seq in range(T * C):
+        t, ch = divmod(seq, C)
+        stage, use = t & 1, (t >> 1) * C + ch
+        b, k = seq & 1, seq >> 1
+        st.append(("wait", f"aempty{stage}", (use & 1) ^ 1, use, "producers"))
+        if ch == 0:
+            st.append(("wait", f"accempty{t % A}", ((t // A) & 1) ^ 1, t // A, "producers"))
+        st += [("wait", f"hfull{b}", k & 1, k + 1, "producers"), ("owns", f"aempty{stage}", use, "producers"),
+               ("arrive", f"hempty{b}", k, 8, "producers"), ("arrive", f"afull{stage}", use, 8, "producers")]
+    sim.agents.append(st)
+    add_issuers(sim, T, C, A, 1, lambda t, sub: t & 1)
+    return sim
+
+
+SHAPES = [(T, C, A) for T in (1, 2, 3, 4, 7) for C in (1, 2, 3) for A in (2, 3)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "T%d_C%d_A%d" % s)
+def test_sub_chunk_kernel_protocol(shape):
+    for seed in range(30):
+        sub_chunk_kernel(*shape).run(seed)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "T%d_C%d_A%d" % s)
+def test_full_chunk_kernel_protocol(shape):
+    for seed in range(30):
+        full_chunk_kernel(*shape).run(seed)
+
+
+def test_model_catches_shared_stages():
+    """Plant the mistake the stage-per-tile-parity rule prevents: both issuers
+    (even and odd tiles) on the same two A stages, with the use count still
+    advancing every other tile.  The model must report it."""
+    failures = 0
+    for seed in range(50):
+        try:
+            sub_chunk_kernel(6, 2, 3, stage_of=lambda t, g: g).run(seed)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
+
+
+def test_model_catches_a_missing_accumulator_wait():
+    """Plant a data race: the producers stop waiting for the drained
+    accumulator, so an issuer may start a tile on one still being read."""
+    failures = 0
+    for seed in range(100):
+        sim = sub_chunk_kernel(7, 1, 2)
+        for a in sim.agents:
+            a[:] = [st for st in a if not (st[0] == "wait" and st[1].startswith("accempty"))]
+        try:
+            sim.run(seed)
+        except AssertionError as e:
+            failures += "releases done" in str(e)
+    assert failures > 0
