@@ -1,9 +1,9 @@
-"""CPU model of the mbarrier protocol of the tensor-core conv2d kernels.
+"""CPU model of the mbarrier protocol of the tensor-core kernels.
 
 Every role of one CTA (TMA warp, producer warps, MMA issuers, the tensor core
 completing what they issued, drain and pool warps) is an agent that waits on
 and arrives at mbarriers with the parities and counts the kernels in
-csrc/conv2d_tc.cuh use.  The agents run in many random interleavings; for each
+csrc/conv2d_tc.cuh (both conv2d kernels) and csrc/conv1d_tcx.cuh use.  The agents run in many random interleavings; for each
 shape of the work (tiles per CTA, input-channel chunks, accumulator buffers)
 the model checks:
 
@@ -197,6 +197,54 @@ def full_chunk_kernel(T, C, A):
     return sim
 
 
+def conv1d_tma_halo_kernel(T, NK):
+    """dwsep_conv1d_tcx_kernel: T tiles per CTA, NK 32-channel chunks per tile.
+
+    Two smem stages (seq & 1) hold the pw chunk and the x halo, which the TMA
+    warp loads once the MMAs that read the stage are done ("empty", a commit);
+    8 producer warps wait for the loads ("tma"), turn the halo into the A
+    operand in place and arrive at "full"; one issuer waits for "full" per
+    chunk and for the accumulator (local & 1) to be drained ("aempty", 4
+    epilogue warps) per tile, and commits "empty" per chunk and "afull" per
+    tile."""
+    sim = Sim()
+    for s in range(2):
+        sim.bar(f"full{s}", 8)
+        sim.bar(f"empty{s}", 1)
+        sim.bar(f"tma{s}", 1)
+        sim.bar(f"afull{s}", 1)
+        sim.bar(f"aempty{s}", 4)
+    tma, prod = [], []
+    for seq in range(T * NK):
+        st, k = seq & 1, seq >> 1
+        tma += [("wait", f"empty{st}", (k & 1) ^ 1, k, "tma"), ("owns", f"empty{st}", k, "tma"),
+                ("arrive", f"tma{st}", k, 1, "tma")]
+        prod += [("wait", f"tma{st}", k & 1, k + 1, "producers"), ("owns", f"empty{st}", k, "producers"),
+                 ("arrive", f"full{st}", k, 8, "producers")]
+    issue, complete, epi = [], [], []
+    n = 0
+    for t in range(T):
+        buf, bk = t & 1, t >> 1
+        issue += [("wait", f"aempty{buf}", (bk & 1) ^ 1, bk, "issuer"), ("owns", f"aempty{buf}", bk, "issuer")]
+        for c in range(NK):
+            seq = t * NK + c
+            st, k = seq & 1, seq >> 1
+            issue += [("wait", f"full{st}", k & 1, k + 1, "issuer"), ("issue", 0)]
+            complete += [("issued", 0, n), ("arrive", f"empty{st}", k, 1, "mma")]
+            n += 1
+        complete.append(("arrive", f"afull{buf}", bk, 1, "mma"))
+        epi += [("wait", f"afull{buf}", bk & 1, bk + 1, "epilogue"), ("arrive", f"aempty{buf}", bk, 4, "epilogue")]
+    sim.agents += [tma, prod, issue, complete, epi]
+    return sim
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("NK", [1, 2, 3, 8])
+def test_conv1d_tma_halo_kernel_protocol(T, NK):
+    for seed in range(30):
+        conv1d_tma_halo_kernel(T, NK).run(seed)
+
+
 SHAPES = [(T, C, A) for T in (1, 2, 3, 4, 7) for C in (1, 2, 3) for A in (2, 3)]
 
 
@@ -233,6 +281,20 @@ def test_model_catches_a_missing_accumulator_wait():
         sim = sub_chunk_kernel(7, 1, 2)
         for a in sim.agents:
             a[:] = [st for st in a if not (st[0] == "wait" and st[1].startswith("accempty"))]
+        try:
+            sim.run(seed)
+        except AssertionError as e:
+            failures += "releases done" in str(e)
+    assert failures > 0
+
+
+def test_model_catches_a_missing_conv1d_accumulator_wait():
+    """Plant a data race in the conv1d protocol: the issuer stops waiting for
+    the drained accumulator."""
+    failures = 0
+    for seed in range(100):
+        sim = conv1d_tma_halo_kernel(6, 2)
+        sim.agents[2] = [st for st in sim.agents[2] if not (st[0] == "wait" and st[1].startswith("aempty"))]
         try:
             sim.run(seed)
         except AssertionError as e:
