@@ -206,7 +206,9 @@ def conv1d_tma_halo_kernel(T, NK):
     operand in place and arrive at "full"; one issuer waits for "full" per
     chunk and for the accumulator (local & 1) to be drained ("aempty", 4
     epilogue warps) per tile, and commits "empty" per chunk and "afull" per
-    tile."""
+    tile.  The register-halo kernel (dwsep_conv1d_tc_kernel) has the same
+    protocol: its TMA brings only the pw chunk, and its halo goes through a
+    buffer only the producers use, ordered by their own group barrier."""
     sim = Sim()
     for s in range(2):
         sim.bar(f"full{s}", 8)
