@@ -49,6 +49,8 @@ SIGNATURES = {
     "fcv_dwsep_conv1d": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "fcv_dwsep_conv1d_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
     "fcv_conv2d_auto_algo": (_I, [_I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
+    "fcv_conv2d_tc_plan": (_I, [_I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
+                                ctypes.POINTER(ctypes.c_uint)]),
     "fcv_dwsep_conv1d_auto_algo": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)]),
     "fcv_status_string": (ctypes.c_char_p, [_I]),
     "fcv_version": (_I, []),
@@ -274,6 +276,15 @@ def dwsep_conv1d(x, dw, pw, bias, stride, pad, out=None, algo=ALGO_AUTO, stream=
     _check(lib.fcv_dwsep_conv1d_ex(_ptr(xd), _ptr(dwd), _ptr(pwd), _ptr(bd), N, C, T, O, K, stride, pad,
                                    _ptr(out), algo, _stream_ptr(stream)), "fcv_dwsep_conv1d")
     return _result(out, host, stream, out_host)
+
+
+def conv2d_tc_plan(Cin, Cout, pool, use_tma=True) -> dict:
+    """Diagnostic: what one launch of the tensor-core conv2d uses for these sizes."""
+    v, n, t, sm = _I(), _I(), _I(), ctypes.c_uint()
+    _check(load().fcv_conv2d_tc_plan(Cin, Cout, pool, int(bool(use_tma)), ctypes.byref(v), ctypes.byref(n),
+                                     ctypes.byref(t), ctypes.byref(sm)), "fcv_conv2d_tc_plan")
+    return {"variant": "sub-chunk" if v.value else "full-chunk", "nacc": n.value, "tmem_cols": t.value,
+            "smem_bytes": sm.value}
 
 
 def conv2d_auto_algo(N, Cin, H, W, Cout, pool) -> int:

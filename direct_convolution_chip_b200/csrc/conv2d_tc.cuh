@@ -125,7 +125,7 @@ struct Params {
     int tiles_img;    // tiles per image
     int total_tiles;
     int use_tma;      // halo by one 4-D TMA box (W % 4 == 0, aligned x), else by cp.async
-    int nacc;         // accumulator buffers in TMEM: 3 when 3 * NP + 2 * A_COLS <= 512, else 2
+    int nacc;         // accumulator buffers in TMEM: 3 when they fit next to the kernel's A stages, else 2
 };
 
 // Shared-memory layout (bytes, from a 1024-aligned base).
@@ -920,6 +920,45 @@ inline bool conv2d_tc_supported(int Cin, int Cout, int P)
     return s <= (uint32_t)c2tc::SMEM_LIMIT;
 }
 
+// What one launch of the tensor-core conv2d uses for given sizes: the kernel
+// (the sub-chunk kernel when the halo comes by TMA and Cout' <= 96), its
+// accumulator count, the TMEM columns it addresses of the 512 it allocates,
+// and the dynamic shared memory it requests.
+struct Conv2dTcPlan {
+    int sub;          // 1: conv2d_tc4_kernel, 0: conv2d_tc_kernel
+    int NP;           // Cout rounded up to 16 (MMA N)
+    int nacc;         // accumulator buffers of NP columns
+    int tmem_cols;    // accumulators + A stages
+    uint32_t smem;    // bytes, including the 1 KB alignment slack
+};
+
+template <int P>
+inline Conv2dTcPlan conv2d_tc_plan(int Cin, int Cout, bool use_tma)
+{
+    Conv2dTcPlan pl;
+    pl.NP = (Cout + 15) & ~15;
+    pl.sub = (use_tma && pl.NP <= c2tc::NP_MAX_SUB) ? 1 : 0;
+    const int a_cols = pl.sub ? 4 * c2tc::SUB_COLS : 2 * c2tc::A_COLS;
+    pl.nacc = (3 * pl.NP + a_cols <= (int)c2tc::TMEM_COLS) ? 3 : 2;
+    pl.tmem_cols = pl.nacc * pl.NP + a_cols;
+    // At least 120 KB, so that two CTAs never share an SM: each allocates all
+    // 512 TMEM columns.
+    pl.smem = conv2d_tc_smem<P>(Cin, Cout);
+    if (pl.smem < 120u * 1024u) pl.smem = 120u * 1024u;
+    return pl;
+}
+
+inline bool conv2d_tc_plan_for(int Cin, int Cout, int P, bool use_tma, Conv2dTcPlan* pl)
+{
+    switch (P) {
+    case 1: *pl = conv2d_tc_plan<1>(Cin, Cout, use_tma); return true;
+    case 2: *pl = conv2d_tc_plan<2>(Cin, Cout, use_tma); return true;
+    case 4: *pl = conv2d_tc_plan<4>(Cin, Cout, use_tma); return true;
+    case 8: *pl = conv2d_tc_plan<8>(Cin, Cout, use_tma); return true;
+    default: return false;
+    }
+}
+
 template <int P, int MODE>
 inline int launch_conv2d_tc_p(c2tc::Params prm, int N, int grid, cudaStream_t stream)
 {
@@ -944,19 +983,15 @@ inline int launch_conv2d_tc_p(c2tc::Params prm, int N, int grid, cudaStream_t st
             return FCV_ERR_CUDA;
         prm.use_tma = 1;
     }
-    // At least 120 KB, so that two CTAs never share an SM: each allocates all
-    // 512 TMEM columns.
-    uint32_t smem = conv2d_tc_smem<P>(prm.Cin, prm.Cout);
-    if (smem < 120u * 1024u) smem = 120u * 1024u;
     // With the halo by TMA and Cout <= 96, the sub-chunk kernel: four smaller A
     // stages let a producer group refill half a chunk while the MMAs of the
     // other half run.
-    const bool sub = prm.use_tma && prm.NP <= c2tc::NP_MAX_SUB;
-    if (sub) prm.nacc = (3 * prm.NP + 4 * c2tc::SUB_COLS <= (int)c2tc::TMEM_COLS) ? 3 : 2;
-    auto kern = sub ? c2tc::conv2d_tc4_kernel<P, MODE> : c2tc::conv2d_tc_kernel<P, MODE>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    const Conv2dTcPlan pl = conv2d_tc_plan<P>(prm.Cin, prm.Cout, prm.use_tma != 0);
+    prm.nacc = pl.nacc;
+    auto kern = pl.sub ? c2tc::conv2d_tc4_kernel<P, MODE> : c2tc::conv2d_tc_kernel<P, MODE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) != cudaSuccess)
         return FCV_ERR_CUDA;
-    kern<<<grid, c2tc::NTHREADS, smem, stream>>>(prm, map);
+    kern<<<grid, c2tc::NTHREADS, pl.smem, stream>>>(prm, map);
     return launch_status();
 }
 
@@ -980,7 +1015,7 @@ inline int launch_conv2d_tc(const float* x, const float* w, const float* b, int 
     prm.tiles_img = (int)per_img;
     prm.total_tiles = (int)total;
     prm.use_tma = 0;
-    prm.nacc = (3 * prm.NP + 2 * c2tc::A_COLS <= (int)c2tc::TMEM_COLS) ? 3 : 2;
+    prm.nacc = 2;  // set with the kernel choice in launch_conv2d_tc_p
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;

@@ -238,6 +238,21 @@ int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* 
     return FCV_OK;
 }
 
+int fcv_conv2d_tc_plan(int Cin, int Cout, int pool, int use_tma, int* variant, int* nacc, int* tmem_cols,
+                       unsigned int* smem_bytes)
+{
+    if (!variant || !nacc || !tmem_cols || !smem_bytes) return FCV_ERR_INVALID_ARG;
+    if (Cin < 1 || Cout < 1 || pool < 1) return FCV_ERR_INVALID_ARG;
+    if (!fcv::conv2d_tc_supported(Cin, Cout, pool)) return FCV_ERR_UNSUPPORTED;
+    fcv::Conv2dTcPlan pl;
+    if (!fcv::conv2d_tc_plan_for(Cin, Cout, pool, use_tma != 0, &pl)) return FCV_ERR_UNSUPPORTED;
+    *variant = pl.sub;
+    *nacc = pl.nacc;
+    *tmem_cols = pl.tmem_cols;
+    *smem_bytes = pl.smem;
+    return FCV_OK;
+}
+
 int fcv_dwsep_conv1d_auto_algo(const float* x, const float* pw_w, int N, int C, int T, int O, int K, int stride,
                                int pad, int* algo)
 {

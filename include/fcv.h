@@ -209,6 +209,16 @@ int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* 
 int fcv_dwsep_conv1d_auto_algo(const float* x, const float* pw_w, int N, int C, int T, int O, int K,
                                int stride, int pad, int* algo);
 
+/* Diagnostic (layout may change between versions): what one launch of
+ * FCV_CONV2D_TC_3XTF32 uses for these sizes.  use_tma says whether the input
+ * halo comes by TMA (W % 4 == 0 and a 16-byte aligned x).  Writes the kernel
+ * variant (1 = sub-chunk, 0 = full-chunk), the accumulator buffers, the tensor
+ * memory columns the kernel addresses (of the 512 it allocates) and the dynamic
+ * shared memory it requests.  FCV_ERR_UNSUPPORTED outside that kernel's
+ * envelope, FCV_ERR_INVALID_ARG for a NULL output or sizes < 1.  No CUDA call. */
+int fcv_conv2d_tc_plan(int Cin, int Cout, int pool, int use_tma, int* variant, int* nacc, int* tmem_cols,
+                       unsigned int* smem_bytes);
+
 /* Human-readable name of a status code (static storage). */
 const char* fcv_status_string(int status);
 

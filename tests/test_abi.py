@@ -205,3 +205,38 @@ def test_binding_calls_run_on_their_stream_argument(monkeypatch):
     assert call(1, 2, "s1") == (1, 2, "s1") and seen == ["s1"]
     assert call(1, stream="s2") == (1, 1, "s2") and seen == ["s1", "s2"]
     assert call(1, 3) == (1, 3, None) and seen == ["s1", "s2"]
+
+
+def test_conv2d_tc_plan_fits_tensor_memory_and_shared_memory(lib):
+    """For every shape the tensor-core conv2d accepts, the launch plan stays
+    within the 512 TMEM columns the kernel allocates and the 227 KB of shared
+    memory a CTA may request; the sub-chunk kernel runs exactly where it
+    applies (TMA halo, Cout rounded to 16 at most 96)."""
+    v, n, t, sm = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_uint()
+    q = lib.fcv_conv2d_tc_plan
+    supported = 0
+    for cin in (1, 3, 8, 9, 16, 24, 32, 40, 48, 64, 65):
+        for cout in range(1, 121):
+            for pool in (1, 2, 4, 8):
+                for tma in (0, 1):
+                    st = q(cin, cout, pool, tma, ctypes.byref(v), ctypes.byref(n), ctypes.byref(t), ctypes.byref(sm))
+                    if cout > 112:
+                        assert st == UNSUPPORTED
+                        continue
+                    if st == UNSUPPORTED:
+                        continue  # weights too large for shared memory
+                    assert st == OK
+                    supported += 1
+                    np_ = (cout + 15) // 16 * 16
+                    assert v.value == int(bool(tma) and np_ <= 96)
+                    a_cols = 4 * 80 if v.value else 2 * 144
+                    assert n.value in (2, 3) and t.value == n.value * np_ + a_cols <= 512
+                    assert n.value == (3 if 3 * np_ + a_cols <= 512 else 2)
+                    assert 120 * 1024 <= sm.value <= 227 * 1024
+    assert supported > 3000
+    # the full-size workload: sub-chunk kernel, three accumulators, all 512 columns
+    assert q(8, 64, 4, 1, ctypes.byref(v), ctypes.byref(n), ctypes.byref(t), ctypes.byref(sm)) == OK
+    assert (v.value, n.value, t.value) == (1, 3, 512)
+    assert q(8, 64, 3, 1, ctypes.byref(v), ctypes.byref(n), ctypes.byref(t), ctypes.byref(sm)) == UNSUPPORTED
+    assert q(0, 64, 4, 1, ctypes.byref(v), ctypes.byref(n), ctypes.byref(t), ctypes.byref(sm)) == INVALID
+    assert q(8, 64, 4, 1, None, ctypes.byref(n), ctypes.byref(t), ctypes.byref(sm)) == INVALID

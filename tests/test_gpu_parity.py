@@ -108,7 +108,8 @@ EDGE_2D = [
     (2, 8, 50, 52, 112, 2),    # the widest Cout: full-chunk kernel, two accumulators, TMA halo
     (1, 24, 40, 44, 48, 4),    # sub-chunk kernel: three input-channel chunks, three accumulators
     (3, 5, 66, 64, 20, 1),     # sub-chunk kernel, pool 1, Cout padded to 32
-    (1, 16, 36, 68, 96, 2),    # sub-chunk kernel at its widest Cout: two accumulators, two chunks
+    (1, 8, 36, 68, 96, 2),     # sub-chunk kernel at its widest Cout: two accumulators, all 512 TMEM columns
+    (1, 16, 36, 68, 96, 2),    # weights too large for the tensor-core kernel: AUTO and FMA only
     (2, 8, 48, 40, 80, 8),     # sub-chunk kernel, pool 8, Cout 80 (two accumulators)
     (1, 9, 30, 34, 64, 4),     # W % 4 != 0: full-chunk kernel with the cp.async halo
 ]
