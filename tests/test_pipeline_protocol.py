@@ -3,7 +3,8 @@
 Every role of one CTA (TMA warp, producer warps, MMA issuers, the tensor core
 completing what they issued, drain and pool warps) is an agent that waits on
 and arrives at mbarriers with the parities and counts the kernels in
-csrc/conv2d_tc.cuh (both conv2d kernels) and csrc/conv1d_tcx.cuh use.  The agents run in many random interleavings; for each
+csrc/conv2d_tc.cuh (both conv2d kernels), csrc/conv1d_tcx.cuh and
+csrc/conv1d_tc2.cuh (two CTAs of a cluster) use.  The agents run in many random interleavings; for each
 shape of the work (tiles per CTA, input-channel chunks, accumulator buffers)
 the model checks:
 
@@ -48,7 +49,9 @@ class Sim:
     ("wait", barrier, parity, phases that must be done, who),
     ("arrive", barrier, use, arrivals, who),
     ("issue", counter), ("issued", counter, k)  -- ordering of a commit after its issue,
-    ("owns", barrier, phases done, who)  -- a write that needs the buffer released."""
+    ("owns", barrier, phases done, who)  -- a write that needs the buffer released,
+    ("release", key), ("owns_all", keys, releases done, who)  -- the same with
+    explicit per-buffer release counts, for buffers in several CTAs."""
 
     def __init__(self):
         self.bars, self.agents, self.counters = {}, [], {}
@@ -76,6 +79,13 @@ class Sim:
                 self.bars[name].arrive(use, who)
         elif st[0] == "issue":
             self.counters[st[1]] = self.counters.get(st[1], 0) + 1
+        elif st[0] == "release":
+            self.counters[st[1]] = self.counters.get(st[1], 0) + 1
+        elif st[0] == "owns_all":
+            _, keys, need, who = st
+            for key in keys:
+                assert self.counters.get(key, 0) >= need, (f"{who}: writes {key} with "
+                                                           f"{self.counters.get(key, 0)} of {need} releases done")
         elif st[0] == "owns":
             _, name, need, who = st
             assert self.bars[name].phase >= need, (f"{who}: writes the buffer of {name} with "
@@ -240,6 +250,66 @@ def conv1d_tma_halo_kernel(T, NK):
     return sim
 
 
+def conv1d_pair_kernel(T, NK, stages=3):
+    """dwsep_conv1d_tc2_kernel: a cluster of two CTAs (rank 0 leads) shares
+    every MMA (cta_group::2).  Each CTA's TMA warp fills its own stage once
+    the MMAs that read it are done (its "empty", which the leader's
+    multicast commit completes in both CTAs); each CTA's 8 producer warps
+    arrive at the leader's "full" (16 arrivals); the leader's issuer waits for
+    "full" per chunk and for the accumulator to be drained by both CTAs'
+    epilogues (its "aempty", 8 arrivals) per tile; its multicast commits
+    complete "empty" and "afull" in both CTAs."""
+    sim = Sim()
+    for r in range(2):
+        for s_ in range(stages):
+            sim.bar(f"empty{s_}@{r}", 1)
+            sim.bar(f"tma{s_}@{r}", 1)
+        for b_ in range(2):
+            sim.bar(f"afull{b_}@{r}", 1)
+    for s_ in range(stages):
+        sim.bar(f"full{s_}@0", 16)
+    for b_ in range(2):
+        sim.bar(f"aempty{b_}@0", 8)
+    for r in range(2):
+        tma, prod = [], []
+        for seq in range(T * NK):
+            st, k = seq % stages, seq // stages
+            tma += [("wait", f"empty{st}@{r}", (k & 1) ^ 1, k, f"tma{r}"), ("owns", f"empty{st}@{r}", k, f"tma{r}"),
+                    ("arrive", f"tma{st}@{r}", k, 1, f"tma{r}")]
+            prod += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"producers{r}"),
+                     ("owns", f"empty{st}@{r}", k, f"producers{r}"),
+                     ("arrive", f"full{st}@0", k, 8, f"producers{r}")]
+        epi = []
+        for t in range(T):
+            buf, bk = t & 1, t >> 1
+            epi += [("wait", f"afull{buf}@{r}", bk & 1, bk + 1, f"epilogue{r}"),
+                    ("release", f"acc{buf}@{r}"),
+                    ("arrive", f"aempty{buf}@0", bk, 4, f"epilogue{r}")]
+        sim.agents += [tma, prod, epi]
+    issue, complete = [], []
+    n = 0
+    for t in range(T):
+        buf, bk = t & 1, t >> 1
+        issue += [("wait", f"aempty{buf}@0", (bk & 1) ^ 1, bk, "issuer"),
+                  ("owns_all", [f"acc{buf}@0", f"acc{buf}@1"], bk, "issuer")]
+        for c in range(NK):
+            seq = t * NK + c
+            st, k = seq % stages, seq // stages
+            issue += [("wait", f"full{st}@0", k & 1, k + 1, "issuer"), ("issue", 0)]
+            complete += [("issued", 0, n), ("arrive", f"empty{st}@0", k, 1, "mma"), ("arrive", f"empty{st}@1", k, 1, "mma")]
+            n += 1
+        complete += [("arrive", f"afull{buf}@0", bk, 1, "mma"), ("arrive", f"afull{buf}@1", bk, 1, "mma")]
+    sim.agents += [issue, complete]
+    return sim
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("NK", [1, 2, 3, 4, 8])
+def test_conv1d_pair_kernel_protocol(T, NK):
+    for seed in range(30):
+        conv1d_pair_kernel(T, NK).run(seed)
+
+
 @pytest.mark.parametrize("T", [1, 2, 3, 5, 8])
 @pytest.mark.parametrize("NK", [1, 2, 3, 8])
 def test_conv1d_tma_halo_kernel_protocol(T, NK):
@@ -297,6 +367,24 @@ def test_model_catches_a_missing_conv1d_accumulator_wait():
     for seed in range(100):
         sim = conv1d_tma_halo_kernel(6, 2)
         sim.agents[2] = [st for st in sim.agents[2] if not (st[0] == "wait" and st[1].startswith("aempty"))]
+        try:
+            sim.run(seed)
+        except AssertionError as e:
+            failures += "releases done" in str(e)
+    assert failures > 0
+
+
+def test_model_catches_a_leader_that_ignores_the_peer_epilogue():
+    """Plant a cluster race: the leader's "accumulator drained" barrier counts
+    only its own epilogue warps, so an MMA may overwrite the peer CTA's
+    accumulator rows while the peer still reads them."""
+    failures = 0
+    for seed in range(100):
+        sim = conv1d_pair_kernel(5, 3)
+        for b in range(2):
+            sim.bars[f"aempty{b}@0"].count = 4
+        peer_epilogue = sim.agents[5]
+        peer_epilogue[:] = [st for st in peer_epilogue if st[0] != "arrive"]
         try:
             sim.run(seed)
         except AssertionError as e:
