@@ -56,3 +56,22 @@ def test_reference_arm_runs_only_on_rank_zero(capsys, monkeypatch):
     monkeypatch.setenv("RANK", "1")
     bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_json_line(capsys, monkeypatch):
+    """Rank 0 prints one JSON line with the keys the benchmark contract needs
+    for the CPU-oracle arm: the arm's own metric and unit, a cpu_baseline that
+    describes the run, and an e2e with no host-device traffic."""
+    import json
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.delenv("RANK", raising=False)
+    bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3
+    assert d["value"] > 0 and d["unit"] == "GFLOP/s" and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] and d["data"] == "synthetic"
