@@ -38,6 +38,7 @@ SPEC_FMA_LANES_PER_SM = 128       # FP32 FMA units per SM
 SPEC_SM_MAX_MHZ = 1965.0          # clocks.max.sm
 TF32_OVER_BF16 = 1.1 / 2.25       # nominal dense TF32 : BF16 tensor throughput
 ALGO_NAMES = {10: "conv2d_direct_fma", 11: "conv2d_poolfirst_fma", 12: "conv2d_tc_3xtf32",
+              13: "conv2d_tc_shift_3xtf32",
               20: "dwsep_conv1d_fma", 21: "dwsep_conv1d_tc_register_halo", 22: "dwsep_conv1d_tc_2sm",
               23: "dwsep_conv1d_tc_tma_halo"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -110,6 +111,73 @@ def fma_peak_tflops(props):
 
 def roofline_time_s(macs, nbytes, peak_tflops, hbm_gbs):
     return max(2.0 * macs / (peak_tflops * 1e12), nbytes / (hbm_gbs * 1e9))
+
+
+def op_roofline(c, tensor, tc_peak, fma_peak, hbm):
+    """Roofline time of one workload.  FP32-FMA kernels: every MAC on the FMA
+    pipe.  Tensor-core kernels: conv2d's MACs on the 3xTF32 tensor pipe;
+    conv1d's pointwise MACs on the tensor pipe while its depthwise MACs run
+    on the FMA pipe beside them.  Then the slower of that and the compulsory
+    bytes at HBM bandwidth."""
+    nbytes = case_bytes(c)
+    t_mem = nbytes / (hbm * 1e9)
+    if not tensor:
+        return max(2.0 * case_macs(c) / (fma_peak * 1e12), t_mem)
+    if c.op == "conv2d":
+        return max(2.0 * case_macs(c) / (tc_peak * 1e12), t_mem)
+    pw = macs_conv1d_pointwise(c.N, c.C, c.T, c.O, c.K, c.stride, c.pad)
+    dw = case_macs(c) - pw
+    return max(2.0 * pw / (tc_peak * 1e12), 2.0 * dw / (fma_peak * 1e12), t_mem)
+
+
+def stats_ms(values):
+    """Median, min and 90th percentile of a list of times (ms)."""
+    v = sorted(values)
+    return {"median": v[len(v) // 2], "min": v[0], "p90": v[min(len(v) - 1, int(0.9 * len(v)))], "n": len(v)}
+
+
+def source_info():
+    """Git commit when the checkout has one, and a hash of the library and bench sources."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "direct_convolution_chip_b200", "csrc")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for f in files + [os.path.join(ROOT, "include", "fcv.h"), os.path.abspath(__file__)]:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    try:
+        sha = subprocess.run(["git", "-C", ROOT, "rev-parse", "HEAD"], capture_output=True, text=True,
+                             timeout=10).stdout.strip() or None
+    except (OSError, subprocess.SubprocessError):
+        sha = None
+    return {"git_sha": sha, "source_sha256": h.hexdigest()}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def probe_tf32_tflops():
+    """Dense TF32 tensor rate measured now on this GPU: one CTA per SM issuing
+    tcgen05.mma kind::tf32 M = 128, N = 256, K = 8 back to back (best of 3)."""
+    import ctypes
+    from direct_convolution_chip_b200 import build as fcv_build
+    try:
+        lib = ctypes.CDLL(fcv_build.build_probes())
+    except (OSError, subprocess.SubprocessError):
+        return None
+    best = None
+    for _ in range(3):
+        f, ms, cyc = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+        if lib.fcvprobe_tf32_mma_rate(256, 0, 1, 1, 24000, ctypes.byref(f), ctypes.byref(ms), ctypes.byref(cyc)) == 0:
+            best = max(best or 0.0, f.value / 1e12)
+    return best
 
 
 # ----------------------------------------------------------------------------
@@ -277,6 +345,49 @@ def run_oracle_sample(budget_s=12.0):
                       f"({ta:.2f} s), op B {items_b} batch items ({tb:.2f} s); double-precision OpenMP loops"}
 
 
+def time_small_case(lib, fcv, c, stream, flush_buf, iters=60):
+    """Device time of one named small workload through its C entry point: warm
+    L2 (inputs resident) and cold L2 (a 256 MB buffer written between calls),
+    each over `iters` timed calls with CUDA events on the launching stream."""
+    import ctypes
+    P = ctypes.c_void_p
+    sp = P(stream.cuda_stream)
+    if c.op == "conv2d":
+        x, w, b = [t.cuda() for t in wl.conv2d_inputs(c)]
+        out = torch.empty((c.N,), device="cuda")
+
+        def fn():
+            return lib.fcv_conv2d_pool_sigmoid_sum(P(x.data_ptr()), P(w.data_ptr()), P(b.data_ptr()), c.N, c.Cin,
+                                                   c.H, c.W, c.Cout, c.P, P(out.data_ptr()), sp)
+        algo = fcv.conv2d_auto_algo(c.N, c.Cin, c.H, c.W, c.Cout, c.P)
+    else:
+        x, dw, pw, b = [t.cuda() for t in wl.conv1d_inputs(c)]
+        To = (c.T + 2 * c.pad - c.K) // c.stride + 1
+        out = torch.empty((c.N, c.O, To), device="cuda")
+
+        def fn():
+            return lib.fcv_dwsep_conv1d(P(x.data_ptr()), P(dw.data_ptr()), P(pw.data_ptr()), P(b.data_ptr()),
+                                        c.N, c.C, c.T, c.O, c.K, c.stride, c.pad, P(out.data_ptr()), sp)
+        algo = fcv.dwsep_conv1d_auto_algo(x, dw, pw, c.stride, c.pad)
+    for _ in range(5):
+        if fn() != 0:
+            raise RuntimeError(f"{c.name}: launch failed")
+    res = {}
+    for leg in ("warm_l2", "cold_l2"):
+        ts = []
+        for _ in range(iters):
+            if leg == "cold_l2":
+                flush_buf.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        res[leg] = stats_ms(ts)
+    return algo, res
+
+
 def run_gpu(args):
     import direct_convolution_chip_b200 as fcv
 
@@ -286,6 +397,7 @@ def run_gpu(args):
     use_dist = init_dist(world, local)
     lib = fcv.load()
     props = torch.cuda.get_device_properties(device)
+    tf32_probe = probe_tf32_tflops() if world == 1 else None
 
     # Inputs: seeded synthetic data of the pages' shapes, resident in HBM.
     xa, wa, ba = wl.conv2d_inputs(CASE_A)
@@ -340,31 +452,46 @@ def run_gpu(args):
     clocks = sampler.stop()
     barrier(use_dist, device)
     total_ms = t_start.elapsed_time(t_end)
-    ta_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
-    tb_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
+    la = [e[0].elapsed_time(e[1]) for e in ev]
+    lb = [e[1].elapsed_time(e[2]) for e in ev]
+    ta_ms, tb_ms = sum(la), sum(lb)
     total_ms, ta_ms, tb_ms = max_over_ranks([total_ms, ta_ms, tb_ms], use_dist, device)
 
-    # End to end through the public API with pinned host buffers.
-    e2e_steps = max(2, min(8, K // 25))
+    # End to end through the public API with pinned host buffers: every step
+    # copies its inputs host -> device, runs both ops and copies both results
+    # back.  Steps alternate between two streams and the binding does not wait
+    # for its copies (wait=False), so one step's results travel device -> host
+    # while the next step's inputs travel host -> device; the timed region
+    # ends when the last copy has landed.
+    e2e_steps = max(8, min(16, K // 10))
     xa_h, wa_h, ba_h, xb_h, dwb_h, pwb_h, bb_h = host
-    # results land in pinned host buffers allocated once, as an application would
-    ra_h = torch.empty((CASE_A.N,), dtype=torch.float32, pin_memory=True)
-    rb_h = torch.empty((CASE_B.N, CASE_B.O, To), dtype=torch.float32, pin_memory=True)
-    for _ in range(1):
-        fcv.conv2d_pool_sigmoid_sum(xa_h, wa_h, ba_h, CASE_A.P, out=ra_h)
-        fcv.dwsep_conv1d(xb_h, dwb_h, pwb_h, bb_h, CASE_B.stride, CASE_B.pad, out=rb_h)
+    streams = [stream, torch.cuda.Stream(device)]
+    ra_h = [torch.empty((CASE_A.N,), dtype=torch.float32, pin_memory=True) for _ in range(2)]
+    rb_h = [torch.empty((CASE_B.N, CASE_B.O, To), dtype=torch.float32, pin_memory=True) for _ in range(2)]
+
+    def e2e_step(i):
+        s_ = streams[i & 1]
+        fcv.conv2d_pool_sigmoid_sum(xa_h, wa_h, ba_h, CASE_A.P, out=ra_h[i & 1], stream=s_, wait=False)
+        fcv.dwsep_conv1d(xb_h, dwb_h, pwb_h, bb_h, CASE_B.stride, CASE_B.pad, out=rb_h[i & 1], stream=s_,
+                         wait=False)
+
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize(device)
     barrier(use_dist, device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(device)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        ra = fcv.conv2d_pool_sigmoid_sum(xa_h, wa_h, ba_h, CASE_A.P, out=ra_h)
-        rb = fcv.dwsep_conv1d(xb_h, dwb_h, pwb_h, bb_h, CASE_B.stride, CASE_B.pad, out=rb_h)
-    e1.record(stream)
+    e0.record(streams[0])
+    streams[1].wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    done1 = torch.cuda.Event()
+    done1.record(streams[1])
+    streams[0].wait_event(done1)
+    e1.record(streams[0])
     torch.cuda.synchronize(device)
     e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], use_dist, device)[0]
     h2d = sum(t.numel() * t.element_size() for t in host)
-    d2h = ra.numel() * 4 + rb.numel() * 4
+    d2h = ra_h[0].numel() * 4 + rb_h[0].numel() * 4
 
     macs_a, macs_b = case_macs(CASE_A), case_macs(CASE_B)
     bytes_a, bytes_b = case_bytes(CASE_A), case_bytes(CASE_B)
@@ -374,46 +501,74 @@ def run_gpu(args):
     hbm = peaks["hbm_gbs"]
     fma_peak = fma_peak_tflops(props)
     tf32_peak = peaks["bf16_tflops"] * TF32_OVER_BF16
+    tc_rule = tf32_peak / 3.0
+    tc_probe = tf32_probe / 3.0 if tf32_probe else None
     ta_s, tb_s = ta_ms / K / 1e3, tb_ms / K / 1e3
 
     # The algorithms AUTO runs here (the library reports its own choice).
     algo_a = fcv.conv2d_auto_algo(CASE_A.N, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout, CASE_A.P)
     algo_b = fcv.dwsep_conv1d_auto_algo(xb_d, dwb_d, pwb_d, CASE_B.stride, CASE_B.pad)
-    tc_a = algo_a == fcv.CONV2D_TC_3XTF32
+    tc_a = algo_a in (fcv.CONV2D_TC_3XTF32, fcv.CONV2D_TC_SHIFT_3XTF32)
     tc_b = algo_b in (fcv.CONV1D_TC_3XTF32, fcv.CONV1D_TC_TMA_3XTF32, fcv.CONV1D_TC2_3XTF32)
-    pw_macs_b = macs_conv1d_pointwise(CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K, CASE_B.stride, CASE_B.pad)
-    per_op = {
-        "conv2d": {"workload": CASE_A.name, "algo": ALGO_NAMES.get(algo_a, algo_a), "ms": ta_s * 1e3,
-                   "gflops": 2 * macs_a / ta_s / 1e9, "macs": macs_a, "compulsory_bytes": bytes_a,
-                   "roofline_frac_fp32_fma": roofline_time_s(macs_a, bytes_a, fma_peak, hbm) / ta_s,
-                   "roofline_frac_3xtf32": roofline_time_s(macs_a, bytes_a, tf32_peak / 3.0, hbm) / ta_s},
-        "dwsep_conv1d": {"workload": CASE_B.name, "algo": ALGO_NAMES.get(algo_b, algo_b), "ms": tb_s * 1e3,
-                         "gflops": 2 * macs_b / tb_s / 1e9, "macs": macs_b, "compulsory_bytes": bytes_b,
-                         "roofline_frac_fp32_fma": roofline_time_s(macs_b, bytes_b, fma_peak, hbm) / tb_s,
-                         "roofline_frac_3xtf32": roofline_time_s(pw_macs_b, bytes_b, tf32_peak / 3.0, hbm) / tb_s},
-    }
+
+    def op_entry(c, algo, tensor, t_s, samples):
+        e = {"workload": c.name, "algo": ALGO_NAMES.get(algo, algo), "ms": t_s * 1e3,
+             "ms_stats": stats_ms(samples) if samples else None,
+             "gflops": 2 * case_macs(c) / t_s / 1e9, "macs": case_macs(c), "compulsory_bytes": case_bytes(c),
+             "roofline_frac_fp32_fma": op_roofline(c, False, None, fma_peak, hbm) / t_s,
+             "roofline_frac_3xtf32": op_roofline(c, True, tc_rule, fma_peak, hbm) / t_s,
+             "roofline_frac_3xtf32_probe": (op_roofline(c, True, tc_probe, fma_peak, hbm) / t_s
+                                            if tc_probe else None),
+             "pipe": "3xtf32" if tensor else "fp32_fma"}
+        e["roofline_frac"] = e["roofline_frac_3xtf32"] if tensor else e["roofline_frac_fp32_fma"]
+        return e
+
+    per_op = {"conv2d": op_entry(CASE_A, algo_a, tc_a, ta_s, la),
+              "dwsep_conv1d": op_entry(CASE_B, algo_b, tc_b, tb_s, lb)}
+    if rank == 0 and world == 1:
+        flush_buf = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)  # 256 MB > L2
+        for key, c in (("conv2d_small", wl.CONV2D_SMALL), ("dwsep_conv1d_small", wl.CONV1D_SMALL)):
+            algo, legs = time_small_case(lib, fcv, c, stream, flush_buf)
+            tensor = algo in (fcv.CONV2D_TC_3XTF32, fcv.CONV2D_TC_SHIFT_3XTF32, fcv.CONV1D_TC_3XTF32,
+                              fcv.CONV1D_TC_TMA_3XTF32, fcv.CONV1D_TC2_3XTF32)
+            e = op_entry(c, algo, tensor, legs["warm_l2"]["median"] / 1e3, None)
+            e["ms_stats"] = legs
+            e["note"] = "launch-latency bound; reported, no target"
+            per_op[key] = e
+        del flush_buf
     fma_src = "148 SMs x 128 FP32 FMA lanes x 2 FLOP x 1965 MHz (spec clocks)"
-    tc_src = ("measured bf16 GEMM x nominal TF32/BF16 (1.1/2.25), / 3 for the three TF32 products of the "
-              "3xTF32 split; FLOPs are the fp32 method's (2 per MAC)")
+    tc_src = ("measured bf16 GEMM (MEASURED_PEAKS) x nominal TF32/BF16 (1.1/2.25), / 3 for the three TF32 "
+              "products of the 3xTF32 split; FLOPs are the fp32 method's (2 per MAC)")
+    tc_probe_src = ("tcgen05.mma kind::tf32 M128 N256 K8 rate probed on this GPU at the start of this run "
+                    "(libfcv_probes.so), / 3")
     dom = "conv2d" if ta_s >= tb_s else "dwsep_conv1d"
     if dom == "conv2d":
         achieved = 2 * macs_a / ta_s / 1e12
         if tc_a:
-            kname = ("c2tc::conv2d_tc4_kernel<4, sum>" if CASE_A.Cout <= 96 and CASE_A.W % 4 == 0
-                     else "c2tc::conv2d_tc_kernel<4, sum>")
-            roof = {"kernel": kname, "bound": "tensor", "achieved": achieved,
-                    "peak": tf32_peak / 3.0, "unit": "TFLOP/s", "frac": achieved / (tf32_peak / 3.0),
-                    "traffic": traffic_per_launch("conv2d_tc_p4"), "peak_source": tc_src}
+            if algo_a == fcv.CONV2D_TC_SHIFT_3XTF32:
+                kname, tkey = "c2s::conv2d_tcs_kernel<4, 1, sum>", "conv2d_tcs_p4"
+            else:
+                kname = ("c2tc::conv2d_tc4_kernel<4, sum>" if CASE_A.Cout <= 96 and CASE_A.W % 4 == 0
+                         else "c2tc::conv2d_tc_kernel<4, sum>")
+                tkey = "conv2d_tc_p4"
+            roof = {"kernel": kname, "bound": "tensor", "achieved": achieved, "peak": tc_rule, "unit": "TFLOP/s",
+                    "frac": achieved / tc_rule, "traffic": traffic_per_launch(tkey), "peak_source": tc_src,
+                    "peak_probe": tc_probe, "frac_probe": achieved / tc_probe if tc_probe else None,
+                    "peak_probe_source": tc_probe_src}
         else:
             roof = {"kernel": "conv2d_direct_kernel<4, sum>", "bound": "alu", "achieved": achieved,
                     "peak": fma_peak, "unit": "TFLOP/s", "frac": achieved / fma_peak,
                     "traffic": traffic_per_launch("conv2d_direct_p4"), "peak_source": fma_src}
     else:
         if tc_b:
+            pw_macs_b = macs_conv1d_pointwise(CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K, CASE_B.stride,
+                                              CASE_B.pad)
             achieved = 2 * pw_macs_b / tb_s / 1e12
             roof = {"kernel": "dwsep_conv1d (tensor-core)", "bound": "tensor", "achieved": achieved,
-                    "peak": tf32_peak / 3.0, "unit": "TFLOP/s", "frac": achieved / (tf32_peak / 3.0),
-                    "traffic": traffic_per_launch("dwsep_conv1d"), "peak_source": tc_src}
+                    "peak": tc_rule, "unit": "TFLOP/s", "frac": achieved / tc_rule,
+                    "traffic": traffic_per_launch("dwsep_conv1d"), "peak_source": tc_src,
+                    "achieved_basis": "pointwise MACs (the depthwise MACs run on the FMA pipe)",
+                    "peak_probe": tc_probe, "frac_probe": achieved / tc_probe if tc_probe else None}
         else:
             achieved = 2 * macs_b / tb_s / 1e12
             roof = {"kernel": "dwsep_conv1d_fma_kernel", "bound": "alu", "achieved": achieved, "peak": fma_peak,
@@ -428,12 +583,16 @@ def run_gpu(args):
                    "algos": {"conv2d": ALGO_NAMES.get(algo_a, algo_a),
                              "dwsep_conv1d": ALGO_NAMES.get(algo_b, algo_b)}},
         "per_op": per_op, "roofline": roof,
-        "peaks": {"hbm_gbs": hbm, "fp32_fma_tflops": fma_peak, "tf32_tflops": tf32_peak, "source": peak_src},
+        "peaks": {"hbm_gbs": hbm, "fp32_fma_tflops": fma_peak, "tf32_tflops": tf32_peak,
+                  "tf32_tflops_probe": tf32_probe, "source": peak_src},
         "e2e": {"value": job_throughput(2.0 * (macs_a + macs_b), world, e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "steps": e2e_steps},
-        "gpu_launches": 2 * K,
+                "steps": e2e_steps, "overlap": "two streams, alternating steps; copies not waited for per call"},
+        # op A: one launch per block of 64 output channels on the shifted-operand kernel, else one; op B: one
+        "gpu_launches": K * (((CASE_A.Cout + 63) // 64 if algo_a == fcv.CONV2D_TC_SHIFT_3XTF32 else 1) + 1),
         "clocks": clocks,
+        "host": {"cpu_model": cpu_model(), "cores": len(os.sched_getaffinity(0))},
+        "source": source_info(),
     }
     if rank == 0 and world == 1:
         # The library's other algorithms on the same inputs (not part of the step).
@@ -453,15 +612,18 @@ def run_gpu(args):
                     raise fcv.FcvError(st, f"conv1d algorithm {algo}")
             return fn
 
-        def alt_a_fma():
-            st = lib.fcv_conv2d_pool_sigmoid_sum_ex(P(xa_d.data_ptr()), P(wa_d.data_ptr()), P(ba_d.data_ptr()),
-                                                    CASE_A.N, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout, CASE_A.P,
-                                                    P(out_a.data_ptr()), fcv.CONV2D_DIRECT, P(sp))
-            if st:
-                raise fcv.FcvError(st, "FMA direct conv2d")
+        def alt_a_algo(algo):
+            def fn():
+                st = lib.fcv_conv2d_pool_sigmoid_sum_ex(P(xa_d.data_ptr()), P(wa_d.data_ptr()), P(ba_d.data_ptr()),
+                                                        CASE_A.N, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout,
+                                                        CASE_A.P, P(out_a.data_ptr()), algo, P(sp))
+                if st:
+                    raise fcv.FcvError(st, f"conv2d algorithm {algo}")
+            return fn
 
         ta2 = _event_ms(alt_a, 10, stream)
-        ta3 = _event_ms(alt_a_fma, 10, stream)
+        ta3 = _event_ms(alt_a_algo(fcv.CONV2D_DIRECT), 10, stream)
+        ta4 = _event_ms(alt_a_algo(fcv.CONV2D_TC_3XTF32), 10, stream)
         tb = {name: _event_ms(alt_b(algo), 10, stream)
               for name, algo in (("dwsep_conv1d_fma", fcv.CONV1D_FMA),
                                  ("dwsep_conv1d_tc_register_halo", fcv.CONV1D_TC_3XTF32),
@@ -475,6 +637,8 @@ def run_gpu(args):
                                  "note": "pools the input first (exact identity): 9*Cin MACs per pooled value"},
             "conv2d_direct_fma": {"ms": ta3, "gflops": 2.0 * macs_a / (ta3 / 1e3) / 1e9,
                                   "frac_of_fp32_fma_peak": 2.0 * macs_a / (ta3 / 1e3) / 1e12 / fma_peak},
+            "conv2d_tc_im2col_3xtf32": {"ms": ta4, "gflops": 2.0 * macs_a / (ta4 / 1e3) / 1e9,
+                                        "note": "im2col rows in tensor memory, M = 128 positions, N = Cout"},
         }
         for name, ms in tb.items():
             result["variants"][name] = {"ms": ms, "gflops": 2.0 * macs_b / (ms / 1e3) / 1e9}

@@ -11,7 +11,11 @@ too: they are copied to the current device (asynchronously when pinned), the
 kernel runs, and the result is copied back into `out` when a CPU tensor is
 given (pinned for an asynchronous copy), else into a new pinned CPU tensor --
 the path an application with host-resident data takes.  A `stream` argument
-orders all of it (copies, allocations, kernel) on that stream.
+orders all of it (copies, allocations, kernel) on that stream.  Host-mode
+calls wait for their result copy unless wait=False: the returned CPU tensor
+is then valid once that stream has passed the copy, so that a caller can
+overlap one call's result copy with the next call's input copy on another
+stream.
 """
 import ctypes
 import functools
@@ -28,6 +32,7 @@ ALGO_AUTO = 0
 CONV2D_DIRECT = 10
 CONV2D_POOLFIRST = 11
 CONV2D_TC_3XTF32 = 12
+CONV2D_TC_SHIFT_3XTF32 = 13
 CONV1D_FMA = 20
 CONV1D_TC_3XTF32 = 21
 CONV1D_TC2_3XTF32 = 22
@@ -56,6 +61,9 @@ SIGNATURES = {
     "fcv_version": (_I, []),
     "fcv_device_error": (_I, [_P]),
     "fcv_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
+    "fcv_selftest_conv2d_stall": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _I, ctypes.c_ulonglong, _P]),
+    "fcv_selftest_conv1d_stall": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _I, ctypes.c_ulonglong,
+                                       _P]),
 }
 
 
@@ -153,9 +161,11 @@ def _host_mode(*ts):
     return True
 
 
-def _result(out_dev, host, stream, out_host=None):
+def _result(out_dev, host, stream, out_host=None, wait=True):
     """Host mode: copy the device result into `out_host` (a caller's CPU tensor,
-    best pinned) or into a new pinned tensor, and wait for the copy."""
+    best pinned) or into a new pinned tensor, and wait for the copy -- or, with
+    wait=False, return at once: the CPU tensor then holds the result once the
+    stream has reached the end of the copy (e.g. after stream.synchronize())."""
     if not host:
         return out_dev
     if out_host is not None:
@@ -165,9 +175,11 @@ def _result(out_dev, host, stream, out_host=None):
         res = out_host
     else:
         res = torch.empty(out_dev.shape, dtype=out_dev.dtype, pin_memory=True)
-    with torch.cuda.stream(stream or torch.cuda.current_stream()):
+    s = stream or torch.cuda.current_stream()
+    with torch.cuda.stream(s):
         res.copy_(out_dev, non_blocking=True)
-    (stream or torch.cuda.current_stream()).synchronize()
+    if wait:
+        s.synchronize()
     return res
 
 
@@ -177,7 +189,7 @@ def conv2d_out_shape(H, W, pool):
 
 
 @_on_stream
-def conv2d_pool_sigmoid_sum(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None):
+def conv2d_pool_sigmoid_sum(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None, wait=True):
     """out[N] = sum over (C, PH, PW) of sigmoid(avgpool_pool(conv3x3(x, w) + b))."""
     lib = load()
     host = _host_mode(x, w, b)
@@ -193,7 +205,7 @@ def conv2d_pool_sigmoid_sum(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None
     _check(lib.fcv_conv2d_pool_sigmoid_sum_ex(_ptr(xd), _ptr(wd), _ptr(bd), N, Cin, H, W, Cout, pool,
                                               _ptr(out), algo, _stream_ptr(stream)),
            "fcv_conv2d_pool_sigmoid_sum")
-    return _result(out, host, stream, out_host)
+    return _result(out, host, stream, out_host, wait)
 
 
 def conv2d_workspace_bytes(N, Cin, H, W, Cout, pool) -> int:
@@ -205,7 +217,7 @@ def conv2d_workspace_bytes(N, Cin, H, W, Cout, pool) -> int:
 
 
 @_on_stream
-def conv2d_pool_sigmoid_sum_det(x, w, b, pool, out=None, workspace=None, stream=None):
+def conv2d_pool_sigmoid_sum_det(x, w, b, pool, out=None, workspace=None, stream=None, wait=True):
     """Bitwise-reproducible variant of conv2d_pool_sigmoid_sum.
 
     `workspace` is a device tensor of at least conv2d_workspace_bytes(...) bytes
@@ -228,11 +240,11 @@ def conv2d_pool_sigmoid_sum_det(x, w, b, pool, out=None, workspace=None, stream=
     _check(lib.fcv_conv2d_pool_sigmoid_sum_det(_ptr(xd), _ptr(wd), _ptr(bd), N, Cin, H, W, Cout, pool, _ptr(out),
                                                _ptr(workspace) if need else None, nbytes, _stream_ptr(stream)),
            "fcv_conv2d_pool_sigmoid_sum_det")
-    return _result(out, host, stream, out_host)
+    return _result(out, host, stream, out_host, wait)
 
 
 @_on_stream
-def conv2d_pool_tap(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None):
+def conv2d_pool_tap(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None, wait=True):
     """Pooled pre-sigmoid values [N, Cout, PH, PW] of the same fused kernel."""
     lib = load()
     host = _host_mode(x, w, b)
@@ -248,7 +260,7 @@ def conv2d_pool_tap(x, w, b, pool, out=None, algo=ALGO_AUTO, stream=None):
         out = torch.empty((N, Cout, max(PH, 0), max(PW, 0)), dtype=torch.float32, device=xd.device)
     _check(lib.fcv_conv2d_pool_tap(_ptr(xd), _ptr(wd), _ptr(bd), N, Cin, H, W, Cout, pool,
                                    _ptr(out), algo, _stream_ptr(stream)), "fcv_conv2d_pool_tap")
-    return _result(out, host, stream, out_host)
+    return _result(out, host, stream, out_host, wait)
 
 
 def conv1d_out_len(T, K, stride, pad):
@@ -257,7 +269,7 @@ def conv1d_out_len(T, K, stride, pad):
 
 
 @_on_stream
-def dwsep_conv1d(x, dw, pw, bias, stride, pad, out=None, algo=ALGO_AUTO, stream=None):
+def dwsep_conv1d(x, dw, pw, bias, stride, pad, out=None, algo=ALGO_AUTO, stream=None, wait=True):
     """out[N, O, To] = pointwise(depthwise(x)) + bias; bias may be None."""
     lib = load()
     host = _host_mode(x, dw, pw, bias)
@@ -275,7 +287,7 @@ def dwsep_conv1d(x, dw, pw, bias, stride, pad, out=None, algo=ALGO_AUTO, stream=
         out = torch.empty((N, O, max(To, 0)), dtype=torch.float32, device=xd.device)
     _check(lib.fcv_dwsep_conv1d_ex(_ptr(xd), _ptr(dwd), _ptr(pwd), _ptr(bd), N, C, T, O, K, stride, pad,
                                    _ptr(out), algo, _stream_ptr(stream)), "fcv_dwsep_conv1d")
-    return _result(out, host, stream, out_host)
+    return _result(out, host, stream, out_host, wait)
 
 
 def conv2d_tc_plan(Cin, Cout, pool, use_tma=True) -> dict:

@@ -256,7 +256,23 @@ struct Params {
     int C, T, O, K, pad, To;
     int tiles_t, tiles_o, total_tiles;
     int out_vec;  // output rows 16-byte aligned (To % 4 == 0, aligned base)
+    // Failure-path test (all 0 in normal calls): role stall_role (1 TMA warp,
+    // 2 producers, 3 MMA issuer, 4 epilogue) of every CTA waits, before its
+    // stall_at-th tile, on a barrier nothing completes, with limit stall_ns.
+    int stall_role = 0, stall_at = 0;
+    unsigned long long stall_ns = 0;
 };
+
+// The failure-path test hook: true unless role `role` is to stall before its
+// `local`-th tile and its wait on `gate` (a barrier nothing completes) ran out,
+// which also sets the abort flag and the device error word.  gate == 0: the
+// kernel has no gate.
+__device__ __forceinline__ bool stall_ok(const Params& p, int role, int local, uint32_t gate,
+                                         volatile uint32_t* abort_flag)
+{
+    if (gate == 0 || p.stall_role != role || local != p.stall_at) return true;
+    return wait_bounded(gate, 0, abort_flag, p.stall_ns);
+}
 
 struct TileCoord {
     int n, t0, o0;
@@ -298,12 +314,14 @@ __device__ __forceinline__ void quad_transpose(float& x0, float& x1, float& x2, 
 // barrier.  Finally drain every MMA issued (bounded) so TMEM can be freed.
 __device__ __forceinline__ void mma_issuer(const Params& p, uint32_t tmem, uint32_t sbase, uint32_t bar_full,
                                            uint32_t bar_empty, uint32_t bar_afull, uint32_t bar_aempty,
-                                           uint32_t bar_drain, volatile uint32_t* abort_flag, int nk)
+                                           uint32_t bar_drain, volatile uint32_t* abort_flag, int nk,
+                                           uint32_t gate = 0)
 {
     int seq = 0, local = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++local) {
         const int buf = local & 1;
+        if (!stall_ok(p, 3, local, gate, abort_flag)) break;
         if (!wait_bounded(bar_aempty + 8 * buf, ((local >> 1) & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
@@ -347,14 +365,16 @@ __device__ __forceinline__ void mma_issuer(const Params& p, uint32_t tmem, uint3
 // adds the bias and stores the tile's outputs, then frees the buffer.
 __device__ __forceinline__ void epilogue_warp(const Params& p, uint32_t tmem, uint32_t bar_afull,
                                               uint32_t bar_aempty, volatile uint32_t* abort_flag, int warp,
-                                              int lane)
+                                              int lane, uint32_t gate = 0)
 {
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int local = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++local) {
         const int buf = local & 1;
         int ok = 1;
-        if (lane == 0) ok = wait_bounded(bar_afull + 8 * buf, (local >> 1) & 1, abort_flag) ? 1 : 0;
+        if (lane == 0)
+            ok = (stall_ok(p, 4, local, gate, abort_flag) &&
+                  wait_bounded(bar_afull + 8 * buf, (local >> 1) & 1, abort_flag)) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
@@ -640,8 +660,10 @@ dwsep_conv1d_tc_kernel(const Params p, const __grid_constant__ CUtensorMap pw_ma
                     pending[stage] = true;
                 }
             }
-            // On an abort, wait (bounded) for copies still in flight before the CTA can exit.
-            if (!ok) {
+            // Wait (bounded) for copies still in flight before the CTA can exit,
+            // also when another role gave up and they were never consumed
+            // (normally they have all landed and this returns at once).
+            {
                 for (int st = 0; st < 2; ++st) {
                     if (!pending[st]) continue;
                     const int last = seq - 1 - ((seq - 1 - st) & 1);  // latest sequence number on this stage

@@ -376,9 +376,11 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                     }
                 }
             }
-            if (!ok) {
-                // After an abort, wait (bounded) for copies still in flight: the
-                // latest use of stage s is number u = issued-1-((issued-1-s) mod 3).
+            {
+                // Wait (bounded) for copies still in flight before the CTA can
+                // exit, also when another role gave up and they were never
+                // consumed (normally they have all landed): the latest use of
+                // stage s is number u = issued-1-((issued-1-s) mod 3).
                 for (int st = 0; st < STAGES; ++st) {
                     if (!pending[st]) continue;
                     const int u = issued - 1 - ((issued - 1 - st) % STAGES);

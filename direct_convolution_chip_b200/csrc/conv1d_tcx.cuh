@@ -41,7 +41,7 @@ constexpr uint32_t X_BYTES = (uint32_t)XW * KC * 4;         // 18,944 B per chun
 constexpr int DWX_MAX = 8192;                               // resident depthwise weights, [K][32*nk]
 constexpr uint32_t OFF_DWS = STAGES * STAGE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_DWS + DWX_MAX * 4;
-constexpr uint32_t NBAR = 11;
+constexpr uint32_t NBAR = 12;  // full[2] empty[2] afull[2] aempty[2] drain tma[2] gate
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;           // slack to align the base to 1024 B
@@ -103,6 +103,7 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     const uint32_t bar_aempty = bar_full + 48;       // + 8 * buf
     const uint32_t bar_drain = bar_full + 64;
     const uint32_t bar_tma = bar_full + 72;          // + 8 * stage
+    const uint32_t bar_gate = bar_full + 88;         // never completed (failure-path test)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
     volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 8);
@@ -119,6 +120,7 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         mbar_init(bar_drain, 1);
         mbar_init(bar_tma, 1);       // expect_tx arrival + TMA bytes
         mbar_init(bar_tma + 8, 1);
+        mbar_init(bar_gate, 1);
         *abort_flag = 0u;
         *prod_abort = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -148,14 +150,16 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         // ------------------------------------------------------------ producers
         const int ptid = threadIdx.x;
         const int K = KT > 0 ? KT : p.K;
-        int seq = 0;
+        int seq = 0, local = 0;
         bool run = true;
-        for (int tile = blockIdx.x; run && tile < p.total_tiles; tile += gridDim.x) {
+        for (int tile = blockIdx.x; run && tile < p.total_tiles; tile += gridDim.x, ++local) {
             for (int kc = 0; kc < nk; ++kc, ++seq) {
                 const int stage = seq & 1;
                 const uint32_t parity = (seq >> 1) & 1;
+                if (ptid == 0 && kc == 0 && !stall_ok(p, 2, local, bar_gate, abort_flag)) *prod_abort = 1u;
                 // The TMA copies of this stage (pw chunk and halo) have landed.
-                if (ptid == 0 && !wait_bounded(bar_tma + 8 * stage, parity, abort_flag)) *prod_abort = 1u;
+                if (ptid == 0 && !*prod_abort && !wait_bounded(bar_tma + 8 * stage, parity, abort_flag))
+                    *prod_abort = 1u;
                 asm volatile("bar.sync 1, 256;\n" ::: "memory");
                 if (*prod_abort) {
                     run = false;
@@ -232,7 +236,8 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     } else if (warp == MMA_WARP) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0)
-            mma_issuer(p, tmem, sbase, bar_full, bar_empty, bar_afull, bar_aempty, bar_drain, abort_flag, nk);
+            mma_issuer(p, tmem, sbase, bar_full, bar_empty, bar_afull, bar_aempty, bar_drain, abort_flag, nk,
+                       bar_gate);
         __syncwarp();
     } else if (warp == TMA_WARP) {
         // -------------------------------------------------------- TMA issuer
@@ -240,7 +245,9 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             int seq = 0;
             bool pending[2] = {false, false};
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+            int local = 0;
+            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++local) {
+                if (!stall_ok(p, 1, local, bar_gate, abort_flag)) break;
                 const TileCoord tcd = decode_tile(p, tile);
                 const int x0 = tcd.t0 - p.pad - R;  // a multiple of 4: 16-byte aligned time coordinate
                 // Pull the next tile's halo boxes into L2 now, so its TMA loads
@@ -263,8 +270,10 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                     pending[stage] = true;
                 }
             }
-            // On an abort, wait (bounded) for copies still in flight before the CTA can exit.
-            if (!ok) {
+            // Wait (bounded) for copies still in flight before the CTA can exit,
+            // also when another role gave up and they were never consumed
+            // (normally they have all landed and this returns at once).
+            {
                 for (int st = 0; st < 2; ++st) {
                     if (!pending[st]) continue;
                     const int last = seq - 1 - ((seq - 1 - st) & 1);  // latest sequence number on this stage
@@ -278,7 +287,7 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        epilogue_warp(p, tmem, bar_afull, bar_aempty, abort_flag, warp, lane);
+        epilogue_warp(p, tmem, bar_afull, bar_aempty, abort_flag, warp, lane, bar_gate);
     }
 
     tc_fence_before();
@@ -302,9 +311,13 @@ inline bool conv1d_tcx_supported(int C, int T, int O, int K, int stride, const v
 }
 
 inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float* pw, const float* bias, int N,
-                                   int C, int T, int O, int K, int pad, int To, float* out, cudaStream_t stream)
+                                   int C, int T, int O, int K, int pad, int To, float* out, cudaStream_t stream,
+                                   int stall_role = 0, int stall_at = 0, unsigned long long stall_ns = 0)
 {
     tc::Params prm;
+    prm.stall_role = stall_role;
+    prm.stall_at = stall_at;
+    prm.stall_ns = stall_ns;
     prm.x = x; prm.dw = dw; prm.pw = pw; prm.bias = bias; prm.out = out;
     prm.C = C; prm.T = T; prm.O = O; prm.K = K; prm.pad = pad; prm.To = To;
     prm.tiles_t = (To + tc::TM - 1) / tc::TM;

@@ -257,8 +257,10 @@ __device__ __forceinline__ void tma_halo_warp(const Params& p, const CUtensorMap
                 pending[b] = true;
             }
         }
-        if (!ok) {
-            // After an abort, wait (bounded) for boxes still in flight.
+        {
+            // Wait (bounded) for boxes still in flight before the CTA may leave,
+            // also when another role gave up and they were never consumed
+            // (normally they have all landed and this returns at once).
             for (int b = 0; b < 2; ++b) {
                 if (!pending[b]) continue;
                 const int last = seq - 1 - ((seq - 1 - b) & 1);  // latest sequence number on buffer b

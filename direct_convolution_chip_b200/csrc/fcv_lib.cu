@@ -13,6 +13,7 @@
 #include "conv2d_direct.cuh"
 #include "conv2d_poolfirst.cuh"
 #include "conv2d_tc.cuh"
+#include "conv2d_tcs.cuh"
 
 #define FCV_VERSION_MAJOR 0
 #define FCV_VERSION_MINOR 1
@@ -77,22 +78,24 @@ int check_conv1d(const float* x, const float* dw, const float* pw, const float* 
 // kernel, which spreads any grid over every SM, wins.
 constexpr long long kConv2dFmaMinCtas = 128;
 
-// What AUTO runs for op A: the tensor-core kernel where it applies, unless
-// the layer is narrow (Cin < 4 or Cout <= 32) and the FMA kernel's grid fills
-// at least kConv2dFmaMinCtas CTAs.  Every tile costs the tensor-core kernel the same 27 MMAs
-// and A-operand build whatever Cout is, while the FMA kernel's time scales
-// with Cin * Cout: on x[16,Cin,509,509], pool 4, FMA measured 880 vs 1,069 us
-// at Cin 16, Cout 32, 1,709 vs 2,280 at Cin 32, Cout 32 and 338 vs 451 at
-// Cin 3, Cout 48, and the other way 830 vs 489 at Cin 8, Cout 48.  On a small
-// grid the FMA kernel leaves most SMs idle: x[2,8,64,64], Cout 16, pool 4 runs
-// 34.8 us on its 4 CTAs against 10.3 us on the tensor cores.
-bool conv2d_auto_tc(int N, int Cin, int Cout, int pool, int PH, int PW)
+// What AUTO runs for op A.  Narrow layers (Cin < 4 or Cout <= 32) whose FMA
+// grid fills at least kConv2dFmaMinCtas CTAs stay on FP32 FMA; otherwise the
+// shifted-operand tensor-core kernel where it applies (Cin <= 16, pool 1, 2, 4
+// or 8, 16-byte aligned x), else the im2col tensor-core kernel where it
+// applies, else FP32 FMA.
+int conv2d_auto_algo_for(int N, int Cin, int Cout, int pool, int PH, int PW, bool x_aligned16)
 {
-    if (!fcv::conv2d_tc_supported(Cin, Cout, pool)) return false;
-    if (Cin >= 4 && Cout > 32) return true;
-    int ty = 0, tx = 0, cb = 0;
-    if (!fcv::conv2d_grid(pool, PH, PW, Cout, &ty, &tx, &cb)) return true;
-    return (long long)N * ty * tx * cb < kConv2dFmaMinCtas;
+    const bool tcs = fcv::conv2d_tcs_supported(Cin, pool, x_aligned16 ? reinterpret_cast<const void*>(16)
+                                                                      : reinterpret_cast<const void*>(4));
+    const bool tc = fcv::conv2d_tc_supported(Cin, Cout, pool);
+    if (!tcs && !tc) return FCV_CONV2D_DIRECT;
+    if (Cin < 4 || Cout <= 32) {
+        int ty = 0, tx = 0, cb = 0;
+        if (fcv::conv2d_grid(pool, PH, PW, Cout, &ty, &tx, &cb) &&
+            (long long)N * ty * tx * cb >= kConv2dFmaMinCtas)
+            return FCV_CONV2D_DIRECT;
+    }
+    return tcs ? FCV_CONV2D_TC_SHIFT_3XTF32 : FCV_CONV2D_TC_3XTF32;
 }
 
 int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin, int H, int W,
@@ -101,31 +104,34 @@ int conv2d_common(const float* x, const float* w, const float* b, int N, int Cin
     int st = check_conv2d(x, w, b, N, Cin, H, W, Cout, pool, out, tap);
     if (st != FCV_OK) return st;
     if (algo != FCV_ALGO_AUTO && algo != FCV_CONV2D_DIRECT && algo != FCV_CONV2D_POOLFIRST &&
-        algo != FCV_CONV2D_TC_3XTF32)
+        algo != FCV_CONV2D_TC_3XTF32 && algo != FCV_CONV2D_TC_SHIFT_3XTF32)
         return FCV_ERR_INVALID_ARG;
     if (algo == FCV_CONV2D_TC_3XTF32 && !fcv::conv2d_tc_supported(Cin, Cout, pool)) return FCV_ERR_UNSUPPORTED;
+    if (algo == FCV_CONV2D_TC_SHIFT_3XTF32 && !fcv::conv2d_tcs_supported(Cin, pool, x)) return FCV_ERR_UNSUPPORTED;
     if (N == 0) return FCV_OK;
     cudaStream_t s = fcv::as_stream(stream);
     const int PH = (H - 2) / pool, PW = (W - 2) / pool;
     if (!tap) {
-        // The kernel accumulates one atomic add per CTA into out[n]; start from zero.
+        // The kernels accumulate atomic adds into out[n]; start from zero.
         if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N, s) != cudaSuccess) return FCV_ERR_CUDA;
     }
     if (PH == 0 || PW == 0) return FCV_OK;  // empty sum: out stays 0; the tap has no elements
-    if (algo == FCV_CONV2D_TC_3XTF32) {
+    if (algo == FCV_ALGO_AUTO)
+        algo = conv2d_auto_algo_for(N, Cin, Cout, pool, PH, PW, (reinterpret_cast<uintptr_t>(x) & 15) == 0);
+    switch (algo) {
+    case FCV_CONV2D_TC_SHIFT_3XTF32:
+        return tap ? fcv::launch_conv2d_tcs<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
+                   : fcv::launch_conv2d_tcs<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
+    case FCV_CONV2D_TC_3XTF32:
         return tap ? fcv::launch_conv2d_tc<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
                    : fcv::launch_conv2d_tc<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
-    }
-    if (algo == FCV_CONV2D_POOLFIRST) {
+    case FCV_CONV2D_POOLFIRST:
         return tap ? fcv::launch_conv2d_poolfirst<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
                    : fcv::launch_conv2d_poolfirst<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
+    default:
+        return tap ? fcv::launch_conv2d_direct<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
+                   : fcv::launch_conv2d_direct<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
     }
-    if (algo == FCV_ALGO_AUTO && conv2d_auto_tc(N, Cin, Cout, pool, PH, PW)) {
-        return tap ? fcv::launch_conv2d_tc<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
-                   : fcv::launch_conv2d_tc<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
-    }
-    return tap ? fcv::launch_conv2d_direct<fcv::kTap>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s)
-               : fcv::launch_conv2d_direct<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s);
 }
 
 }  // namespace
@@ -227,6 +233,39 @@ int fcv_selftest_wait_timeout(unsigned long long limit_ns, void* stream)
     return fcv::launch_status();
 }
 
+int fcv_selftest_conv2d_stall(const float* x, const float* w, const float* b, int N, int Cin, int H, int W,
+                              int Cout, int pool, float* out, int role, int at_unit, unsigned long long limit_ns,
+                              void* stream)
+{
+    int st = check_conv2d(x, w, b, N, Cin, H, W, Cout, pool, out, false);
+    if (st != FCV_OK) return st;
+    if (role < 1 || role > 4 || at_unit < 0 || limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000)
+        return FCV_ERR_INVALID_ARG;
+    if (!fcv::conv2d_tcs_supported(Cin, pool, x)) return FCV_ERR_UNSUPPORTED;
+    if (N == 0) return FCV_OK;
+    cudaStream_t s = fcv::as_stream(stream);
+    const int PH = (H - 2) / pool, PW = (W - 2) / pool;
+    if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)N, s) != cudaSuccess) return FCV_ERR_CUDA;
+    if (PH == 0 || PW == 0) return FCV_OK;
+    return fcv::launch_conv2d_tcs<fcv::kSumAtomic>(x, w, b, N, Cin, H, W, Cout, pool, PH, PW, out, s, limit_ns, role,
+                                                   at_unit);
+}
+
+int fcv_selftest_conv1d_stall(const float* x, const float* dw_w, const float* pw_w, const float* bias, int N, int C,
+                              int T, int O, int K, int stride, int pad, float* out, int role, int at_tile,
+                              unsigned long long limit_ns, void* stream)
+{
+    int To = 0;
+    int st = check_conv1d(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, out, &To);
+    if (st != FCV_OK) return st;
+    if (role < 1 || role > 4 || at_tile < 0 || limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000)
+        return FCV_ERR_INVALID_ARG;
+    if (!fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w)) return FCV_ERR_UNSUPPORTED;
+    if (N == 0) return FCV_OK;
+    return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, fcv::as_stream(stream), role,
+                                        at_tile, limit_ns);
+}
+
 int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* algo)
 {
     if (!algo) return FCV_ERR_INVALID_ARG;
@@ -234,7 +273,7 @@ int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* 
     if (!mul_ok(N, Cin, H, W) || !mul_ok(N, Cout, H, W)) return FCV_ERR_INVALID_ARG;
     if (pool > 8) return FCV_ERR_UNSUPPORTED;
     const int PH = (H - 2) / pool, PW = (W - 2) / pool;
-    *algo = conv2d_auto_tc(N, Cin, Cout, pool, PH, PW) ? FCV_CONV2D_TC_3XTF32 : FCV_CONV2D_DIRECT;
+    *algo = conv2d_auto_algo_for(N, Cin, Cout, pool, PH, PW, true);
     return FCV_OK;
 }
 
@@ -328,21 +367,26 @@ constexpr size_t kNoAllocScratchBytes = 256 * 1024;  // the largest workspace th
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kNoAllocMaxDevices = 64;
-std::once_flag g_noalloc_once[kNoAllocMaxDevices];
-void* g_noalloc_ptr[kNoAllocMaxDevices];
-cudaError_t g_noalloc_status[kNoAllocMaxDevices];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices];  // cached device address per device; NULL until a lookup succeeds
 
-// Device address of g_noalloc_scratch on the current device, looked up once per
-// device (with that device current) and then cached.
+// Device address of g_noalloc_scratch on the current device, looked up with
+// that device current the first time it is needed and then cached.  A failed
+// lookup is not cached: the next call tries again.
 int noalloc_scratch(void** ptr)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
     if (dev < 0 || dev >= kNoAllocMaxDevices) return FCV_ERR_UNSUPPORTED;
-    std::call_once(g_noalloc_once[dev], [dev] {
-        g_noalloc_status[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
-    });
-    if (g_noalloc_status[dev] != cudaSuccess || g_noalloc_ptr[dev] == nullptr) return FCV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            (void)cudaGetLastError();  // leave no sticky status behind for the caller's next call
+            return FCV_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
     *ptr = g_noalloc_ptr[dev];
     return FCV_OK;
 }

@@ -38,7 +38,10 @@
  *     returns early.
  *   - N == 0 (an empty batch) is valid and enqueues nothing.
  *   - The library holds no per-call state; concurrent calls on different
- *     streams with disjoint outputs are safe.
+ *     streams with disjoint outputs are safe.  The one exception is
+ *     fcv_conv2d_pool_sigmoid_sum_noalloc: all its calls on a device share one
+ *     library-owned 256 KiB array, so calls that overlap on the GPU race and
+ *     must be serialised by the caller.
  */
 #ifndef FCV_H
 #define FCV_H
@@ -76,6 +79,12 @@ typedef enum {
     FCV_CONV2D_TC_3XTF32 = 12,    /* the direct method as an implicit GEMM on tcgen05 tensor
                                      cores (K = 9*Cin, N = Cout), fp32-accurate through a
                                      3xTF32 split; pool 1, 2, 4 or 8 and Cout <= 112 only,
+                                     UNSUPPORTED otherwise */
+    FCV_CONV2D_TC_SHIFT_3XTF32 = 13, /* the direct method on tcgen05 tensor cores with four images
+                                     side by side in the MMA's N dimension, so that each of the
+                                     nine taps reads the staged input rows in place (no im2col);
+                                     M = 64 output channels x (TF32 hi | lo weights), fp32-accurate;
+                                     Cin <= 16, pool 1, 2, 4 or 8 and a 16-byte aligned x only,
                                      UNSUPPORTED otherwise */
     /* op B */
     FCV_CONV1D_FMA = 20,          /* depthwise + pointwise on FP32 FMA */
@@ -141,7 +150,11 @@ int fcv_conv2d_pool_sigmoid_sum_det(const float* x, const float* w, const float*
  * The workspace is a 256 KiB array in the library's own device memory (every
  * GPU that loads the library holds it until the process exits).  The first
  * call on each device looks up that array's address (cudaGetSymbolAddress) with
- * the device current; make that first call before any stream capture.  Sizes
+ * the device current and keeps it for later calls; make that first call before
+ * any stream capture.  A failed lookup returns FCV_ERR_CUDA and is tried again
+ * on the next call.  The kept address belongs to the device's context at the
+ * time of the lookup: after cudaDeviceReset it is no longer valid, so do not
+ * use this entry point in a process after resetting the device.  Sizes
  * whose workspace (fcv_conv2d_workspace_bytes) exceeds 256 KiB are rejected
  * with FCV_ERR_UNSUPPORTED before anything is enqueued.  All calls on a device
  * share the one array: calls that overlap on the GPU (other streams, other
@@ -237,6 +250,36 @@ int fcv_device_error(void* stream);
  * following fcv_device_error(stream) returns FCV_ERR_TIMEOUT and the context
  * stays usable.  Nothing faults, traps or hangs.  Asynchronous on `stream`. */
 int fcv_selftest_wait_timeout(unsigned long long limit_ns, void* stream);
+
+/* Test of the failure path of the shifted-operand tensor-core conv2d
+ * (FCV_CONV2D_TC_SHIFT_3XTF32; no counterpart on the pages).  Runs that kernel
+ * on op A's arguments, except that one role of every thread block waits, just
+ * before its `at_unit`-th unit of work, on a barrier nothing completes, with a
+ * wait limit of `limit_ns` (1 ns .. 10 s; the same limit then bounds that
+ * block's other main-loop waits).  The wait gives up, records FCV_ERR_TIMEOUT
+ * in the device error word and sets the block's abort flag; every role leaves
+ * its loop, the copies and MMAs already issued are waited for, tensor memory
+ * is freed and the kernel exits.  `out` is zeroed first and then holds a
+ * partial sum.  role: 1 loader, 2 producers, 3 MMA issuer, 4 epilogue.
+ * INVALID_ARG for a role outside 1..4, at_unit < 0 or limit_ns outside its
+ * range, UNSUPPORTED where that kernel does not apply; otherwise as
+ * fcv_conv2d_pool_sigmoid_sum.  Asynchronous on `stream`. */
+int fcv_selftest_conv2d_stall(const float* x, const float* w, const float* b,
+                              int N, int Cin, int H, int W, int Cout, int pool,
+                              float* out, int role, int at_unit, unsigned long long limit_ns,
+                              void* stream);
+
+/* The same test for op B's TMA-halo tensor-core kernel (FCV_CONV1D_TC_TMA_3XTF32):
+ * one role of every thread block (1 TMA warp, 2 producers, 3 MMA issuer, 4
+ * epilogue) waits, before its `at_tile`-th output tile, on a barrier nothing
+ * completes, with limit `limit_ns` (1 ns .. 10 s); the block then takes its
+ * abort path and FCV_ERR_TIMEOUT is recorded.  `out` holds partial results.
+ * INVALID_ARG / UNSUPPORTED as for fcv_selftest_conv2d_stall, with that
+ * kernel's envelope; otherwise as fcv_dwsep_conv1d. */
+int fcv_selftest_conv1d_stall(const float* x, const float* dw_w, const float* pw_w, const float* bias,
+                              int N, int C, int T, int O, int K, int stride, int pad,
+                              float* out, int role, int at_tile, unsigned long long limit_ns,
+                              void* stream);
 
 #ifdef __cplusplus
 }

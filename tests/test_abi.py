@@ -17,6 +17,7 @@ OK, INVALID, UNSUPPORTED = 0, 1, 2
 P = ctypes.c_void_p
 FAKE = P(0x10000)     # never dereferenced: every call below returns during validation
 MISALIGNED = P(0x10002)
+ALIGNED4 = P(0x10004)  # 4-byte aligned, not 16-byte aligned
 
 
 def declared_functions():
@@ -65,10 +66,45 @@ def c1d(lib, x=FAKE, dw=FAKE, pw=FAKE, bias=FAKE, N=2, C=8, T=64, O=16, K=9, s=1
     dict(N=-1), dict(Cin=0), dict(Cout=0), dict(H=2), dict(W=2), dict(pool=0),
     dict(x=MISALIGNED), dict(out=MISALIGNED),
     dict(N=1 << 30, Cin=1 << 30, H=1 << 20, W=1 << 20),  # element count overflows int64
-    dict(algo=999), dict(algo=21), dict(algo=13),
+    dict(algo=999), dict(algo=21), dict(algo=14),
 ])
 def test_conv2d_invalid(lib, kw):
     assert c2d(lib, **kw) == INVALID
+
+
+@pytest.mark.parametrize("kw", [dict(Cin=17), dict(pool=3), dict(x=ALIGNED4)])
+def test_conv2d_shifted_tensor_core_envelope(lib, kw):
+    """The shifted-operand tensor-core kernel takes Cin <= 16, pool 1/2/4/8 and a
+    16-byte aligned x; outside that an explicit request is UNSUPPORTED."""
+    assert c2d(lib, algo=13, **kw) == UNSUPPORTED
+
+
+def stall2d(lib, role=1, at=0, limit=1000, **kw):
+    a = dict(x=FAKE, w=FAKE, b=FAKE, N=2, Cin=8, H=64, W=64, Cout=16, pool=4, out=FAKE)
+    a.update(kw)
+    return lib.fcv_selftest_conv2d_stall(a["x"], a["w"], a["b"], a["N"], a["Cin"], a["H"], a["W"], a["Cout"],
+                                         a["pool"], a["out"], role, at, limit, None)
+
+
+def stall1d(lib, role=1, at=0, limit=1000, **kw):
+    a = dict(x=FAKE, dw=FAKE, pw=FAKE, bias=FAKE, N=2, C=32, T=64, O=16, K=9, s=1, p=4, out=FAKE)
+    a.update(kw)
+    return lib.fcv_selftest_conv1d_stall(a["x"], a["dw"], a["pw"], a["bias"], a["N"], a["C"], a["T"], a["O"], a["K"],
+                                         a["s"], a["p"], a["out"], role, at, limit, None)
+
+
+@pytest.mark.parametrize("fn", [stall2d, stall1d])
+@pytest.mark.parametrize("kw,want", [(dict(role=0), "inv"), (dict(role=5), "inv"), (dict(at=-1), "inv"),
+                                     (dict(limit=0), "inv"), (dict(limit=11 * 10**9), "inv"), (dict(N=0), "ok")])
+def test_stall_selftests_validate_on_the_host(lib, fn, kw, want):
+    """The failure-path test entry points reject bad roles, units and limits
+    before any CUDA call (N == 0 enqueues nothing)."""
+    assert fn(lib, **kw) == {"inv": INVALID, "ok": OK}[want]
+
+
+def test_stall_selftests_outside_their_kernels(lib):
+    assert stall2d(lib, Cin=20) == UNSUPPORTED
+    assert stall1d(lib, s=2) == UNSUPPORTED
 
 
 def test_conv2d_unsupported_pool(lib):
@@ -141,23 +177,27 @@ def test_selftest_rejects_bad_limits(lib):
 
 
 def test_auto_algo_conv2d(lib):
-    """AUTO runs the tensor-core direct conv where it covers the shape, else the FMA kernel."""
+    """AUTO: FMA for narrow layers (Cin < 4 or Cout <= 32) once the FMA grid has
+    128 CTAs; else the shifted-operand tensor-core kernel (Cin <= 16, pool 1, 2,
+    4 or 8), else the im2col tensor-core kernel where it fits, else FMA."""
     a = ctypes.c_int()
     q = lib.fcv_conv2d_auto_algo
-    assert q(128, 8, 384, 384, 64, 4, ctypes.byref(a)) == OK and a.value == 12  # the full-size workload
+    assert q(128, 8, 384, 384, 64, 4, ctypes.byref(a)) == OK and a.value == 13  # the full-size workload
     for pool in (1, 2, 8):
-        assert q(2, 8, 40, 40, 48, pool, ctypes.byref(a)) == OK and a.value == 12
+        assert q(2, 8, 40, 40, 48, pool, ctypes.byref(a)) == OK and a.value == 13
     # narrow layers (Cin < 4 or Cout <= 32): FMA once its grid has 128 CTAs
     assert q(16, 3, 130, 130, 32, 4, ctypes.byref(a)) == OK and a.value == 10   # exactly 128
-    assert q(15, 3, 130, 130, 32, 4, ctypes.byref(a)) == OK and a.value == 12   # 120
+    assert q(15, 3, 130, 130, 32, 4, ctypes.byref(a)) == OK and a.value == 13   # 120
     assert q(16, 3, 509, 509, 32, 4, ctypes.byref(a)) == OK and a.value == 10
     assert q(16, 3, 509, 509, 48, 4, ctypes.byref(a)) == OK and a.value == 10
     assert q(16, 16, 509, 509, 32, 4, ctypes.byref(a)) == OK and a.value == 10
-    assert q(2, 3, 40, 40, 32, 4, ctypes.byref(a)) == OK and a.value == 12      # 8 FMA CTAs: tensor cores
-    assert q(2, 8, 64, 64, 16, 4, ctypes.byref(a)) == OK and a.value == 12      # the small workload
-    assert q(2, 4, 40, 40, 33, 4, ctypes.byref(a)) == OK and a.value == 12      # Cin >= 4, Cout > 32
+    assert q(2, 3, 40, 40, 32, 4, ctypes.byref(a)) == OK and a.value == 13      # 8 FMA CTAs: tensor cores
+    assert q(2, 8, 64, 64, 16, 4, ctypes.byref(a)) == OK and a.value == 13      # the small workload
+    assert q(2, 4, 40, 40, 33, 4, ctypes.byref(a)) == OK and a.value == 13      # Cin >= 4, Cout > 32
+    assert q(2, 8, 40, 40, 128, 4, ctypes.byref(a)) == OK and a.value == 13     # two launches of 64 channels
+    assert q(2, 20, 40, 40, 48, 4, ctypes.byref(a)) == OK and a.value == 12     # Cin > 16: im2col kernel
     assert q(2, 8, 40, 40, 16, 3, ctypes.byref(a)) == OK and a.value == 10      # pool 3: FMA path
-    assert q(2, 8, 40, 40, 128, 4, ctypes.byref(a)) == OK and a.value == 10     # Cout > 112: FMA path
+    assert q(2, 40, 40, 40, 128, 4, ctypes.byref(a)) == OK and a.value == 10    # neither tensor-core kernel
     assert q(2, 3, 40, 40, 16, 9, ctypes.byref(a)) == UNSUPPORTED
     assert q(2, 0, 40, 40, 16, 4, ctypes.byref(a)) == INVALID
     assert q(2, 3, 40, 40, 16, 4, None) == INVALID

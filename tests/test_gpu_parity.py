@@ -17,7 +17,8 @@ from tests.parity import assert_close, requires_cuda, sample_indices
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
 
-CONV2D_ALGOS = [fcv.CONV2D_DIRECT, fcv.CONV2D_POOLFIRST, fcv.CONV2D_TC_3XTF32]
+CONV2D_ALGOS = [fcv.CONV2D_DIRECT, fcv.CONV2D_POOLFIRST, fcv.CONV2D_TC_3XTF32, fcv.CONV2D_TC_SHIFT_3XTF32]
+CONV2D_TC_ALGOS = (fcv.CONV2D_TC_3XTF32, fcv.CONV2D_TC_SHIFT_3XTF32)
 CONV1D_ALGOS = [fcv.CONV1D_FMA, fcv.CONV1D_TC_3XTF32, fcv.CONV1D_TC2_3XTF32, fcv.CONV1D_TC_TMA_3XTF32]
 
 
@@ -47,8 +48,8 @@ def conv2d_or_skip(fn, x, w, b, pool, algo):
     try:
         return fn(x, w, b, pool, algo=algo)
     except fcv.FcvError as e:
-        if e.status == 2 and algo == fcv.CONV2D_TC_3XTF32:
-            pytest.skip("tensor-core conv2d does not cover this shape")
+        if e.status == 2 and algo in CONV2D_TC_ALGOS:
+            pytest.skip("this tensor-core conv2d does not cover this shape")
         raise
 
 
@@ -112,6 +113,13 @@ EDGE_2D = [
     (1, 16, 36, 68, 96, 2),    # weights too large for the tensor-core kernel: AUTO and FMA only
     (2, 8, 48, 40, 80, 8),     # sub-chunk kernel, pool 8, Cout 80 (two accumulators)
     (1, 9, 30, 34, 64, 4),     # W % 4 != 0: full-chunk kernel with the cp.async halo
+    # shifted-operand tensor-core conv2d envelope
+    (5, 8, 40, 76, 64, 4),     # N % 4 != 0: the last image group is partial (TMA rows)
+    (6, 16, 30, 41, 200, 2),   # two K chunks, four launches of <= 64 channels, cp.async rows, N % 4 != 0
+    (9, 3, 21, 134, 64, 8),    # Cin padded to 8, pool 8, three column tiles with a ragged last one
+    (4, 12, 19, 20, 65, 1),    # pool 1, Cout one past a block, W % 4 == 0 with two K chunks
+    (2, 7, 67, 257, 31, 4),    # W % 4 == 1 (every row a different 16-byte phase), ragged tiles
+    (1, 16, 10, 10, 1, 2),     # a single unit: the CTA has no continuation
 ]
 
 

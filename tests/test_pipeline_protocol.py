@@ -390,3 +390,259 @@ def test_model_catches_a_leader_that_ignores_the_peer_epilogue():
         except AssertionError as e:
             failures += "releases done" in str(e)
     assert failures > 0
+
+
+
+# ------------------------------------------------------------------------------
+# conv2d_tcs_kernel (csrc/conv2d_tcs.cuh): the input rows of a CTA's contiguous
+# range of units stream through NSTG staging buffers (loader -> producers) and
+# NSLOT row slots (producers -> MMA issuer); the issuer releases a slot after
+# the last conv row that reads it and hands two accumulators to the epilogue.
+# The abort model lets any main-loop wait give up (a timeout): every role then
+# leaves its loop, the loader waits for the last box it issued on each staging
+# buffer, the issuer commits a drain barrier and waits for it, and the CTA
+# leaves.  At that point no TMA box and no MMA may still be in flight.
+
+
+def shifted_units(P, u0, u1, PH):
+    """(base row sequence number, continues into the next unit) per unit, and
+    the number of rows loaded, as every role of the kernel derives them."""
+    units, s = [], 0
+    for u in range(u0, u1):
+        ph = u % PH
+        fj = 2 if (u > u0 and ph > 0) else 0
+        units.append((s - fj, u + 1 < u1 and ph + 1 < PH))
+        s += P + 2 - fj
+    return units, s
+
+
+class AbortSim(Sim):
+    """Sim whose role agents are (loop steps, steps after the loop).  A "wait"
+    inside the loop may give up once the abort flag is set, or start the abort
+    with probability p_abort; the role then runs its after-loop steps, whose
+    waits always end (drain waits).  Asynchronous work (TMA boxes, MMAs with
+    their commits) goes into FIFO queues, one per unit, which complete in order
+    at any later time.
+
+    Extra steps: ("enqueue", queue, actions) issues asynchronous work whose
+    completion runs `actions`; ("mark", s, nstg) records the last box issued on
+    a staging buffer; ("tma_drain", nstg, who) passes once the last box issued
+    on every staging buffer has landed; ("write", buf, use) fills a buffer and
+    ("read", buf, use, who) -- run when an MMA completes, i.e. at the end of its
+    asynchronous read -- checks that the buffer still holds that use."""
+
+    def __init__(self):
+        super().__init__()
+        self.roles, self.queues, self.done, self.last_issue, self.content = [], {}, {}, {}, {}
+
+    def can_run(self, st):
+        if st[0] in ("write", "read"):
+            return True
+        if st[0] == "tma_drain":
+            _, nstg, _who = st
+            for b in range(nstg):
+                last = self.last_issue.get(b)
+                if last is not None and self.bars[f"stgf{b}"].phase < last // nstg + 1:
+                    return False
+            return True
+        if st[0] in ("enqueue", "mark", "end_loop"):
+            return True
+        return super().can_run(st)
+
+    def step(self, st):
+        if st[0] == "enqueue":
+            self.queues.setdefault(st[1], []).append(st[2])
+            self.counters[st[1]] = self.counters.get(st[1], 0) + 1
+        elif st[0] == "mark":
+            self.last_issue[st[1] % st[2]] = st[1]
+        elif st[0] == "write":
+            self.content[st[1]] = st[2]
+        elif st[0] == "read":
+            _, buf, use, who = st
+            assert self.content.get(buf) == use, (f"{who}: {buf} use {use} overwritten by use "
+                                                  f"{self.content.get(buf)} before the read completed")
+        elif st[0] in ("tma_drain", "end_loop"):
+            pass
+        else:
+            super().step(st)
+
+    def complete(self, q):
+        self.done[q] = self.done.get(q, 0) + 1
+        for act in self.queues[q].pop(0):
+            self.step(act)
+
+    def run(self, seed, p_abort=0.0):
+        rng = random.Random(seed)
+        steps = [list(m) + [("end_loop",)] + list(post) for m, post in self.roles]
+        post_at = [len(m) for m, _ in self.roles]
+        pcs = [0] * len(steps)
+        aborted = False
+        while True:
+            if all(pcs[i] >= len(a) for i, a in enumerate(steps)):
+                # The CTA leaves (__syncthreads, TMEM dealloc, exit): nothing it
+                # issued may still be in flight.
+                for q, n in self.counters.items():
+                    assert self.done.get(q, 0) == n, f"{q}: {n - self.done.get(q, 0)} still in flight at exit"
+                break
+            moves = []
+            for i, a in enumerate(steps):
+                if pcs[i] >= len(a):
+                    continue
+                st = a[pcs[i]]
+                if st[0] == "wait" and pcs[i] < post_at[i] and (aborted or p_abort > 0):
+                    moves.append(("giveup", i))
+                if self.can_run(st):
+                    moves.append(("role", i))
+            for q, items in self.queues.items():
+                if items:
+                    moves.append(("complete", q))
+            assert moves, "deadlock at " + str([a[pcs[i]] for i, a in enumerate(steps) if pcs[i] < len(a)])
+            kind, i = rng.choice(moves)
+            if kind == "giveup":
+                if not aborted and rng.random() > p_abort:
+                    continue
+                aborted = True
+                pcs[i] = post_at[i] + 1
+            elif kind == "role":
+                self.step(steps[i][pcs[i]])
+                pcs[i] += 1
+            else:
+                self.complete(i)
+        if not aborted:
+            for bar in self.bars.values():
+                assert bar.pending == 0, f"{bar.name}: {bar.pending} arrivals left over"
+        return aborted
+
+
+def shifted_kernel(P, u0, u1, PH, nslot, nstg, nprod=4, planted=None):
+    """The roles of conv2d_tcs_kernel for one CTA with units [u0, u1) of strips of
+    PH pooled rows.  `planted` names a mistake to plant: "drain_only_if_aborted"
+    (the loader skips its drain when its own loop ended normally), "early_release"
+    (a slot is released one conv row early), "no_acc_wait" (the issuer does not
+    wait for a drained accumulator)."""
+    units, S = shifted_units(P, u0, u1, PH)
+    sim = AbortSim()
+    for b in range(nstg):
+        sim.bar(f"stgf{b}", 1)
+        sim.bar(f"stge{b}", 1)
+    for b in range(nslot):
+        sim.bar(f"slotf{b}", 1)
+        sim.bar(f"slote{b}", 1)
+    for b in range(2):
+        sim.bar(f"accf{b}", 1)
+        sim.bar(f"acce{b}", 4)
+    sim.bar("drain", 1)
+    # loader: one box per row into staging buffer s % nstg (the TMA unit lands it later)
+    loop = []
+    for s in range(S):
+        b, k = s % nstg, s // nstg
+        loop += [("wait", f"stge{b}", (k & 1) ^ 1, k, "loader"), ("owns", f"stge{b}", k, "loader"),
+                 ("enqueue", "tma", [("arrive", f"stgf{b}", k, 1, "tma")]), ("mark", s, nstg)]
+    sim.roles.append((loop, [] if planted == "drain_only_if_aborted" else [("tma_drain", nstg, "loader")]))
+    # producers: row s -> warp s % nprod
+    for w in range(nprod):
+        loop = []
+        for s in range(w, S, nprod):
+            b, k, sl, ks = s % nstg, s // nstg, s % nslot, s // nslot
+            loop += [("wait", f"slote{sl}", (ks & 1) ^ 1, ks, f"prod{w}"),
+                     ("wait", f"stgf{b}", k & 1, k + 1, f"prod{w}"),
+                     ("owns", f"slote{sl}", ks, f"prod{w}"), ("write", f"slot{sl}", ks),
+                     ("arrive", f"slotf{sl}", ks, 1, f"prod{w}"), ("arrive", f"stge{b}", k, 1, f"prod{w}")]
+        sim.roles.append((loop, []))
+    # MMA issuer; a commit arrives once the MMAs before it have completed
+    loop = []
+    shift = 1 if planted == "early_release" else 0
+    released = set()
+
+    def commit(bar, use):
+        loop.append(("enqueue", "mma", [("arrive", bar, use, 1, "tcore")]))
+
+    for i, (base, cont) in enumerate(units):
+        ab, ak = i & 1, i >> 1
+        if planted != "no_acc_wait":
+            loop.append(("wait", f"acce{ab}", (ak & 1) ^ 1, ak, "mma"))
+        loop.append(("owns", f"acce{ab}", ak, "mma"))
+        for dy in range(P):
+            for ky in range(3):
+                q = base + dy + ky
+                loop.append(("wait", f"slotf{q % nslot}", (q // nslot) & 1, q // nslot + 1, "mma"))
+            # the conv row's MMAs read the three rows until they complete
+            loop.append(("enqueue", "mma", [("read", f"slot{q % nslot}", q // nslot, "mma")
+                                            for q in range(base + dy, base + dy + 3)]))
+            r = base + dy + shift
+            if r not in released:
+                released.add(r)
+                commit(f"slote{r % nslot}", r // nslot)
+        if not cont:
+            for r in (base + P, base + P + 1):
+                if r not in released:
+                    released.add(r)
+                    commit(f"slote{r % nslot}", r // nslot)
+        commit(f"accf{ab}", ak)
+    sim.roles.append((loop, [("enqueue", "mma", [("arrive", "drain", 0, 1, "tcore")]),
+                             ("wait", "drain", 0, 1, "mma")]))
+    # epilogue: its four warps take one decision per unit (one thread waits)
+    loop = []
+    for i in range(len(units)):
+        ab, ak = i & 1, i >> 1
+        loop += [("wait", f"accf{ab}", ak & 1, ak + 1, "epilogue"), ("arrive", f"acce{ab}", ak, 4, "epilogue")]
+    sim.roles.append((loop, []))
+    return sim
+
+
+SHIFT_UNITS = [(0, 1, 5), (0, 3, 5), (2, 9, 5), (0, 12, 4), (3, 4, 1), (0, 6, 2), (4, 11, 3)]
+
+
+@pytest.mark.parametrize("P", [1, 2, 4, 8])
+@pytest.mark.parametrize("units", SHIFT_UNITS, ids=lambda u: "u%d-%d_ph%d" % u)
+@pytest.mark.parametrize("nslot,nstg", [(8, 4), (4, 4)])
+def test_shifted_kernel_protocol(P, units, nslot, nstg):
+    for seed in range(15):
+        shifted_kernel(P, *units, nslot, nstg).run(seed)
+
+
+@pytest.mark.parametrize("P", [1, 4])
+@pytest.mark.parametrize("units", SHIFT_UNITS, ids=lambda u: "u%d-%d_ph%d" % u)
+def test_shifted_kernel_abort_leaves_nothing_in_flight(P, units):
+    """Any main-loop wait may give up: afterwards every role leaves, and when the
+    CTA exits no TMA box or MMA is in flight."""
+    aborted = 0
+    for seed in range(60):
+        aborted += shifted_kernel(P, *units, 8, 4).run(seed, p_abort=0.05)
+        aborted += shifted_kernel(P, *units, 4, 4).run(seed, p_abort=0.05)
+    assert aborted > 0
+
+
+def _planted_failures(planted, P=2, units=(0, 9, 4), p_abort=0.0, seeds=200, match="", nslot=8, nstg=4):
+    failures = 0
+    for seed in range(seeds):
+        try:
+            shifted_kernel(P, *units, nslot, nstg, planted=planted).run(seed, p_abort=p_abort)
+        except AssertionError as e:
+            failures += match in str(e)
+    return failures
+
+
+def test_shifted_model_catches_a_loader_that_drains_only_after_its_own_timeout():
+    """The mistake fixed in every TMA-issuing warp: a loader whose own loop ends
+    normally, while another role gave up, leaves boxes in flight at exit."""
+    assert _planted_failures("drain_only_if_aborted", p_abort=0.05, match="still in flight") > 0
+
+
+def test_shifted_model_catches_an_early_slot_release():
+    """A slot released one conv row early is refilled while the MMAs of the
+    next conv row still read it."""
+    assert _planted_failures("early_release", match="overwritten") + \
+        _planted_failures("early_release", match="deadlock") > 0
+
+
+def test_shifted_model_catches_a_missing_accumulator_wait():
+    assert _planted_failures("no_acc_wait", match="releases done") > 0
+
+
+def test_shifted_model_catches_buffers_shared_between_producer_warps():
+    """Four producer warps taking rows in turn over three staging buffers:
+    successive uses of one buffer then belong to different warps, and a warp
+    can wait on a buffer two phases ahead of it, where the parity wait passes
+    on a stale phase."""
+    assert _planted_failures(None, nslot=8, nstg=3, match="needs") > 0

@@ -6,8 +6,9 @@ cannot take the device synchronisation cudaMalloc/cudaFree can cause, a fixed
 memory budget): its workspace is a fixed 256 KiB array that lives in the
 library's own device memory.  These tests call it through the C ABI and check
 it against the workspace-taking entry point, fcv_conv2d_pool_sigmoid_sum_det,
-on two calls in a row (the shared array keeps the previous call's contents,
-so the second call shows the call clears what it must).
+bit for bit on two calls in a row (the shared array keeps the previous call's
+contents, so the second call shows the call clears what it must), and against
+the CPU oracle.
 
 This file sorts last so that a run stopping at its first failure has already
 run every other test; it also passes on its own in a fresh process.
@@ -17,6 +18,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from direct_convolution_chip_b200 import binding
 from direct_convolution_chip_b200 import build as fcv_build
 from direct_convolution_chip_b200 import workloads as wl
@@ -72,6 +74,12 @@ def test_noalloc_matches_workspace_entry_point_twice(lib, case):
         results.append(out)
     torch.cuda.synchronize()
     assert lib.fcv_device_error(stream) == 0
+    # Both entry points run the same kernel and add the partial sums in the
+    # same fixed order, so the results agree bit for bit.
     for i, out in enumerate(results):
-        assert_close(out.cpu().double().numpy(), ref.cpu().double().numpy(), f"{case.name} call {i}")
-    assert torch.equal(results[0], results[1])
+        assert torch.equal(out, ref), f"{case.name} call {i}: differs from the workspace entry point"
+    # ... and they match the CPU oracle on the first and last batch items.
+    xn, wn, bn = [t.cpu().numpy() for t in (x, w, b)]
+    for bi in sorted({0, case.N - 1}):
+        want = oracle.conv2d_pool_sigmoid_sum(xn[bi:bi + 1], wn, bn, case.P)
+        assert_close(results[1][bi:bi + 1].cpu().double().numpy(), want, f"{case.name} item {bi} vs oracle")
