@@ -185,17 +185,40 @@ def probe_tf32_tflops():
 # ----------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled while the timed region
+    runs: NVML every ~2 ms in a thread (nvidia-smi every 100 ms when NVML is
+    not importable); mark() brackets the samples that count."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    NVML_REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+                    0x4: "sw_power_cap"}
 
     def __init__(self, device_index):
         self.dev = device_index
         self.proc = None
         self.lines = []
         self.thread = None
+        self.samples = []  # (time, sm_mhz, max_mhz, power_w, reason bits) from NVML
+        self.stop_flag = False
+        self.window = None
+        self.nvml = None
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            handle = pynvml.nvmlDeviceGetHandleByUUID(sel.encode() if isinstance(sel, str) else sel)
+            self.nvml = (pynvml, handle)
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return
         try:
             uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
             sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
@@ -208,11 +231,33 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def _poll_nvml(self):
+        nv, h = self.nvml
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.perf_counter(), sm, mx, pw, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def mark(self, t0, t1):
+        """Host-time window that contains the timed region."""
+        self.window = (t0, t1)
+
     def stop(self):
+        if self.nvml is not None:
+            self.stop_flag = True
+            if self.thread:
+                self.thread.join(timeout=5)
+            return self.summary_nvml()
         if self.proc is None:
             return None
         time.sleep(0.15)
@@ -224,6 +269,18 @@ class ClockSampler:
         if self.thread:
             self.thread.join(timeout=5)
         return self.summary()
+
+    def summary_nvml(self):
+        rows = self.samples
+        if self.window:
+            inside = [r for r in rows if self.window[0] <= r[0] <= self.window[1]]
+            rows = inside or rows
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "nvml"}
+        reasons = sorted({name for r in rows for bit, name in self.NVML_REASONS.items() if r[4] & bit})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": max(r[2] for r in rows),
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(r[3] for r in rows),
+                "source": "nvml, every ~2 ms during the timed region"}
 
     def summary(self):
         sm, mx, pw = [], [], []
@@ -440,6 +497,7 @@ def run_gpu(args):
     torch.cuda.synchronize(device)
     sampler.start()
     time.sleep(0.2)  # let the sampler attach before the timed region
+    h0 = time.perf_counter()
     t_start.record(stream)
     for i in range(K):
         ev[i][0].record(stream)
@@ -449,6 +507,7 @@ def run_gpu(args):
         ev[i][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(device)
+    sampler.mark(h0, time.perf_counter())
     clocks = sampler.stop()
     barrier(use_dist, device)
     total_ms = t_start.elapsed_time(t_end)
@@ -819,6 +878,38 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_profile(args):
+    """Only one fused op, `--steps` times after `--warmup` calls, nothing else
+    launched: the target of the committed ncu captures.  `--batch` replaces the
+    batch size (a smaller case for full-section captures)."""
+    import direct_convolution_chip_b200 as fcv
+    import dataclasses
+    torch.cuda.set_device(0)
+    c = CASE_A if args.profile == "conv2d" else CASE_B
+    if args.batch:
+        c = dataclasses.replace(c, N=args.batch, name=f"{c.name}_n{args.batch}")
+    if c.op == "conv2d":
+        x, w, b = [t.cuda() for t in wl.conv2d_inputs(c)]
+        out = torch.empty((c.N,), device="cuda")
+        fn = lambda: fcv.conv2d_pool_sigmoid_sum(x, w, b, c.P, out=out)
+    else:
+        x, dw, pw, b = [t.cuda() for t in wl.conv1d_inputs(c)]
+        To = (c.T + 2 * c.pad - c.K) // c.stride + 1
+        out = torch.empty((c.N, c.O, To), device="cuda")
+        fn = lambda: fcv.dwsep_conv1d(x, dw, pw, b, c.stride, c.pad, out=out)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": c.name, "steps": args.steps, "ms_per_call": e0.elapsed_time(e1) / args.steps,
+                      "device_error": fcv.device_error()}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -830,12 +921,17 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true", help="with --configs: the 48-point shape sweep as well")
     ap.add_argument("--probe", action="store_true",
                     help="run the FP32-FMA and tcgen05 TF32 peak probes, one JSON line each")
+    ap.add_argument("--profile", choices=["conv2d", "dwsep_conv1d"],
+                    help="run only this op of the step (the target of ncu captures)")
+    ap.add_argument("--batch", type=int, default=0, help="with --profile: batch size instead of the full one")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
     elif args.probe:
         run_probes()
+    elif args.profile:
+        run_profile(args)
     elif args.configs:
         run_configs(args)
     else:

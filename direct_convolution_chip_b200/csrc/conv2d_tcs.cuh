@@ -14,7 +14,8 @@
 // tap (ky, kx) one MMA adds
 //     D[m, j] += sum_ci A_t[m, ci] * X[ci, j],   j = 4 * c + i,
 // with m = 128 weight rows (output channels 0-63 with the TF32 hi part of w,
-// then the same 64 with the lo part), c = conv column of the tile, i = image
+// then the same 64 with the lo part; the A operand, resident in tensor memory
+// for the whole kernel), c = conv column of the tile, i = image
 // of the group and X[ci, j] = x[4g + i, ci, r + ky, c0 + c + kx].  The input
 // row r + ky is staged in shared memory as the MMA's K-major B operand without
 // swizzle: position j = 4c + i owns one 16-byte row holding 4 channels, the
@@ -47,10 +48,12 @@
 //     [channel quad][column][image][4 channels] and split it into TF32 hi/lo
 //     rows of a ring of NSLOT row slots.  Staging buffer and slot of row s are s % 4 and
 //     s % NSLOT, so each belongs to one producer warp.
-//   * warp 2: allocates TMEM (two accumulators of 4 * NCOL columns); one
-//     thread issues 2 * 9 * CCH MMAs per conv row (M = 128, N = 4 * NCOL,
-//     K = 8, both operands from shared memory), releases each row slot after
-//     the last conv row that reads it, and commits a unit's accumulator.
+//   * warp 2: allocates TMEM (two accumulators of 4 * NCOL columns and the
+//     weights, 72 * CCH columns); one thread issues 2 * 9 * CCH MMAs per conv
+//     row (M = 128, N = 4 * NCOL = 192 or 128, K = 8, A from tensor memory, B
+//     from shared memory: measured 18 % faster per MMA than both operands from
+//     shared memory), releases each row slot after the last conv row that
+//     reads it, and commits a unit's accumulator.
 //   * warps 7-10 (epilogue, one per TMEM lane quarter): tcgen05.ld 32 columns
 //     at a time, add the P columns of each window, exchange the hi and lo
 //     halves through shared memory (the two pairs of warps take alternate
@@ -94,34 +97,36 @@ constexpr int SMEM_LIMIT = 227 * 1024;
 // Compile-time geometry of one instance.
 template <int P, int CCH>
 struct Geo {
-    static constexpr int NCOL = CCH == 1 ? 64 : 32;       // conv columns per tile
+    static constexpr int NCOL = CCH == 1 ? 48 : 32;       // conv columns per tile
     static constexpr int NMMA = IMG * NCOL;               // MMA N = accumulator columns
     static constexpr int WPT = NCOL / P;                  // pooled windows per tile
     static constexpr int XC = NCOL + 2;                   // staged columns per row (all read by some tap)
     static constexpr uint32_t PLANE = XC * IMG * 16u;     // one quad of channels: 16 bytes per (column, image)
     static constexpr uint32_t HALF = 2u * CCH * PLANE;    // one hi or lo row copy (2 quads per K chunk)
     static constexpr uint32_t SLOT = 2u * HALF;
-    static constexpr int NSLOT = CCH == 1 ? 8 : 4;        // ring of staged rows (slot s belongs to warp s % 4)
-    // Staging: [channel][image][column] with pitch SP = NCOL + 8 floats (8 mod
-    // 32, so lanes (column 0-7, image 0-3) read distinct banks); a TMA box is
-    // SP columns wide, the cp.async path fills NJ aligned 16-byte copies.
+    static constexpr int NSLOT = 8;                       // ring of staged rows (slot s belongs to warp s % 4)
+    // Staging: [channel][image][column] with pitch SP = NCOL + 8 floats (8 or
+    // 24 mod 32, so lanes (image 0-3, column 0-7) read distinct banks); a TMA
+    // box is SP columns wide, the cp.async path fills NJ aligned 16-byte copies.
     static constexpr int SP = NCOL + 8;
     static constexpr int NJ = SP / 4;
     static constexpr uint32_t STG = IMG * 8u * CCH * SP * 4u;
     static constexpr int V = 32 / P;                      // pooled values per 32-column chunk (8/P windows x 4 images)
     static constexpr int XP = V == 4 ? 4 : V + 4;         // exchange row pitch (floats), conflict-free
     static constexpr int NCHK = NMMA / 32;                // 32-column chunks per accumulator
-    static constexpr uint32_t W_BYTES = 9u * CCH * 4096u; // A operand: 9 taps x CCH chunks of 128 x 8
-    static constexpr uint32_t TMEM_COLS = 2u * NMMA;
+    static constexpr uint32_t WCOL0 = 2u * NMMA;          // TMEM: weights (A) after the two accumulators
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(2 * NMMA + 72 * CCH <= 512, "two accumulators and the weights fit tensor memory");
     static_assert(NCOL % P == 0 && 8 % P == 0, "pool must divide a chunk of 8 columns");
-    static_assert(SP % 32 == 8 && SP >= XC + 3 + 3, "staging pitch: bank spread, and room for the cp.async shift");
+    static_assert((SP % 32 == 8 || SP % 32 == 24) && SP >= XC + 3 + 3,
+                  "staging pitch: bank spread, and room for the cp.async shift");
     static_assert(NSTG % NPRODW == 0 && NSLOT % NPRODW == 0,
                   "every staging buffer and row slot is used by one producer warp only");
 };
 
 // Shared-memory layout (bytes from a 1024-aligned base).
 struct Layout {
-    uint32_t w, slots, stg, xbuf, red, bar, misc, total;
+    uint32_t slots, stg, xbuf, red, bar, misc, total;
 };
 
 template <int P, int CCH>
@@ -129,8 +134,7 @@ __host__ __device__ constexpr Layout make_layout()
 {
     using G = Geo<P, CCH>;
     Layout L{};
-    L.w = 0;
-    L.slots = G::W_BYTES;
+    L.slots = 0;
     L.stg = L.slots + G::NSLOT * G::SLOT;
     L.xbuf = L.stg + NSTG * G::STG;
     L.red = L.xbuf + 2u * CO_BLK * G::XP * 4u;
@@ -141,8 +145,14 @@ __host__ __device__ constexpr Layout make_layout()
     return L;
 }
 
+// Dynamic shared memory requested: the layout plus alignment slack, and at
+// least 120 KB so that two CTAs never share an SM (each allocates all 512 TMEM
+// columns; a second one on the same SM would wait in tcgen05.alloc).
 template <int P, int CCH>
-constexpr uint32_t smem_bytes() { return make_layout<P, CCH>().total + 1024u; }
+constexpr uint32_t smem_bytes()
+{
+    return make_layout<P, CCH>().total + 1024u > 120u * 1024u ? make_layout<P, CCH>().total + 1024u : 120u * 1024u;
+}
 
 struct Params {
     const float* x;
@@ -180,23 +190,25 @@ __device__ __forceinline__ Unit decode(const Params& p, long long u)
     return t;
 }
 
+// The unit after t (ph fastest, then column tile, then image group): every
+// role walks its units this way instead of dividing per unit.
+__device__ __forceinline__ void next_unit(const Params& p, Unit& t)
+{
+    if (++t.ph == p.PH) {
+        t.ph = 0;
+        if (++t.ct == p.CT) {
+            t.ct = 0;
+            ++t.g;
+        }
+    }
+}
+
 // Shared-memory matrix descriptor, no swizzle (canonical interleaved layout):
 // LBO and SBO in bytes, version 1.
 __device__ __forceinline__ uint64_t desc_none(uint32_t saddr, uint32_t lbo, uint32_t sbo)
 {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
            ((uint64_t)1 << 46);
-}
-
-// D[tmem] (+)= A[smem] * B[smem], kind::tf32.
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate)
-{
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
 }
 
 // 32 consecutive 32-bit TMEM columns of the warp's 32 lanes.
@@ -238,24 +250,45 @@ __device__ __forceinline__ float tf32_trunc(float v) { return __uint_as_float(__
 // two input rows.
 __device__ __forceinline__ int first_row(long long u, long long u0, int ph) { return (u > u0 && ph > 0) ? 2 : 0; }
 
-// Weights of this launch as the A operand, K-major without swizzle: block
-// (tap t, chunk c) holds 128 rows x 8 channels, rows 0-63 the TF32 hi part of
-// output channels 0-63 and rows 64-127 their lo part; element (m, k) at
-// (m % 8) * 16 + (m / 8) * 256 + (k / 4) * 128 + (k % 4) * 4.
+// Weights of this launch as the A operand in tensor memory: block (tap t,
+// chunk c) is 8 consecutive columns from WCOL0 + 8 * (t * CCH + c); lane m holds
+// row m, rows 0-63 the TF32 hi part of output channels 0-63 and rows 64-127
+// their lo part; column k of a block is input channel 8c + k.  Written by the
+// four epilogue warps (warp quarter q owns lanes 32q .. 32q + 31).
 template <int CCH>
-__device__ __forceinline__ void stage_weights(const Params& p, uint8_t* smem)
+__device__ __forceinline__ void weights_to_tmem(const Params& p, uint32_t tmem, uint32_t wcol0, int q, int lane)
 {
-    for (int idx = threadIdx.x; idx < 9 * CCH * 1024; idx += NTHREADS) {
-        const int blk = idx >> 10, e = idx & 1023;
-        const int m = e >> 3, k = e & 7;
+    const int m = 32 * q + lane;
+    const int co = m & 63;
+    const bool hi_part = m < 64;
+    const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + wcol0;
+#pragma unroll 1
+    for (int blk = 0; blk < 9 * CCH; ++blk) {
         const int t = blk / CCH, c = blk - t * CCH;
-        const int co = m & 63, ci = 8 * c + k;
-        const float v = (co < p.Cout && ci < p.Cin) ? __ldg(p.w + ((size_t)co * p.Cin + ci) * 9 + t) : 0.f;
-        const float hi = tf32_trunc(v);
-        const uint32_t off = (uint32_t)blk * 4096u + (uint32_t)(m & 7) * 16u + (uint32_t)(m >> 3) * 256u +
-                             (uint32_t)(k >> 2) * 128u + (uint32_t)(k & 3) * 4u;
-        *reinterpret_cast<float*>(smem + off) = (m < 64) ? hi : v - hi;
+        uint32_t r[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int ci = 8 * c + k;
+            const float v = (co < p.Cout && ci < p.Cin) ? __ldg(p.w + ((size_t)co * p.Cin + ci) * 9 + t) : 0.f;
+            const float hi = tf32_trunc(v);
+            r[k] = __float_as_uint(hi_part ? hi : v - hi);
+        }
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"r"(
+                         taddr + (uint32_t)(8 * blk)),
+                     "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]));
     }
+    asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], kind::tf32.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 template <int P, int CCH, int MODE>
@@ -314,12 +347,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
-    stage_weights<CCH>(p, smem + L.w);
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // weights visible to the tensor core
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    if (warp >= EPI_WARP0) weights_to_tmem<CCH>(p, tmem, G::WCOL0, warp & 3, lane);
+    tc_fence_before();
+    __syncthreads();  // weights in tensor memory before the first MMA
+    tc_fence_after();
 
     if (warp < MMA_WARP) {
         // ------------------------------------------------------------- loaders
@@ -329,8 +364,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 long long last[NSTG];
                 for (int i = 0; i < NSTG; ++i) last[i] = -1;
                 bool ok = true;
-                for (long long u = u0; ok && u < u1; ++u) {
-                    const Unit t = decode(p, u);
+                Unit ut = decode(p, u0);
+                for (long long u = u0; ok && u < u1; ++u, next_unit(p, ut)) {
+                    const Unit t = ut;
                     if (!not_stalled(1, u)) break;
                     for (int j = first_row(u, u0, t.ph); j < P + 2; ++j, ++s) {
                         const int st = (int)(s % NSTG);
@@ -367,8 +403,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // zeros for them); bytes past the end of x are zero-filled.
             long long s = 0;
             bool ok = true;
-            for (long long u = u0; ok && u < u1; ++u) {
-                const Unit t = decode(p, u);
+            Unit ut = decode(p, u0);
+            for (long long u = u0; ok && u < u1; ++u, next_unit(p, ut)) {
+                const Unit t = ut;
                 int go = 1;
                 if (lane == 0) go = not_stalled(1, u);
                 if (!__shfl_sync(0xffffffffu, go, 0)) break;
@@ -405,25 +442,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     } else if (warp == MMA_WARP) {
         // --------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            // D fp32, A and B tf32, both K-major, N = 4 * NCOL, M = 128.
+            // D fp32, A (tensor memory) and B tf32, B K-major, N = 4 * NCOL, M = 128.
             constexpr uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(G::NMMA >> 3) << 17) |
                                        ((uint32_t)(128 >> 4) << 24);
-            uint64_t adesc[9 * CCH];
-#pragma unroll
-            for (int i = 0; i < 9 * CCH; ++i) adesc[i] = desc_none(sbase + L.w + (uint32_t)i * 4096u, 128u, 256u);
+            const uint32_t a_tmem0 = tmem + G::WCOL0;  // weights: 8 columns per (tap, chunk)
             // B: position rows 16 bytes apart (8-row groups 128 bytes apart), the
             // second channel quad one plane further (leading-byte offset).
             const uint64_t bconst = desc_none(0u, G::PLANE, 128u);
-            long long s = 0;
+            // Rows are first needed in sequence order, and a row seen full stays
+            // until this thread releases it: `confirmed` is the last row seen full,
+            // so each conv row waits for one new row at most.  (Checking ahead
+            // without blocking -- test_wait on the next row and the next unit's
+            // accumulator while MMAs are queued -- measured no faster for the rows
+            // and 13-17 % slower for the accumulator.)
+            long long s = 0, confirmed = -1;
             bool ok = true;
-            for (long long u = u0; ok && u < u1; ++u) {
-                const Unit t = decode(p, u);
+            Unit ut = decode(p, u0);
+            for (long long u = u0; ok && u < u1; ++u, next_unit(p, ut)) {
+                const Unit t = ut;
                 if (!not_stalled(3, u)) break;
                 const int fj = first_row(u, u0, t.ph);
                 const long long base = s - fj;
                 s += P + 2 - fj;
                 const long long i = u - u0;
                 const int abuf = (int)(i & 1);
+                const bool cont_next = u + 1 < u1 && t.ph + 1 < p.PH;  // the next unit continues this strip
                 if (!wait_bounded(bar_acc_empty + 8 * abuf, (uint32_t)((i >> 1) & 1) ^ 1u, abort_flag, p.wait_ns)) {
                     ok = false;
                     break;
@@ -432,33 +475,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const uint32_t d = tmem + (uint32_t)(abuf * G::NMMA);
                 uint32_t acc = 0u;
                 for (int dy = 0; ok && dy < P; ++dy) {
-#pragma unroll
-                    for (int ky = 0; ky < 3; ++ky) {
-                        const long long q = base + dy + ky;
-                        const int sl = (int)(q % G::NSLOT);
-                        if (!wait_bounded(bar_slot_full + 8 * sl, (uint32_t)((q / G::NSLOT) & 1), abort_flag,
-                                          p.wait_ns)) {
+                    // rows base+dy .. base+dy+2, in order
+                    while (confirmed < base + dy + 2) {
+                        const long long q = confirmed + 1;
+                        if (!wait_bounded(bar_slot_full + 8 * (int)(q % G::NSLOT), (uint32_t)((q / G::NSLOT) & 1),
+                                          abort_flag, p.wait_ns)) {
                             ok = false;
                             break;
                         }
+                        confirmed = q;
                         tc_fence_after();
-                        const uint32_t sh = sbase + L.slots + (uint32_t)sl * G::SLOT;
+                    }
+                    if (!ok) break;
+#pragma unroll
+                    for (int ky = 0; ky < 3; ++ky) {
+                        const uint32_t sh = sbase + L.slots + (uint32_t)((base + dy + ky) % G::NSLOT) * G::SLOT;
 #pragma unroll
                         for (int kx = 0; kx < 3; ++kx) {
 #pragma unroll
                             for (int c = 0; c < CCH; ++c) {
                                 const uint32_t off = (uint32_t)kx * (IMG * 16u) + (uint32_t)(2 * c) * G::PLANE;
-                                const uint64_t a = adesc[(3 * ky + kx) * CCH + c];
-                                mma_ss(d, a, bconst | (uint64_t)(((sh + off) & 0x3FFFFu) >> 4), idesc, acc);
-                                mma_ss(d, a, bconst | (uint64_t)(((sh + G::HALF + off) & 0x3FFFFu) >> 4), idesc, 1u);
+                                const uint32_t a = a_tmem0 + 8u * (uint32_t)((3 * ky + kx) * CCH + c);
+                                mma_ts(d, a, bconst | (uint64_t)(((sh + off) & 0x3FFFFu) >> 4), idesc, acc);
+                                mma_ts(d, a, bconst | (uint64_t)(((sh + G::HALF + off) & 0x3FFFFu) >> 4), idesc, 1u);
                                 acc = 1u;
                             }
                         }
                     }
-                    if (ok) tc_commit(bar_slot_empty + 8 * (int)((base + dy) % G::NSLOT));  // row base+dy read for the last time
+                    tc_commit(bar_slot_empty + 8 * (int)((base + dy) % G::NSLOT));  // row base+dy read for the last time
                 }
                 if (!ok) break;
-                if (!(u + 1 < u1 && t.ph + 1 < p.PH)) {
+                if (!cont_next) {
                     // No continuation: the unit's last two rows are not read again.
                     tc_commit(bar_slot_empty + 8 * (int)((base + P) % G::NSLOT));
                     tc_commit(bar_slot_empty + 8 * (int)((base + P + 1) % G::NSLOT));
@@ -483,15 +530,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // copies.  NSTG and NSLOT are multiples of 4, so each buffer and slot is
         // only ever used by one warp, in order: a parity wait is then never more
         // than one phase behind and cannot pass on a stale phase.  Lane
-        // (column lane % 8, image lane / 8) makes both the staging reads (pitch
-        // 8 mod 32 floats) and the 16-byte slot stores (512 contiguous bytes)
-        // conflict-free.
+        // (image lane % 4, column lane / 4) makes both the staging reads (pitch
+        // 8 or 24 mod 32 floats) and the 16-byte slot stores conflict-free: the
+        // 8 lanes a store serves at a time write 128 contiguous bytes.
         const int pw = warp - PROD_WARP0;
-        const int col_lo = lane & 7, img = lane >> 3;
+        const int img = lane & 3, col_lo = lane >> 2;
         long long s = 0;
         bool ok = true;
-        for (long long u = u0; ok && u < u1; ++u) {
-            const Unit t = decode(p, u);
+        Unit ut = decode(p, u0);
+        for (long long u = u0; ok && u < u1; ++u, next_unit(p, ut)) {
+            const Unit t = ut;
             int go = 1;
             if (lane == 0 && pw == 0) go = not_stalled(2, u);
             if (!__shfl_sync(0xffffffffu, go, 0)) break;
@@ -586,8 +634,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             asm volatile("bar.sync 1, 128;\n" ::: "memory");
         };
         bool ok = true;
-        for (long long u = u0; u < u1; ++u) {
-            const Unit t = decode(p, u);
+        Unit ut = decode(p, u0);
+        for (long long u = u0; u < u1; ++u, next_unit(p, ut)) {
+            const Unit t = ut;
             const long long i = u - u0;
             const int abuf = (int)(i & 1);
             // One thread waits (bounded); the barrier makes the abort decision the
@@ -720,7 +769,7 @@ inline int launch_conv2d_tcs(const float* x, const float* w, const float* b, int
 {
     if (!conv2d_tcs_supported(Cin, P, x)) return FCV_ERR_UNSUPPORTED;
     const int CCH = Cin <= 8 ? 1 : 2;
-    const int ncol = CCH == 1 ? 64 : 32;
+    const int ncol = CCH == 1 ? c2s::Geo<1, 1>::NCOL : c2s::Geo<1, 2>::NCOL;
     c2s::Params prm;
     prm.x = x; prm.out = out;
     prm.N = N; prm.Cin = Cin; prm.H = H; prm.W = W;

@@ -557,6 +557,7 @@ def shifted_kernel(P, u0, u1, PH, nslot, nstg, nprod=4, planted=None):
     def commit(bar, use):
         loop.append(("enqueue", "mma", [("arrive", bar, use, 1, "tcore")]))
 
+    confirmed = -1  # the issuer waits for a row only the first time it needs it
     for i, (base, cont) in enumerate(units):
         ab, ak = i & 1, i >> 1
         if planted != "no_acc_wait":
@@ -565,7 +566,9 @@ def shifted_kernel(P, u0, u1, PH, nslot, nstg, nprod=4, planted=None):
         for dy in range(P):
             for ky in range(3):
                 q = base + dy + ky
-                loop.append(("wait", f"slotf{q % nslot}", (q // nslot) & 1, q // nslot + 1, "mma"))
+                if q > confirmed:
+                    loop.append(("wait", f"slotf{q % nslot}", (q // nslot) & 1, q // nslot + 1, "mma"))
+                    confirmed = q
             # the conv row's MMAs read the three rows until they complete
             loop.append(("enqueue", "mma", [("read", f"slot{q % nslot}", q // nslot, "mma")
                                             for q in range(base + dy, base + dy + 3)]))
