@@ -56,9 +56,9 @@
 //     reads it, and commits a unit's accumulator.
 //   * warps 7-10 (epilogue, one per TMEM lane quarter): tcgen05.ld 32 columns
 //     at a time, add the P columns of each window, exchange the hi and lo
-//     halves through shared memory (the two pairs of warps take alternate
-//     column chunks), add the bias, apply the sigmoid and accumulate per
-//     image; one atomic add per CTA and image.
+//     halves through shared memory (each pair of warps finishes half of every
+//     chunk's pooled values), add the bias, apply the sigmoid and accumulate
+//     per image; one atomic add per CTA and image.
 //   * Every wait is bounded; a wait that runs out sets the CTA abort flag and
 //     the device error word, every role leaves its loop, TMA copies and MMAs
 //     still in flight are waited for (bounded) and TMEM is freed.
@@ -679,38 +679,36 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         pv[w * IMG + img] = s;
                     }
                 }
-                const bool owner = ((k & 1) == 0) == hi_half;  // even chunks: hi warps; odd: lo warps
+                // Each warp pair finishes half of the chunk's pooled values: the hi
+                // warps values [0, V/2), the lo warps [V/2, V).  Each writes its
+                // partial sums of the other half to shared memory, then adds the
+                // partner's partial sums of its own half.
+                constexpr int HV = G::V / 2;
+                const int mine = hi_half ? 0 : HV, theirs = hi_half ? HV : 0;
                 float* xb = xbuf + ((k & 1) * CO_BLK + co) * G::XP;
-                if (!owner) {
+                if constexpr (HV % 4 == 0) {
 #pragma unroll
-                    for (int e = 0; e < G::V; e += 4)
-                        *reinterpret_cast<float4*>(xb + e) = make_float4(pv[e], pv[e + 1], pv[e + 2], pv[e + 3]);
+                    for (int e = 0; e < HV; e += 4)
+                        *reinterpret_cast<float4*>(xb + theirs + e) =
+                            make_float4(pv[theirs + e], pv[theirs + e + 1], pv[theirs + e + 2], pv[theirs + e + 3]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < HV; e += 2)
+                        *reinterpret_cast<float2*>(xb + theirs + e) = make_float2(pv[theirs + e], pv[theirs + e + 1]);
                 }
                 asm volatile("bar.sync 1, 128;\n" ::: "memory");
-                if (owner) {
 #pragma unroll
-                    for (int e = 0; e < G::V; e += 4) {
-                        const float4 o = *reinterpret_cast<const float4*>(xb + e);
-                        pv[e] += o.x;
-                        pv[e + 1] += o.y;
-                        pv[e + 2] += o.z;
-                        pv[e + 3] += o.w;
-                    }
-#pragma unroll
-                    for (int w = 0; w < 8 / P; ++w) {
-                        const int pwx = t.ct * G::WPT + k * (8 / P) + w;
-                        if (!co_ok || pwx >= p.PW) continue;
-#pragma unroll
-                        for (int img = 0; img < IMG; ++img) {
-                            const int n = IMG * t.g + img;
-                            if (n >= p.N) continue;
-                            const float pooled = pv[w * IMG + img] * inv_area + bias;
-                            if (MODE == kTap) {
-                                p.out[(((size_t)n * p.Cout_total + p.co0 + co) * p.PH + t.ph) * p.PW + pwx] = pooled;
-                            } else {
-                                acc[img] += __fdividef(1.f, 1.f + __expf(-pooled));  // sigmoid; 0 once exp overflows
-                            }
-                        }
+                for (int e = 0; e < HV; ++e) {
+                    const int v = mine + e;           // value index = window * 4 + image
+                    const int w = v / IMG, img = v % IMG;
+                    const int pwx = t.ct * G::WPT + k * (8 / P) + w;
+                    const int n = IMG * t.g + img;
+                    if (!co_ok || pwx >= p.PW || n >= p.N) continue;
+                    const float pooled = (pv[v] + xb[v]) * inv_area + bias;
+                    if (MODE == kTap) {
+                        p.out[(((size_t)n * p.Cout_total + p.co0 + co) * p.PH + t.ph) * p.PW + pwx] = pooled;
+                    } else {
+                        acc[img] += __fdividef(1.f, 1.f + __expf(-pooled));  // sigmoid; 0 once exp overflows
                     }
                 }
             }
@@ -799,7 +797,7 @@ inline int launch_conv2d_tcs(const float* x, const float* w, const float* b, int
         const cuuint32_t box[4] = {(cuuint32_t)(ncol + 8), (cuuint32_t)c2s::IMG, (cuuint32_t)(8 * CCH), 1};
         const cuuint32_t estride[4] = {1, 1, 1, 1};
         if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(x), gdim, gstride, box, estride,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return FCV_ERR_CUDA;
         prm.use_tma = 1;

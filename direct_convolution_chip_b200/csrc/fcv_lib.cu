@@ -73,23 +73,24 @@ int check_conv1d(const float* x, const float* dw, const float* pw, const float* 
 }
 
 // Smallest FMA-kernel grid (CTAs) at which AUTO lets it take a narrow layer.
-// Measured on x[16,Cin,130,130], Cout 32, pool 4 (128 FMA CTAs): FMA 20.5 vs
-// 40.9 us at Cin 3 and 73.8 vs 78.0 us at Cin 16; below that the tensor-core
-// kernel, which spreads any grid over every SM, wins.
 constexpr long long kConv2dFmaMinCtas = 128;
 
-// What AUTO runs for op A.  Narrow layers (Cin < 4 or Cout <= 32) whose FMA
-// grid fills at least kConv2dFmaMinCtas CTAs stay on FP32 FMA; otherwise the
-// shifted-operand tensor-core kernel where it applies (Cin <= 16, pool 1, 2, 4
-// or 8, 16-byte aligned x), else the im2col tensor-core kernel where it
-// applies, else FP32 FMA.
+// What AUTO runs for op A.  Narrow layers (Cin <= 4 and Cout <= 32) whose FMA
+// grid fills at least kConv2dFmaMinCtas CTAs stay on FP32 FMA: the tensor-core
+// kernels pad Cin to 8 input channels and Cout to 64, so the FMA kernel, whose
+// time scales with Cin * Cout, does less work there (x[16,3,509,509], Cout 32,
+// pool 4: FMA 187 us, shifted-operand tensor cores 201 us; Cin 4: 240 against
+// 214, Cout 48: 339 against 203).  Otherwise the shifted-operand tensor-core
+// kernel where it applies (Cin <= 16, pool 1, 2, 4 or 8, 16-byte aligned x;
+// it beat FMA by 1.7-3.2x at Cin 8 and 16 on 509 x 509 images), else the
+// im2col tensor-core kernel where it applies, else FP32 FMA.
 int conv2d_auto_algo_for(int N, int Cin, int Cout, int pool, int PH, int PW, bool x_aligned16)
 {
     const bool tcs = fcv::conv2d_tcs_supported(Cin, pool, x_aligned16 ? reinterpret_cast<const void*>(16)
                                                                       : reinterpret_cast<const void*>(4));
     const bool tc = fcv::conv2d_tc_supported(Cin, Cout, pool);
     if (!tcs && !tc) return FCV_CONV2D_DIRECT;
-    if (Cin < 4 || Cout <= 32) {
+    if (Cin <= 4 && Cout <= 32) {
         int ty = 0, tx = 0, cb = 0;
         if (fcv::conv2d_grid(pool, PH, PW, Cout, &ty, &tx, &cb) &&
             (long long)N * ty * tx * cb >= kConv2dFmaMinCtas)

@@ -63,11 +63,12 @@ typedef enum {
 /* Algorithm selectors for the *_ex entry points.  FCV_ALGO_AUTO picks the
  * fastest path valid for the shape and pointers (fcv_conv2d_auto_algo and
  * fcv_dwsep_conv1d_auto_algo report which).  For op A it is always the direct
- * method (every conv output is computed): on tensor cores where
- * FCV_CONV2D_TC_3XTF32 covers the shape, except narrow layers (Cin < 4 or
- * Cout <= 32) whose FP32-FMA grid has at least 128 CTAs (there FP32 FMA
- * measured faster), else on FP32 FMA; the pool-first identity is never chosen
- * automatically. */
+ * method (every conv output is computed): FCV_CONV2D_TC_SHIFT_3XTF32 where it
+ * covers the shape, else FCV_CONV2D_TC_3XTF32 where that one does, except narrow
+ * layers (Cin <= 4 and Cout <= 32) whose FP32-FMA grid has at least 128 CTAs
+ * (there FP32 FMA measured faster), else FP32 FMA; the pool-first identity is
+ * never chosen automatically.  The AUTO report for op A assumes a 16-byte
+ * aligned x. */
 typedef enum {
     FCV_ALGO_AUTO = 0,
     /* op A */
@@ -110,8 +111,8 @@ typedef enum {
  * INVALID_ARG: x, w, b or out NULL while N > 0; N < 0; Cin, Cout < 1; H, W < 3; pool < 1;
  *              element counts beyond 2^31 * 2^31; misaligned pointers.
  * UNSUPPORTED: pool > 8.
- * The per-batch sum is accumulated with atomic adds (one per thread block on
- * the FMA path, one per warp and image on the tensor-core path), so the last
+ * The per-batch sum is accumulated with atomic adds (one per thread block and
+ * image; one per warp and image on the im2col tensor-core path), so the last
  * bits may differ between runs. */
 int fcv_conv2d_pool_sigmoid_sum(const float* x, const float* w, const float* b,
                                 int N, int Cin, int H, int W, int Cout, int pool,

@@ -177,23 +177,24 @@ def test_selftest_rejects_bad_limits(lib):
 
 
 def test_auto_algo_conv2d(lib):
-    """AUTO: FMA for narrow layers (Cin < 4 or Cout <= 32) once the FMA grid has
-    128 CTAs; else the shifted-operand tensor-core kernel (Cin <= 16, pool 1, 2,
-    4 or 8), else the im2col tensor-core kernel where it fits, else FMA."""
+    """AUTO: FMA for narrow layers (Cin <= 4 and Cout <= 32) once the FMA grid
+    has 128 CTAs; else the shifted-operand tensor-core kernel (Cin <= 16, pool
+    1, 2, 4 or 8), else the im2col tensor-core kernel where it fits, else FMA."""
     a = ctypes.c_int()
     q = lib.fcv_conv2d_auto_algo
     assert q(128, 8, 384, 384, 64, 4, ctypes.byref(a)) == OK and a.value == 13  # the full-size workload
     for pool in (1, 2, 8):
         assert q(2, 8, 40, 40, 48, pool, ctypes.byref(a)) == OK and a.value == 13
-    # narrow layers (Cin < 4 or Cout <= 32): FMA once its grid has 128 CTAs
+    # narrow layers (Cin <= 4 and Cout <= 32): FMA once its grid has 128 CTAs
     assert q(16, 3, 130, 130, 32, 4, ctypes.byref(a)) == OK and a.value == 10   # exactly 128
     assert q(15, 3, 130, 130, 32, 4, ctypes.byref(a)) == OK and a.value == 13   # 120
     assert q(16, 3, 509, 509, 32, 4, ctypes.byref(a)) == OK and a.value == 10
-    assert q(16, 3, 509, 509, 48, 4, ctypes.byref(a)) == OK and a.value == 10
-    assert q(16, 16, 509, 509, 32, 4, ctypes.byref(a)) == OK and a.value == 10
+    assert q(16, 4, 509, 509, 16, 2, ctypes.byref(a)) == OK and a.value == 10
+    assert q(16, 3, 509, 509, 48, 4, ctypes.byref(a)) == OK and a.value == 13   # Cout > 32
+    assert q(16, 16, 509, 509, 32, 4, ctypes.byref(a)) == OK and a.value == 13  # Cin > 4
+    assert q(16, 5, 130, 130, 16, 4, ctypes.byref(a)) == OK and a.value == 13
     assert q(2, 3, 40, 40, 32, 4, ctypes.byref(a)) == OK and a.value == 13      # 8 FMA CTAs: tensor cores
     assert q(2, 8, 64, 64, 16, 4, ctypes.byref(a)) == OK and a.value == 13      # the small workload
-    assert q(2, 4, 40, 40, 33, 4, ctypes.byref(a)) == OK and a.value == 13      # Cin >= 4, Cout > 32
     assert q(2, 8, 40, 40, 128, 4, ctypes.byref(a)) == OK and a.value == 13     # two launches of 64 channels
     assert q(2, 20, 40, 40, 48, 4, ctypes.byref(a)) == OK and a.value == 12     # Cin > 16: im2col kernel
     assert q(2, 8, 40, 40, 16, 3, ctypes.byref(a)) == OK and a.value == 10      # pool 3: FMA path
