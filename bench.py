@@ -780,6 +780,42 @@ def run_probes():
                     print(json.dumps({"probe": "tcgen05_tf32_mma", "n": n, "a_tmem": a_tmem, "chains": chains,
                                       "issuers": issuers, "status": st, "tflops": f.value / 1e12, "ms": ms.value,
                                       "cycles_per_mma": cyc.value}), flush=True)
+    run_layout_probes(lib)
+
+
+def run_layout_probes(lib):
+    """The tcgen05 kind::tf32 operand facts the shifted-operand conv2d relies
+    on: the B address map for K-major and MN-major descriptors without swizzle,
+    the TMEM lanes of an M = 64 accumulator, and SM cycles per MMA."""
+    import ctypes
+    import numpy as np
+    buf = (ctypes.c_float * 2048)()
+    for b_major, lbo, sbo in ((0, 128, 128), (0, 256, 128), (1, 128, 128), (1, 256, 128)):
+        st = lib.fcvprobe_umma_b_map(b_major, lbo, sbo, buf)
+        d = np.frombuffer(buf, dtype=np.float32).reshape(8, 256)
+        n = np.arange(256)
+        kmajor = np.array([4 * n + (k % 4) + (lbo // 4) * (k // 4) for k in range(8)])  # rows 16 B apart
+        mnmajor = np.array([(n % 4) + (sbo // 4) * (n // 4) + 4 * k for k in range(8)])
+        print(json.dumps({"probe": "umma_b_map", "b_major": b_major, "lbo": lbo, "sbo": sbo, "status": st,
+                          "all_zero": bool(np.all(d == 0)),
+                          "matches_k_major_rows_16B": bool(np.array_equal(d, kmajor % 2048)),
+                          "matches_mn_major_interleave": bool(np.array_equal(d, mnmajor % 2048)),
+                          "k0_n0_7": d[0, :8].astype(int).tolist(), "k4_n0_7": d[4, :8].astype(int).tolist()}),
+              flush=True)
+    rows = (ctypes.c_float * 128)()
+    st = lib.fcvprobe_umma_m64_rows(rows)
+    r = np.frombuffer(rows, dtype=np.float32).astype(int)
+    print(json.dumps({"probe": "umma_m64_rows", "status": st,
+                      "lanes_written": [int(i) for i in np.nonzero(r != -7)[0]],
+                      "row_of_lane": {int(i): int(r[i]) - 1 for i in np.nonzero(r != -7)[0]}}), flush=True)
+    for m, n, a_tmem in ((128, 256, 0), (128, 256, 1), (64, 256, 1), (128, 192, 1), (64, 192, 1)):
+        best = None
+        for _ in range(3):
+            c = ctypes.c_double()
+            st = lib.fcvprobe_umma_cycles(m, n, a_tmem, 2000, ctypes.byref(c))
+            best = c.value if best is None else min(best, c.value)
+        print(json.dumps({"probe": "umma_cycles", "m": m, "n": n, "a": "tmem" if a_tmem else "smem",
+                          "b": "smem, K-major, no swizzle", "status": st, "sm_cycles_per_mma": best}), flush=True)
 
 
 def run_configs(args):

@@ -27,8 +27,9 @@ def sources():
 
 
 def build_probes(force: bool = False) -> str:
-    """Compile libfcv_probes.so (the FP32-FMA and tcgen05 TF32 peak probes) if missing or stale."""
-    srcs = [os.path.join(CSRC, "probes", f) for f in ("fma_peak.cu", "tf32_mma_rate.cu")]
+    """Compile libfcv_probes.so (the FP32-FMA and tcgen05 TF32 peak probes, the
+    tcgen05 operand-layout probes) if missing or stale."""
+    srcs = [os.path.join(CSRC, "probes", f) for f in ("fma_peak.cu", "tf32_mma_rate.cu", "umma_layout.cu")]
     if not force and os.path.exists(PROBE_LIB) and all(
             os.path.getmtime(PROBE_LIB) >= os.path.getmtime(s) for s in srcs):
         return PROBE_LIB

@@ -164,6 +164,7 @@ struct Params {
     int co0, Cout_total;
     int PH, PW;
     int CT;             // column tiles per pooled row
+    int PHB;            // pooled rows per block of the unit walk
     long long U;        // units = groups * CT * PH
     long long x_elems;  // N * Cin * H * W
     int use_tma;
@@ -175,8 +176,15 @@ struct Params {
     int stall_role, stall_at;
 };
 
+// Units are walked image group by image group; within a group, in blocks of
+// PHB pooled rows: every column tile of a block, each down its PHB pooled rows,
+// then the next block.  Consecutive units of one column tile share two input
+// rows (loaded once), and the column tiles of a block follow each other
+// closely, so the columns their boxes share and the rows between blocks are
+// still in L2 when the next box needs them.
 struct Unit {
     int g, ct, ph;
+    int b0, bh;  // first pooled row and height of the block
 };
 
 __device__ __forceinline__ Unit decode(const Params& p, long long u)
@@ -185,22 +193,30 @@ __device__ __forceinline__ Unit decode(const Params& p, long long u)
     const long long per_g = (long long)p.CT * p.PH;
     t.g = (int)(u / per_g);
     const int r = (int)(u - (long long)t.g * per_g);
-    t.ct = r / p.PH;
-    t.ph = r - t.ct * p.PH;
+    const int full = p.PHB * p.CT;  // units of a full block
+    const int blk = r / full;
+    t.b0 = blk * p.PHB;
+    t.bh = min(p.PHB, p.PH - t.b0);
+    const int rb = r - blk * full;
+    t.ct = rb / t.bh;
+    t.ph = t.b0 + (rb - t.ct * t.bh);
     return t;
 }
 
-// The unit after t (ph fastest, then column tile, then image group): every
-// role walks its units this way instead of dividing per unit.
+// The unit after t: every role walks its units this way instead of dividing.
 __device__ __forceinline__ void next_unit(const Params& p, Unit& t)
 {
-    if (++t.ph == p.PH) {
-        t.ph = 0;
-        if (++t.ct == p.CT) {
-            t.ct = 0;
-            ++t.g;
-        }
+    if (++t.ph < t.b0 + t.bh) return;
+    t.ph = t.b0;
+    if (++t.ct < p.CT) return;
+    t.ct = 0;
+    t.b0 += t.bh;
+    if (t.b0 == p.PH) {
+        t.b0 = 0;
+        ++t.g;
     }
+    t.bh = min(p.PHB, p.PH - t.b0);
+    t.ph = t.b0;
 }
 
 // Shared-memory matrix descriptor, no swizzle (canonical interleaved layout):
@@ -246,9 +262,12 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar)
 __device__ __forceinline__ float tf32_trunc(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
 
 // First row (0 or 2) of unit u that its CTA has to load: a unit that directly
-// follows the previous pooled row of the same strip reuses that unit's last
-// two input rows.
-__device__ __forceinline__ int first_row(long long u, long long u0, int ph) { return (u > u0 && ph > 0) ? 2 : 0; }
+// follows the previous pooled row of the same column tile reuses that unit's
+// last two input rows.
+__device__ __forceinline__ int first_row(long long u, long long u0, const Unit& t)
+{
+    return (u > u0 && t.ph > t.b0) ? 2 : 0;
+}
 
 // Weights of this launch as the A operand in tensor memory: block (tap t,
 // chunk c) is 8 consecutive columns from WCOL0 + 8 * (t * CCH + c); lane m holds
@@ -368,7 +387,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 for (long long u = u0; ok && u < u1; ++u, next_unit(p, ut)) {
                     const Unit t = ut;
                     if (!not_stalled(1, u)) break;
-                    for (int j = first_row(u, u0, t.ph); j < P + 2; ++j, ++s) {
+                    for (int j = first_row(u, u0, t); j < P + 2; ++j, ++s) {
                         const int st = (int)(s % NSTG);
                         if (!wait_bounded(bar_stg_empty + 8 * st, (uint32_t)((s / NSTG) & 1) ^ 1u, abort_flag,
                                           p.wait_ns)) {
@@ -409,7 +428,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 int go = 1;
                 if (lane == 0) go = not_stalled(1, u);
                 if (!__shfl_sync(0xffffffffu, go, 0)) break;
-                for (int j = first_row(u, u0, t.ph); j < P + 2; ++j, ++s) {
+                for (int j = first_row(u, u0, t); j < P + 2; ++j, ++s) {
                     if ((int)(s & 1) != warp) continue;
                     const int st = (int)(s % NSTG);
                     int good = 1;
@@ -461,12 +480,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (long long u = u0; ok && u < u1; ++u, next_unit(p, ut)) {
                 const Unit t = ut;
                 if (!not_stalled(3, u)) break;
-                const int fj = first_row(u, u0, t.ph);
+                const int fj = first_row(u, u0, t);
                 const long long base = s - fj;
                 s += P + 2 - fj;
                 const long long i = u - u0;
                 const int abuf = (int)(i & 1);
-                const bool cont_next = u + 1 < u1 && t.ph + 1 < p.PH;  // the next unit continues this strip
+                const bool cont_next = u + 1 < u1 && t.ph + 1 < t.b0 + t.bh;  // the next unit continues this column tile
                 if (!wait_bounded(bar_acc_empty + 8 * abuf, (uint32_t)((i >> 1) & 1) ^ 1u, abort_flag, p.wait_ns)) {
                     ok = false;
                     break;
@@ -543,7 +562,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int go = 1;
             if (lane == 0 && pw == 0) go = not_stalled(2, u);
             if (!__shfl_sync(0xffffffffu, go, 0)) break;
-            for (int j = first_row(u, u0, t.ph); j < P + 2; ++j, ++s) {
+            for (int j = first_row(u, u0, t); j < P + 2; ++j, ++s) {
                 if ((int)(s % NPRODW) != pw) continue;
                 const int st = (int)(s % NSTG), sl = (int)(s % G::NSLOT);
                 int good = 1;
@@ -697,6 +716,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         *reinterpret_cast<float2*>(xb + theirs + e) = make_float2(pv[theirs + e], pv[theirs + e + 1]);
                 }
                 asm volatile("bar.sync 1, 128;\n" ::: "memory");
+                // the partner's sums of this half, read as 16- or 8-byte vectors
+                // (lanes XP floats apart: conflict-free, like the stores)
+                float part[HV];
+                if constexpr (HV % 4 == 0) {
+#pragma unroll
+                    for (int e = 0; e < HV; e += 4) {
+                        const float4 o = *reinterpret_cast<const float4*>(xb + mine + e);
+                        part[e] = o.x; part[e + 1] = o.y; part[e + 2] = o.z; part[e + 3] = o.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < HV; e += 2) {
+                        const float2 o = *reinterpret_cast<const float2*>(xb + mine + e);
+                        part[e] = o.x; part[e + 1] = o.y;
+                    }
+                }
 #pragma unroll
                 for (int e = 0; e < HV; ++e) {
                     const int v = mine + e;           // value index = window * 4 + image
@@ -704,7 +739,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const int pwx = t.ct * G::WPT + k * (8 / P) + w;
                     const int n = IMG * t.g + img;
                     if (!co_ok || pwx >= p.PW || n >= p.N) continue;
-                    const float pooled = (pv[v] + xb[v]) * inv_area + bias;
+                    const float pooled = (pv[v] + part[e]) * inv_area + bias;
                     if (MODE == kTap) {
                         p.out[(((size_t)n * p.Cout_total + p.co0 + co) * p.PH + t.ph) * p.PW + pwx] = pooled;
                     } else {
@@ -757,6 +792,12 @@ inline int launch_conv2d_tcs_p(const c2s::Params& prm, int CCH, int grid, const 
                     : launch_conv2d_tcs_inst<P, 2, MODE>(prm, grid, map, stream);
 }
 
+#ifndef FCV_TCS_BLOCK_ROWS
+#define FCV_TCS_BLOCK_ROWS 8
+#endif
+// Pooled rows per block of the shifted-operand kernel's unit walk.
+constexpr int kConv2dTcsBlockRows = FCV_TCS_BLOCK_ROWS;
+
 // MODE: kSumAtomic (out[N], zeroed by the caller) or kTap (pooled values).
 // One launch per block of 64 output channels; wait_ns bounds the main-loop
 // waits of every launch.
@@ -778,6 +819,7 @@ inline int launch_conv2d_tcs(const float* x, const float* w, const float* b, int
     const long long groups = (N + c2s::IMG - 1) / c2s::IMG;
     prm.U = groups * prm.CT * PH;
     prm.x_elems = (long long)N * Cin * H * W;
+    prm.PHB = kConv2dTcsBlockRows;
     prm.wait_ns = wait_ns;
     prm.stall_role = stall_role;
     prm.stall_at = stall_at;

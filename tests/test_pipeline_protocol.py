@@ -404,14 +404,24 @@ def test_model_catches_a_leader_that_ignores_the_peer_epilogue():
 # leaves.  At that point no TMA box and no MMA may still be in flight.
 
 
-def shifted_units(P, u0, u1, PH):
+def shifted_walk(u, PH, CT, PHB):
+    """(ph, first pooled row of its block, block height) of unit u: image groups,
+    then blocks of PHB pooled rows, then column tiles, then pooled rows."""
+    r = u % (CT * PH)
+    blk = r // (PHB * CT)
+    b0 = blk * PHB
+    bh = min(PHB, PH - b0)
+    return b0 + (r - blk * PHB * CT) % bh, b0, bh
+
+
+def shifted_units(P, u0, u1, PH, CT=1, PHB=1 << 30):
     """(base row sequence number, continues into the next unit) per unit, and
     the number of rows loaded, as every role of the kernel derives them."""
     units, s = [], 0
     for u in range(u0, u1):
-        ph = u % PH
-        fj = 2 if (u > u0 and ph > 0) else 0
-        units.append((s - fj, u + 1 < u1 and ph + 1 < PH))
+        ph, b0, bh = shifted_walk(u, PH, CT, PHB)
+        fj = 2 if (u > u0 and ph > b0) else 0
+        units.append((s - fj, u + 1 < u1 and ph + 1 < b0 + bh))
         s += P + 2 - fj
     return units, s
 
@@ -514,13 +524,13 @@ class AbortSim(Sim):
         return aborted
 
 
-def shifted_kernel(P, u0, u1, PH, nslot, nstg, nprod=4, planted=None):
+def shifted_kernel(P, u0, u1, PH, nslot, nstg, nprod=4, planted=None, CT=1, PHB=1 << 30):
     """The roles of conv2d_tcs_kernel for one CTA with units [u0, u1) of strips of
     PH pooled rows.  `planted` names a mistake to plant: "drain_only_if_aborted"
     (the loader skips its drain when its own loop ended normally), "early_release"
     (a slot is released one conv row early), "no_acc_wait" (the issuer does not
     wait for a drained accumulator)."""
-    units, S = shifted_units(P, u0, u1, PH)
+    units, S = shifted_units(P, u0, u1, PH, CT, PHB)
     sim = AbortSim()
     for b in range(nstg):
         sim.bar(f"stgf{b}", 1)
@@ -602,6 +612,18 @@ SHIFT_UNITS = [(0, 1, 5), (0, 3, 5), (2, 9, 5), (0, 12, 4), (3, 4, 1), (0, 6, 2)
 def test_shifted_kernel_protocol(P, units, nslot, nstg):
     for seed in range(15):
         shifted_kernel(P, *units, nslot, nstg).run(seed)
+
+
+@pytest.mark.parametrize("P", [2, 4])
+@pytest.mark.parametrize("walk", [(0, 40, 7, 3, 2), (5, 33, 9, 2, 4), (1, 20, 5, 4, 8), (0, 12, 3, 5, 1)],
+                         ids=lambda w: "u%d-%d_ph%d_ct%d_b%d" % w)
+def test_shifted_kernel_blocked_walk_protocol(P, walk):
+    """The walk in blocks of PHB pooled rows (every column tile of a block, then
+    the next block): continuations only inside a block and column tile."""
+    u0, u1, PH, CT, PHB = walk
+    for seed in range(15):
+        shifted_kernel(P, u0, u1, PH, 8, 4, CT=CT, PHB=PHB).run(seed)
+        shifted_kernel(P, u0, u1, PH, 8, 4, CT=CT, PHB=PHB).run(seed, p_abort=0.05)
 
 
 @pytest.mark.parametrize("P", [1, 4])
