@@ -21,12 +21,18 @@
 //     32-bit stores that fill one 128-byte row per warp instruction.
 //   * The pw operand's hi part is the raw fp32 chunk itself (the tensor core
 //     ignores the 13 low mantissa bits); only lo = v - truncate(v) is written.
-//   * r = (t0 - pad) mod 4 (the same for every tile) keeps the box's first
+//   * r = (t0*s - pad) mod 4 (the same for every tile) keeps the box's first
 //     time on a 16-byte boundary, as TMA requires; it is a template parameter
 //     so the window indexing stays in registers.
+//   * Stride s = 2 (the op's stride argument; output t reads x[2t + k - pad]):
+//     a 128-output tile spans up to 2*127 + K + r = 270 input samples, more
+//     than one TMA box can hold (256 per dimension), so the halo comes as two
+//     boxes of 140 samples, the first into the A region, the second into the
+//     B_lo region; the producers then write B_lo only after the barrier that
+//     follows their window reads.  A thread's window covers 2*15 + K samples.
 //
-// Requirements beyond the register-staged kernel: T % 4 == 0 and a 16-byte
-// aligned x (the TMA map's row strides are T*4 and C*T*4 bytes).
+// Requirements beyond the register-staged kernel: stride 1 or 2, T % 4 == 0
+// and a 16-byte aligned x (the TMA map's row strides are T*4 and C*T*4 bytes).
 #pragma once
 
 #include "conv1d_tc.cuh"
@@ -36,8 +42,10 @@ namespace tcx {
 
 using namespace tc;
 
-constexpr int XW = 148;                                     // halo box width = smem row pitch (floats)
+constexpr int XW = 148;                                     // halo box width = smem row pitch (floats), stride 1
 constexpr uint32_t X_BYTES = (uint32_t)XW * KC * 4;         // 18,944 B per chunk
+constexpr int XW2 = 140;                                    // stride 2: two boxes of this width (row pitch)
+constexpr uint32_t X2_BYTES = (uint32_t)XW2 * KC * 4;       // 17,920 B per box
 constexpr int DWX_MAX = 8192;                               // resident depthwise weights, [K][32*nk]
 constexpr uint32_t OFF_DWS = STAGES * STAGE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_DWS + DWX_MAX * 4;
@@ -47,6 +55,8 @@ constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;           // slack to align the base to 1024 B
 
 static_assert(X_BYTES <= 2 * A_BYTES, "the halo box must fit the stage's A region");
+static_assert(X2_BYTES <= 2 * A_BYTES && X2_BYTES <= B_BYTES, "stride-2 halo boxes: A region and B_lo region");
+static_assert((XW2 * 4) % 16 == 0 && XW2 % 4 == 0, "second stride-2 box starts 16-byte aligned");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert((XW * 4) % 16 == 0, "TMA box inner extent must be a multiple of 16 bytes");
 
@@ -83,15 +93,19 @@ __device__ __forceinline__ void sts32(uint32_t addr, float v)
 }
 
 // KT: depthwise kernel size when fixed at compile time (0: any K <= KMAXW).
-// R: (t0 - pad) mod 4, the offset of the first needed sample inside the box.
-template <int KT, int R>
+// R: (t0*S - pad) mod 4, the offset of the first needed sample inside the box.
+// S: the stride, 1 or 2.
+template <int KT, int R, int S>
 __global__ void __launch_bounds__(NTHREADS, 1)
 dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_map,
                         const __grid_constant__ CUtensorMap x_map)
 {
-    constexpr int KW = KT > 0 ? KT : KMAXW;            // taps the window must cover
-    constexpr int NV = (R + 15 + KW + 3) / 4;          // 16-byte window loads per thread
-    static_assert(16 * 7 + 4 * NV <= XW, "window inside the halo box");
+    static_assert(S == 1 || S == 2, "stride 1 or 2");
+    constexpr int KW = KT > 0 ? KT : KMAXW;              // taps the window must cover
+    constexpr int NV = (R + S * 15 + KW + 3) / 4;        // 16-byte window loads per thread
+    constexpr int PITCH = S == 1 ? XW : XW2;             // halo row pitch (floats)
+    static_assert(S == 2 || 16 * 7 + 4 * NV <= XW, "window inside the halo box");
+    static_assert(S == 1 || 32 * 7 + 4 * NV <= 2 * XW2, "window inside the two halo boxes");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -179,21 +193,31 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                 // reads only the TF32 bits of an fp32 operand (the 13 low mantissa
                 // bits are ignored, i.e. hi = truncate(v)); B_lo = v - truncate(v)
                 // is exact and |B_lo| < 2^-10 |v|.  This saves the in-place rewrite.
+                // At stride 2 the second halo box occupies the B_lo region, so
+                // B_lo is written after the barrier below.
+                auto split_pw = [&]() {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int row = warp * 32 + i * 4 + (lane >> 3);
-                    const uint32_t off = sw128_off(row, lane & 7);
-                    sts128(b_lo + off, tf32_trunc_rest4(lds128(b_hi + off)));
-                }
+                    for (int i = 0; i < 8; ++i) {
+                        const int row = warp * 32 + i * 4 + (lane >> 3);
+                        const uint32_t off = sw128_off(row, lane & 7);
+                        sts128(b_lo + off, tf32_trunc_rest4(lds128(b_hi + off)));
+                    }
+                };
+                if constexpr (S == 1) split_pw();
 
                 // Depthwise: channel lane, times 16*warp .. 16*warp+15 of the tile.
-                // Sample j of the halo row is x[t0 - pad - R + j]; output time
-                // 16*warp + i takes samples 16*warp + R + i + k, k < K.
-                const float* xrow = reinterpret_cast<const float*>(smem + stage * STAGE_BYTES) + lane * XW + 16 * warp;
+                // Sample j of the halo is x[t0*S - pad - R + j]; output time
+                // 16*warp + i takes samples S*(16*warp + i) + R + k, k < K.  At
+                // stride 2, samples j >= XW2 sit in the second box (B_lo region).
+                const float* xs0 = reinterpret_cast<const float*>(smem + stage * STAGE_BYTES) + lane * PITCH;
+                const float* xs1 =
+                    reinterpret_cast<const float*>(smem + stage * STAGE_BYTES + 2 * A_BYTES + B_BYTES) + lane * PITCH;
                 float win[4 * NV];
 #pragma unroll
                 for (int q = 0; q < NV; ++q) {
-                    const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
+                    const int j = S * 16 * warp + 4 * q;
+                    const float* src = (S == 1 || j < XW2) ? xs0 + j : xs1 + (j - XW2);
+                    const float4 v = *reinterpret_cast<const float4*>(src);
                     win[4 * q] = v.x;
                     win[4 * q + 1] = v.y;
                     win[4 * q + 2] = v.z;
@@ -210,11 +234,14 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                         const float2 w2 = make_float2(w, w);
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
-                            d2[j] = __ffma2_rn(make_float2(win[R + 2 * j + k], win[R + 2 * j + k + 1]), w2, d2[j]);
+                            d2[j] = __ffma2_rn(make_float2(win[R + 2 * S * j + k], win[R + 2 * S * j + S + k]), w2,
+                                               d2[j]);
                     }
                 }
-                // Every producer has read its halo window before the A operand overwrites it.
+                // Every producer has read its halo window before the A operand (and,
+                // at stride 2, B_lo) overwrites it.
                 asm volatile("bar.sync 1, 256;\n" ::: "memory");
+                if constexpr (S == 2) split_pw();
 
                 // A operand: row t = 16*warp + i, column = channel lane; one warp
                 // store fills one 128-byte swizzled row.
@@ -249,12 +276,15 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++local) {
                 if (!stall_ok(p, 1, local, bar_gate, abort_flag)) break;
                 const TileCoord tcd = decode_tile(p, tile);
-                const int x0 = tcd.t0 - p.pad - R;  // a multiple of 4: 16-byte aligned time coordinate
+                const int x0 = tcd.t0 * S - p.pad - R;  // a multiple of 4: 16-byte aligned time coordinate
                 // Pull the next tile's halo boxes into L2 now, so its TMA loads
                 // wait on L2 rather than on DRAM latency.
                 if (tile + (int)gridDim.x < p.total_tiles) {
                     const TileCoord nx = decode_tile(p, tile + gridDim.x);
-                    for (int k = 0; k < nk; ++k) tma_prefetch_3d(&x_map, nx.t0 - p.pad - R, k * KC, nx.n);
+                    for (int k = 0; k < nk; ++k) {
+                        tma_prefetch_3d(&x_map, nx.t0 * S - p.pad - R, k * KC, nx.n);
+                        if (S == 2) tma_prefetch_3d(&x_map, nx.t0 * S - p.pad - R + XW2, k * KC, nx.n);
+                    }
                 }
                 for (int k = 0; k < nk; ++k, ++seq) {
                     const int stage = seq & 1;
@@ -264,9 +294,11 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                     }
                     pending[stage] = false;  // the producers consumed its previous loads before the MMA ran
                     const uint32_t st = sbase + stage * STAGE_BYTES;
-                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES + X_BYTES);
+                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES + (S == 1 ? X_BYTES : 2 * X2_BYTES));
                     tma_load_2d(st + 2 * A_BYTES, &pw_map, k * KC, tcd.o0, bar_tma + 8 * stage);
                     tma_load_3d(st, &x_map, x0, k * KC, tcd.n, bar_tma + 8 * stage);
+                    if (S == 2)
+                        tma_load_3d(st + 2 * A_BYTES + B_BYTES, &x_map, x0 + XW2, k * KC, tcd.n, bar_tma + 8 * stage);
                     pending[stage] = true;
                 }
             }
@@ -305,14 +337,15 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
 inline bool conv1d_tcx_supported(int C, int T, int O, int K, int stride, const void* x, const void* pw)
 {
     const long long cw = (long long)tc::KC * ((C + tc::KC - 1) / tc::KC);
-    return stride == 1 && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1 && T >= 1 && (C & 3) == 0 &&
+    return (stride == 1 || stride == 2) && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1 && T >= 1 && (C & 3) == 0 &&
            (T & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 &&
            (reinterpret_cast<uintptr_t>(pw) & 15) == 0 && cw * K <= tcx::DWX_MAX;
 }
 
 inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float* pw, const float* bias, int N,
-                                   int C, int T, int O, int K, int pad, int To, float* out, cudaStream_t stream,
-                                   int stall_role = 0, int stall_at = 0, unsigned long long stall_ns = 0)
+                                   int C, int T, int O, int K, int stride, int pad, int To, float* out,
+                                   cudaStream_t stream, int stall_role = 0, int stall_at = 0,
+                                   unsigned long long stall_ns = 0)
 {
     tc::Params prm;
     prm.stall_role = stall_role;
@@ -341,12 +374,13 @@ inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float*
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return FCV_ERR_CUDA;
     }
-    // x [N][C][T]: 148 times x 32 channels x 1 batch item per box, rows packed
-    // (no swizzle); times and channels outside the tensor read as zero.
+    // x [N][C][T]: 148 (stride 2: 140) times x 32 channels x 1 batch item per
+    // box, rows packed (no swizzle); times and channels outside the tensor read
+    // as zero.
     {
         const cuuint64_t gdim[3] = {(cuuint64_t)T, (cuuint64_t)C, (cuuint64_t)N};
         const cuuint64_t gstride[2] = {(cuuint64_t)T * sizeof(float), (cuuint64_t)C * T * sizeof(float)};
-        const cuuint32_t box[3] = {(cuuint32_t)tcx::XW, (cuuint32_t)tc::KC, 1};
+        const cuuint32_t box[3] = {(cuuint32_t)(stride == 1 ? tcx::XW : tcx::XW2), (cuuint32_t)tc::KC, 1};
         const cuuint32_t estride[3] = {1, 1, 1};
         if (encode(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(x), gdim, gstride, box, estride,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -357,14 +391,23 @@ inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float*
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
-    const int r = (-pad) & 3;  // (t0 - pad) mod 4 with t0 a multiple of 128
-    decltype(&tcx::dwsep_conv1d_tcx_kernel<0, 0>) kern;
-    if (K == 9 && r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<9, 0>;
-    else if (K == 3 && r == 3) kern = tcx::dwsep_conv1d_tcx_kernel<3, 3>;
-    else if (r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<0, 0>;
-    else if (r == 1) kern = tcx::dwsep_conv1d_tcx_kernel<0, 1>;
-    else if (r == 2) kern = tcx::dwsep_conv1d_tcx_kernel<0, 2>;
-    else kern = tcx::dwsep_conv1d_tcx_kernel<0, 3>;
+    const int r = (-pad) & 3;  // (t0*stride - pad) mod 4 with t0 a multiple of 128
+    decltype(&tcx::dwsep_conv1d_tcx_kernel<0, 0, 1>) kern;
+    if (stride == 1) {
+        if (K == 9 && r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<9, 0, 1>;
+        else if (K == 3 && r == 3) kern = tcx::dwsep_conv1d_tcx_kernel<3, 3, 1>;
+        else if (r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<0, 0, 1>;
+        else if (r == 1) kern = tcx::dwsep_conv1d_tcx_kernel<0, 1, 1>;
+        else if (r == 2) kern = tcx::dwsep_conv1d_tcx_kernel<0, 2, 1>;
+        else kern = tcx::dwsep_conv1d_tcx_kernel<0, 3, 1>;
+    } else {
+        if (K == 9 && r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<9, 0, 2>;
+        else if (K == 3 && r == 3) kern = tcx::dwsep_conv1d_tcx_kernel<3, 3, 2>;
+        else if (r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<0, 0, 2>;
+        else if (r == 1) kern = tcx::dwsep_conv1d_tcx_kernel<0, 1, 2>;
+        else if (r == 2) kern = tcx::dwsep_conv1d_tcx_kernel<0, 2, 2>;
+        else kern = tcx::dwsep_conv1d_tcx_kernel<0, 3, 2>;
+    }
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcx::SMEM_BYTES) != cudaSuccess)
         return FCV_ERR_CUDA;
     const int grid = (int)(total < sms ? total : sms);

@@ -200,7 +200,7 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
     switch (algo) {
     case FCV_ALGO_AUTO:
         if (fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w))
-            return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, s);
+            return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
         if (fcv::conv1d_tc_supported(C, O, K, stride, pw_w)) {
             return fcv::launch_dwsep_conv1d_tc(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
         }
@@ -215,7 +215,7 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
         return fcv::launch_dwsep_conv1d_tc(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     case FCV_CONV1D_TC_TMA_3XTF32:
         if (!fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w)) return FCV_ERR_UNSUPPORTED;
-        return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, s);
+        return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     default:
         return FCV_ERR_INVALID_ARG;
     }
@@ -263,8 +263,8 @@ int fcv_selftest_conv1d_stall(const float* x, const float* dw_w, const float* pw
         return FCV_ERR_INVALID_ARG;
     if (!fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w)) return FCV_ERR_UNSUPPORTED;
     if (N == 0) return FCV_OK;
-    return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, fcv::as_stream(stream), role,
-                                        at_tile, limit_ns);
+    return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out,
+                                        fcv::as_stream(stream), role, at_tile, limit_ns);
 }
 
 int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* algo)

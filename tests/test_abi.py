@@ -104,7 +104,7 @@ def test_stall_selftests_validate_on_the_host(lib, fn, kw, want):
 
 def test_stall_selftests_outside_their_kernels(lib):
     assert stall2d(lib, Cin=20) == UNSUPPORTED
-    assert stall1d(lib, s=2) == UNSUPPORTED
+    assert stall1d(lib, s=3) == UNSUPPORTED
 
 
 def test_conv2d_unsupported_pool(lib):
@@ -205,15 +205,17 @@ def test_auto_algo_conv2d(lib):
 
 
 def test_auto_algo_conv1d(lib):
-    """AUTO: TMA-halo tensor cores for aligned x/pw and T % 4 == 0, then the
-    register-halo tensor-core kernel, then FMA (stride > 1)."""
+    """AUTO: TMA-halo tensor cores for aligned x/pw, T % 4 == 0 and stride 1 or
+    2, then the register-halo tensor-core kernel (stride 1), then FMA."""
     a = ctypes.c_int()
     q = lib.fcv_dwsep_conv1d_auto_algo
     X, PW = P(0x10000), P(0x20000)
     assert q(X, PW, 32, 256, 4096, 512, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 23  # full-size workload
     assert q(X, PW, 2, 64, 1001, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21    # T % 4 != 0
     assert q(P(0x10004), PW, 2, 64, 1000, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21  # x not 16-B aligned
-    assert q(X, PW, 2, 64, 1000, 128, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 20    # stride 2
+    assert q(X, PW, 2, 64, 1000, 128, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 23    # stride 2
+    assert q(X, PW, 2, 64, 1001, 128, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 20    # stride 2, T % 4 != 0
+    assert q(X, PW, 2, 64, 1000, 128, 9, 3, 4, ctypes.byref(a)) == OK and a.value == 20    # stride 3
     assert q(X, PW, 2, 62, 1000, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 20    # C % 4 != 0
     assert q(X, PW, 2, 64, 1000, 128, 33, 1, 4, ctypes.byref(a)) == UNSUPPORTED           # K > 32
     assert q(X, PW, 2, 64, 1000, 128, 9, 1, -1, ctypes.byref(a)) == INVALID

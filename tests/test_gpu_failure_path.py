@@ -68,8 +68,11 @@ def test_conv2d_stall_every_role(lib, case):
         assert_close(tap[bi:bi + 1], oracle.conv2d_pool_tap(xn[bi:bi + 1], wn, bn, case.P), f"tap[{bi}]")
 
 
-def test_conv1d_stall_every_role(lib):
-    case = wl.Conv1dCase("stall", 40, 64, 1024, 256, 9, 1, 4, seed=33)  # 320 tiles: every block has >= 2
+@pytest.mark.parametrize("stride", [1, 2])
+def test_conv1d_stall_every_role(lib, stride):
+    # 320 tiles either way: every block has >= 2
+    T = 1024 * stride
+    case = wl.Conv1dCase("stall", 40, 64, T, 256, 9, stride, 4, seed=33 + stride)
     x, dw, pw, bias = [t.cuda() for t in wl.conv1d_inputs(case)]
     To = binding.conv1d_out_len(case.T, case.K, case.stride, case.pad)
     out = torch.empty((case.N, case.O, To), device="cuda")

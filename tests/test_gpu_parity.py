@@ -222,6 +222,14 @@ EDGE_1D = [
     (2, 36, 512, 48, 7, 1, 3, True),    # r = 1, a partial second channel chunk
     (1, 64, 256, 300, 13, 1, 5, False), # r = 3 with the largest tensor-core K, partial output tile
     (1, 8, 4, 8, 3, 1, 1, True),        # T = 4: one partial time tile
+    # the same kernel at stride 2 (the halo in two TMA boxes): every r, ragged tiles
+    (2, 32, 1000, 64, 9, 2, 4, True),   # r = 0, K = 9
+    (1, 36, 516, 300, 13, 2, 5, False), # r = 3 with the largest tensor-core K, partial output tile
+    (3, 17, 260, 33, 3, 2, 1, True),    # r = 3, K = 3, C not a multiple of 4 (register/FMA paths)
+    (2, 64, 2048, 256, 5, 2, 2, True),  # r = 2
+    (1, 40, 300, 20, 4, 2, 0, True),    # even K, no padding
+    (1, 16, 256, 40, 3, 2, 7, True),    # pad larger than K, r = 1
+    (1, 8, 4, 8, 3, 2, 1, True),        # T = 4: To = 2
 ]
 
 
