@@ -282,12 +282,14 @@ struct TileCoord {
 // CTAs running at the same moment write neighbouring 512-byte segments of the
 // same output rows, and both output-channel tiles of a batch item read its
 // input while it is still in L2.
+// TN_T: output channels per tile.
+template <int TN_T = TN>
 __device__ __forceinline__ TileCoord decode_tile(const Params& p, int tile)
 {
     TileCoord tc;
     tc.t0 = (tile % p.tiles_t) * TM;
     const int rest = tile / p.tiles_t;
-    tc.o0 = (rest % p.tiles_o) * TN;
+    tc.o0 = (rest % p.tiles_o) * TN_T;
     tc.n = rest / p.tiles_o;
     return tc;
 }
@@ -361,8 +363,10 @@ __device__ __forceinline__ void mma_issuer(const Params& p, uint32_t tmem, uint3
     }
 }
 
-// One epilogue warp: drains its 32 TMEM lanes of each finished accumulator,
-// adds the bias and stores the tile's outputs, then frees the buffer.
+// One epilogue warp: drains its 32 TMEM lanes of each finished accumulator
+// (TN_E columns, buffer b at column b * TN_E), adds the bias and stores the
+// tile's outputs, then frees the buffer.
+template <int TN_E = TN>
 __device__ __forceinline__ void epilogue_warp(const Params& p, uint32_t tmem, uint32_t bar_afull,
                                               uint32_t bar_aempty, volatile uint32_t* abort_flag, int warp,
                                               int lane, uint32_t gate = 0)
@@ -378,9 +382,9 @@ __device__ __forceinline__ void epilogue_warp(const Params& p, uint32_t tmem, ui
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
-        const TileCoord tcd = decode_tile(p, tile);
+        const TileCoord tcd = decode_tile<TN_E>(p, tile);
         const int tw = tcd.t0 + 32 * q;  // first time of this warp's 32 TMEM lanes
-        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TN);
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TN_E);
         // Fast path: all 32 times in range and 16-byte aligned rows.  After a
         // 4x4 transpose inside each lane quad, lane 4k+j holds times
         // tw+4k .. tw+4k+3 of output channels 4j .. 4j+3 (of the 16 loaded), so
@@ -395,10 +399,10 @@ __device__ __forceinline__ void epilogue_warp(const Params& p, uint32_t tmem, ui
         };
         float bnext = bias_at(0), bcur = 0.f;
 #pragma unroll 1
-        for (int cb = 0; cb < TN / 16; ++cb) {
+        for (int cb = 0; cb < TN_E / 16; ++cb) {
             if ((cb & 1) == 0) {
                 bcur = bnext;
-                if (cb + 2 < TN / 16) bnext = bias_at((cb >> 1) + 1);
+                if (cb + 2 < TN_E / 16) bnext = bias_at((cb >> 1) + 1);
             }
             uint32_t r[16];
             tmem_ld16(taddr + (uint32_t)(cb * 16), r);

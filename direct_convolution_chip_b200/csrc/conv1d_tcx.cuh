@@ -47,17 +47,36 @@ constexpr uint32_t X_BYTES = (uint32_t)XW * KC * 4;         // 18,944 B per chun
 constexpr int XW2 = 140;                                    // stride 2: two boxes of this width (row pitch)
 constexpr uint32_t X2_BYTES = (uint32_t)XW2 * KC * 4;       // 17,920 B per box
 constexpr int DWX_MAX = 8192;                               // resident depthwise weights, [K][32*nk]
-constexpr uint32_t OFF_DWS = STAGES * STAGE_BYTES;
-constexpr uint32_t OFF_BAR = OFF_DWS + DWX_MAX * 4;
-constexpr uint32_t NBAR = 12;  // full[2] empty[2] afull[2] aempty[2] drain tma[2] gate
-constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr uint32_t SMEM_USED = OFF_MISC + 16;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;           // slack to align the base to 1024 B
 
-static_assert(X_BYTES <= 2 * A_BYTES, "the halo box must fit the stage's A region");
-static_assert(X2_BYTES <= 2 * A_BYTES && X2_BYTES <= B_BYTES, "stride-2 halo boxes: A region and B_lo region");
+// Geometry per output-channel tile width TN_ (the UMMA N): 256 (two 96 KB
+// stages) or 128 (three 64 KB stages; for O <= 128, where half of a 256-wide
+// tile would be zero).  A stage is A_hi | A_lo | B_lo | B_hi: the halo boxes
+// land from its start (stride 1: one box in the A region; stride 2: two boxes
+// over the A and B_lo regions), never over B_hi, which the TMA fills at once.
+template <int TN_>
+struct Geo {
+    static constexpr int TN = TN_;
+    static constexpr int STAGES = TN_ == 256 ? 2 : 3;
+    static constexpr uint32_t B_BYTES = (uint32_t)TN_ * KC * 4;
+    static constexpr uint32_t OFF_BLO = 2 * A_BYTES;
+    static constexpr uint32_t OFF_BHI = 2 * A_BYTES + B_BYTES;
+    static constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
+    static constexpr uint32_t OFF_DWS = STAGES * STAGE_BYTES;
+    static constexpr uint32_t OFF_BAR = OFF_DWS + DWX_MAX * 4;
+    static constexpr uint32_t NBAR = 3 * STAGES + 6;  // full, empty, tma per stage; afull[2] aempty[2] drain gate
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // slack to align the base to 1024 B
+    static constexpr uint32_t TMEM_COLS = 2 * TN_;
+    // Instruction descriptor: D fp32, A/B tf32, both K-major, N = TN, M = TM.
+    static constexpr uint32_t IDESC = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(TN_ >> 3) << 17) |
+                                      ((uint32_t)(TM >> 4) << 24);
+    static_assert(TN_ == 256 || TN_ == 128, "tile widths");
+    static_assert(X_BYTES <= 2 * A_BYTES, "the stride-1 halo box must fit the stage's A region");
+    static_assert(2 * X2_BYTES <= OFF_BHI, "the stride-2 halo boxes must stay below B_hi");
+    static_assert(OFF_BHI % 1024 == 0 && STAGE_BYTES % 1024 == 0, "128B-swizzled operands on 1024-byte boundaries");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
 static_assert((XW2 * 4) % 16 == 0 && XW2 % 4 == 0, "second stride-2 box starts 16-byte aligned");
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert((XW * 4) % 16 == 0, "TMA box inner extent must be a multiple of 16 bytes");
 
 // 3-D tiled TMA load (no multicast) completing on `bar`.
@@ -92,14 +111,82 @@ __device__ __forceinline__ void sts32(uint32_t addr, float v)
     asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(addr), "f"(v) : "memory");
 }
 
+// tcgen05.mma kind::tf32 with the instruction descriptor as a parameter.
+__device__ __forceinline__ void mma_tf32_id(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Single-thread MMA issuer (the register-halo kernel's protocol, for G's
+// stage count, stage layout and N): per tile wait until its accumulator buffer
+// is drained; per chunk wait until the producers filled the stage, issue its
+// 12 MMAs (4 K-steps x A_hi.B_hi + A_hi.B_lo + A_lo.B_hi) and commit them to
+// the stage's "empty" barrier; after the last chunk commit "afull".  Finally
+// drain every MMA issued (bounded) so TMEM can be freed.
+template <class G>
+__device__ __forceinline__ void mma_issuer_g(const Params& p, uint32_t tmem, uint32_t sbase, uint32_t bar_full,
+                                             uint32_t bar_empty, uint32_t bar_afull, uint32_t bar_aempty,
+                                             uint32_t bar_drain, volatile uint32_t* abort_flag, int nk, uint32_t gate)
+{
+    int seq = 0, local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++local) {
+        const int buf = local & 1;
+        if (!stall_ok(p, 3, local, gate, abort_flag)) break;
+        if (!wait_bounded(bar_aempty + 8 * buf, ((local >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * G::TN);
+        for (int k = 0; k < nk; ++k, ++seq) {
+            const int stage = seq % G::STAGES;
+            if (!wait_bounded(bar_full + 8 * stage, (seq / G::STAGES) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a_hi = sbase + stage * G::STAGE_BYTES;
+            const uint32_t a_lo = a_hi + A_BYTES;
+            const uint32_t b_lo = a_hi + G::OFF_BLO;
+            const uint32_t b_hi = a_hi + G::OFF_BHI;
+#pragma unroll
+            for (int kk = 0; kk < KC / 8; ++kk) {
+                const uint32_t koff = 32u * kk;
+                const uint64_t dah = sw128_desc(a_hi + koff), dal = sw128_desc(a_lo + koff);
+                const uint64_t dbh = sw128_desc(b_hi + koff), dbl = sw128_desc(b_lo + koff);
+                mma_tf32_id(d_tmem, dah, dbh, G::IDESC, (k > 0 || kk > 0) ? 1u : 0u);
+                mma_tf32_id(d_tmem, dah, dbl, G::IDESC, 1u);
+                mma_tf32_id(d_tmem, dal, dbh, G::IDESC, 1u);
+            }
+            tc_commit(bar_empty + 8 * stage);  // stage free once these MMAs have read it
+        }
+        if (ok) tc_commit(bar_afull + 8 * buf);  // accumulator complete
+    }
+    // Drain: every MMA this thread issued has completed before TMEM is freed.
+    tc_commit(bar_drain);
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(bar_drain, 0)) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1u;
+            record_device_error(kErrTimeout);
+            break;
+        }
+    }
+}
+
 // KT: depthwise kernel size when fixed at compile time (0: any K <= KMAXW).
 // R: (t0*S - pad) mod 4, the offset of the first needed sample inside the box.
-// S: the stride, 1 or 2.
-template <int KT, int R, int S>
+// S: the stride, 1 or 2.  TN_: output channels per tile, 256 or 128.
+template <int KT, int R, int S, int TN_>
 __global__ void __launch_bounds__(NTHREADS, 1)
 dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_map,
                         const __grid_constant__ CUtensorMap x_map)
 {
+    using G = Geo<TN_>;
+    constexpr int NS = G::STAGES;
     static_assert(S == 1 || S == 2, "stride 1 or 2");
     constexpr int KW = KT > 0 ? KT : KMAXW;              // taps the window must cover
     constexpr int NV = (R + S * 15 + KW + 3) / 4;        // 16-byte window loads per thread
@@ -110,30 +197,31 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
-    float* dws = reinterpret_cast<float*>(smem + OFF_DWS);
-    const uint32_t bar_full = sbase + OFF_BAR;       // + 8 * stage
-    const uint32_t bar_empty = bar_full + 16;        // + 8 * stage
-    const uint32_t bar_afull = bar_full + 32;        // + 8 * buf
-    const uint32_t bar_aempty = bar_full + 48;       // + 8 * buf
-    const uint32_t bar_drain = bar_full + 64;
-    const uint32_t bar_tma = bar_full + 72;          // + 8 * stage
-    const uint32_t bar_gate = bar_full + 88;         // never completed (failure-path test)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
-    volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 8);
+    float* dws = reinterpret_cast<float*>(smem + G::OFF_DWS);
+    const uint32_t bar_full = sbase + G::OFF_BAR;    // + 8 * stage
+    const uint32_t bar_empty = bar_full + 8 * NS;    // + 8 * stage
+    const uint32_t bar_tma = bar_full + 16 * NS;     // + 8 * stage
+    const uint32_t bar_afull = bar_full + 24 * NS;   // + 8 * buf
+    const uint32_t bar_aempty = bar_afull + 16;      // + 8 * buf
+    const uint32_t bar_drain = bar_afull + 32;
+    const uint32_t bar_gate = bar_afull + 40;        // never completed (failure-path test)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + G::OFF_MISC);
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + G::OFF_MISC + 4);
+    volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + G::OFF_MISC + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NS; ++i) {
             mbar_init(bar_full + 8 * i, 8);    // one arrival per producer warp
             mbar_init(bar_empty + 8 * i, 1);   // tcgen05.commit
+            mbar_init(bar_tma + 8 * i, 1);     // expect_tx arrival + TMA bytes
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(bar_afull + 8 * i, 1);   // tcgen05.commit
             mbar_init(bar_aempty + 8 * i, 4);  // one arrival per epilogue warp
         }
         mbar_init(bar_drain, 1);
-        mbar_init(bar_tma, 1);       // expect_tx arrival + TMA bytes
-        mbar_init(bar_tma + 8, 1);
         mbar_init(bar_gate, 1);
         *abort_flag = 0u;
         *prod_abort = 0u;
@@ -141,7 +229,7 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     }
     if (warp == MMA_WARP) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_holder)),
-                     "r"(TMEM_COLS)
+                     "r"(G::TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
@@ -168,8 +256,8 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         bool run = true;
         for (int tile = blockIdx.x; run && tile < p.total_tiles; tile += gridDim.x, ++local) {
             for (int kc = 0; kc < nk; ++kc, ++seq) {
-                const int stage = seq & 1;
-                const uint32_t parity = (seq >> 1) & 1;
+                const int stage = seq % NS;
+                const uint32_t parity = (seq / NS) & 1;
                 if (ptid == 0 && kc == 0 && !stall_ok(p, 2, local, bar_gate, abort_flag)) *prod_abort = 1u;
                 // The TMA copies of this stage (pw chunk and halo) have landed.
                 if (ptid == 0 && !*prod_abort && !wait_bounded(bar_tma + 8 * stage, parity, abort_flag))
@@ -184,10 +272,10 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                 for (int spin = 0; !mbar_try_wait(bar_tma + 8 * stage, parity) && spin < (1 << 20); ++spin) {
                 }
 
-                const uint32_t a_hi = sbase + stage * STAGE_BYTES;
+                const uint32_t a_hi = sbase + stage * G::STAGE_BYTES;
                 const uint32_t a_lo = a_hi + A_BYTES;
-                const uint32_t b_hi = a_lo + A_BYTES;
-                const uint32_t b_lo = b_hi + B_BYTES;
+                const uint32_t b_lo = a_hi + G::OFF_BLO;
+                const uint32_t b_hi = a_hi + G::OFF_BHI;
 
                 // pw chunk: B_hi stays the raw fp32 the TMA wrote, because the MMA
                 // reads only the TF32 bits of an fp32 operand (the 13 low mantissa
@@ -197,8 +285,8 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                 // B_lo is written after the barrier below.
                 auto split_pw = [&]() {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int row = warp * 32 + i * 4 + (lane >> 3);
+                    for (int i = 0; i < G::TN / 32; ++i) {
+                        const int row = warp * (G::TN / 8) + i * 4 + (lane >> 3);
                         const uint32_t off = sw128_off(row, lane & 7);
                         sts128(b_lo + off, tf32_trunc_rest4(lds128(b_hi + off)));
                     }
@@ -209,9 +297,8 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                 // Sample j of the halo is x[t0*S - pad - R + j]; output time
                 // 16*warp + i takes samples S*(16*warp + i) + R + k, k < K.  At
                 // stride 2, samples j >= XW2 sit in the second box (B_lo region).
-                const float* xs0 = reinterpret_cast<const float*>(smem + stage * STAGE_BYTES) + lane * PITCH;
-                const float* xs1 =
-                    reinterpret_cast<const float*>(smem + stage * STAGE_BYTES + 2 * A_BYTES + B_BYTES) + lane * PITCH;
+                const float* xs0 = reinterpret_cast<const float*>(smem + stage * G::STAGE_BYTES) + lane * PITCH;
+                const float* xs1 = xs0 + KC * XW2;  // the second stride-2 box follows the first
                 float win[4 * NV];
 #pragma unroll
                 for (int q = 0; q < NV; ++q) {
@@ -263,42 +350,41 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     } else if (warp == MMA_WARP) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0)
-            mma_issuer(p, tmem, sbase, bar_full, bar_empty, bar_afull, bar_aempty, bar_drain, abort_flag, nk,
-                       bar_gate);
+            mma_issuer_g<G>(p, tmem, sbase, bar_full, bar_empty, bar_afull, bar_aempty, bar_drain, abort_flag, nk,
+                            bar_gate);
         __syncwarp();
     } else if (warp == TMA_WARP) {
         // -------------------------------------------------------- TMA issuer
         if (lane == 0) {
             int seq = 0;
-            bool pending[2] = {false, false};
+            bool pending[NS] = {};
             bool ok = true;
             int local = 0;
             for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++local) {
                 if (!stall_ok(p, 1, local, bar_gate, abort_flag)) break;
-                const TileCoord tcd = decode_tile(p, tile);
+                const TileCoord tcd = decode_tile<TN_>(p, tile);
                 const int x0 = tcd.t0 * S - p.pad - R;  // a multiple of 4: 16-byte aligned time coordinate
                 // Pull the next tile's halo boxes into L2 now, so its TMA loads
                 // wait on L2 rather than on DRAM latency.
                 if (tile + (int)gridDim.x < p.total_tiles) {
-                    const TileCoord nx = decode_tile(p, tile + gridDim.x);
+                    const TileCoord nx = decode_tile<TN_>(p, tile + gridDim.x);
                     for (int k = 0; k < nk; ++k) {
                         tma_prefetch_3d(&x_map, nx.t0 * S - p.pad - R, k * KC, nx.n);
                         if (S == 2) tma_prefetch_3d(&x_map, nx.t0 * S - p.pad - R + XW2, k * KC, nx.n);
                     }
                 }
                 for (int k = 0; k < nk; ++k, ++seq) {
-                    const int stage = seq & 1;
-                    if (!wait_bounded(bar_empty + 8 * stage, ((seq >> 1) & 1) ^ 1, abort_flag)) {
+                    const int stage = seq % NS;
+                    if (!wait_bounded(bar_empty + 8 * stage, ((seq / NS) & 1) ^ 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                     pending[stage] = false;  // the producers consumed its previous loads before the MMA ran
-                    const uint32_t st = sbase + stage * STAGE_BYTES;
-                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES + (S == 1 ? X_BYTES : 2 * X2_BYTES));
-                    tma_load_2d(st + 2 * A_BYTES, &pw_map, k * KC, tcd.o0, bar_tma + 8 * stage);
+                    const uint32_t st = sbase + stage * G::STAGE_BYTES;
+                    mbar_arrive_expect_tx(bar_tma + 8 * stage, G::B_BYTES + (S == 1 ? X_BYTES : 2 * X2_BYTES));
+                    tma_load_2d(st + G::OFF_BHI, &pw_map, k * KC, tcd.o0, bar_tma + 8 * stage);
                     tma_load_3d(st, &x_map, x0, k * KC, tcd.n, bar_tma + 8 * stage);
-                    if (S == 2)
-                        tma_load_3d(st + 2 * A_BYTES + B_BYTES, &x_map, x0 + XW2, k * KC, tcd.n, bar_tma + 8 * stage);
+                    if (S == 2) tma_load_3d(st + X2_BYTES, &x_map, x0 + XW2, k * KC, tcd.n, bar_tma + 8 * stage);
                     pending[stage] = true;
                 }
             }
@@ -306,11 +392,11 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             // also when another role gave up and they were never consumed
             // (normally they have all landed and this returns at once).
             {
-                for (int st = 0; st < 2; ++st) {
+                for (int st = 0; st < NS; ++st) {
                     if (!pending[st]) continue;
-                    const int last = seq - 1 - ((seq - 1 - st) & 1);  // latest sequence number on this stage
+                    const int last = seq - 1 - ((seq - 1 - st) % NS);  // latest sequence number on this stage
                     const unsigned long long t0 = globaltimer();
-                    while (last >= 0 && !mbar_try_wait(bar_tma + 8 * st, (last >> 1) & 1)) {
+                    while (last >= 0 && !mbar_try_wait(bar_tma + 8 * st, (last / NS) & 1)) {
                         if (globaltimer() - t0 > kWaitLimitNs) break;
                     }
                 }
@@ -319,14 +405,14 @@ dwsep_conv1d_tcx_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        epilogue_warp(p, tmem, bar_afull, bar_aempty, abort_flag, warp, lane, bar_gate);
+        epilogue_warp<TN_>(p, tmem, bar_afull, bar_aempty, abort_flag, warp, lane, bar_gate);
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == MMA_WARP) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(TMEM_COLS)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(G::TMEM_COLS)
                      : "memory");
     }
 }
@@ -342,11 +428,46 @@ inline bool conv1d_tcx_supported(int C, int T, int O, int K, int stride, const v
            (reinterpret_cast<uintptr_t>(pw) & 15) == 0 && cw * K <= tcx::DWX_MAX;
 }
 
+namespace tcx {
+using KernelPtr = void (*)(const tc::Params, const CUtensorMap, const CUtensorMap);
+
+// The instance for (K, r, stride) at tile width TN_: K = 9 with r = 0 and K = 3
+// with r = 3 (the pages' kernel sizes with pad K/2) have their taps unrolled
+// at 256 columns; every other K runs the generic K <= 13 loop.
+template <int TN_>
+inline KernelPtr select_kernel(int K, int r, int stride)
+{
+    if (stride == 1) {
+        if constexpr (TN_ == 256) {
+            if (K == 9 && r == 0) return dwsep_conv1d_tcx_kernel<9, 0, 1, TN_>;
+            if (K == 3 && r == 3) return dwsep_conv1d_tcx_kernel<3, 3, 1, TN_>;
+        }
+        if (r == 0) return dwsep_conv1d_tcx_kernel<0, 0, 1, TN_>;
+        if (r == 1) return dwsep_conv1d_tcx_kernel<0, 1, 1, TN_>;
+        if (r == 2) return dwsep_conv1d_tcx_kernel<0, 2, 1, TN_>;
+        return dwsep_conv1d_tcx_kernel<0, 3, 1, TN_>;
+    }
+    if constexpr (TN_ == 256) {
+        if (K == 9 && r == 0) return dwsep_conv1d_tcx_kernel<9, 0, 2, TN_>;
+        if (K == 3 && r == 3) return dwsep_conv1d_tcx_kernel<3, 3, 2, TN_>;
+    }
+    if (r == 0) return dwsep_conv1d_tcx_kernel<0, 0, 2, TN_>;
+    if (r == 1) return dwsep_conv1d_tcx_kernel<0, 1, 2, TN_>;
+    if (r == 2) return dwsep_conv1d_tcx_kernel<0, 2, 2, TN_>;
+    return dwsep_conv1d_tcx_kernel<0, 3, 2, TN_>;
+}
+}  // namespace tcx
+
+// Output channels per tile of the TMA-halo kernel: 128 when O fits in one such
+// tile (a 256-wide tile would be half zero), else 256.
+inline int conv1d_tcx_tile_n(int O) { return O <= 128 ? 128 : 256; }
+
 inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float* pw, const float* bias, int N,
                                    int C, int T, int O, int K, int stride, int pad, int To, float* out,
                                    cudaStream_t stream, int stall_role = 0, int stall_at = 0,
                                    unsigned long long stall_ns = 0)
 {
+    const int tn = conv1d_tcx_tile_n(O);
     tc::Params prm;
     prm.stall_role = stall_role;
     prm.stall_at = stall_at;
@@ -354,7 +475,7 @@ inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float*
     prm.x = x; prm.dw = dw; prm.pw = pw; prm.bias = bias; prm.out = out;
     prm.C = C; prm.T = T; prm.O = O; prm.K = K; prm.pad = pad; prm.To = To;
     prm.tiles_t = (To + tc::TM - 1) / tc::TM;
-    prm.tiles_o = (O + tc::TN - 1) / tc::TN;
+    prm.tiles_o = (O + tn - 1) / tn;
     const long long total = (long long)N * prm.tiles_t * prm.tiles_o;
     if (total > 0x7fffffffLL) return FCV_ERR_UNSUPPORTED;
     prm.total_tiles = (int)total;
@@ -362,12 +483,12 @@ inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float*
 
     auto encode = tensor_map_encoder();
     if (!encode) return FCV_ERR_CUDA;
-    // pw [O][C]: 32 channels x 256 output channels per box, 128B-swizzled.
+    // pw [O][C]: 32 channels x tn output channels per box, 128B-swizzled.
     CUtensorMap pw_map, x_map;
     {
         const cuuint64_t gdim[2] = {(cuuint64_t)C, (cuuint64_t)O};
         const cuuint64_t gstride[1] = {(cuuint64_t)C * sizeof(float)};
-        const cuuint32_t box[2] = {(cuuint32_t)tc::KC, (cuuint32_t)tc::TN};
+        const cuuint32_t box[2] = {(cuuint32_t)tc::KC, (cuuint32_t)tn};
         const cuuint32_t estride[2] = {1, 1};
         if (encode(&pw_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pw), gdim, gstride, box, estride,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -392,26 +513,12 @@ inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float*
     if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
     const int r = (-pad) & 3;  // (t0*stride - pad) mod 4 with t0 a multiple of 128
-    decltype(&tcx::dwsep_conv1d_tcx_kernel<0, 0, 1>) kern;
-    if (stride == 1) {
-        if (K == 9 && r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<9, 0, 1>;
-        else if (K == 3 && r == 3) kern = tcx::dwsep_conv1d_tcx_kernel<3, 3, 1>;
-        else if (r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<0, 0, 1>;
-        else if (r == 1) kern = tcx::dwsep_conv1d_tcx_kernel<0, 1, 1>;
-        else if (r == 2) kern = tcx::dwsep_conv1d_tcx_kernel<0, 2, 1>;
-        else kern = tcx::dwsep_conv1d_tcx_kernel<0, 3, 1>;
-    } else {
-        if (K == 9 && r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<9, 0, 2>;
-        else if (K == 3 && r == 3) kern = tcx::dwsep_conv1d_tcx_kernel<3, 3, 2>;
-        else if (r == 0) kern = tcx::dwsep_conv1d_tcx_kernel<0, 0, 2>;
-        else if (r == 1) kern = tcx::dwsep_conv1d_tcx_kernel<0, 1, 2>;
-        else if (r == 2) kern = tcx::dwsep_conv1d_tcx_kernel<0, 2, 2>;
-        else kern = tcx::dwsep_conv1d_tcx_kernel<0, 3, 2>;
-    }
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcx::SMEM_BYTES) != cudaSuccess)
+    const tcx::KernelPtr kern = tn == 256 ? tcx::select_kernel<256>(K, r, stride) : tcx::select_kernel<128>(K, r, stride);
+    const int smem = (int)(tn == 256 ? tcx::Geo<256>::SMEM_BYTES : tcx::Geo<128>::SMEM_BYTES);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return FCV_ERR_CUDA;
     const int grid = (int)(total < sms ? total : sms);
-    kern<<<grid, tc::NTHREADS, tcx::SMEM_BYTES, stream>>>(prm, pw_map, x_map);
+    kern<<<grid, tc::NTHREADS, smem, stream>>>(prm, pw_map, x_map);
     return launch_status();
 }
 

@@ -277,6 +277,58 @@ def test_guard_bands_untouched():
         assert torch.isfinite(o_).all()
 
 
+def _guarded_copy(t, guard=1024):
+    """t's values inside a NaN-filled device buffer with `guard` floats on each
+    side (4 KiB: the 16-byte alignment the TMA paths need is kept)."""
+    buf = torch.full((t.numel() + 2 * guard,), float("nan"), device="cuda")
+    view = buf[guard:guard + t.numel()].view(t.shape)
+    view.copy_(t)
+    return buf, view
+
+
+def _check_guards_and_inputs(guarded, originals, guard=1024):
+    for (buf, view), orig in zip(guarded, originals):
+        assert torch.isnan(buf[:guard]).all() and torch.isnan(buf[-guard:]).all(), "a guard region changed"
+        assert torch.equal(view, orig), "an input changed"
+
+
+@pytest.mark.parametrize("W", [48, 47], ids=["tma", "cp_async"])
+@pytest.mark.parametrize("algo", CONV2D_ALGOS)
+def test_conv2d_inputs_in_guard_regions(algo, W):
+    """Every input inside NaN guard regions: a read past an input's ends would
+    turn outputs into NaN, so oracle parity shows none happens; the inputs and
+    their guards are unchanged afterwards."""
+    case = wl.Conv2dCase("inguard", 3, 5, 61, W, 19, 4, seed=7)
+    x, w, b = wl.conv2d_inputs(case)
+    originals = cuda(x, w, b)
+    guarded = [_guarded_copy(t) for t in originals]
+    xg, wg, bg = [v for _, v in guarded]
+    out = conv2d_or_skip(fcv.conv2d_pool_sigmoid_sum, xg, wg, bg, case.P, algo)
+    tap = conv2d_or_skip(fcv.conv2d_pool_tap, xg, wg, bg, case.P, algo)
+    torch.cuda.synchronize()
+    _check_guards_and_inputs(guarded, originals)
+    xn, wn, bn = x.numpy(), w.numpy(), b.numpy()
+    assert_close(out, oracle.conv2d_pool_sigmoid_sum(xn, wn, bn, case.P), "out")
+    assert_close(tap, oracle.conv2d_pool_tap(xn, wn, bn, case.P), "tap")
+
+
+@pytest.mark.parametrize("shape", [(2, 36, 516, 40, 9, 1, 4), (2, 36, 516, 40, 9, 2, 4), (2, 36, 517, 40, 7, 1, 3)],
+                         ids=["s1", "s2", "s1_ragged_T"])
+@pytest.mark.parametrize("algo", CONV1D_ALGOS)
+def test_conv1d_inputs_in_guard_regions(algo, shape):
+    """The same for op B, at stride 1 and 2 and with T % 4 != 0 (register halo)."""
+    case = wl.Conv1dCase("inguard", *shape, seed=8)
+    x, dw, pw, bias = wl.conv1d_inputs(case)
+    originals = cuda(x, dw, pw, bias)
+    guarded = [_guarded_copy(t) for t in originals]
+    xg, dwg, pwg, bg = [v for _, v in guarded]
+    out = conv1d_or_skip(xg, dwg, pwg, bg, case.stride, case.pad, algo)
+    torch.cuda.synchronize()
+    _check_guards_and_inputs(guarded, originals)
+    ref = oracle.dwsep_conv1d(x.numpy(), dw.numpy(), pw.numpy(), bias.numpy(), case.stride, case.pad)
+    assert_close(out, ref, "out")
+
+
 def test_conv1d_bitwise_repeatable():
     case = wl.CONV1D_SMALL
     x, dw, pw, bias = cuda(*wl.conv1d_inputs(case))

@@ -207,28 +207,30 @@ def full_chunk_kernel(T, C, A):
     return sim
 
 
-def conv1d_tma_halo_kernel(T, NK):
+def conv1d_tma_halo_kernel(T, NK, stages=2):
     """dwsep_conv1d_tcx_kernel: T tiles per CTA, NK 32-channel chunks per tile.
 
-    Two smem stages (seq & 1) hold the pw chunk and the x halo, which the TMA
-    warp loads once the MMAs that read the stage are done ("empty", a commit);
-    8 producer warps wait for the loads ("tma"), turn the halo into the A
-    operand in place and arrive at "full"; one issuer waits for "full" per
-    chunk and for the accumulator (local & 1) to be drained ("aempty", 4
-    epilogue warps) per tile, and commits "empty" per chunk and "afull" per
-    tile.  The register-halo kernel (dwsep_conv1d_tc_kernel) has the same
-    protocol: its TMA brings only the pw chunk, and its halo goes through a
+    `stages` smem stages (seq % stages; two for 256-wide tiles, three for
+    128-wide ones) hold the pw chunk and the x halo, which the TMA warp loads
+    once the MMAs that read the stage are done ("empty", a commit); 8 producer
+    warps wait for the loads ("tma"), turn the halo into the A operand in place
+    and arrive at "full"; one issuer waits for "full" per chunk and for the
+    accumulator (local & 1) to be drained ("aempty", 4 epilogue warps) per
+    tile, and commits "empty" per chunk and "afull" per tile.  The
+    register-halo kernel (dwsep_conv1d_tc_kernel) has the same protocol with
+    two stages: its TMA brings only the pw chunk, and its halo goes through a
     buffer only the producers use, ordered by their own group barrier."""
     sim = Sim()
-    for s in range(2):
+    for s in range(stages):
         sim.bar(f"full{s}", 8)
         sim.bar(f"empty{s}", 1)
         sim.bar(f"tma{s}", 1)
-        sim.bar(f"afull{s}", 1)
-        sim.bar(f"aempty{s}", 4)
+    for b in range(2):
+        sim.bar(f"afull{b}", 1)
+        sim.bar(f"aempty{b}", 4)
     tma, prod = [], []
     for seq in range(T * NK):
-        st, k = seq & 1, seq >> 1
+        st, k = seq % stages, seq // stages
         tma += [("wait", f"empty{st}", (k & 1) ^ 1, k, "tma"), ("owns", f"empty{st}", k, "tma"),
                 ("arrive", f"tma{st}", k, 1, "tma")]
         prod += [("wait", f"tma{st}", k & 1, k + 1, "producers"), ("owns", f"empty{st}", k, "producers"),
@@ -240,7 +242,7 @@ def conv1d_tma_halo_kernel(T, NK):
         issue += [("wait", f"aempty{buf}", (bk & 1) ^ 1, bk, "issuer"), ("owns", f"aempty{buf}", bk, "issuer")]
         for c in range(NK):
             seq = t * NK + c
-            st, k = seq & 1, seq >> 1
+            st, k = seq % stages, seq // stages
             issue += [("wait", f"full{st}", k & 1, k + 1, "issuer"), ("issue", 0)]
             complete += [("issued", 0, n), ("arrive", f"empty{st}", k, 1, "mma")]
             n += 1
@@ -310,11 +312,12 @@ def test_conv1d_pair_kernel_protocol(T, NK):
         conv1d_pair_kernel(T, NK).run(seed)
 
 
+@pytest.mark.parametrize("stages", [2, 3])
 @pytest.mark.parametrize("T", [1, 2, 3, 5, 8])
 @pytest.mark.parametrize("NK", [1, 2, 3, 8])
-def test_conv1d_tma_halo_kernel_protocol(T, NK):
+def test_conv1d_tma_halo_kernel_protocol(T, NK, stages):
     for seed in range(30):
-        conv1d_tma_halo_kernel(T, NK).run(seed)
+        conv1d_tma_halo_kernel(T, NK, stages).run(seed)
 
 
 SHAPES = [(T, C, A) for T in (1, 2, 3, 4, 7) for C in (1, 2, 3) for A in (2, 3)]
