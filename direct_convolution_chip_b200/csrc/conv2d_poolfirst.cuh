@@ -14,11 +14,18 @@
 // pooled value), taken to its end: the conv output is never formed at all.
 //
 // Kernel: a CTA covers 8 x 16 pooled positions x 64 output channels of one
-// image, in chunks of 4 input channels:
-//   1. cp.async stages the input halo [4][8P+2][16P+2] and the weights
-//      [4*9][64] (zero past the image / past Cin / past Cout);
-//   2. each thread forms the box sums S of two (position, channel) pairs with
-//      separable running sums over its (P+2)x(P+2) patch -> smem S[36][128];
+// image, in chunks of ICC input channels (4; 2 from P = 5 on, so that two CTAs
+// still fit an SM):
+//   1. cp.async stages the input halo [ICC][8P+2][16P+2] (16-byte copies of
+//      whole rows when W % 4 == 0 and x is 16-byte aligned, else 4-byte ones)
+//      and the weights [ICC*9][64] (zero past the image / Cin / Cout);
+//   2. the box sums S[ic][ky][kx][pos] in two separable passes, both with the
+//      lanes of a warp on consecutive pooled columns: horizontal sums of P
+//      samples at the three column offsets kx (one vector read of P+2 samples
+//      per row and pooled column) into H[ic][kx][row][px], then vertical
+//      running sums over P rows at the three row offsets ky.  H's row pitch
+//      puts the two half-warps of the vertical pass (pooled rows 2j, 2j+1) in
+//      opposite halves of the banks;
 //   3. the contraction out[pos][c] += sum_k S[k][pos] * W[k][c] runs as a
 //      register-blocked FP32 GEMM: 4 positions x 8 channels per thread, packed
 //      fma.rn.f32x2 over channel pairs.
@@ -36,20 +43,58 @@ struct PoolFirstGeom {
     static constexpr int TPH = 8, TPW = 16;          // pooled positions per CTA: 8 x 16
     static constexpr int NPOS = TPH * TPW;           // 128
     static constexpr int CB = 64;                    // output channels per CTA
-    static constexpr int ICC = 4;                    // input channels per chunk
+    static constexpr int ICC = P <= 4 ? 4 : 2;       // input channels per chunk
     static constexpr int NT = 256;
     static constexpr int KC = ICC * 9;               // contraction length per chunk
     static constexpr int HY = P * TPH + 2, HX = P * TPW + 2;
-    static constexpr int HXP = HX + 1;               // odd pitch: patch rows of adjacent positions spread over banks
+    static constexpr int HXP = (HX + 3) & ~3;        // halo row pitch: rows start 16-byte aligned
+    static constexpr int NF4 = HXP / 4;              // 16-byte pieces per staged row
+    // Row pitch of the horizontal sums H: (P * HRP) mod 32 == 16, so pooled
+    // rows 2j and 2j+1 (the two half-warps of the vertical pass) use opposite
+    // bank halves.
+    static constexpr int HRP = (P & 1) ? 16 : (P == 4 ? 20 : (P == 8 ? 18 : 24));
     static constexpr int RP = 4, RC = 8;             // per-thread register block: 4 positions x 8 channels
     static constexpr int HALO_FLOATS = ICC * HY * HXP;
+    static constexpr int H_FLOATS = ICC * 3 * HY * HRP;
     static constexpr int S_FLOATS = KC * NPOS;
     static constexpr int W_FLOATS = KC * CB;
-    static constexpr size_t SMEM_BYTES = sizeof(float) * (HALO_FLOATS + S_FLOATS + W_FLOATS + NT / 32 + 4);
+    static constexpr size_t SMEM_BYTES =
+        sizeof(float) * (HALO_FLOATS + H_FLOATS + S_FLOATS + W_FLOATS + NT / 32 + 4);
     static_assert((NPOS / RP) * (CB / RC) == NT, "thread layout");
+    static_assert((P * HRP) % 32 == 16 && HRP >= TPW, "vertical-pass bank halves");
+    static_assert(SMEM_BYTES * 2 <= 227 * 1024, "two CTAs per SM");
+    static_assert(HALO_FLOATS % 4 == 0 && H_FLOATS % 4 == 0 && S_FLOATS % 4 == 0, "16-byte aligned smem arrays");
 };
 
-template <int P, int MODE>
+// The P + 2 consecutive samples v[0..P+1] at p, with the widest loads the
+// alignment of p allows (p = row + P * px: 16 bytes when P % 4 == 0, 8 when P
+// is even, else 4; lanes on consecutive px then read consecutive words).
+template <int P>
+__device__ __forceinline__ void load_run(const float* p, float (&v)[P + 2])
+{
+    if constexpr (P % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < P / 4; ++q) {
+            const float4 t = *reinterpret_cast<const float4*>(p + 4 * q);
+            v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+        }
+        const float2 t = *reinterpret_cast<const float2*>(p + P);
+        v[P] = t.x; v[P + 1] = t.y;
+    } else if constexpr (P % 2 == 0) {
+#pragma unroll
+        for (int q = 0; q < (P + 2) / 2; ++q) {
+            const float2 t = *reinterpret_cast<const float2*>(p + 2 * q);
+            v[2 * q] = t.x; v[2 * q + 1] = t.y;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < P + 2; ++q) v[q] = p[q];
+    }
+}
+
+// VEC: the halo rows are staged as 16-byte copies (W % 4 == 0 and x 16-byte
+// aligned), else as 4-byte ones.
+template <int P, int MODE, bool VEC>
 __global__ void __launch_bounds__(256, 2)
 conv2d_poolfirst_kernel(const float* __restrict__ x, const float* __restrict__ w,
                         const float* __restrict__ bias, int Cin, int H, int W, int Cout,
@@ -58,11 +103,12 @@ conv2d_poolfirst_kernel(const float* __restrict__ x, const float* __restrict__ w
 {
     using G = PoolFirstGeom<P>;
     constexpr int NT = G::NT, NPOS = G::NPOS, CB = G::CB, ICC = G::ICC, KC = G::KC;
-    constexpr int HY = G::HY, HX = G::HX, HXP = G::HXP, RP = G::RP, RC = G::RC;
+    constexpr int HY = G::HY, HX = G::HX, HXP = G::HXP, RP = G::RP, RC = G::RC, HRP = G::HRP;
 
     extern __shared__ __align__(16) float smem[];
     float* halo = smem;                       // [ICC][HY][HXP]
-    float* Ss = halo + G::HALO_FLOATS;        // [KC][NPOS]   box sums, k = icl*9 + ky*3 + kx
+    float* Hs = halo + G::HALO_FLOATS;        // [ICC][3][HY][HRP]  horizontal sums at column offsets kx
+    float* Ss = Hs + G::H_FLOATS;             // [KC][NPOS]   box sums, k = icl*9 + ky*3 + kx
     float* Ws = Ss + G::S_FLOATS;             // [KC][CB]
     float* red = Ws + G::W_FLOATS;            // [NT/32 + 4]
 
@@ -86,14 +132,31 @@ conv2d_poolfirst_kernel(const float* __restrict__ x, const float* __restrict__ w
         for (int j = 0; j < RC / 2; ++j) acc[i][j] = make_float2(0.f, 0.f);
 
     const float* xn = x + (size_t)n * Cin * H * W;
+    const int warp = tid >> 5, lane = tid & 31;
     for (int ic0 = 0; ic0 < Cin; ic0 += ICC) {
-        for (int i = tid; i < ICC * HY * HX; i += NT) {
-            const int icl = i / (HY * HX);
-            const int rem = i - icl * (HY * HX);
-            const int r = rem / HX, sc = rem - (rem / HX) * HX;
-            const int ic = ic0 + icl, yy = y0 + r, xx = x0 + sc;
-            const bool in = ic < Cin && yy < H && xx < W;
-            cp_async4(halo + (icl * HY + r) * HXP + sc, in ? xn + ((size_t)ic * H + yy) * W + xx : x, in);
+        if constexpr (VEC) {
+            // one staged row per warp iteration: x0 is a multiple of 16 and W of
+            // 4, so a 16-byte piece lies wholly inside or wholly outside the row
+            for (int row = warp; row < ICC * HY; row += NT / 32) {
+                const int icl = row / HY, r = row - (row / HY) * HY;
+                const int ic = ic0 + icl, yy = y0 + r;
+                const bool row_in = ic < Cin && yy < H;
+                const float* src = xn + ((size_t)(row_in ? ic : 0) * H + (row_in ? yy : 0)) * W;
+                for (int f = lane; f < G::NF4; f += 32) {
+                    const int xx = x0 + 4 * f;
+                    const bool in = row_in && xx < W;
+                    cp_async16(halo + row * HXP + 4 * f, in ? src + xx : x, in ? 16 : 0);
+                }
+            }
+        } else {
+            for (int i = tid; i < ICC * HY * HX; i += NT) {
+                const int icl = i / (HY * HX);
+                const int rem = i - icl * (HY * HX);
+                const int r = rem / HX, sc = rem - (rem / HX) * HX;
+                const int ic = ic0 + icl, yy = y0 + r, xx = x0 + sc;
+                const bool in = ic < Cin && yy < H && xx < W;
+                cp_async4(halo + (icl * HY + r) * HXP + sc, in ? xn + ((size_t)ic * H + yy) * W + xx : x, in);
+            }
         }
         for (int i = tid; i < KC * CB; i += NT) {
             const int cl = i % CB, k = i / CB;
@@ -106,33 +169,44 @@ conv2d_poolfirst_kernel(const float* __restrict__ x, const float* __restrict__ w
         cp_async_wait<0>();
         __syncthreads();
 
-        // Box sums: (position, input channel) pairs, two per thread.
-        for (int q = tid; q < NPOS * ICC; q += NT) {
-            const int pos = q % NPOS, icl = q / NPOS;
+        // Horizontal pass: for every staged row and pooled column px, the sums of
+        // P samples starting at columns P*px + kx, kx = 0, 1, 2.
+        for (int i = tid; i < ICC * HY * G::TPW; i += NT) {
+            const int px = i % G::TPW, row = i / G::TPW;
+            const int icl = row / HY, r = row - (row / HY) * HY;
+            float v[P + 2];
+            load_run<P>(halo + row * HXP + P * px, v);
+            float h = 0.f;
+#pragma unroll
+            for (int dx = 0; dx < P; ++dx) h += v[dx];
+            float* hd = Hs + ((icl * 3) * HY + r) * HRP + px;
+            hd[0] = h;
+            h = h - v[0] + v[P];
+            hd[HY * HRP] = h;
+            h = h - v[1] + v[P + 1];
+            hd[2 * HY * HRP] = h;
+        }
+        __syncthreads();
+
+        // Vertical pass: for every (input channel, kx) and pooled position, the
+        // sums of P horizontal sums starting at rows P*py + ky, ky = 0, 1, 2:
+        // the box sums S[ic][ky][kx][pos].
+        for (int i = tid; i < ICC * 3 * NPOS; i += NT) {
+            const int pos = i % NPOS, g = i / NPOS;
+            const int icl = g / 3, kx = g - (g / 3) * 3;
             const int py = pos / G::TPW, px = pos % G::TPW;
-            const float* hp = halo + (icl * HY + py * P) * HXP + px * P;
-            // row sums over P columns at the 3 column offsets, for the P+2 rows
-            float R[P + 2][3];
+            const float* hp = Hs + ((icl * 3 + kx) * HY + P * py) * HRP + px;
+            float v[P + 2];
 #pragma unroll
-            for (int r = 0; r < P + 2; ++r) {
-                float s0 = 0.f;
+            for (int j = 0; j < P + 2; ++j) v[j] = hp[j * HRP];
+            float s = 0.f;
 #pragma unroll
-                for (int dx = 0; dx < P; ++dx) s0 += hp[r * HXP + dx];
-                R[r][0] = s0;
-                R[r][1] = s0 - hp[r * HXP] + hp[r * HXP + P];
-                R[r][2] = R[r][1] - hp[r * HXP + 1] + hp[r * HXP + P + 1];
-            }
-#pragma unroll
-            for (int kx = 0; kx < 3; ++kx) {
-                float s = 0.f;
-#pragma unroll
-                for (int dy = 0; dy < P; ++dy) s += R[dy][kx];
-                Ss[(icl * 9 + 0 * 3 + kx) * NPOS + pos] = s;
-                s = s - R[0][kx] + R[P][kx];
-                Ss[(icl * 9 + 1 * 3 + kx) * NPOS + pos] = s;
-                s = s - R[1][kx] + R[P + 1][kx];
-                Ss[(icl * 9 + 2 * 3 + kx) * NPOS + pos] = s;
-            }
+            for (int dy = 0; dy < P; ++dy) s += v[dy];
+            Ss[(icl * 9 + kx) * NPOS + pos] = s;
+            s = s - v[0] + v[P];
+            Ss[(icl * 9 + 3 + kx) * NPOS + pos] = s;
+            s = s - v[1] + v[P + 1];
+            Ss[(icl * 9 + 6 + kx) * NPOS + pos] = s;
         }
         __syncthreads();
 
@@ -214,7 +288,8 @@ int launch_conv2d_poolfirst_p(const float* x, const float* w, const float* b, in
     const long long nblk = (long long)N * tiles_y * tiles_x;
     const int cblk = (Cout + G::CB - 1) / G::CB;
     if (nblk > 0x7fffffffLL || cblk > 65535) return FCV_ERR_UNSUPPORTED;
-    auto kern = conv2d_poolfirst_kernel<P, MODE>;
+    const bool vec = (W & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0;
+    auto kern = vec ? conv2d_poolfirst_kernel<P, MODE, true> : conv2d_poolfirst_kernel<P, MODE, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::SMEM_BYTES) != cudaSuccess)
         return FCV_ERR_CUDA;
     dim3 grid((unsigned)nblk, (unsigned)cblk);
