@@ -917,22 +917,24 @@ def run_reference(args):
 def run_profile(args):
     """Only one fused op, `--steps` times after `--warmup` calls, nothing else
     launched: the target of the committed ncu captures.  `--batch` replaces the
-    batch size (a smaller case for full-section captures)."""
+    batch size (a smaller case for full-section captures), `--algo` the
+    algorithm (default AUTO)."""
     import direct_convolution_chip_b200 as fcv
     import dataclasses
     torch.cuda.set_device(0)
     c = CASE_A if args.profile == "conv2d" else CASE_B
     if args.batch:
         c = dataclasses.replace(c, N=args.batch, name=f"{c.name}_n{args.batch}")
+    algo = args.algo
     if c.op == "conv2d":
         x, w, b = [t.cuda() for t in wl.conv2d_inputs(c)]
         out = torch.empty((c.N,), device="cuda")
-        fn = lambda: fcv.conv2d_pool_sigmoid_sum(x, w, b, c.P, out=out)
+        fn = lambda: fcv.conv2d_pool_sigmoid_sum(x, w, b, c.P, out=out, algo=algo)
     else:
         x, dw, pw, b = [t.cuda() for t in wl.conv1d_inputs(c)]
         To = (c.T + 2 * c.pad - c.K) // c.stride + 1
         out = torch.empty((c.N, c.O, To), device="cuda")
-        fn = lambda: fcv.dwsep_conv1d(x, dw, pw, b, c.stride, c.pad, out=out)
+        fn = lambda: fcv.dwsep_conv1d(x, dw, pw, b, c.stride, c.pad, out=out, algo=algo)
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
@@ -942,8 +944,8 @@ def run_profile(args):
         fn()
     e1.record()
     torch.cuda.synchronize()
-    print(json.dumps({"profile": c.name, "steps": args.steps, "ms_per_call": e0.elapsed_time(e1) / args.steps,
-                      "device_error": fcv.device_error()}), flush=True)
+    print(json.dumps({"profile": c.name, "algo": algo, "steps": args.steps,
+                      "ms_per_call": e0.elapsed_time(e1) / args.steps, "device_error": fcv.device_error()}), flush=True)
 
 
 def main(argv=None):
@@ -960,6 +962,7 @@ def main(argv=None):
     ap.add_argument("--profile", choices=["conv2d", "dwsep_conv1d"],
                     help="run only this op of the step (the target of ncu captures)")
     ap.add_argument("--batch", type=int, default=0, help="with --profile: batch size instead of the full one")
+    ap.add_argument("--algo", type=int, default=0, help="with --profile: algorithm selector (0: AUTO)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":

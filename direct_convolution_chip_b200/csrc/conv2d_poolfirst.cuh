@@ -68,7 +68,10 @@ struct PoolFirstGeom {
 
 // The P + 2 consecutive samples v[0..P+1] at p, with the widest loads the
 // alignment of p allows (p = row + P * px: 16 bytes when P % 4 == 0, 8 when P
-// is even, else 4; lanes on consecutive px then read consecutive words).
+// is even, else 4; lanes on consecutive px then read consecutive words).  For
+// P % 4 == 0 the last two samples come with a 16-byte load too (at a 16-byte
+// lane stride an 8-byte load would meet another lane's banks); it stays inside
+// the row, whose pitch is 16P + 4 floats then.
 template <int P>
 __device__ __forceinline__ void load_run(const float* p, float (&v)[P + 2])
 {
@@ -78,7 +81,7 @@ __device__ __forceinline__ void load_run(const float* p, float (&v)[P + 2])
             const float4 t = *reinterpret_cast<const float4*>(p + 4 * q);
             v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
         }
-        const float2 t = *reinterpret_cast<const float2*>(p + P);
+        const float4 t = *reinterpret_cast<const float4*>(p + P);
         v[P] = t.x; v[P + 1] = t.y;
     } else if constexpr (P % 2 == 0) {
 #pragma unroll
@@ -122,7 +125,9 @@ conv2d_poolfirst_kernel(const float* __restrict__ x, const float* __restrict__ w
     const int y0 = ph0 * P, x0 = pw0 * P;
     const int tid = threadIdx.x;
 
-    // GEMM thread block: positions 4*pg .. 4*pg+3, channels 8*cgi .. 8*cgi+7
+    // GEMM thread block: positions 4*pg .. 4*pg+3, channels 4*cgi .. 4*cgi+3 and
+    // 32+4*cgi .. 32+4*cgi+3 (a quarter-warp's weight loads then cover 128
+    // contiguous bytes)
     const int cgi = tid & 7, pg = tid >> 3;
 
     float2 acc[RP][RC / 2];
@@ -215,8 +220,8 @@ conv2d_poolfirst_kernel(const float* __restrict__ x, const float* __restrict__ w
 #pragma unroll 4
         for (int k = 0; k < kc; ++k) {
             const float4 sv = *reinterpret_cast<const float4*>(Ss + k * NPOS + RP * pg);
-            const float4 w0 = *reinterpret_cast<const float4*>(Ws + k * CB + RC * cgi);
-            const float4 w1 = *reinterpret_cast<const float4*>(Ws + k * CB + RC * cgi + 4);
+            const float4 w0 = *reinterpret_cast<const float4*>(Ws + k * CB + 4 * cgi);
+            const float4 w1 = *reinterpret_cast<const float4*>(Ws + k * CB + CB / 2 + 4 * cgi);
             const float2 wp[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w), make_float2(w1.x, w1.y),
                                   make_float2(w1.z, w1.w)};
             const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
@@ -239,7 +244,7 @@ conv2d_poolfirst_kernel(const float* __restrict__ x, const float* __restrict__ w
         const bool valid = ph < PH && pw < PW;
 #pragma unroll
         for (int j = 0; j < RC; ++j) {
-            const int cc = c_base + RC * cgi + j;
+            const int cc = c_base + (j < 4 ? 4 * cgi + j : CB / 2 + 4 * cgi + (j - 4));
             if (valid && cc < Cout) {
                 const float a = (j & 1) ? acc[i][j / 2].y : acc[i][j / 2].x;
                 const float avg = a / (float)(P * P) + __ldg(bias + cc);
