@@ -816,6 +816,40 @@ def run_layout_probes(lib):
             best = c.value if best is None else min(best, c.value)
         print(json.dumps({"probe": "umma_cycles", "m": m, "n": n, "a": "tmem" if a_tmem else "smem",
                           "b": "smem, K-major, no swizzle", "status": st, "sm_cycles_per_mma": best}), flush=True)
+    # Swizzled K-major B with shifted start addresses (the column taps of the
+    # shifted-operand conv2d): which word each (k, n) reads, under two readings
+    # of the swizzle -- on the matrix-relative row, or on the absolute address.
+    n = np.arange(256)
+    for layout, row_bytes, starts in ((6, 32, (0, 128, 256, 384)), (4, 64, (0, 256, 512))):
+        atom = 8 * row_bytes
+        for start in starts:
+            for base_off in sorted({0, (start >> 7) & 7}):
+                st = lib.fcvprobe_umma_b_map_ex(layout, 16, atom, start, base_off, buf)
+                d = np.frombuffer(buf, dtype=np.float32).reshape(8, 256).astype(np.int64)
+                rel, ab = [], []
+                chunks = row_bytes // 16  # 16-byte chunks per row; the swizzle XORs their index
+                for k in range(8):
+                    off = start + (n // 8) * atom + (n % 8) * row_bytes
+                    swz_rel = (((n % 8) * row_bytes) >> 7) & (chunks - 1)  # from the row inside the matrix
+                    swz_abs = (off >> 7) & (chunks - 1)                      # from the shared-memory address
+                    rel.append((off + ((k // 4) ^ swz_rel) * 16 + (k % 4) * 4) // 4)
+                    ab.append((off + ((k // 4) ^ swz_abs) * 16 + (k % 4) * 4) // 4)
+                rel, ab = np.array(rel) % 2048, np.array(ab) % 2048
+                print(json.dumps({"probe": "umma_b_map_swizzled", "layout": {6: "SW32", 4: "SW64"}[layout],
+                                  "start_offset": start, "base_offset": base_off, "status": st,
+                                  "matches_relative_row_swizzle": bool(np.array_equal(d, rel)),
+                                  "matches_absolute_address_swizzle": bool(np.array_equal(d, ab)),
+                                  "k0_n0_7": d[0, :8].tolist(), "k4_n0_7": d[4, :8].tolist()}), flush=True)
+    for name, layout, lbo, sbo, shift in (("none, planes 3200 B apart, rows 16 B (conv2d today)", 0, 3200, 128, 64),
+                                          ("SW32, rows 32 B", 6, 16, 256, 128), ("SW32, rows 32 B, no shift", 6, 16, 256, 0),
+                                          ("SW64, rows 64 B", 4, 16, 512, 256)):
+        best = None
+        for _ in range(3):
+            c = ctypes.c_double()
+            st = lib.fcvprobe_umma_cycles_ex(128, 192, 1, layout, lbo, sbo, shift, 2001, ctypes.byref(c))
+            best = c.value if best is None else min(best, c.value)
+        print(json.dumps({"probe": "umma_cycles_shifted_b", "m": 128, "n": 192, "a": "tmem", "b": name,
+                          "start_shift_bytes": shift, "status": st, "sm_cycles_per_mma": best}), flush=True)
 
 
 def run_configs(args):
@@ -830,6 +864,7 @@ def run_configs(args):
     peaks, _ = load_peaks()
     fma_peak = fma_peak_tflops(props)
     tf32_peak = peaks["bf16_tflops"] * TF32_OVER_BF16
+    tf32_probe = probe_tf32_tflops()  # the on-box tcgen05 TF32 rate, for the second fraction
     stream = torch.cuda.current_stream()
     sp = P(stream.cuda_stream)
     cases = list(wl.NAMED) + (wl.sweep_cases() if args.sweep else [])
@@ -840,7 +875,8 @@ def run_configs(args):
             fn = lambda: lib.fcv_conv2d_pool_sigmoid_sum(P(x.data_ptr()), P(w.data_ptr()), P(b.data_ptr()), c.N,
                                                          c.Cin, c.H, c.W, c.Cout, c.P, P(out.data_ptr()), sp)
             algo = fcv.conv2d_auto_algo(c.N, c.Cin, c.H, c.W, c.Cout, c.P)
-            pipe, peak = ("3xtf32", tf32_peak / 3.0) if algo == fcv.CONV2D_TC_3XTF32 else ("fp32_fma", fma_peak)
+            tc = algo in (fcv.CONV2D_TC_3XTF32, fcv.CONV2D_TC_SHIFT_3XTF32)
+            pipe, peak = ("3xtf32", tf32_peak / 3.0) if tc else ("fp32_fma", fma_peak)
         else:
             x, dw, pw, b = [t.cuda() for t in wl.conv1d_inputs(c)]
             To = (c.T + 2 * c.pad - c.K) // c.stride + 1
@@ -854,13 +890,17 @@ def run_configs(args):
         macs, nbytes = case_macs(c), case_bytes(c)
         iters = max(3, min(200, int(0.2 / max(2.0 * macs / (peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)))))
         ms = _event_ms(fn, iters, stream)
-        roof = roofline_time_s(macs if (pipe == "fp32_fma" or c.op == "conv2d") else
-                               (macs_conv1d_pointwise(c.N, c.C, c.T, c.O, c.K, c.stride, c.pad)),
-                               nbytes, peak, peaks["hbm_gbs"])
-        print(json.dumps({"config": c.name, "op": c.op, "algo": ALGO_NAMES.get(algo, algo), "ms": ms,
-                          "gflops": 2.0 * macs / (ms / 1e3) / 1e9,
-                          "macs": macs, "bytes": nbytes, "pipe": pipe, "roofline_ms": roof * 1e3,
-                          "roofline_frac": roof / (ms / 1e3), "l2": "inputs resident; no flush"}), flush=True)
+        roof_macs = macs if (pipe == "fp32_fma" or c.op == "conv2d") else \
+            macs_conv1d_pointwise(c.N, c.C, c.T, c.O, c.K, c.stride, c.pad)
+        roof = roofline_time_s(roof_macs, nbytes, peak, peaks["hbm_gbs"])
+        line = {"config": c.name, "op": c.op, "algo": ALGO_NAMES.get(algo, algo), "ms": ms,
+                "gflops": 2.0 * macs / (ms / 1e3) / 1e9,
+                "macs": macs, "bytes": nbytes, "pipe": pipe, "roofline_ms": roof * 1e3,
+                "roofline_frac": roof / (ms / 1e3), "l2": "inputs resident; no flush"}
+        if pipe == "3xtf32" and tf32_probe:
+            roof_p = roofline_time_s(roof_macs, nbytes, tf32_probe / 3.0, peaks["hbm_gbs"])
+            line["roofline_frac_3xtf32_probe"] = roof_p / (ms / 1e3)
+        print(json.dumps(line), flush=True)
         del x, out
 
 

@@ -15,6 +15,13 @@
 //   fcvprobe_umma_cycles  one CTA per SM, one thread issuing `iters` MMAs
 //       back to back (M = 64 or 128, N = 192 or 256, A from shared memory or
 //       tensor memory, both K-major without swizzle); SM cycles per MMA.
+//   fcvprobe_umma_b_map_ex  the B address map of a K-major descriptor with a
+//       given layout type (none, 128/64/32-byte swizzle), leading and stride
+//       byte offsets, start address offset from a 1024-byte aligned image and
+//       descriptor base-offset field.
+//   fcvprobe_umma_cycles_ex  the rate probe with such a B descriptor whose
+//       start address cycles through 0, shift, 2*shift bytes (the three column
+//       taps of a shifted-operand convolution).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -26,6 +33,14 @@ __device__ __forceinline__ uint64_t desc_none(uint32_t addr, uint32_t lbo, uint3
 {
     return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
            ((uint64_t)1 << 46);
+}
+
+// Descriptor with a layout type (bits 61-63: 0 none, 2 SW128, 4 SW64, 6 SW32)
+// and base-offset field (bits 49-51).
+__device__ __forceinline__ uint64_t desc_gen(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout,
+                                             uint32_t base_off)
+{
+    return desc_none(addr, lbo, sbo) | ((uint64_t)(base_off & 7u) << 49) | ((uint64_t)(layout & 7u) << 61);
 }
 
 __device__ __forceinline__ uint32_t idesc_tf32(int m, int n, int b_major)
@@ -56,6 +71,7 @@ constexpr uint32_t SMEM_BYTES = 65536;
 // mode 0: B address map (k0 = 0..7, one MMA each, row 0 of D copied out per k0)
 // mode 1: M = 64 row layout
 __global__ void __launch_bounds__(128, 1) layout_kernel(int mode, int b_major, uint32_t lbo, uint32_t sbo,
+                                                        uint32_t layout, uint32_t start_off, uint32_t base_off,
                                                         float* d_out, unsigned* status)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -107,7 +123,8 @@ __global__ void __launch_bounds__(128, 1) layout_kernel(int mode, int b_major, u
         fence_after();
         if (threadIdx.x == 0) {
             const uint64_t ad = desc_none(su32(A), 128, 256);
-            const uint64_t bd = mode == 0 ? desc_none(su32(B), lbo, sbo) : desc_none(su32(B), 128, 256);
+            const uint64_t bd =
+                mode == 0 ? desc_gen(su32(B) + start_off, lbo, sbo, layout, base_off) : desc_none(su32(B), 128, 256);
             const uint32_t id = mode == 0 ? idesc_tf32(128, 256, b_major) : idesc_tf32(64, 64, 0);
             asm volatile("tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, 0;\n" ::"r"(tmem), "l"(ad), "l"(bd),
                          "r"(id)
@@ -155,7 +172,8 @@ __global__ void __launch_bounds__(128, 1) layout_kernel(int mode, int b_major, u
 
 // Rate: one thread per CTA issues `iters` MMAs into one accumulator, then
 // commits and waits (bounded); SM cycles from clock64.
-__global__ void __launch_bounds__(128, 1) cycles_kernel(int m, int n, int a_tmem, int iters,
+__global__ void __launch_bounds__(128, 1) cycles_kernel(int m, int n, int a_tmem, int iters, uint32_t layout,
+                                                        uint32_t lbo, uint32_t sbo, uint32_t shift,
                                                         unsigned long long* cycles, unsigned* status)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -181,19 +199,35 @@ __global__ void __launch_bounds__(128, 1) cycles_kernel(int m, int n, int a_tmem
     fence_after();
     const uint32_t tmem = tmem_holder;
     if (threadIdx.x == 0) {
-        const uint64_t ad = desc_none(su32(A), 128, 256), bd = desc_none(su32(B), 128, 256);
+        const uint64_t ad = desc_none(su32(A), 128, 256);
+        const uint64_t bd0 = desc_gen(su32(B), lbo, sbo, layout, 0);
+        const uint64_t bd1 = desc_gen(su32(B) + shift, lbo, sbo, layout, 0);
+        const uint64_t bd2 = desc_gen(su32(B) + 2 * shift, lbo, sbo, layout, 0);
         const uint32_t id = idesc_tf32(m, n, 0);
         const uint32_t a_t = tmem + 256;  // A in tensor memory: columns 256..263 (contents do not matter)
         const long long t0 = clock64();
-        for (int i = 0; i < iters; ++i) {
-            if (a_tmem)
+        for (int i = 0; i < iters; i += 3) {
+            if (a_tmem) {
                 asm volatile("tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, 1;\n" ::"r"(tmem), "r"(a_t),
-                             "l"(bd), "r"(id)
+                             "l"(bd0), "r"(id)
                              : "memory");
-            else
+                asm volatile("tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, 1;\n" ::"r"(tmem), "r"(a_t),
+                             "l"(bd1), "r"(id)
+                             : "memory");
+                asm volatile("tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, 1;\n" ::"r"(tmem), "r"(a_t),
+                             "l"(bd2), "r"(id)
+                             : "memory");
+            } else {
                 asm volatile("tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, 1;\n" ::"r"(tmem), "l"(ad),
-                             "l"(bd), "r"(id)
+                             "l"(bd0), "r"(id)
                              : "memory");
+                asm volatile("tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, 1;\n" ::"r"(tmem), "l"(ad),
+                             "l"(bd1), "r"(id)
+                             : "memory");
+                asm volatile("tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, 1;\n" ::"r"(tmem), "l"(ad),
+                             "l"(bd2), "r"(id)
+                             : "memory");
+            }
         }
         asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
                          su32(&bar))
@@ -227,7 +261,7 @@ int fcvprobe_umma_b_map(int b_major, unsigned lbo, unsigned sbo, float* out_host
         return 2;
     }
     cudaFuncSetAttribute(layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    layout_kernel<<<1, 128, SMEM_BYTES>>>(0, b_major, lbo, sbo, d, st);
+    layout_kernel<<<1, 128, SMEM_BYTES>>>(0, b_major, lbo, sbo, 0, 0, 0, d, st);
     unsigned ok = 0;
     int rc = cudaDeviceSynchronize() == cudaSuccess ? 0 : 2;
     if (!rc && cudaMemcpy(out_host, d, 8 * 256 * sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess) rc = 2;
@@ -249,7 +283,7 @@ int fcvprobe_umma_m64_rows(float* out_host)
         return 2;
     }
     cudaFuncSetAttribute(layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    layout_kernel<<<1, 128, SMEM_BYTES>>>(1, 0, 128, 256, d, st);
+    layout_kernel<<<1, 128, SMEM_BYTES>>>(1, 0, 128, 256, 0, 0, 0, d, st);
     unsigned ok = 0;
     int rc = cudaDeviceSynchronize() == cudaSuccess ? 0 : 2;
     if (!rc && cudaMemcpy(out_host, d, 128 * sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess) rc = 2;
@@ -275,7 +309,7 @@ int fcvprobe_umma_cycles(int m, int n, int a_tmem, int iters, double* cycles_per
     }
     // 200 KB of shared memory: one CTA per SM (each allocates all 512 TMEM columns)
     cudaFuncSetAttribute(cycles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    cycles_kernel<<<sms, 128, 200 * 1024>>>(m, n, a_tmem ? 1 : 0, iters, c, st);
+    cycles_kernel<<<sms, 128, 200 * 1024>>>(m, n, a_tmem ? 1 : 0, iters, 0, 128, 256, 0, c, st);
     unsigned long long cyc = 0;
     unsigned ok = 0;
     int rc = cudaDeviceSynchronize() == cudaSuccess ? 0 : 2;
@@ -283,7 +317,71 @@ int fcvprobe_umma_cycles(int m, int n, int a_tmem, int iters, double* cycles_per
     if (!rc && cudaMemcpy(&ok, st, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) rc = 2;
     cudaFree(c);
     cudaFree(st);
-    *cycles_per_mma = (double)cyc / iters;
+    *cycles_per_mma = (double)cyc / (3 * ((iters + 2) / 3));  // the loop issues MMAs three at a time
+    return rc ? rc : (ok ? 0 : 3);
+}
+
+// B address map of a K-major descriptor with layout type `layout` (0 none, 2
+// SW128, 4 SW64, 6 SW32), byte offsets lbo/sbo, start address `start_off`
+// bytes after a 1024-byte aligned image and base-offset field `base_off`;
+// out_host[k * 256 + n] = index (mod 2048) of the word read for (k, n).
+int fcvprobe_umma_b_map_ex(int layout, unsigned lbo, unsigned sbo, unsigned start_off, unsigned base_off,
+                           float* out_host)
+{
+    if ((layout != 0 && layout != 2 && layout != 4 && layout != 6) || lbo > 8192 || sbo > 8192 || (lbo & 15) ||
+        (sbo & 15) || start_off > 4096 || (start_off & 15) || base_off > 7 || !out_host)
+        return 1;
+    // N = 256 rows at most 32 * sbo + one 128-byte row past the start: inside the 48 KB B image
+    if (start_off + 32u * sbo + lbo + 128u > (unsigned)(B_WORDS * 4)) return 1;
+    float* d = nullptr;
+    unsigned* st = nullptr;
+    if (cudaMalloc(&d, 8 * 256 * sizeof(float)) != cudaSuccess) return 2;
+    if (cudaMalloc(&st, sizeof(unsigned)) != cudaSuccess) {
+        cudaFree(d);
+        return 2;
+    }
+    cudaFuncSetAttribute(layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    layout_kernel<<<1, 128, SMEM_BYTES>>>(0, 0, lbo, sbo, (uint32_t)layout, start_off, base_off, d, st);
+    unsigned ok = 0;
+    int rc = cudaDeviceSynchronize() == cudaSuccess ? 0 : 2;
+    if (!rc && cudaMemcpy(out_host, d, 8 * 256 * sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess) rc = 2;
+    if (!rc && cudaMemcpy(&ok, st, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) rc = 2;
+    cudaFree(d);
+    cudaFree(st);
+    return rc ? rc : (ok ? 0 : 3);
+}
+
+// SM cycles per MMA with a B descriptor of the given layout whose start
+// address cycles through 0, shift, 2 * shift bytes.
+int fcvprobe_umma_cycles_ex(int m, int n, int a_tmem, int layout, unsigned lbo, unsigned sbo, unsigned shift,
+                            int iters, double* cycles_per_mma)
+{
+    if ((m != 64 && m != 128) || (n != 192 && n != 256) || iters < 3 || iters > 100000 || !cycles_per_mma ||
+        (layout != 0 && layout != 2 && layout != 4 && layout != 6) || lbo > 8192 || sbo > 8192 || (lbo & 15) ||
+        (sbo & 15) || shift > 1024 || (shift & 15))
+        return 1;
+    // B image: 200 KB - 16 KB for A; rows reach 2 * shift + (n / 8) * sbo + lbo + 128 bytes
+    if (2u * shift + (unsigned)(n / 8) * sbo + lbo + 128u > 184u * 1024u) return 1;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 2;
+    unsigned long long* c = nullptr;
+    unsigned* st = nullptr;
+    if (cudaMalloc(&c, sizeof(unsigned long long)) != cudaSuccess) return 2;
+    if (cudaMalloc(&st, sizeof(unsigned)) != cudaSuccess) {
+        cudaFree(c);
+        return 2;
+    }
+    cudaFuncSetAttribute(cycles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cycles_kernel<<<sms, 128, 200 * 1024>>>(m, n, a_tmem ? 1 : 0, iters, (uint32_t)layout, lbo, sbo, shift, c, st);
+    unsigned long long cyc = 0;
+    unsigned ok = 0;
+    int rc = cudaDeviceSynchronize() == cudaSuccess ? 0 : 2;
+    if (!rc && cudaMemcpy(&cyc, c, sizeof(cyc), cudaMemcpyDeviceToHost) != cudaSuccess) rc = 2;
+    if (!rc && cudaMemcpy(&ok, st, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) rc = 2;
+    cudaFree(c);
+    cudaFree(st);
+    *cycles_per_mma = (double)cyc / (3 * ((iters + 2) / 3));
     return rc ? rc : (ok ? 0 : 3);
 }
 
