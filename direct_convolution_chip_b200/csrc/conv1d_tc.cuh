@@ -185,6 +185,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
+// tcgen05.wait::ld that also names the 16 registers of the load it completes,
+// so no use of them can be scheduled above the wait.
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])
+                 :
+                 : "memory");
+}
+
 // Shared-memory descriptor of a K-major operand in the canonical 128-byte
 // swizzle layout: rows of 128 B, 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
@@ -391,48 +403,64 @@ __device__ __forceinline__ void epilogue_warp(const Params& p, uint32_t tmem, ui
         // each 16-byte store instruction covers 128 contiguous bytes of 4 rows.
         const bool vec = tw + 32 <= p.To && p.out_vec;
         const int kq = lane >> 2, jq = lane & 3;
-        // bias of output channels o0 + 32*i + lane, one load per lane per 32
-        // columns, fetched a step ahead and broadcast by shuffle
-        auto bias_at = [&](int i) {
-            const int o = tcd.o0 + 32 * i + lane;
-            return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f;
-        };
-        float bnext = bias_at(0), bcur = 0.f;
-#pragma unroll 1
-        for (int cb = 0; cb < TN_E / 16; ++cb) {
-            if ((cb & 1) == 0) {
-                bcur = bnext;
-                if (cb + 2 < TN_E / 16) bnext = bias_at((cb >> 1) + 1);
-            }
-            uint32_t r[16];
-            tmem_ld16(taddr + (uint32_t)(cb * 16), r);
-            tmem_wait_ld();
-            const int obase = tcd.o0 + cb * 16;
-            float v[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                v[j] = __uint_as_float(r[j]) + __shfl_sync(0xffffffffu, bcur, (cb & 1) * 16 + j);
+        auto bias_of = [&](int o) { return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f; };
+        // Blocks of 16 columns, two at a time: their eight 4x4 transposes are
+        // independent, so their shuffles overlap.  The bias is added after the
+        // transpose, where a lane's four values belong to one output channel.
+        auto store_pair = [&](int cb, const uint32_t (&ra)[16], const uint32_t (&rb)[16]) {
             if (vec) {
+                float x[2][4][4];
+                float bv[2][4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    // block m: rows = the 4 lanes' times, columns = channels m, 4+m, 8+m, 12+m
-                    float x0 = v[m], x1 = v[4 + m], x2 = v[8 + m], x3 = v[12 + m];
-                    quad_transpose(x0, x1, x2, x3, jq);
-                    const int o = obase + 4 * jq + m;
-                    if (o < p.O) {
-                        float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
-                        __stcs(reinterpret_cast<float4*>(dst), make_float4(x0, x1, x2, x3));  // streaming store
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const uint32_t(&r)[16] = h ? rb : ra;
+                        x[h][m][0] = __uint_as_float(r[m]);
+                        x[h][m][1] = __uint_as_float(r[4 + m]);
+                        x[h][m][2] = __uint_as_float(r[8 + m]);
+                        x[h][m][3] = __uint_as_float(r[12 + m]);
+                        bv[h][m] = bias_of(tcd.o0 + (cb + h) * 16 + 4 * jq + m);
                     }
-                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) quad_transpose(x[h][m][0], x[h][m][1], x[h][m][2], x[h][m][3], jq);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        // rows = the 4 lanes' times, one output channel per lane
+                        const int o = tcd.o0 + (cb + h) * 16 + 4 * jq + m;
+                        if (o < p.O) {
+                            float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
+                            const float b = bv[h][m];
+                            __stcs(reinterpret_cast<float4*>(dst),
+                                   make_float4(x[h][m][0] + b, x[h][m][1] + b, x[h][m][2] + b, x[h][m][3] + b));
+                        }
+                    }
             } else {
                 const int t = tw + lane;
                 float* out_nt = p.out + (size_t)tcd.n * p.O * p.To + t;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int o = obase + j;
-                    if (t < p.To && o < p.O) out_nt[(size_t)o * p.To] = v[j];
-                }
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int o = tcd.o0 + (cb + h) * 16 + j;
+                        if (t < p.To && o < p.O) out_nt[(size_t)o * p.To] = __uint_as_float((h ? rb : ra)[j]) + bias_of(o);
+                    }
             }
+        };
+        constexpr int NB = TN_E / 16;
+        static_assert(NB % 2 == 0, "blocks come in pairs");
+#pragma unroll 1
+        for (int cb = 0; cb < NB; cb += 2) {
+            uint32_t ra[16], rb[16];
+            tmem_ld16(taddr + (uint32_t)(cb * 16), ra);
+            tmem_ld16(taddr + (uint32_t)((cb + 1) * 16), rb);
+            tmem_wait_ld16(ra);
+            tmem_wait_ld16(rb);
+            store_pair(cb, ra, rb);
         }
         tc_fence_before();
         __syncwarp();
