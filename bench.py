@@ -362,12 +362,16 @@ def traffic_per_launch(kernel_key):
     e = d.get(kernel_key)
     if not e:
         return None
-    src = os.path.join(ROOT, e["source"])
+    # "source" is one file or a list of files: the sha256 of their contents,
+    # concatenated in order
+    srcs = e["source"] if isinstance(e["source"], list) else [e["source"]]
+    h = hashlib.sha256()
     try:
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        for src in srcs:
+            h.update(open(os.path.join(ROOT, src), "rb").read())
     except OSError:
         return None
-    return e["bytes_per_launch"] if h == e["source_sha256"] else None
+    return e["bytes_per_launch"] if h.hexdigest() == e["source_sha256"] else None
 
 
 def job_throughput(flops_per_rank_step, world, max_step_s):
@@ -596,7 +600,9 @@ def run_gpu(args):
             per_op[key] = e
         del flush_buf
     fma_src = "148 SMs x 128 FP32 FMA lanes x 2 FLOP x 1965 MHz (spec clocks)"
-    tc_src = ("measured bf16 GEMM (MEASURED_PEAKS) x nominal TF32/BF16 (1.1/2.25), / 3 for the three TF32 "
+    gemm_src = ("measured bf16 GEMM (MEASURED_PEAKS.json, %.1f TFLOP/s)" if peak_src == "measured" else
+                "bf16 GEMM figure of the profiling recipe's fallback (%.1f TFLOP/s; MEASURED_PEAKS.json absent)")
+    tc_src = (gemm_src % peaks["bf16_tflops"] + " x nominal TF32/BF16 (1.1/2.25), / 3 for the three TF32 "
               "products of the 3xTF32 split; FLOPs are the fp32 method's (2 per MAC)")
     tc_probe_src = ("tcgen05.mma kind::tf32 M128 N256 K8 rate probed on this GPU at the start of this run "
                     "(libfcv_probes.so), / 3")
