@@ -16,9 +16,12 @@
 // CTAs) and, in the leader CTA only, one thread issues the MMAs for the pair;
 // warps 9-12 drain this CTA's accumulator rows; warp 13 loads, per chunk, this
 // CTA's half of the pw chunk and its input halo by TMA.  The leader's "full"
-// and "aempty" barriers collect arrivals from both CTAs (remote mbarrier
-// arrives); MMA completion is committed to both CTAs' "empty"/"afull" barriers
-// with a multicast commit.  Every mbarrier wait is bounded; a cluster barrier
+// collects its own 8 producer warps and one forwarded arrival per chunk from
+// the other CTA, whose producers arrive locally and whose warp-8 lane 0 relays
+// (a cluster-scope release per producer warp cost ~1,600 cycles on the
+// producers' path); the leader's "aempty" collects both CTAs' epilogues
+// (remote arrives).  MMA completion is committed to both CTAs' "empty"/"afull"
+// barriers with a multicast commit.  Every mbarrier wait is bounded; a cluster barrier
 // follows initialisation and precedes exit, so no CTA leaves while its peer
 // may still signal it.  No TMA multicast.
 #pragma once
@@ -49,8 +52,8 @@ constexpr uint32_t B_BYTES = TNH * KC * 4;   // 16 KB
 constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
 constexpr uint32_t OFF_DWS = STAGES * STAGE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_DWS + DWX_MAX * 4;
-constexpr uint32_t NBAR = 14;    // full[3] empty[3] afull[2] aempty[2] drain tma[3]
-constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
+constexpr uint32_t NBAR = 17;    // full[3] empty[3] afull[2] aempty[2] drain tma[3] lfull[3]
+constexpr uint32_t OFF_MISC = OFF_BAR + 24 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(X_BYTES <= 2 * A_BYTES, "the halo box must fit the stage's A region");
@@ -174,6 +177,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     const uint32_t bar_aempty = bar_full + 64;   // + 8 * buf (leader's collects both CTAs)
     const uint32_t bar_drain = bar_full + 80;
     const uint32_t bar_tma = bar_full + 88;      // + 8 * stage
+    const uint32_t bar_lfull = bar_full + 112;   // + 8 * stage (rank 1: its producers, forwarded by the relay)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
     volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 8);
@@ -185,7 +189,8 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
-            mbar_init(bar_full + 8 * i, 16);   // 8 producer warps x 2 CTAs (used in the leader)
+            mbar_init(bar_full + 8 * i, 9);    // the leader's 8 producer warps + the other CTA's relay
+            mbar_init(bar_lfull + 8 * i, 8);   // the other CTA's 8 producer warps (used in rank 1)
             mbar_init(bar_empty + 8 * i, 1);   // multicast commit
             mbar_init(bar_tma + 8 * i, 1);     // expect_tx arrival + TMA bytes
         }
@@ -220,7 +225,6 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         // ------------------------------------------------------------ producers
         const int ptid = threadIdx.x;
         const int K = KT > 0 ? KT : p.K;
-        const uint32_t full_leader = mapa(bar_full, 0);
         int stage = 0;
         uint32_t phase = 0;
         bool run = true;
@@ -287,7 +291,10 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                 }
                 asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(full_leader + 8 * stage);
+                // The leader's producers arrive at its "full" directly; the other
+                // CTA's arrive locally and its relay thread forwards one cluster
+                // arrival, so no producer warp waits out a cluster-scope release.
+                if (lane == 0) mbar_arrive(leader ? bar_full + 8 * stage : bar_lfull + 8 * stage);
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
@@ -333,6 +340,30 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                 if (ok) commit2(bar_afull + 8 * buf);  // both CTAs' accumulator rows complete
             }
             commit2(bar_drain);  // every MMA issued for the pair has completed once this fires
+        }
+        if (lane == 0 && !leader) {
+            // Relay: once this CTA's 8 producer warps have filled a stage (local
+            // barrier, CTA-scope release/acquire), one cluster-scope arrival
+            // at the leader's "full" carries their writes to the leader's
+            // issuer.  Bounded like every wait; after an abort the leader's
+            // barrier is still alive (the closing cluster barrier).
+            const uint32_t full_leader = mapa(bar_full, 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < p.total_tiles; tile += npairs) {
+                for (int k = 0; k < nk; ++k) {
+                    if (!wait_bounded(bar_lfull + 8 * stage, phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_cluster(full_leader + 8 * stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
         }
         if (lane == 0) {
             const unsigned long long t0 = globaltimer();

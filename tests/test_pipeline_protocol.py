@@ -252,15 +252,18 @@ def conv1d_tma_halo_kernel(T, NK, stages=2):
     return sim
 
 
-def conv1d_pair_kernel(T, NK, stages=3):
+def conv1d_pair_kernel(T, NK, stages=3, relay=True):
     """dwsep_conv1d_tc2_kernel: a cluster of two CTAs (rank 0 leads) shares
     every MMA (cta_group::2).  Each CTA's TMA warp fills its own stage once
     the MMAs that read it are done (its "empty", which the leader's
-    multicast commit completes in both CTAs); each CTA's 8 producer warps
-    arrive at the leader's "full" (16 arrivals); the leader's issuer waits for
-    "full" per chunk and for the accumulator to be drained by both CTAs'
-    epilogues (its "aempty", 8 arrivals) per tile; its multicast commits
-    complete "empty" and "afull" in both CTAs."""
+    multicast commit completes in both CTAs).  The leader's 8 producer warps
+    arrive at its "full" directly; the other CTA's 8 arrive at a local "lfull",
+    and one relay thread there forwards a single cluster arrival to the
+    leader's "full" (9 arrivals; relay=False: all 16 producer warps arrive at
+    the leader's "full" themselves).  The leader's issuer waits for "full" per
+    chunk and for the accumulator to be drained by both CTAs' epilogues (its
+    "aempty", 8 arrivals) per tile; its multicast commits complete "empty"
+    and "afull" in both CTAs."""
     sim = Sim()
     for r in range(2):
         for s_ in range(stages):
@@ -269,7 +272,9 @@ def conv1d_pair_kernel(T, NK, stages=3):
         for b_ in range(2):
             sim.bar(f"afull{b_}@{r}", 1)
     for s_ in range(stages):
-        sim.bar(f"full{s_}@0", 16)
+        sim.bar(f"full{s_}@0", 9 if relay else 16)
+        if relay:
+            sim.bar(f"lfull{s_}@1", 8)
     for b_ in range(2):
         sim.bar(f"aempty{b_}@0", 8)
     for r in range(2):
@@ -278,9 +283,10 @@ def conv1d_pair_kernel(T, NK, stages=3):
             st, k = seq % stages, seq // stages
             tma += [("wait", f"empty{st}@{r}", (k & 1) ^ 1, k, f"tma{r}"), ("owns", f"empty{st}@{r}", k, f"tma{r}"),
                     ("arrive", f"tma{st}@{r}", k, 1, f"tma{r}")]
+            target = f"lfull{st}@1" if (relay and r == 1) else f"full{st}@0"
             prod += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"producers{r}"),
                      ("owns", f"empty{st}@{r}", k, f"producers{r}"),
-                     ("arrive", f"full{st}@0", k, 8, f"producers{r}")]
+                     ("arrive", target, k, 8, f"producers{r}")]
         epi = []
         for t in range(T):
             buf, bk = t & 1, t >> 1
@@ -288,6 +294,12 @@ def conv1d_pair_kernel(T, NK, stages=3):
                     ("release", f"acc{buf}@{r}"),
                     ("arrive", f"aempty{buf}@0", bk, 4, f"epilogue{r}")]
         sim.agents += [tma, prod, epi]
+    if relay:
+        rel = []
+        for seq in range(T * NK):
+            st, k = seq % stages, seq // stages
+            rel += [("wait", f"lfull{st}@1", k & 1, k + 1, "relay"), ("arrive", f"full{st}@0", k, 1, "relay")]
+        sim.agents.append(rel)
     issue, complete = [], []
     n = 0
     for t in range(T):
@@ -310,6 +322,7 @@ def conv1d_pair_kernel(T, NK, stages=3):
 def test_conv1d_pair_kernel_protocol(T, NK):
     for seed in range(30):
         conv1d_pair_kernel(T, NK).run(seed)
+        conv1d_pair_kernel(T, NK, relay=False).run(seed)
 
 
 @pytest.mark.parametrize("stages", [2, 3])
