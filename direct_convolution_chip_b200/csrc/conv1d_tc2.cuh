@@ -389,6 +389,13 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             for (int tile = pair; ok && tile < p.total_tiles; tile += npairs) {
                 const TileCoord tcd = decode_pair_tile(p, tile);
                 const int x0 = tcd.t0 + (int)rank * TM - p.pad - R;  // a multiple of 4
+                // Pull the next tile's halo boxes into L2 now, so its TMA loads
+                // wait on L2 rather than on DRAM latency.
+                if (tile + npairs < p.total_tiles) {
+                    const TileCoord nx = decode_pair_tile(p, tile + npairs);
+                    for (int k = 0; k < nk; ++k)
+                        tcx::tma_prefetch_3d(&x_map, nx.t0 + (int)rank * TM - p.pad - R, k * KC, nx.n);
+                }
                 for (int k = 0; k < nk; ++k) {
                     if (!wait_bounded_cluster(bar_empty + 8 * stage, phase ^ 1, abort_flag)) {
                         ok = false;
@@ -440,46 +447,59 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TN);
             const bool vec = tw + 32 <= p.To && p.out_vec;
             const int kq = lane >> 2, jq = lane & 3;
-            // bias of output channels o0 + 32*i + lane, one load per lane per 32
-            // columns, fetched a step ahead and broadcast by shuffle
-            auto bias_at = [&](int i) {
-                const int o = tcd.o0 + 32 * i + lane;
-                return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f;
-            };
-            float bnext = bias_at(0), bcur = 0.f;
+            auto bias_of = [&](int o) { return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f; };
+            // Blocks of 16 columns, two at a time, so that their eight 4x4
+            // transposes (lane 4k+j ends with times tw+4k..tw+4k+3 of channels
+            // 4j..4j+3) overlap; the bias is added after the transpose, where a
+            // lane's four values belong to one output channel.
 #pragma unroll 1
-            for (int cb = 0; cb < TN / 16; ++cb) {
-                if ((cb & 1) == 0) {
-                    bcur = bnext;
-                    if (cb + 2 < TN / 16) bnext = bias_at((cb >> 1) + 1);
-                }
-                uint32_t r[16];
-                tmem_ld16(taddr + (uint32_t)(cb * 16), r);
-                tmem_wait_ld();
-                const int obase = tcd.o0 + cb * 16;
-                float v[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    v[j] = __uint_as_float(r[j]) + __shfl_sync(0xffffffffu, bcur, (cb & 1) * 16 + j);
+            for (int cb = 0; cb < TN / 16; cb += 2) {
+                uint32_t ra[16], rb[16];
+                tmem_ld16(taddr + (uint32_t)(cb * 16), ra);
+                tmem_ld16(taddr + (uint32_t)((cb + 1) * 16), rb);
+                tmem_wait_ld16(ra);
+                tmem_wait_ld16(rb);
                 if (vec) {
+                    float x[2][4][4];
+                    float bv[2][4];
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        float x0 = v[m], x1 = v[4 + m], x2 = v[8 + m], x3 = v[12 + m];
-                        quad_transpose(x0, x1, x2, x3, jq);
-                        const int o = obase + 4 * jq + m;
-                        if (o < p.O) {
-                            float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
-                            __stcs(reinterpret_cast<float4*>(dst), make_float4(x0, x1, x2, x3));  // streaming store
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            const uint32_t(&r)[16] = h ? rb : ra;
+                            x[h][m][0] = __uint_as_float(r[m]);
+                            x[h][m][1] = __uint_as_float(r[4 + m]);
+                            x[h][m][2] = __uint_as_float(r[8 + m]);
+                            x[h][m][3] = __uint_as_float(r[12 + m]);
+                            bv[h][m] = bias_of(tcd.o0 + (cb + h) * 16 + 4 * jq + m);
                         }
-                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) quad_transpose(x[h][m][0], x[h][m][1], x[h][m][2], x[h][m][3], jq);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            const int o = tcd.o0 + (cb + h) * 16 + 4 * jq + m;
+                            if (o < p.O) {
+                                float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
+                                const float b = bv[h][m];
+                                __stcs(reinterpret_cast<float4*>(dst),  // streaming store
+                                       make_float4(x[h][m][0] + b, x[h][m][1] + b, x[h][m][2] + b, x[h][m][3] + b));
+                            }
+                        }
                 } else {
                     const int t = tw + lane;
                     float* out_nt = p.out + (size_t)tcd.n * p.O * p.To + t;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int o = obase + j;
-                        if (t < p.To && o < p.O) out_nt[(size_t)o * p.To] = v[j];
-                    }
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int o = tcd.o0 + (cb + h) * 16 + j;
+                            if (t < p.To && o < p.O)
+                                out_nt[(size_t)o * p.To] = __uint_as_float((h ? rb : ra)[j]) + bias_of(o);
+                        }
                 }
             }
             tc_fence_before();
