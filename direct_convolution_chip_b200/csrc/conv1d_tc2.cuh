@@ -11,13 +11,18 @@
 // and three 64 KB stages fit where the single-SM kernel has two of 96 KB: the
 // extra stage hides the TMA latency that bounds the single-SM pipeline.
 //
-// Roles per CTA (448 threads): warps 0-7 produce (pw split of this CTA's half,
-// depthwise from the TMA-staged halo, A split); warp 8 allocates TMEM (both
-// CTAs) and, in the leader CTA only, one thread issues the MMAs for the pair;
-// warps 9-12 drain this CTA's accumulator rows; warp 13 loads, per chunk, this
-// CTA's half of the pw chunk and its input halo by TMA.  The leader's "full"
-// collects its own 8 producer warps and one forwarded arrival per chunk from
-// the other CTA, whose producers arrive locally and whose warp-8 lane 0 relays
+// Roles per CTA (512 threads): warps 0-7 produce (depthwise from the
+// TMA-staged halo, A split); warp 8 allocates TMEM (both CTAs) and, in the
+// leader CTA only, one thread issues the MMAs for the pair; warps 9-12 drain
+// this CTA's accumulator rows; warp 13 loads, per chunk, this CTA's half of
+// the pw chunk and its input halo by TMA; warps 14-15 form the pw lo part
+// beside the producers (taking that pass off the depthwise warps shortens
+// their per-chunk chain; sixteen depthwise warps of 8 times each, or two
+// groups of eight on alternate chunks, measured slower: the shared-memory
+// data path, which the MMAs' operand reads also use, sets the pace, not the
+// warps' latency).  The leader's "full" collects its own 10 producer and
+// split warps and one forwarded arrival per chunk from the other CTA, whose
+// warps arrive locally and whose warp-8 lane 0 relays
 // (a cluster-scope release per producer warp cost ~1,600 cycles on the
 // producers' path); the leader's "aempty" collects both CTAs' epilogues
 // (remote arrives).  MMA completion is committed to both CTAs' "empty"/"afull"
@@ -38,9 +43,13 @@ constexpr int TN = 256;          // output channels per pair tile (UMMA N)
 constexpr int TNH = TN / 2;      // pw rows held by each CTA
 constexpr int KC = 32;
 constexpr int STAGES = 3;
-constexpr int NPROD = 256;
-constexpr int MMA_WARP = 8, TMA_WARP = 13;
-constexpr int NTHREADS = 14 * 32;
+constexpr int NPW = 8;                  // depthwise producer warps
+constexpr int TPW = TM / NPW;                // times per producer warp
+constexpr int MMA_WARP = NPW, TMA_WARP = NPW + 5;
+constexpr int SPLIT_WARP = NPW + 6, NSPLIT = 2;  // warps that form B_lo
+constexpr int NTHREADS = (SPLIT_WARP + NSPLIT) * 32;
+constexpr int FULL_ARRIVALS = NPW + NSPLIT;  // per CTA and chunk: producer and split warps
+static_assert(TPW % 4 == 0 && TPW * NPW == TM, "16-byte window loads cover the CTA's times");
 constexpr int KMAXW = tc::KMAXW;
 constexpr int XW = 148;          // halo box width = smem row pitch (floats)
 constexpr uint32_t X_BYTES = (uint32_t)XW * KC * 4;
@@ -165,8 +174,8 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
 {
     using namespace tc;
     constexpr int KW = KT > 0 ? KT : KMAXW;            // taps the window must cover
-    constexpr int NV = (R + 15 + KW + 3) / 4;          // 16-byte window loads per thread
-    static_assert(16 * 7 + 4 * NV <= XW, "window inside the halo box");
+    constexpr int NV = (R + TPW - 1 + KW + 3) / 4;     // 16-byte window loads per thread
+    static_assert(TPW * (NPW - 1) + 4 * NV <= XW, "window inside the halo box");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
@@ -189,8 +198,8 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
-            mbar_init(bar_full + 8 * i, 9);    // the leader's 8 producer warps + the other CTA's relay
-            mbar_init(bar_lfull + 8 * i, 8);   // the other CTA's 8 producer warps (used in rank 1)
+            mbar_init(bar_full + 8 * i, FULL_ARRIVALS + 1);  // the leader's warps + the other CTA's relay
+            mbar_init(bar_lfull + 8 * i, FULL_ARRIVALS);     // the other CTA's warps (used in rank 1)
             mbar_init(bar_empty + 8 * i, 1);   // multicast commit
             mbar_init(bar_tma + 8 * i, 1);     // expect_tx arrival + TMA bytes
         }
@@ -221,7 +230,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp < 8) {
+    if (warp < NPW) {
         // ------------------------------------------------------------ producers
         const int ptid = threadIdx.x;
         const int K = KT > 0 ? KT : p.K;
@@ -232,7 +241,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             for (int kc = 0; kc < nk; ++kc) {
                 // The TMA copies of this stage (pw half and halo) have landed.
                 if (ptid == 0 && !wait_bounded(bar_tma + 8 * stage, phase, abort_flag)) *prod_abort = 1u;
-                asm volatile("bar.sync 1, 256;\n" ::: "memory");
+                asm volatile("bar.sync 1, %0;\n" ::"n"(NPW * 32) : "memory");
                 if (*prod_abort) {
                     run = false;
                     break;
@@ -241,20 +250,10 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                 }
                 const uint32_t a_hi = sbase + stage * STAGE_BYTES;
                 const uint32_t a_lo = a_hi + A_BYTES;
-                const uint32_t b_hi = a_lo + A_BYTES;
-                const uint32_t b_lo = b_hi + B_BYTES;
 
-                // This CTA's half of the pw chunk: B_hi stays raw (the MMA reads
-                // its TF32 bits); B_lo = v - truncate(v).
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t off = sw128_off(warp * 16 + i * 4 + (lane >> 3), lane & 7);
-                    sts128(b_lo + off, tcx::tf32_trunc_rest4(lds128(b_hi + off)));
-                }
-
-                // Depthwise: channel lane, this CTA's times 16*warp .. +15; halo
-                // sample j is x[t0 + 128*rank - pad - R + j].
-                const float* xrow = reinterpret_cast<const float*>(smem + stage * STAGE_BYTES) + lane * XW + 16 * warp;
+                // Depthwise: channel lane, this CTA's times TPW*warp .. +TPW-1;
+                // halo sample j is x[t0 + 128*rank - pad - R + j].
+                const float* xrow = reinterpret_cast<const float*>(smem + stage * STAGE_BYTES) + lane * XW + TPW * warp;
                 float win[4 * NV];
 #pragma unroll
                 for (int q = 0; q < NV; ++q) {
@@ -264,9 +263,9 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                     win[4 * q + 2] = v.z;
                     win[4 * q + 3] = v.w;
                 }
-                float2 d2[8];
+                float2 d2[TPW / 2];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) d2[j] = make_float2(0.f, 0.f);
+                for (int j = 0; j < TPW / 2; ++j) d2[j] = make_float2(0.f, 0.f);
                 const float* wcol = dws + KC * kc + lane;
 #pragma unroll
                 for (int k = 0; k < KW; ++k) {
@@ -274,18 +273,18 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                         const float w = wcol[k * CW];
                         const float2 w2 = make_float2(w, w);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
+                        for (int j = 0; j < TPW / 2; ++j)
                             d2[j] = __ffma2_rn(make_float2(win[R + 2 * j + k], win[R + 2 * j + k + 1]), w2, d2[j]);
                     }
                 }
                 // Every producer has read its halo window before the A operand overwrites it.
-                asm volatile("bar.sync 1, 256;\n" ::: "memory");
+                asm volatile("bar.sync 1, %0;\n" ::"n"(NPW * 32) : "memory");
                 const uint32_t col = ((uint32_t)(lane & 3) << 2);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < TPW; ++i) {
                     const float v = (i & 1) ? d2[i >> 1].y : d2[i >> 1].x;
                     const float hi = tf32_round(v);
-                    const uint32_t off = sw128_off(16 * warp + i, lane >> 2) + col;
+                    const uint32_t off = sw128_off(TPW * warp + i, lane >> 2) + col;
                     tcx::sts32(a_hi + off, hi);
                     tcx::sts32(a_lo + off, v - hi);
                 }
@@ -376,6 +375,53 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             }
         }
         __syncwarp();
+    } else if (warp >= SPLIT_WARP) {
+        // ------------------------------------------------------ pw split
+        // This CTA's half of each pw chunk, once its TMA copy has landed: B_hi
+        // stays raw (the MMA reads its TF32 bits), B_lo = v - truncate(v).
+        // Off the depthwise warps' path, so their chunk time is the
+        // depthwise alone.
+        const int sl = (warp - SPLIT_WARP) * 32 + lane;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = pair; ok && tile < p.total_tiles; tile += npairs) {
+            for (int k = 0; k < nk; ++k) {
+                int good = 1;
+                if (lane == 0) good = wait_bounded(bar_tma + 8 * stage, phase, abort_flag) ? 1 : 0;
+                good = __shfl_sync(0xffffffffu, good, 0);
+                if (!good) {
+                    ok = false;
+                    break;
+                }
+                for (int spin = 0; !mbar_try_wait(bar_tma + 8 * stage, phase) && spin < (1 << 20); ++spin) {
+                }
+                const uint32_t b_hi = sbase + stage * STAGE_BYTES + 2 * A_BYTES;
+                const uint32_t b_lo = b_hi + B_BYTES;
+                // 1024 16-byte slots (128 rows x 8), 16 per thread in two batches
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float4 v[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int slot = (8 * h + i) * 32 * NSPLIT + sl;
+                        v[i] = lds128(b_hi + sw128_off(slot >> 3, slot & 7));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int slot = (8 * h + i) * 32 * NSPLIT + sl;
+                        sts128(b_lo + sw128_off(slot >> 3, slot & 7), tcx::tf32_trunc_rest4(v[i]));
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(leader ? bar_full + 8 * stage : bar_lfull + 8 * stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
     } else if (warp == TMA_WARP) {
         // -------------------------------------------------------- TMA issuer
         // Per chunk: this CTA's half of the pw chunk into B_hi and its input

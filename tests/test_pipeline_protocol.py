@@ -252,7 +252,7 @@ def conv1d_tma_halo_kernel(T, NK, stages=2):
     return sim
 
 
-def conv1d_pair_kernel(T, NK, stages=3, relay=True):
+def conv1d_pair_kernel(T, NK, stages=3, relay=True, split=2, npw=8):
     """dwsep_conv1d_tc2_kernel: a cluster of two CTAs (rank 0 leads) shares
     every MMA (cta_group::2).  Each CTA's TMA warp fills its own stage once
     the MMAs that read it are done (its "empty", which the leader's
@@ -263,7 +263,8 @@ def conv1d_pair_kernel(T, NK, stages=3, relay=True):
     the leader's "full" themselves).  The leader's issuer waits for "full" per
     chunk and for the accumulator to be drained by both CTAs' epilogues (its
     "aempty", 8 arrivals) per tile; its multicast commits complete "empty"
-    and "afull" in both CTAs."""
+    and "afull" in both CTAs.  `split` more warps per CTA (one agent) form
+    the pw lo part of each chunk and arrive beside the producers."""
     sim = Sim()
     for r in range(2):
         for s_ in range(stages):
@@ -272,13 +273,13 @@ def conv1d_pair_kernel(T, NK, stages=3, relay=True):
         for b_ in range(2):
             sim.bar(f"afull{b_}@{r}", 1)
     for s_ in range(stages):
-        sim.bar(f"full{s_}@0", 9 if relay else 16)
+        sim.bar(f"full{s_}@0", npw + split + 1 if relay else 2 * (npw + split))
         if relay:
-            sim.bar(f"lfull{s_}@1", 8)
+            sim.bar(f"lfull{s_}@1", npw + split)
     for b_ in range(2):
         sim.bar(f"aempty{b_}@0", 8)
     for r in range(2):
-        tma, prod = [], []
+        tma, prod, spl = [], [], []
         for seq in range(T * NK):
             st, k = seq % stages, seq // stages
             tma += [("wait", f"empty{st}@{r}", (k & 1) ^ 1, k, f"tma{r}"), ("owns", f"empty{st}@{r}", k, f"tma{r}"),
@@ -286,14 +287,17 @@ def conv1d_pair_kernel(T, NK, stages=3, relay=True):
             target = f"lfull{st}@1" if (relay and r == 1) else f"full{st}@0"
             prod += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"producers{r}"),
                      ("owns", f"empty{st}@{r}", k, f"producers{r}"),
-                     ("arrive", target, k, 8, f"producers{r}")]
+                     ("arrive", target, k, npw, f"producers{r}")]
+            spl += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"split{r}"),
+                    ("owns", f"empty{st}@{r}", k, f"split{r}"),
+                    ("arrive", target, k, split, f"split{r}")]
         epi = []
         for t in range(T):
             buf, bk = t & 1, t >> 1
             epi += [("wait", f"afull{buf}@{r}", bk & 1, bk + 1, f"epilogue{r}"),
                     ("release", f"acc{buf}@{r}"),
                     ("arrive", f"aempty{buf}@0", bk, 4, f"epilogue{r}")]
-        sim.agents += [tma, prod, epi]
+        sim.agents += [tma, prod, epi] + ([spl] if split else [])
     if relay:
         rel = []
         for seq in range(T * NK):
@@ -323,6 +327,7 @@ def test_conv1d_pair_kernel_protocol(T, NK):
     for seed in range(30):
         conv1d_pair_kernel(T, NK).run(seed)
         conv1d_pair_kernel(T, NK, relay=False).run(seed)
+        conv1d_pair_kernel(T, NK, split=0).run(seed)
 
 
 @pytest.mark.parametrize("stages", [2, 3])
