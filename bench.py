@@ -636,9 +636,13 @@ def run_gpu(args):
             pw_macs_b = macs_conv1d_pointwise(CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K, CASE_B.stride,
                                               CASE_B.pad)
             achieved = 2 * pw_macs_b / tb_s / 1e12
-            roof = {"kernel": "dwsep_conv1d (tensor-core)", "bound": "tensor", "achieved": achieved,
+            if algo_b == fcv.CONV1D_TC2_3XTF32:
+                kname, tkey = "tc2::dwsep_conv1d_tc2_kernel<9, 0>", "dwsep_conv1d_tc2"
+            else:
+                kname, tkey = "tcx::dwsep_conv1d_tcx_kernel<9, 0, 1, 256>", "dwsep_conv1d"
+            roof = {"kernel": kname, "bound": "tensor", "achieved": achieved,
                     "peak": tc_rule, "unit": "TFLOP/s", "frac": achieved / tc_rule,
-                    "traffic": traffic_per_launch("dwsep_conv1d"), "peak_source": tc_src,
+                    "traffic": traffic_per_launch(tkey), "peak_source": tc_src,
                     "achieved_basis": "pointwise MACs (the depthwise MACs run on the FMA pipe)",
                     "peak_probe": tc_probe, "frac_probe": achieved / tc_probe if tc_probe else None}
         else:

@@ -575,6 +575,17 @@ inline bool conv1d_tc2_supported(int C, int T, int O, int K, int stride, const v
            (reinterpret_cast<uintptr_t>(pw) & 15) == 0 && cw * K <= tc2::DWX_MAX;
 }
 
+// Where AUTO takes the SM pair over the single-SM TMA-halo kernel: at least
+// eight 32-channel chunks per tile (C >= 256), so the pair's per-tile
+// start-up and drain are amortised, and O >= 256, so the 256-wide tile is
+// not half empty.  Measured on B200 over the stride-1 points of the conv1d
+// shape sweep: 1.05-1.20x faster there, 0.80-0.98x at C = 64, about even at
+// O = 128.
+inline bool conv1d_tc2_preferred(int C, int T, int O, int K, int stride, const void* x, const void* pw)
+{
+    return C >= 256 && O >= 256 && conv1d_tc2_supported(C, T, O, K, stride, x, pw);
+}
+
 inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float* pw, const float* bias, int N,
                                    int C, int T, int O, int K, int pad, int To, float* out, cudaStream_t stream)
 {

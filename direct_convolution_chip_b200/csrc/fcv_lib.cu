@@ -199,6 +199,8 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
     cudaStream_t s = fcv::as_stream(stream);
     switch (algo) {
     case FCV_ALGO_AUTO:
+        if (fcv::conv1d_tc2_preferred(C, T, O, K, stride, x, pw_w))
+            return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, s);
         if (fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w))
             return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
         if (fcv::conv1d_tc_supported(C, O, K, stride, pw_w)) {
@@ -305,7 +307,8 @@ int fcv_dwsep_conv1d_auto_algo(const float* x, const float* pw_w, int N, int C, 
     const int st = check_conv1d(N > 0 && !x ? dummy : x, dummy, N > 0 && !pw_w ? dummy : pw_w, nullptr, N, C, T, O,
                                 K, stride, pad, odummy, &To);
     if (st != FCV_OK) return st;
-    if (fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w)) *algo = FCV_CONV1D_TC_TMA_3XTF32;
+    if (fcv::conv1d_tc2_preferred(C, T, O, K, stride, x, pw_w)) *algo = FCV_CONV1D_TC2_3XTF32;
+    else if (fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w)) *algo = FCV_CONV1D_TC_TMA_3XTF32;
     else if (fcv::conv1d_tc_supported(C, O, K, stride, pw_w)) *algo = FCV_CONV1D_TC_3XTF32;
     else *algo = FCV_CONV1D_FMA;
     return FCV_OK;

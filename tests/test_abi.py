@@ -205,12 +205,20 @@ def test_auto_algo_conv2d(lib):
 
 
 def test_auto_algo_conv1d(lib):
-    """AUTO: TMA-halo tensor cores for aligned x/pw, T % 4 == 0 and stride 1 or
-    2, then the register-halo tensor-core kernel (stride 1), then FMA."""
+    """AUTO: the SM-pair kernel for C >= 256 and O >= 256 (stride 1, aligned
+    x/pw, T % 4 == 0), then TMA-halo tensor cores for aligned x/pw, T % 4 == 0
+    and stride 1 or 2, then the register-halo tensor-core kernel (stride 1),
+    then FMA."""
     a = ctypes.c_int()
     q = lib.fcv_dwsep_conv1d_auto_algo
     X, PW = P(0x10000), P(0x20000)
-    assert q(X, PW, 32, 256, 4096, 512, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 23  # full-size workload
+    assert q(X, PW, 32, 256, 4096, 512, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 22  # full-size workload
+    assert q(X, PW, 8, 384, 1000, 768, 3, 1, 1, ctypes.byref(a)) == OK and a.value == 22   # SM pair
+    assert q(X, PW, 8, 64, 1000, 768, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 23    # C < 256
+    assert q(X, PW, 8, 384, 1000, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 23   # O < 256
+    assert q(X, PW, 8, 384, 1000, 768, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 23   # stride 2
+    assert q(X, PW, 8, 384, 1001, 768, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21   # T % 4 != 0
+    assert q(P(0x10004), PW, 8, 384, 1000, 768, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21  # x misaligned
     assert q(X, PW, 2, 64, 1001, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21    # T % 4 != 0
     assert q(P(0x10004), PW, 2, 64, 1000, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21  # x not 16-B aligned
     assert q(X, PW, 2, 64, 1000, 128, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 23    # stride 2

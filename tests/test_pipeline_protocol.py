@@ -404,7 +404,7 @@ def test_model_catches_a_leader_that_ignores_the_peer_epilogue():
         sim = conv1d_pair_kernel(5, 3)
         for b in range(2):
             sim.bars[f"aempty{b}@0"].count = 4
-        peer_epilogue = sim.agents[5]
+        peer_epilogue = next(a for a in sim.agents if any(st[-1] == "epilogue1" for st in a))
         peer_epilogue[:] = [st for st in peer_epilogue if st[0] != "arrive"]
         try:
             sim.run(seed)
