@@ -4,6 +4,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+#include <vector>
+
 #include "../../include/fcv.h"
 
 namespace fcv {
@@ -69,6 +73,103 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 inline int launch_status()
 {
     return cudaGetLastError() == cudaSuccess ? FCV_OK : FCV_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launch state kept between calls.  A call on a small problem
+// should cost little more than its launch, so the SM count is looked up once
+// per device and each kernel's dynamic shared-memory limit is raised once per
+// device; a context reset (cudaDeviceReset) drops that limit, which shows as a
+// failed launch, after which launch_cached sets it again and launches once
+// more.
+
+constexpr int kMaxCachedDevices = 64;
+
+// Number of SMs of the current device.
+inline int device_sm_count(int* sms)
+{
+    static std::atomic<int> cache[kMaxCachedDevices];  // static storage: zero until looked up
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
+    const bool cached = dev >= 0 && dev < kMaxCachedDevices;
+    if (cached) {
+        const int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) {
+            *sms = v;
+            return FCV_OK;
+        }
+    }
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return FCV_ERR_CUDA;
+    if (cached) cache[dev].store(v, std::memory_order_relaxed);
+    *sms = v;
+    return FCV_OK;
+}
+
+struct SmemLimit {
+    const void* fn;
+    int dev;
+    int bytes;
+};
+
+inline std::mutex& smem_limit_mu()
+{
+    static std::mutex m;
+    return m;
+}
+
+inline std::vector<SmemLimit>& smem_limits()
+{
+    static std::vector<SmemLimit> v;
+    return v;
+}
+
+// Raise `fn`'s dynamic shared-memory limit to `bytes` on the current device
+// unless an earlier call already did.
+inline int ensure_smem_limit(const void* fn, int bytes)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(smem_limit_mu());
+    for (const SmemLimit& e : smem_limits())
+        if (e.fn == fn && e.dev == dev && e.bytes >= bytes) return FCV_OK;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return FCV_ERR_CUDA;
+    for (SmemLimit& e : smem_limits())
+        if (e.fn == fn && e.dev == dev) {
+            e.bytes = bytes;
+            return FCV_OK;
+        }
+    smem_limits().push_back({fn, dev, bytes});
+    return FCV_OK;
+}
+
+inline void forget_smem_limit(const void* fn)
+{
+    std::lock_guard<std::mutex> lock(smem_limit_mu());
+    auto& v = smem_limits();
+    for (size_t i = 0; i < v.size();)
+        if (v[i].fn == fn) {
+            v[i] = v.back();
+            v.pop_back();
+        } else {
+            ++i;
+        }
+}
+
+// Launch through `go` (a callable that issues the <<<...>>> launch) with the
+// kernel's shared-memory limit raised; after a failed launch the limit is set
+// again and the launch repeated once.
+template <typename Kern, typename Go>
+inline int launch_cached(Kern kern, int smem_bytes, Go&& go)
+{
+    const void* fn = reinterpret_cast<const void*>(kern);
+    if (ensure_smem_limit(fn, smem_bytes) != FCV_OK) return FCV_ERR_CUDA;
+    go();
+    if (cudaGetLastError() == cudaSuccess) return FCV_OK;
+    forget_smem_limit(fn);
+    if (ensure_smem_limit(fn, smem_bytes) != FCV_OK) return FCV_ERR_CUDA;
+    go();
+    return launch_status();
 }
 
 }  // namespace fcv

@@ -180,11 +180,10 @@ inline int launch_dwsep_conv1d_fma(const float* x, const float* dw, const float*
     if (nblk > 0x7fffffffLL) return FCV_ERR_UNSUPPORTED;
     const size_t smem = conv1d_fma_smem(K, s).bytes;
     auto kern = (s == 1) ? dwsep_conv1d_fma_kernel<1> : dwsep_conv1d_fma_kernel<0>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return FCV_ERR_CUDA;
-    kern<<<(unsigned)nblk, G::NT, smem, stream>>>(x, dw, pw, bias, C, T, O, K, s, pad, To, tiles_t,
-                                                  tiles_o, out);
-    return launch_status();
+    return launch_cached(kern, (int)smem, [&] {
+        kern<<<(unsigned)nblk, G::NT, smem, stream>>>(x, dw, pw, bias, C, T, O, K, s, pad, To, tiles_t, tiles_o,
+                                                      out);
+    });
 }
 
 }  // namespace fcv

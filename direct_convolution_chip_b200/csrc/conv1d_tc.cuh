@@ -776,16 +776,13 @@ inline int launch_dwsep_conv1d_tc(const float* x, const float* dw, const float* 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return FCV_ERR_CUDA;
 
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
+    int sms = 0;
+    if (device_sm_count(&sms) != FCV_OK) return FCV_ERR_CUDA;
     auto kern = K == 9 ? tc::dwsep_conv1d_tc_kernel<9>
               : K == 3 ? tc::dwsep_conv1d_tc_kernel<3> : tc::dwsep_conv1d_tc_kernel<0>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM_BYTES) != cudaSuccess)
-        return FCV_ERR_CUDA;
     const int grid = (int)(total < sms ? total : sms);
-    kern<<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(prm, map);
-    return launch_status();
+    return launch_cached(kern, (int)tc::SMEM_BYTES,
+                         [&] { kern<<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(prm, map); });
 }
 
 }  // namespace fcv

@@ -623,9 +623,8 @@ inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float*
             return FCV_ERR_CUDA;
     }
 
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
+    int sms = 0;
+    if (device_sm_count(&sms) != FCV_OK) return FCV_ERR_CUDA;
     const int r = (-pad) & 3;  // (t0 - pad) mod 4 with t0 a multiple of 128
     decltype(&tc2::dwsep_conv1d_tc2_kernel<0, 0>) kern;
     if (K == 9 && r == 0) kern = tc2::dwsep_conv1d_tc2_kernel<9, 0>;
@@ -634,12 +633,10 @@ inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float*
     else if (r == 1) kern = tc2::dwsep_conv1d_tc2_kernel<0, 1>;
     else if (r == 2) kern = tc2::dwsep_conv1d_tc2_kernel<0, 2>;
     else kern = tc2::dwsep_conv1d_tc2_kernel<0, 3>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc2::SMEM_BYTES) != cudaSuccess)
-        return FCV_ERR_CUDA;
     const long long pairs = total < sms / 2 ? total : sms / 2;
     dim3 grid((unsigned)(2 * pairs));
-    kern<<<grid, tc2::NTHREADS, tc2::SMEM_BYTES, stream>>>(prm, pw_map, x_map);
-    return launch_status();
+    return launch_cached(kern, (int)tc2::SMEM_BYTES,
+                         [&] { kern<<<grid, tc2::NTHREADS, tc2::SMEM_BYTES, stream>>>(prm, pw_map, x_map); });
 }
 
 }  // namespace fcv

@@ -509,17 +509,13 @@ inline int launch_dwsep_conv1d_tcx(const float* x, const float* dw, const float*
             return FCV_ERR_CUDA;
     }
 
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
+    int sms = 0;
+    if (device_sm_count(&sms) != FCV_OK) return FCV_ERR_CUDA;
     const int r = (-pad) & 3;  // (t0*stride - pad) mod 4 with t0 a multiple of 128
     const tcx::KernelPtr kern = tn == 256 ? tcx::select_kernel<256>(K, r, stride) : tcx::select_kernel<128>(K, r, stride);
     const int smem = (int)(tn == 256 ? tcx::Geo<256>::SMEM_BYTES : tcx::Geo<128>::SMEM_BYTES);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return FCV_ERR_CUDA;
     const int grid = (int)(total < sms ? total : sms);
-    kern<<<grid, tc::NTHREADS, smem, stream>>>(prm, pw_map, x_map);
-    return launch_status();
+    return launch_cached(kern, smem, [&] { kern<<<grid, tc::NTHREADS, smem, stream>>>(prm, pw_map, x_map); });
 }
 
 }  // namespace fcv

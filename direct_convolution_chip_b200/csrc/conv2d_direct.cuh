@@ -352,15 +352,14 @@ int launch_conv2d_direct_pn(const float* x, const float* w, const float* b, int 
     const long long nblk = (long long)N * tiles_y * tiles_x;
     if (nblk > 0x7fffffffLL || cblk > 65535) return FCV_ERR_UNSUPPORTED;
     auto kern = conv2d_direct_kernel<P, MODE, NARROW>;
-    if (G::SMEM_BYTES > 48 * 1024) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)G::SMEM_BYTES) != cudaSuccess)
-            return FCV_ERR_CUDA;
-    }
     dim3 grid((unsigned)nblk, (unsigned)cblk);
     const int vec16 = ((W & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 && (P * G::TILE_PW) % 4 == 0) ? 1 : 0;
-    kern<<<grid, G::NT, G::SMEM_BYTES, stream>>>(x, w, b, Cin, H, W, Cout, PH, PW, tiles_y, tiles_x, out,
-                                                  partials, counters, vec16);
+    auto go = [&] {
+        kern<<<grid, G::NT, G::SMEM_BYTES, stream>>>(x, w, b, Cin, H, W, Cout, PH, PW, tiles_y, tiles_x, out,
+                                                      partials, counters, vec16);
+    };
+    if (G::SMEM_BYTES > 48 * 1024) return launch_cached(kern, (int)G::SMEM_BYTES, go);
+    go();
     return launch_status();
 }
 

@@ -295,12 +295,11 @@ int launch_conv2d_poolfirst_p(const float* x, const float* w, const float* b, in
     if (nblk > 0x7fffffffLL || cblk > 65535) return FCV_ERR_UNSUPPORTED;
     const bool vec = (W & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0;
     auto kern = vec ? conv2d_poolfirst_kernel<P, MODE, true> : conv2d_poolfirst_kernel<P, MODE, false>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::SMEM_BYTES) != cudaSuccess)
-        return FCV_ERR_CUDA;
     dim3 grid((unsigned)nblk, (unsigned)cblk);
-    kern<<<grid, G::NT, G::SMEM_BYTES, stream>>>(x, w, b, Cin, H, W, Cout, PH, PW, tiles_y, tiles_x, out,
-                                                  partials, counters);
-    return launch_status();
+    return launch_cached(kern, (int)G::SMEM_BYTES, [&] {
+        kern<<<grid, G::NT, G::SMEM_BYTES, stream>>>(x, w, b, Cin, H, W, Cout, PH, PW, tiles_y, tiles_x, out,
+                                                      partials, counters);
+    });
 }
 
 // Tiles per image and channel blocks of the pool-first kernel.

@@ -991,10 +991,7 @@ inline int launch_conv2d_tc_p(c2tc::Params prm, int N, int grid, cudaStream_t st
     const Conv2dTcPlan pl = conv2d_tc_plan<P>(prm.Cin, prm.Cout, prm.use_tma != 0);
     prm.nacc = pl.nacc;
     auto kern = pl.sub ? c2tc::conv2d_tc4_kernel<P, MODE> : c2tc::conv2d_tc_kernel<P, MODE>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) != cudaSuccess)
-        return FCV_ERR_CUDA;
-    kern<<<grid, c2tc::NTHREADS, pl.smem, stream>>>(prm, map);
-    return launch_status();
+    return launch_cached(kern, (int)pl.smem, [&] { kern<<<grid, c2tc::NTHREADS, pl.smem, stream>>>(prm, map); });
 }
 
 // MODE: kSumAtomic (out[N], zeroed by the caller) or kTap (pooled values).
@@ -1018,9 +1015,8 @@ inline int launch_conv2d_tc(const float* x, const float* w, const float* b, int 
     prm.total_tiles = (int)total;
     prm.use_tma = 0;
     prm.nacc = 2;  // set with the kernel choice in launch_conv2d_tc_p
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
+    int sms = 0;
+    if (device_sm_count(&sms) != FCV_OK) return FCV_ERR_CUDA;
     const int grid = (int)(total < sms ? total : sms);
     switch (P) {
     case 1: return launch_conv2d_tc_p<1, MODE>(prm, N, grid, stream);

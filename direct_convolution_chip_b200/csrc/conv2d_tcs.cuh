@@ -778,10 +778,7 @@ inline int launch_conv2d_tcs_inst(const c2s::Params& prm, int grid, const CUtens
     constexpr uint32_t smem = c2s::smem_bytes<P, CCH>();
     static_assert(smem <= (uint32_t)c2s::SMEM_LIMIT, "shared memory budget");
     auto kern = c2s::conv2d_tcs_kernel<P, CCH, MODE>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return FCV_ERR_CUDA;
-    kern<<<grid, c2s::NTHREADS, smem, stream>>>(prm, map);
-    return launch_status();
+    return launch_cached(kern, (int)smem, [&] { kern<<<grid, c2s::NTHREADS, smem, stream>>>(prm, map); });
 }
 
 template <int P, int MODE>
@@ -844,9 +841,8 @@ inline int launch_conv2d_tcs(const float* x, const float* w, const float* b, int
             return FCV_ERR_CUDA;
         prm.use_tma = 1;
     }
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FCV_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FCV_ERR_CUDA;
+    int sms = 0;
+    if (device_sm_count(&sms) != FCV_OK) return FCV_ERR_CUDA;
     const int grid = (int)(prm.U < sms ? prm.U : sms);
     for (int co0 = 0; co0 < Cout; co0 += c2s::CO_BLK) {
         prm.co0 = co0;
