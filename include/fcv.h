@@ -38,7 +38,10 @@
  *     returns early.
  *   - N == 0 (an empty batch) is valid and enqueues nothing.
  *   - The library holds no per-call state; concurrent calls on different
- *     streams with disjoint outputs are safe.  The one exception is
+ *     streams with disjoint outputs are safe.  Between calls it keeps, per
+ *     device, the SM count and each kernel's raised shared-memory limit
+ *     (looked up or set once, under a lock; set again after a failed launch,
+ *     as after cudaDeviceReset).  The one exception is
  *     fcv_conv2d_pool_sigmoid_sum_noalloc: all its calls on a device share one
  *     library-owned 256 KiB array, so calls that overlap on the GPU race and
  *     must be serialised by the caller.
