@@ -230,6 +230,10 @@ EDGE_1D = [
     (1, 40, 300, 20, 4, 2, 0, True),    # even K, no padding
     (1, 16, 256, 40, 3, 2, 7, True),    # pad larger than K, r = 1
     (1, 8, 4, 8, 3, 2, 1, True),        # T = 4: To = 2
+    # where AUTO takes the SM-pair kernel (stride 1, C >= 256, O >= 256): ragged in every dimension
+    (2, 260, 1000, 300, 9, 1, 4, True), # 9 channel chunks (the last 4 wide), last pair tile 232 times, O tile 44 wide
+    (1, 256, 516, 256, 3, 1, 1, False), # K = 3, r = 3, no bias, last pair tile 4 times
+    (3, 288, 4, 512, 9, 1, 4, True),    # T = 4: one 4-time tile per item, fewer tiles than SM pairs
 ]
 
 
