@@ -64,6 +64,8 @@ SIGNATURES = {
     "fcv_selftest_conv2d_stall": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _I, ctypes.c_ulonglong, _P]),
     "fcv_selftest_conv1d_stall": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _I, ctypes.c_ulonglong,
                                        _P]),
+    "fcv_selftest_conv1d_pair_stall": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I,
+                                            ctypes.c_ulonglong, _P]),
 }
 
 

@@ -26,9 +26,10 @@
 // (a cluster-scope release per producer warp cost ~1,600 cycles on the
 // producers' path); the leader's "aempty" collects both CTAs' epilogues
 // (remote arrives).  MMA completion is committed to both CTAs' "empty"/"afull"
-// barriers with a multicast commit.  Every mbarrier wait is bounded; a cluster barrier
-// follows initialisation and precedes exit, so no CTA leaves while its peer
-// may still signal it.  No TMA multicast.
+// barriers with a multicast commit.  Every mbarrier wait is bounded and also
+// watches the peer CTA's abort flag, so the pair gives up together; a cluster
+// barrier follows initialisation and precedes exit, so no CTA leaves while
+// its peer may still signal it.  No TMA multicast.
 #pragma once
 
 #include "conv1d_tcx.cuh"
@@ -61,7 +62,7 @@ constexpr uint32_t B_BYTES = TNH * KC * 4;   // 16 KB
 constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
 constexpr uint32_t OFF_DWS = STAGES * STAGE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_DWS + DWX_MAX * 4;
-constexpr uint32_t NBAR = 17;    // full[3] empty[3] afull[2] aempty[2] drain tma[3] lfull[3]
+constexpr uint32_t NBAR = 18;    // full[3] empty[3] afull[2] aempty[2] drain tma[3] lfull[3] gate
 constexpr uint32_t OFF_MISC = OFF_BAR + 24 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -108,17 +109,40 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     return ok != 0;
 }
 
-// Bounded wait with cluster-scope acquire (barriers that the peer CTA signals).
-__device__ __forceinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag)
+// Abort state of the pair: this CTA's flag and the peer CTA's (its
+// shared::cluster address).  A wait gives up when either is set, so when one
+// role of one CTA gives up the whole pair leaves its loops within microseconds
+// instead of each wait running out on its own.
+struct PairAbort {
+    volatile uint32_t* local;
+    uint32_t peer;
+};
+
+__device__ __forceinline__ bool pair_aborted(const PairAbort& a)
 {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*a.local) return true;
+    uint32_t v;
+    asm volatile("ld.relaxed.cluster.shared::cluster.u32 %0, [%1];\n" : "=r"(v) : "r"(a.peer) : "memory");
+    if (v) *a.local = 1u;
+    return v != 0;
+}
+
+// Bounded wait on a barrier of this CTA, with cluster-scope acquire (CLUSTER:
+// barriers the peer CTA signals) or CTA-scope acquire.  After `limit_ns` it
+// sets this CTA's abort flag and the device error word and returns false.
+template <bool CLUSTER>
+__device__ __forceinline__ bool pair_wait(uint32_t bar, uint32_t parity, const PairAbort& a,
+                                          unsigned long long limit_ns = tc::kWaitLimitNs)
+{
+    auto test = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : tc::mbar_try_wait(bar, parity); };
+    if (test()) return true;
     const unsigned long long t0 = tc::globaltimer();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (test()) return true;
         if ((i & 255u) == 0) {
-            if (*abort_flag) return false;
-            if (tc::globaltimer() - t0 > tc::kWaitLimitNs) {
-                *abort_flag = 1u;
+            if (pair_aborted(a)) return false;
+            if (tc::globaltimer() - t0 > limit_ns) {
+                *a.local = 1u;
                 record_device_error(kErrTimeout);
                 return false;
             }
@@ -153,7 +177,23 @@ struct Params {
     int C, T, O, K, pad, To;
     int tiles_t, tiles_o, total_tiles;  // pair tiles (256 times each)
     int out_vec;                         // output rows 16-byte aligned
+    // Failure-path test (all 0 in normal calls): role stall_role (1 TMA warp,
+    // 2 producers, 3 MMA issuer, 4 epilogue, 5 pw split, 6 relay) of the CTA
+    // of rank stall_rank in every pair waits, before its stall_at-th tile, on a
+    // barrier nothing completes, with limit stall_ns.
+    int stall_role = 0, stall_at = 0, stall_rank = 0;
+    unsigned long long stall_ns = 0;
 };
+
+// The failure-path test hook: true unless this role is to stall before its
+// `local`-th tile in this CTA and its wait on `gate` ran out (which sets the
+// abort flag and the device error word).
+__device__ __forceinline__ bool stall_ok(const Params& p, int role, int local, uint32_t rank, uint32_t gate,
+                                         const PairAbort& ab)
+{
+    if (p.stall_role != role || local != p.stall_at || (int)rank != p.stall_rank) return true;
+    return pair_wait<false>(gate, 0, ab, p.stall_ns);
+}
 
 __device__ __forceinline__ TileCoord decode_pair_tile(const Params& p, int tile)
 {
@@ -187,6 +227,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     const uint32_t bar_drain = bar_full + 80;
     const uint32_t bar_tma = bar_full + 88;      // + 8 * stage
     const uint32_t bar_lfull = bar_full + 112;   // + 8 * stage (rank 1: its producers, forwarded by the relay)
+    const uint32_t bar_gate = bar_full + 136;    // never completed: the failure-path test's stall
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
     volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 8);
@@ -208,6 +249,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             mbar_init(bar_aempty + 8 * i, 8);  // 4 epilogue warps x 2 CTAs (used in the leader)
         }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_gate, 1);
         *abort_flag = 0u;
         *prod_abort = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -229,6 +271,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     cluster_sync();  // barriers of both CTAs initialised, TMEM allocated, weights staged
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    const PairAbort ab{abort_flag, mapa(smem_u32(const_cast<uint32_t*>(abort_flag)), rank ^ 1u)};
 
     if (warp < NPW) {
         // ------------------------------------------------------------ producers
@@ -237,10 +280,13 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         int stage = 0;
         uint32_t phase = 0;
         bool run = true;
-        for (int tile = pair; run && tile < p.total_tiles; tile += npairs) {
+        int local = 0;
+        for (int tile = pair; run && tile < p.total_tiles; tile += npairs, ++local) {
             for (int kc = 0; kc < nk; ++kc) {
                 // The TMA copies of this stage (pw half and halo) have landed.
-                if (ptid == 0 && !wait_bounded(bar_tma + 8 * stage, phase, abort_flag)) *prod_abort = 1u;
+                if (ptid == 0 && ((kc == 0 && !stall_ok(p, 2, local, rank, bar_gate, ab)) ||
+                                  !pair_wait<false>(bar_tma + 8 * stage, phase, ab)))
+                    *prod_abort = 1u;
                 asm volatile("bar.sync 1, %0;\n" ::"n"(NPW * 32) : "memory");
                 if (*prod_abort) {
                     run = false;
@@ -308,11 +354,12 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             bool ok = true;
             for (int tile = pair; ok && tile < p.total_tiles; tile += npairs, ++local) {
                 const int buf = local & 1;
-                if (!wait_bounded_cluster(bar_aempty + 8 * buf, ((local >> 1) & 1) ^ 1, abort_flag)) break;
+                if (!stall_ok(p, 3, local, rank, bar_gate, ab)) break;
+                if (!pair_wait<true>(bar_aempty + 8 * buf, ((local >> 1) & 1) ^ 1, ab)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
                 for (int k = 0; k < nk; ++k) {
-                    if (!wait_bounded_cluster(bar_full + 8 * stage, phase, abort_flag)) {
+                    if (!pair_wait<true>(bar_full + 8 * stage, phase, ab)) {
                         ok = false;
                         break;
                     }
@@ -350,9 +397,11 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = pair; ok && tile < p.total_tiles; tile += npairs) {
+            int local = 0;
+            for (int tile = pair; ok && tile < p.total_tiles; tile += npairs, ++local) {
                 for (int k = 0; k < nk; ++k) {
-                    if (!wait_bounded(bar_lfull + 8 * stage, phase, abort_flag)) {
+                    if ((k == 0 && !stall_ok(p, 6, local, rank, bar_gate, ab)) ||
+                        !pair_wait<false>(bar_lfull + 8 * stage, phase, ab)) {
                         ok = false;
                         break;
                     }
@@ -385,10 +434,13 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int tile = pair; ok && tile < p.total_tiles; tile += npairs) {
+        int local = 0;
+        for (int tile = pair; ok && tile < p.total_tiles; tile += npairs, ++local) {
             for (int k = 0; k < nk; ++k) {
                 int good = 1;
-                if (lane == 0) good = wait_bounded(bar_tma + 8 * stage, phase, abort_flag) ? 1 : 0;
+                if (lane == 0)
+                    good = ((k != 0 || stall_ok(p, 5, local, rank, bar_gate, ab)) &&
+                            pair_wait<false>(bar_tma + 8 * stage, phase, ab)) ? 1 : 0;
                 good = __shfl_sync(0xffffffffu, good, 0);
                 if (!good) {
                     ok = false;
@@ -432,7 +484,9 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             uint32_t phase = 0;
             bool pending[STAGES] = {false, false, false};
             bool ok = true;
-            for (int tile = pair; ok && tile < p.total_tiles; tile += npairs) {
+            int local = 0;
+            for (int tile = pair; ok && tile < p.total_tiles; tile += npairs, ++local) {
+                if (!stall_ok(p, 1, local, rank, bar_gate, ab)) break;
                 const TileCoord tcd = decode_pair_tile(p, tile);
                 const int x0 = tcd.t0 + (int)rank * TM - p.pad - R;  // a multiple of 4
                 // Pull the next tile's halo boxes into L2 now, so its TMA loads
@@ -443,7 +497,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                         tcx::tma_prefetch_3d(&x_map, nx.t0 + (int)rank * TM - p.pad - R, k * KC, nx.n);
                 }
                 for (int k = 0; k < nk; ++k) {
-                    if (!wait_bounded_cluster(bar_empty + 8 * stage, phase ^ 1, abort_flag)) {
+                    if (!pair_wait<true>(bar_empty + 8 * stage, phase ^ 1, ab)) {
                         ok = false;
                         break;
                     }
@@ -484,7 +538,9 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         for (int tile = pair; tile < p.total_tiles; tile += npairs, ++local) {
             const int buf = local & 1;
             int ok = 1;
-            if (lane == 0) ok = wait_bounded_cluster(bar_afull + 8 * buf, (local >> 1) & 1, abort_flag) ? 1 : 0;
+            if (lane == 0)
+                ok = (stall_ok(p, 4, local, rank, bar_gate, ab) &&
+                      pair_wait<true>(bar_afull + 8 * buf, (local >> 1) & 1, ab)) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
@@ -587,9 +643,15 @@ inline bool conv1d_tc2_preferred(int C, int T, int O, int K, int stride, const v
 }
 
 inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float* pw, const float* bias, int N,
-                                   int C, int T, int O, int K, int pad, int To, float* out, cudaStream_t stream)
+                                   int C, int T, int O, int K, int pad, int To, float* out, cudaStream_t stream,
+                                   int stall_role = 0, int stall_at = 0, int stall_rank = 0,
+                                   unsigned long long stall_ns = 0)
 {
     tc2::Params prm;
+    prm.stall_role = stall_role;
+    prm.stall_at = stall_at;
+    prm.stall_rank = stall_rank;
+    prm.stall_ns = stall_ns;
     prm.x = x; prm.dw = dw; prm.pw = pw; prm.bias = bias; prm.out = out;
     prm.C = C; prm.T = T; prm.O = O; prm.K = K; prm.pad = pad; prm.To = To;
     prm.tiles_t = (To + 2 * tc2::TM - 1) / (2 * tc2::TM);

@@ -269,6 +269,22 @@ int fcv_selftest_conv1d_stall(const float* x, const float* dw_w, const float* pw
                                         fcv::as_stream(stream), role, at_tile, limit_ns);
 }
 
+int fcv_selftest_conv1d_pair_stall(const float* x, const float* dw_w, const float* pw_w, const float* bias, int N,
+                                   int C, int T, int O, int K, int stride, int pad, float* out, int role,
+                                   int at_tile, int rank, unsigned long long limit_ns, void* stream)
+{
+    int To = 0;
+    int st = check_conv1d(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, out, &To);
+    if (st != FCV_OK) return st;
+    if (role < 1 || role > 6 || rank < 0 || rank > 1 || (role == 3 && rank != 0) || (role == 6 && rank != 1) ||
+        at_tile < 0 || limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000)
+        return FCV_ERR_INVALID_ARG;
+    if (!fcv::conv1d_tc2_supported(C, T, O, K, stride, x, pw_w)) return FCV_ERR_UNSUPPORTED;
+    if (N == 0) return FCV_OK;
+    return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, fcv::as_stream(stream),
+                                        role, at_tile, rank, limit_ns);
+}
+
 int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* algo)
 {
     if (!algo) return FCV_ERR_INVALID_ARG;

@@ -289,6 +289,21 @@ int fcv_selftest_conv1d_stall(const float* x, const float* dw_w, const float* pw
                               float* out, int role, int at_tile, unsigned long long limit_ns,
                               void* stream);
 
+/* The same test for op B's SM-pair kernel (FCV_CONV1D_TC2_3XTF32): in the CTA
+ * of rank `rank` (0 leads the pair, 1 is its peer) of every pair, role `role`
+ * (1 TMA warp, 2 depthwise producers, 3 MMA issuer -- rank 0 only, 4 epilogue,
+ * 5 pw split warps, 6 relay -- rank 1 only) waits, before its `at_tile`-th
+ * pair tile, on a barrier nothing completes, with limit `limit_ns` (1 ns ..
+ * 10 s).  That CTA takes its abort path, its peer sees the abort flag through
+ * distributed shared memory and leaves as well, and FCV_ERR_TIMEOUT is
+ * recorded; `out` holds partial results.  INVALID_ARG for a role, rank or
+ * limit outside those ranges; UNSUPPORTED outside that kernel's envelope;
+ * otherwise as fcv_dwsep_conv1d. */
+int fcv_selftest_conv1d_pair_stall(const float* x, const float* dw_w, const float* pw_w, const float* bias,
+                                   int N, int C, int T, int O, int K, int stride, int pad,
+                                   float* out, int role, int at_tile, int rank, unsigned long long limit_ns,
+                                   void* stream);
+
 #ifdef __cplusplus
 }
 #endif

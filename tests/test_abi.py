@@ -102,7 +102,28 @@ def test_stall_selftests_validate_on_the_host(lib, fn, kw, want):
     assert fn(lib, **kw) == {"inv": INVALID, "ok": OK}[want]
 
 
+def stall1d_pair(lib, role=1, at=0, rank=0, limit=1000, **kw):
+    a = dict(x=FAKE, dw=FAKE, pw=FAKE, bias=FAKE, N=2, C=256, T=64, O=256, K=9, s=1, p=4, out=FAKE)
+    a.update(kw)
+    return lib.fcv_selftest_conv1d_pair_stall(a["x"], a["dw"], a["pw"], a["bias"], a["N"], a["C"], a["T"], a["O"],
+                                              a["K"], a["s"], a["p"], a["out"], role, at, rank, limit, None)
+
+
+@pytest.mark.parametrize("kw,want", [(dict(role=0), "inv"), (dict(role=7), "inv"), (dict(rank=2), "inv"),
+                                     (dict(rank=-1), "inv"), (dict(role=3, rank=1), "inv"),
+                                     (dict(role=6, rank=0), "inv"), (dict(at=-1), "inv"), (dict(limit=0), "inv"),
+                                     (dict(limit=11 * 10**9), "inv"), (dict(N=0), "ok"),
+                                     (dict(role=6, rank=1, N=0), "ok"), (dict(role=5, rank=1, N=0), "ok")])
+def test_pair_stall_selftest_validates_on_the_host(lib, kw, want):
+    """The SM-pair failure-path entry point rejects bad roles, ranks (the
+    MMA issuer lives in rank 0, the relay in rank 1), tiles and limits before
+    any CUDA call."""
+    assert stall1d_pair(lib, **kw) == {"inv": INVALID, "ok": OK}[want]
+
+
 def test_stall_selftests_outside_their_kernels(lib):
+    assert stall1d_pair(lib, s=2) == UNSUPPORTED
+    assert stall1d_pair(lib, T=66) == UNSUPPORTED
     assert stall2d(lib, Cin=20) == UNSUPPORTED
     assert stall1d(lib, s=3) == UNSUPPORTED
 

@@ -1,7 +1,7 @@
 """The failure path of the production tensor-core kernels, on the GPU, without
 a fault: one role of every thread block waits on a barrier that nothing
 completes, with a short limit (fcv_selftest_conv2d_stall /
-fcv_selftest_conv1d_stall).  The wait must give up and record FCV_ERR_TIMEOUT;
+fcv_selftest_conv1d_stall / fcv_selftest_conv1d_pair_stall).  The wait must give up and record FCV_ERR_TIMEOUT;
 every other role must then leave its loop, the TMA copies and MMAs already in
 flight must be waited for and tensor memory freed, so the context stays usable:
 the next normal call on the same inputs matches the CPU oracle.
@@ -85,6 +85,36 @@ def test_conv1d_stall_every_role(lib, stride):
             assert st == 0, f"role {role} at {at}: launch status {st}"
             assert lib.fcv_device_error(sp) == TIMEOUT, f"role {role} at {at}: no timeout recorded"
     got = binding.dwsep_conv1d(x, dw, pw, bias, case.stride, case.pad, algo=binding.CONV1D_TC_TMA_3XTF32)
+    torch.cuda.synchronize()
+    assert lib.fcv_device_error(sp) == 0
+    xn, dwn, pwn, bn = [t.cpu().numpy() for t in (x, dw, pw, bias)]
+    for bi in (0, case.N - 1):
+        want = oracle.dwsep_conv1d(xn[bi:bi + 1], dwn, pwn, bn, case.stride, case.pad)
+        assert_close(got[bi:bi + 1], want, f"out[{bi}]")
+
+
+def test_conv1d_pair_stall_every_role(lib):
+    """The SM-pair kernel: one role of one CTA of every pair stalls; that CTA
+    gives up, its peer sees the abort flag through distributed shared memory,
+    both drain what is in flight and free tensor memory, and the next normal
+    call matches the oracle.  Roles: 1 TMA warp, 2 producers, 3 MMA issuer
+    (rank 0 only), 4 epilogue, 5 pw split, 6 relay (rank 1 only)."""
+    # 40 x 4 x 2 = 320 pair tiles on 74 pairs: every pair has >= 4
+    case = wl.Conv1dCase("pair_stall", 40, 256, 1024, 512, 9, 1, 4, seed=37)
+    x, dw, pw, bias = [t.cuda() for t in wl.conv1d_inputs(case)]
+    To = binding.conv1d_out_len(case.T, case.K, case.stride, case.pad)
+    out = torch.empty((case.N, case.O, To), device="cuda")
+    sp = P(torch.cuda.current_stream().cuda_stream)
+    assert lib.fcv_device_error(sp) == 0
+    for role, ranks in ((1, (0, 1)), (2, (0, 1)), (3, (0,)), (4, (0, 1)), (5, (0, 1)), (6, (1,))):
+        for rank in ranks:
+            for at in (0, 2):
+                st = lib.fcv_selftest_conv1d_pair_stall(_p(x), _p(dw), _p(pw), _p(bias), case.N, case.C, case.T,
+                                                        case.O, case.K, case.stride, case.pad, _p(out), role, at,
+                                                        rank, LIMIT_NS, sp)
+                assert st == 0, f"role {role} rank {rank} at {at}: launch status {st}"
+                assert lib.fcv_device_error(sp) == TIMEOUT, f"role {role} rank {rank} at {at}: no timeout recorded"
+    got = binding.dwsep_conv1d(x, dw, pw, bias, case.stride, case.pad, algo=binding.CONV1D_TC2_3XTF32)
     torch.cuda.synchronize()
     assert lib.fcv_device_error(sp) == 0
     xn, dwn, pwn, bn = [t.cpu().numpy() for t in (x, dw, pw, bias)]
