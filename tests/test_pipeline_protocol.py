@@ -692,3 +692,125 @@ def test_shifted_model_catches_buffers_shared_between_producer_warps():
     can wait on a buffer two phases ahead of it, where the parity wait passes
     on a stale phase."""
     assert _planted_failures(None, nslot=8, nstg=3, match="needs") > 0
+
+
+# ------------------------------------------------------------------------------
+# dwsep_conv1d_tc2_kernel's abort path (csrc/conv1d_tc2.cuh): both CTAs of the
+# pair watch each other's abort flag, so one flag ends every main-loop wait of
+# the pair (the model's abort is global).  Each TMA warp then waits for the
+# last box it issued on every stage, the leader commits a drain barrier to both
+# CTAs after its last MMA and both wait for it, and the pair leaves together
+# (closing cluster barrier): no box or MMA of either CTA may be in flight.
+
+
+class PairAbortSim(AbortSim):
+    """AbortSim with one TMA queue and drain per CTA: ("mark2", r, s, nstg)
+    records the last box CTA r issued on a stage, ("tma_drain2", r, nstg, who)
+    passes once each of them has landed."""
+
+    def __init__(self):
+        super().__init__()
+        self.last2 = {0: {}, 1: {}}
+
+    def can_run(self, st):
+        if st[0] == "mark2":
+            return True
+        if st[0] == "tma_drain2":
+            _, r, nstg, _who = st
+            for b, last in self.last2[r].items():
+                if self.bars[f"tma{b}@{r}"].phase < last // nstg + 1:
+                    return False
+            return True
+        return super().can_run(st)
+
+    def step(self, st):
+        if st[0] == "mark2":
+            self.last2[st[1]][st[2] % st[3]] = st[2]
+        elif st[0] == "tma_drain2":
+            pass
+        else:
+            super().step(st)
+
+
+def conv1d_pair_abort_kernel(T, NK, stages=3, npw=8, split=2):
+    sim = PairAbortSim()
+    for r in range(2):
+        for s_ in range(stages):
+            sim.bar(f"empty{s_}@{r}", 1)
+            sim.bar(f"tma{s_}@{r}", 1)
+        for b_ in range(2):
+            sim.bar(f"afull{b_}@{r}", 1)
+        sim.bar(f"drain@{r}", 1)
+    for s_ in range(stages):
+        sim.bar(f"full{s_}@0", npw + split + 1)
+        sim.bar(f"lfull{s_}@1", npw + split)
+    for b_ in range(2):
+        sim.bar(f"aempty{b_}@0", 8)
+    n = T * NK
+    for r in range(2):
+        tma, prod, spl = [], [], []
+        target = "full{}@0" if r == 0 else "lfull{}@1"
+        for seq in range(n):
+            st, k = seq % stages, seq // stages
+            tma += [("wait", f"empty{st}@{r}", (k & 1) ^ 1, k, f"tma{r}"), ("owns", f"empty{st}@{r}", k, f"tma{r}"),
+                    ("enqueue", f"box{r}", [("arrive", f"tma{st}@{r}", k, 1, f"box{r}")]), ("mark2", r, seq, stages)]
+            prod += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"producers{r}"),
+                     ("owns", f"empty{st}@{r}", k, f"producers{r}"), ("write", f"A{st}@{r}", k),
+                     ("arrive", target.format(st), k, npw, f"producers{r}")]
+            spl += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"split{r}"),
+                    ("owns", f"empty{st}@{r}", k, f"split{r}"), ("write", f"B{st}@{r}", k),
+                    ("arrive", target.format(st), k, split, f"split{r}")]
+        epi = []
+        for t in range(T):
+            buf, bk = t & 1, t >> 1
+            epi += [("wait", f"afull{buf}@{r}", bk & 1, bk + 1, f"epilogue{r}"),
+                    ("arrive", f"aempty{buf}@0", bk, 4, f"epilogue{r}")]
+        sim.roles += [(tma, [("tma_drain2", r, stages, f"tma{r}")]), (prod, []), (spl, []), (epi, [])]
+    rel = []
+    for seq in range(n):
+        st, k = seq % stages, seq // stages
+        rel += [("wait", f"lfull{st}@1", k & 1, k + 1, "relay"), ("arrive", f"full{st}@0", k, 1, "relay")]
+    sim.roles.append((rel, [("wait", "drain@1", 0, 1, "mma1")]))
+    iss = []
+    for t in range(T):
+        buf, bk = t & 1, t >> 1
+        iss += [("wait", f"aempty{buf}@0", (bk & 1) ^ 1, bk, "issuer"), ("owns", f"aempty{buf}@0", bk, "issuer")]
+        for c in range(NK):
+            seq = t * NK + c
+            st, k = seq % stages, seq // stages
+            iss += [("wait", f"full{st}@0", k & 1, k + 1, "issuer"),
+                    ("enqueue", "mma", [("read", f"{op}{st}@{r}", k, "mma") for op in "AB" for r in range(2)]),
+                    ("enqueue", "mma", [("arrive", f"empty{st}@0", k, 1, "mma"),
+                                        ("arrive", f"empty{st}@1", k, 1, "mma")])]
+        iss.append(("enqueue", "mma", [("arrive", f"afull{buf}@0", bk, 1, "mma"),
+                                       ("arrive", f"afull{buf}@1", bk, 1, "mma")]))
+    sim.roles.append((iss, [("enqueue", "mma", [("arrive", "drain@0", 0, 1, "mma"), ("arrive", "drain@1", 0, 1, "mma")]),
+                            ("wait", "drain@0", 0, 1, "issuer")]))
+    return sim
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5])
+@pytest.mark.parametrize("NK", [1, 2, 3, 8])
+def test_conv1d_pair_abort_leaves_nothing_in_flight(T, NK):
+    """Any main-loop wait of either CTA may give up: afterwards every role of
+    both CTAs leaves, and when the pair exits no TMA box of either CTA and no
+    MMA is in flight; without an abort the protocol runs to the end."""
+    aborted = 0
+    for seed in range(40):
+        conv1d_pair_abort_kernel(T, NK).run(seed)
+        aborted += conv1d_pair_abort_kernel(T, NK).run(seed, p_abort=0.05)
+    assert aborted > 0
+
+
+def test_pair_abort_model_catches_a_missing_tma_drain():
+    """Plant the mistake: the peer CTA's TMA warp leaves without waiting for its
+    boxes.  Some abort must then find a box still in flight at exit."""
+    failures = 0
+    for seed in range(200):
+        sim = conv1d_pair_abort_kernel(3, 3)
+        sim.roles[4] = (sim.roles[4][0], [])  # CTA 1's TMA warp: no drain
+        try:
+            sim.run(seed, p_abort=0.05)
+        except AssertionError as e:
+            failures += "still in flight" in str(e)
+    assert failures > 0
