@@ -960,13 +960,16 @@ def run_reference(args):
     macs = (macs_conv2d(1, CASE_A.Cin, CASE_A.H, CASE_A.W, ca, CASE_A.P)
             + macs_conv1d(1, CASE_B.C, CASE_B.T, cb, CASE_B.K, CASE_B.stride, CASE_B.pad))
     value = 2.0 * macs * args.steps / dt / 1e9
+    full_macs = (macs_conv2d(CASE_A.N, CASE_A.Cin, CASE_A.H, CASE_A.W, CASE_A.Cout, CASE_A.P)
+                 + macs_conv1d(CASE_B.N, CASE_B.C, CASE_B.T, CASE_B.O, CASE_B.K, CASE_B.stride, CASE_B.pad))
     sample = (f"per step: op A on 1 batch item with {ca} of {CASE_A.Cout} output channels, op B on 1 batch "
               f"item with {cb} of {CASE_B.O} output channels")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_name(), "parallelism": "CPU oracle, rank 0 only"},
+        "config": {"workload": workload_name(), "parallelism": "CPU oracle, rank 0 only", "sample": sample,
+                   "sampled_fraction_of_step": macs / full_macs},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
