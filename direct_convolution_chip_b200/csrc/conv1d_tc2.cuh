@@ -62,7 +62,7 @@ constexpr uint32_t B_BYTES = TNH * KC * 4;   // 16 KB
 constexpr uint32_t STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
 constexpr uint32_t OFF_DWS = STAGES * STAGE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_DWS + DWX_MAX * 4;
-constexpr uint32_t NBAR = 18;    // full[3] empty[3] afull[2] aempty[2] drain tma[3] lfull[3] gate
+constexpr uint32_t NBAR = 19;    // full[3] empty[3] afull[2] aempty[2] drain tma[3] lfull[3] gate last
 constexpr uint32_t OFF_MISC = OFF_BAR + 24 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -205,6 +205,76 @@ __device__ __forceinline__ TileCoord decode_pair_tile(const Params& p, int tile)
     return tc;
 }
 
+// Drains the 16-column blocks [cb0, cb1) (both even) of this warp's 32 TMEM
+// lanes of a finished accumulator at `taddr` (times tw .. tw+31 of tile tcd):
+// two blocks at a time, so that their eight 4x4 transposes overlap (lane 4k+j
+// ends with times tw+4k..tw+4k+3 of channels 4j..4j+3), the bias added after
+// the transpose, where a lane's four values belong to one output channel, then
+// 16-byte streaming stores.
+__device__ __forceinline__ void drain_blocks(const Params& p, const TileCoord& tcd, uint32_t taddr, int tw, int cb0,
+                                             int cb1, int lane)
+{
+    const bool vec = tw + 32 <= p.To && p.out_vec;
+    const int kq = lane >> 2, jq = lane & 3;
+    auto bias_of = [&](int o) { return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f; };
+#pragma unroll 1
+    for (int cb = cb0; cb < cb1; cb += 2) {
+        uint32_t ra[16], rb[16];
+        tc::tmem_ld16(taddr + (uint32_t)(cb * 16), ra);
+        tc::tmem_ld16(taddr + (uint32_t)((cb + 1) * 16), rb);
+        tc::tmem_wait_ld16(ra);
+        tc::tmem_wait_ld16(rb);
+        if (vec) {
+            float x[2][4][4];
+            float bv[2][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const uint32_t(&r)[16] = h ? rb : ra;
+                    x[h][m][0] = __uint_as_float(r[m]);
+                    x[h][m][1] = __uint_as_float(r[4 + m]);
+                    x[h][m][2] = __uint_as_float(r[8 + m]);
+                    x[h][m][3] = __uint_as_float(r[12 + m]);
+                    bv[h][m] = bias_of(tcd.o0 + (cb + h) * 16 + 4 * jq + m);
+                }
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int m = 0; m < 4; ++m) tc::quad_transpose(x[h][m][0], x[h][m][1], x[h][m][2], x[h][m][3], jq);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int o = tcd.o0 + (cb + h) * 16 + 4 * jq + m;
+                    if (o < p.O) {
+                        float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
+                        const float b = bv[h][m];
+                        __stcs(reinterpret_cast<float4*>(dst),  // streaming store
+                               make_float4(x[h][m][0] + b, x[h][m][1] + b, x[h][m][2] + b, x[h][m][3] + b));
+                    }
+                }
+        } else {
+            const int t = tw + lane;
+            float* out_nt = p.out + (size_t)tcd.n * p.O * p.To + t;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int o = tcd.o0 + (cb + h) * 16 + j;
+                    if (t < p.To && o < p.O) out_nt[(size_t)o * p.To] = __uint_as_float((h ? rb : ra)[j]) + bias_of(o);
+                }
+        }
+    }
+}
+
+// The last tile of a pair has no successor to overlap its drain with, so the
+// eight producer warps, idle by then, take blocks 6..11 (warps 0-3) and 12..15
+// (warps 4-7) of their TMEM lane quarter while the epilogue warp takes 0..5.
+constexpr int LAST_EPI_BLOCKS = 6, LAST_PROD_SPLIT = 12;
+static_assert(LAST_EPI_BLOCKS % 2 == 0 && LAST_PROD_SPLIT % 2 == 0 && LAST_PROD_SPLIT < TN / 16,
+              "blocks are drained in pairs");
+
 // KT: depthwise kernel size when fixed at compile time (0: any K <= KMAXW).
 // R: (t0 - pad) mod 4, the offset of the first needed sample inside the box.
 template <int KT, int R>
@@ -228,6 +298,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     const uint32_t bar_tma = bar_full + 88;      // + 8 * stage
     const uint32_t bar_lfull = bar_full + 112;   // + 8 * stage (rank 1: its producers, forwarded by the relay)
     const uint32_t bar_gate = bar_full + 136;    // never completed: the failure-path test's stall
+    const uint32_t bar_last = bar_full + 144;    // the 4 epilogue warps have seen the last tile's accumulator
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
     volatile uint32_t* prod_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 8);
@@ -250,6 +321,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         }
         mbar_init(bar_drain, 1);
         mbar_init(bar_gate, 1);
+        mbar_init(bar_last, 4);
         *abort_flag = 0u;
         *prod_abort = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -261,14 +333,9 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
     }
     const int nk = (p.C + KC - 1) / KC;
-    // Depthwise weights resident as [K][CW], CW = 32 * nk, zero beyond C.
     const int CW = KC * nk;
-    for (int e = threadIdx.x; e < p.K * CW; e += NTHREADS) {
-        const int k = e / CW, c = e - (e / CW) * CW;
-        dws[e] = c < p.C ? __ldg(p.dw + (size_t)c * p.K + k) : 0.f;
-    }
     tc_fence_before();
-    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated, weights staged
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const PairAbort ab{abort_flag, mapa(smem_u32(const_cast<uint32_t*>(abort_flag)), rank ^ 1u)};
@@ -276,6 +343,14 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     if (warp < NPW) {
         // ------------------------------------------------------------ producers
         const int ptid = threadIdx.x;
+        // Depthwise weights resident as [K][CW], CW = 32 * nk, zero beyond C,
+        // staged by the producers (their only readers) while the TMA warp
+        // already issues the first copies; the group barrier of the first
+        // chunk orders these writes before any read.
+        for (int e = ptid; e < p.K * CW; e += NPW * 32) {
+            const int k = e / CW, c = e - (e / CW) * CW;
+            dws[e] = c < p.C ? __ldg(p.dw + (size_t)c * p.K + k) : 0.f;
+        }
         const int K = KT > 0 ? KT : p.K;
         int stage = 0;
         uint32_t phase = 0;
@@ -344,6 +419,23 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                     stage = 0;
                     phase ^= 1u;
                 }
+            }
+        }
+        if (run) {
+            // The last tile's drain, beside the epilogue warps, once they have
+            // seen its accumulator complete (a barrier used once: no stale phase).
+            int ok = 1;
+            if (lane == 0) ok = pair_wait<false>(bar_last, 0, ab) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (ok) {
+                tc_fence_after();
+                const int last = local - 1, q = warp & 3;
+                const TileCoord tcd = decode_pair_tile(p, pair + last * npairs);
+                const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((last & 1) * TN);
+                const int cb0 = warp < 4 ? LAST_EPI_BLOCKS : LAST_PROD_SPLIT;
+                const int cb1 = warp < 4 ? LAST_PROD_SPLIT : TN / 16;
+                drain_blocks(p, tcd, taddr, tcd.t0 + (int)rank * TM + 32 * q, cb0, cb1, lane);
+                tc_fence_before();
             }
         }
     } else if (warp == MMA_WARP) {
@@ -547,63 +639,9 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             const TileCoord tcd = decode_pair_tile(p, tile);
             const int tw = tcd.t0 + (int)rank * TM + 32 * q;
             const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TN);
-            const bool vec = tw + 32 <= p.To && p.out_vec;
-            const int kq = lane >> 2, jq = lane & 3;
-            auto bias_of = [&](int o) { return (p.bias && o < p.O) ? __ldg(p.bias + o) : 0.f; };
-            // Blocks of 16 columns, two at a time, so that their eight 4x4
-            // transposes (lane 4k+j ends with times tw+4k..tw+4k+3 of channels
-            // 4j..4j+3) overlap; the bias is added after the transpose, where a
-            // lane's four values belong to one output channel.
-#pragma unroll 1
-            for (int cb = 0; cb < TN / 16; cb += 2) {
-                uint32_t ra[16], rb[16];
-                tmem_ld16(taddr + (uint32_t)(cb * 16), ra);
-                tmem_ld16(taddr + (uint32_t)((cb + 1) * 16), rb);
-                tmem_wait_ld16(ra);
-                tmem_wait_ld16(rb);
-                if (vec) {
-                    float x[2][4][4];
-                    float bv[2][4];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            const uint32_t(&r)[16] = h ? rb : ra;
-                            x[h][m][0] = __uint_as_float(r[m]);
-                            x[h][m][1] = __uint_as_float(r[4 + m]);
-                            x[h][m][2] = __uint_as_float(r[8 + m]);
-                            x[h][m][3] = __uint_as_float(r[12 + m]);
-                            bv[h][m] = bias_of(tcd.o0 + (cb + h) * 16 + 4 * jq + m);
-                        }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) quad_transpose(x[h][m][0], x[h][m][1], x[h][m][2], x[h][m][3], jq);
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            const int o = tcd.o0 + (cb + h) * 16 + 4 * jq + m;
-                            if (o < p.O) {
-                                float* dst = p.out + ((size_t)tcd.n * p.O + o) * p.To + tw + 4 * kq;
-                                const float b = bv[h][m];
-                                __stcs(reinterpret_cast<float4*>(dst),  // streaming store
-                                       make_float4(x[h][m][0] + b, x[h][m][1] + b, x[h][m][2] + b, x[h][m][3] + b));
-                            }
-                        }
-                } else {
-                    const int t = tw + lane;
-                    float* out_nt = p.out + (size_t)tcd.n * p.O * p.To + t;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int o = tcd.o0 + (cb + h) * 16 + j;
-                            if (t < p.To && o < p.O)
-                                out_nt[(size_t)o * p.To] = __uint_as_float((h ? rb : ra)[j]) + bias_of(o);
-                        }
-                }
-            }
+            const bool last = tile + npairs >= p.total_tiles;
+            if (last && lane == 0) mbar_arrive(bar_last);  // the producers take the rest of this tile
+            drain_blocks(p, tcd, taddr, tw, 0, last ? LAST_EPI_BLOCKS : TN / 16, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(aempty_leader + 8 * buf);

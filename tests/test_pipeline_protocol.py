@@ -279,6 +279,8 @@ def conv1d_pair_kernel(T, NK, stages=3, relay=True, split=2, npw=8):
     for b_ in range(2):
         sim.bar(f"aempty{b_}@0", 8)
     for r in range(2):
+        sim.bar(f"last@{r}", 4)
+    for r in range(2):
         tma, prod, spl = [], [], []
         for seq in range(T * NK):
             st, k = seq % stages, seq // stages
@@ -291,11 +293,16 @@ def conv1d_pair_kernel(T, NK, stages=3, relay=True, split=2, npw=8):
             spl += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"split{r}"),
                     ("owns", f"empty{st}@{r}", k, f"split{r}"),
                     ("arrive", target, k, split, f"split{r}")]
+        # the producers help drain the last tile once the epilogue warps have
+        # seen it complete (a barrier used once)
+        prod.append(("wait", f"last@{r}", 0, 1, f"producers{r}"))
         epi = []
         for t in range(T):
             buf, bk = t & 1, t >> 1
-            epi += [("wait", f"afull{buf}@{r}", bk & 1, bk + 1, f"epilogue{r}"),
-                    ("release", f"acc{buf}@{r}"),
+            epi += [("wait", f"afull{buf}@{r}", bk & 1, bk + 1, f"epilogue{r}")]
+            if t == T - 1:
+                epi.append(("arrive", f"last@{r}", 0, 4, f"epilogue{r}"))
+            epi += [("release", f"acc{buf}@{r}"),
                     ("arrive", f"aempty{buf}@0", bk, 4, f"epilogue{r}")]
         sim.agents += [tma, prod, epi] + ([spl] if split else [])
     if relay:
@@ -741,6 +748,7 @@ def conv1d_pair_abort_kernel(T, NK, stages=3, npw=8, split=2):
         for b_ in range(2):
             sim.bar(f"afull{b_}@{r}", 1)
         sim.bar(f"drain@{r}", 1)
+        sim.bar(f"last@{r}", 4)
     for s_ in range(stages):
         sim.bar(f"full{s_}@0", npw + split + 1)
         sim.bar(f"lfull{s_}@1", npw + split)
@@ -760,11 +768,14 @@ def conv1d_pair_abort_kernel(T, NK, stages=3, npw=8, split=2):
             spl += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"split{r}"),
                     ("owns", f"empty{st}@{r}", k, f"split{r}"), ("write", f"B{st}@{r}", k),
                     ("arrive", target.format(st), k, split, f"split{r}")]
+        prod.append(("wait", f"last@{r}", 0, 1, f"producers{r}"))  # skipped after an abort: a loop wait
         epi = []
         for t in range(T):
             buf, bk = t & 1, t >> 1
-            epi += [("wait", f"afull{buf}@{r}", bk & 1, bk + 1, f"epilogue{r}"),
-                    ("arrive", f"aempty{buf}@0", bk, 4, f"epilogue{r}")]
+            epi += [("wait", f"afull{buf}@{r}", bk & 1, bk + 1, f"epilogue{r}")]
+            if t == T - 1:
+                epi.append(("arrive", f"last@{r}", 0, 4, f"epilogue{r}"))
+            epi.append(("arrive", f"aempty{buf}@0", bk, 4, f"epilogue{r}"))
         sim.roles += [(tma, [("tma_drain2", r, stages, f"tma{r}")]), (prod, []), (spl, []), (epi, [])]
     rel = []
     for seq in range(n):
