@@ -25,7 +25,9 @@
 // warps arrive locally and whose warp-8 lane 0 relays
 // (a cluster-scope release per producer warp cost ~1,600 cycles on the
 // producers' path); the leader's "aempty" collects both CTAs' epilogues
-// (remote arrives).  MMA completion is committed to both CTAs' "empty"/"afull"
+// (remote arrives).  The producers stage the depthwise weights after the
+// opening cluster barrier, so the TMA warp starts at once, and help drain the
+// pair's last tile, which has no successor to overlap its drain with.  MMA completion is committed to both CTAs' "empty"/"afull"
 // barriers with a multicast commit.  Every mbarrier wait is bounded and also
 // watches the peer CTA's abort flag, so the pair gives up together; a cluster
 // barrier follows initialisation and precedes exit, so no CTA leaves while
