@@ -5,7 +5,8 @@
 // pointwise as a 3xTF32 tcgen05 contraction with the pw hi part read raw,
 // fp32 accumulation in TMEM).  What changes is the tiling: the two CTAs of a
 // cluster compute one 256-time x 256-output-channel tile with
-// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 8).  Each CTA holds its own
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 8), at stride 1 or 2 (the
+// stride-2 halo in two TMA boxes, as in the single-SM kernel).  Each CTA holds its own
 // 128 rows of A (its times) and HALF of B (128 of the 256 pw rows), so per CTA
 // the pw split work, the B stage and the MMA's shared-memory reads are halved,
 // and three 64 KB stages fit where the single-SM kernel has two of 96 KB: the
@@ -54,8 +55,10 @@ constexpr int NTHREADS = (SPLIT_WARP + NSPLIT) * 32;
 constexpr int FULL_ARRIVALS = NPW + NSPLIT;  // per CTA and chunk: producer and split warps
 static_assert(TPW % 4 == 0 && TPW * NPW == TM, "16-byte window loads cover the CTA's times");
 constexpr int KMAXW = tc::KMAXW;
-constexpr int XW = 148;          // halo box width = smem row pitch (floats)
+constexpr int XW = 148;          // halo box width = smem row pitch (floats), stride 1
 constexpr uint32_t X_BYTES = (uint32_t)XW * KC * 4;
+constexpr int XW2 = tcx::XW2;    // stride 2: two boxes of this width
+constexpr uint32_t X2_BYTES = tcx::X2_BYTES;
 constexpr int DWX_MAX = 8192;    // resident depthwise weights, [K][32*nk]
 constexpr uint32_t TMEM_COLS = 2 * TN;
 
@@ -68,7 +71,13 @@ constexpr uint32_t NBAR = 19;    // full[3] empty[3] afull[2] aempty[2] drain tm
 constexpr uint32_t OFF_MISC = OFF_BAR + 24 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(X_BYTES <= 2 * A_BYTES, "the halo box must fit the stage's A region");
+// Stage: A_hi | A_lo | B_lo | B_hi.  The halo (one box at stride 1, two at
+// stride 2) is staged from the stage's start; at stride 2 it reaches into B_lo,
+// which the producers then form after their halo barrier (the split warps
+// serve stride 1 only), and it never reaches B_hi, where the TMA puts pw.
+constexpr uint32_t OFF_BLO = 2 * A_BYTES, OFF_BHI = 2 * A_BYTES + B_BYTES;
+static_assert(X_BYTES <= 2 * A_BYTES, "the stride-1 halo box must fit the stage's A region");
+static_assert(2 * X2_BYTES <= OFF_BHI, "the stride-2 halo boxes must stay below B_hi");
 
 // D fp32, A/B tf32, K-major, N = 256, M = 256 (the pair).
 constexpr uint32_t kIdesc2 = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(TN >> 3) << 17) |
@@ -278,16 +287,19 @@ static_assert(LAST_EPI_BLOCKS % 2 == 0 && LAST_PROD_SPLIT % 2 == 0 && LAST_PROD_
               "blocks are drained in pairs");
 
 // KT: depthwise kernel size when fixed at compile time (0: any K <= KMAXW).
-// R: (t0 - pad) mod 4, the offset of the first needed sample inside the box.
-template <int KT, int R>
+// R: (t0*S - pad) mod 4, the offset of the first needed sample inside the box.
+// S: stride (1 or 2).
+template <int KT, int R, int S>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_map,
                         const __grid_constant__ CUtensorMap x_map)
 {
     using namespace tc;
     constexpr int KW = KT > 0 ? KT : KMAXW;            // taps the window must cover
-    constexpr int NV = (R + TPW - 1 + KW + 3) / 4;     // 16-byte window loads per thread
-    static_assert(TPW * (NPW - 1) + 4 * NV <= XW, "window inside the halo box");
+    constexpr int NV = (R + S * (TPW - 1) + KW + 3) / 4;  // 16-byte window loads per thread
+    static_assert(S == 1 || S == 2, "stride 1 or 2");
+    static_assert(S * TPW * (NPW - 1) + 4 * NV <= (S == 1 ? XW : 2 * XW2), "window inside the halo boxes");
+    constexpr int FULL_N = S == 1 ? FULL_ARRIVALS : NPW;  // producer (and, at stride 1, split) warps
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
@@ -312,8 +324,8 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
-            mbar_init(bar_full + 8 * i, FULL_ARRIVALS + 1);  // the leader's warps + the other CTA's relay
-            mbar_init(bar_lfull + 8 * i, FULL_ARRIVALS);     // the other CTA's warps (used in rank 1)
+            mbar_init(bar_full + 8 * i, FULL_N + 1);  // the leader's warps + the other CTA's relay
+            mbar_init(bar_lfull + 8 * i, FULL_N);     // the other CTA's warps (used in rank 1)
             mbar_init(bar_empty + 8 * i, 1);   // multicast commit
             mbar_init(bar_tma + 8 * i, 1);     // expect_tx arrival + TMA bytes
         }
@@ -375,12 +387,18 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                 const uint32_t a_lo = a_hi + A_BYTES;
 
                 // Depthwise: channel lane, this CTA's times TPW*warp .. +TPW-1;
-                // halo sample j is x[t0 + 128*rank - pad - R + j].
-                const float* xrow = reinterpret_cast<const float*>(smem + stage * STAGE_BYTES) + lane * XW + TPW * warp;
+                // halo sample j is x[(t0 + 128*rank)*S - pad - R + j], output time
+                // TPW*warp + i takes samples S*(TPW*warp + i) + R + k, k < K; at
+                // stride 2, samples j >= XW2 sit in the second box.
+                const float* xs0 = reinterpret_cast<const float*>(smem + stage * STAGE_BYTES) +
+                                   lane * (S == 1 ? XW : XW2);
+                const float* xs1 = xs0 + KC * XW2;
                 float win[4 * NV];
 #pragma unroll
                 for (int q = 0; q < NV; ++q) {
-                    const float4 v = *reinterpret_cast<const float4*>(xrow + 4 * q);
+                    const int j = S * TPW * warp + 4 * q;
+                    const float* src = (S == 1 || j < XW2) ? xs0 + j : xs1 + (j - XW2);
+                    const float4 v = *reinterpret_cast<const float4*>(src);
                     win[4 * q] = v.x;
                     win[4 * q + 1] = v.y;
                     win[4 * q + 2] = v.z;
@@ -397,11 +415,23 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                         const float2 w2 = make_float2(w, w);
 #pragma unroll
                         for (int j = 0; j < TPW / 2; ++j)
-                            d2[j] = __ffma2_rn(make_float2(win[R + 2 * j + k], win[R + 2 * j + k + 1]), w2, d2[j]);
+                            d2[j] = __ffma2_rn(make_float2(win[R + 2 * S * j + k], win[R + 2 * S * j + S + k]),
+                                               w2, d2[j]);
                     }
                 }
-                // Every producer has read its halo window before the A operand overwrites it.
+                // Every producer has read its halo window before the A operand (and,
+                // at stride 2, B_lo) overwrites it.
                 asm volatile("bar.sync 1, %0;\n" ::"n"(NPW * 32) : "memory");
+                if constexpr (S == 2) {
+                    // This CTA's half of the pw chunk: B_hi stays raw (the MMA reads
+                    // its TF32 bits), B_lo = v - truncate(v); 16 rows per warp.
+                    const uint32_t b_lo = a_hi + OFF_BLO, b_hi = a_hi + OFF_BHI;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t off = sw128_off(warp * 16 + i * 4 + (lane >> 3), lane & 7);
+                        sts128(b_lo + off, tcx::tf32_trunc_rest4(lds128(b_hi + off)));
+                    }
+                }
                 const uint32_t col = ((uint32_t)(lane & 3) << 2);
 #pragma unroll
                 for (int i = 0; i < TPW; ++i) {
@@ -460,8 +490,8 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                     tc_fence_after();
                     const uint32_t a_hi = sbase + stage * STAGE_BYTES;
                     const uint32_t a_lo = a_hi + A_BYTES;
-                    const uint32_t b_hi = a_lo + A_BYTES;
-                    const uint32_t b_lo = b_hi + B_BYTES;
+                    const uint32_t b_lo = a_hi + OFF_BLO;
+                    const uint32_t b_hi = a_hi + OFF_BHI;
 #pragma unroll
                     for (int kk = 0; kk < KC / 8; ++kk) {
                         const uint32_t koff = 32u * kk;
@@ -527,7 +557,7 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
         const int sl = (warp - SPLIT_WARP) * 32 + lane;
         int stage = 0;
         uint32_t phase = 0;
-        bool ok = true;
+        bool ok = S == 1;  // at stride 2 the producers form B_lo after their halo barrier
         int local = 0;
         for (int tile = pair; ok && tile < p.total_tiles; tile += npairs, ++local) {
             for (int k = 0; k < nk; ++k) {
@@ -542,8 +572,8 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                 }
                 for (int spin = 0; !mbar_try_wait(bar_tma + 8 * stage, phase) && spin < (1 << 20); ++spin) {
                 }
-                const uint32_t b_hi = sbase + stage * STAGE_BYTES + 2 * A_BYTES;
-                const uint32_t b_lo = b_hi + B_BYTES;
+                const uint32_t b_hi = sbase + stage * STAGE_BYTES + OFF_BHI;
+                const uint32_t b_lo = sbase + stage * STAGE_BYTES + OFF_BLO;
                 // 1024 16-byte slots (128 rows x 8), 16 per thread in two batches
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -582,13 +612,16 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
             for (int tile = pair; ok && tile < p.total_tiles; tile += npairs, ++local) {
                 if (!stall_ok(p, 1, local, rank, bar_gate, ab)) break;
                 const TileCoord tcd = decode_pair_tile(p, tile);
-                const int x0 = tcd.t0 + (int)rank * TM - p.pad - R;  // a multiple of 4
+                const int x0 = (tcd.t0 + (int)rank * TM) * S - p.pad - R;  // a multiple of 4
                 // Pull the next tile's halo boxes into L2 now, so its TMA loads
                 // wait on L2 rather than on DRAM latency.
                 if (tile + npairs < p.total_tiles) {
                     const TileCoord nx = decode_pair_tile(p, tile + npairs);
-                    for (int k = 0; k < nk; ++k)
-                        tcx::tma_prefetch_3d(&x_map, nx.t0 + (int)rank * TM - p.pad - R, k * KC, nx.n);
+                    const int nx0 = (nx.t0 + (int)rank * TM) * S - p.pad - R;
+                    for (int k = 0; k < nk; ++k) {
+                        tcx::tma_prefetch_3d(&x_map, nx0, k * KC, nx.n);
+                        if (S == 2) tcx::tma_prefetch_3d(&x_map, nx0 + XW2, k * KC, nx.n);
+                    }
                 }
                 for (int k = 0; k < nk; ++k) {
                     if (!pair_wait<true>(bar_empty + 8 * stage, phase ^ 1, ab)) {
@@ -597,9 +630,10 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
                     }
                     pending[stage] = false;
                     const uint32_t st = sbase + stage * STAGE_BYTES;
-                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES + X_BYTES);
-                    tma_load_2d(st + 2 * A_BYTES, &pw_map, k * KC, tcd.o0 + (int)rank * TNH, bar_tma + 8 * stage);
+                    mbar_arrive_expect_tx(bar_tma + 8 * stage, B_BYTES + (S == 1 ? X_BYTES : 2 * X2_BYTES));
+                    tma_load_2d(st + OFF_BHI, &pw_map, k * KC, tcd.o0 + (int)rank * TNH, bar_tma + 8 * stage);
                     tcx::tma_load_3d(st, &x_map, x0, k * KC, tcd.n, bar_tma + 8 * stage);
+                    if (S == 2) tcx::tma_load_3d(st + X2_BYTES, &x_map, x0 + XW2, k * KC, tcd.n, bar_tma + 8 * stage);
                     pending[stage] = true;
                     ++issued;
                     if (++stage == STAGES) {
@@ -660,30 +694,46 @@ dwsep_conv1d_tc2_kernel(const Params p, const __grid_constant__ CUtensorMap pw_m
     }
 }
 
+using KernelPtr = decltype(&dwsep_conv1d_tc2_kernel<0, 0, 1>);
+
+template <int S>
+inline KernelPtr select_kernel(int K, int r)
+{
+    if (K == 9 && r == 0) return dwsep_conv1d_tc2_kernel<9, 0, S>;
+    if (K == 3 && r == 3) return dwsep_conv1d_tc2_kernel<3, 3, S>;
+    if (r == 0) return dwsep_conv1d_tc2_kernel<0, 0, S>;
+    if (r == 1) return dwsep_conv1d_tc2_kernel<0, 1, S>;
+    if (r == 2) return dwsep_conv1d_tc2_kernel<0, 2, S>;
+    return dwsep_conv1d_tc2_kernel<0, 3, S>;
+}
+
 }  // namespace tc2
 
 // The 2-SM path covers the shapes of the single-SM TMA-halo kernel.
 inline bool conv1d_tc2_supported(int C, int T, int O, int K, int stride, const void* x, const void* pw)
 {
     const long long cw = (long long)tc2::KC * ((C + tc2::KC - 1) / tc2::KC);
-    return stride == 1 && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1 && T >= 1 && (C & 3) == 0 &&
+    return (stride == 1 || stride == 2) && K >= 1 && K <= tc::KMAXW && C >= 1 && O >= 1 && T >= 1 && (C & 3) == 0 &&
            (T & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 &&
            (reinterpret_cast<uintptr_t>(pw) & 15) == 0 && cw * K <= tc2::DWX_MAX;
 }
 
 // Where AUTO takes the SM pair over the single-SM TMA-halo kernel: at least
 // eight 32-channel chunks per tile (C >= 256), so the pair's per-tile
-// start-up and drain are amortised, and O >= 256, so the 256-wide tile is
-// not half empty.  Measured on B200 over the stride-1 points of the conv1d
-// shape sweep: 1.05-1.20x faster there, 0.80-0.98x at C = 64, about even at
-// O = 128.
+// start-up and drain are amortised, and, at stride 1, O >= 256, so the
+// 256-wide tile is not half empty.  Measured on B200 over the conv1d shape
+// sweep: stride 1, 1.05-1.20x faster there, 0.80-0.98x at C = 64, about even
+// at O = 128; stride 2 (where the depthwise window work, which the pair
+// splits, is twice as large), 1.03-1.14x at C = 384 and O = 128 and
+// 1.22-1.38x at O = 768, 0.82-0.96x at C = 64 and T = 16384.
 inline bool conv1d_tc2_preferred(int C, int T, int O, int K, int stride, const void* x, const void* pw)
 {
-    return C >= 256 && O >= 256 && conv1d_tc2_supported(C, T, O, K, stride, x, pw);
+    return C >= 256 && (stride == 2 || O >= 256) && conv1d_tc2_supported(C, T, O, K, stride, x, pw);
 }
 
 inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float* pw, const float* bias, int N,
-                                   int C, int T, int O, int K, int pad, int To, float* out, cudaStream_t stream,
+                                   int C, int T, int O, int K, int stride, int pad, int To, float* out,
+                                   cudaStream_t stream,
                                    int stall_role = 0, int stall_at = 0, int stall_rank = 0,
                                    unsigned long long stall_ns = 0)
 {
@@ -714,10 +764,10 @@ inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float*
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return FCV_ERR_CUDA;
     }
-    {   // x [N][C][T]: 148 times x 32 channels x 1 batch item per box; outside reads 0
+    {   // x [N][C][T]: 148 (stride 2: 140) times x 32 channels x 1 batch item per box; outside reads 0
         const cuuint64_t gdim[3] = {(cuuint64_t)T, (cuuint64_t)C, (cuuint64_t)N};
         const cuuint64_t gstride[2] = {(cuuint64_t)T * sizeof(float), (cuuint64_t)C * T * sizeof(float)};
-        const cuuint32_t box[3] = {(cuuint32_t)tc2::XW, (cuuint32_t)tc2::KC, 1};
+        const cuuint32_t box[3] = {(cuuint32_t)(stride == 1 ? tc2::XW : tc2::XW2), (cuuint32_t)tc2::KC, 1};
         const cuuint32_t estride[3] = {1, 1, 1};
         if (encode(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(x), gdim, gstride, box, estride,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -727,14 +777,8 @@ inline int launch_dwsep_conv1d_tc2(const float* x, const float* dw, const float*
 
     int sms = 0;
     if (device_sm_count(&sms) != FCV_OK) return FCV_ERR_CUDA;
-    const int r = (-pad) & 3;  // (t0 - pad) mod 4 with t0 a multiple of 128
-    decltype(&tc2::dwsep_conv1d_tc2_kernel<0, 0>) kern;
-    if (K == 9 && r == 0) kern = tc2::dwsep_conv1d_tc2_kernel<9, 0>;
-    else if (K == 3 && r == 3) kern = tc2::dwsep_conv1d_tc2_kernel<3, 3>;
-    else if (r == 0) kern = tc2::dwsep_conv1d_tc2_kernel<0, 0>;
-    else if (r == 1) kern = tc2::dwsep_conv1d_tc2_kernel<0, 1>;
-    else if (r == 2) kern = tc2::dwsep_conv1d_tc2_kernel<0, 2>;
-    else kern = tc2::dwsep_conv1d_tc2_kernel<0, 3>;
+    const int r = (-pad) & 3;  // (t0*stride - pad) mod 4 with t0 a multiple of 128
+    const tc2::KernelPtr kern = stride == 1 ? tc2::select_kernel<1>(K, r) : tc2::select_kernel<2>(K, r);
     const long long pairs = total < sms / 2 ? total : sms / 2;
     dim3 grid((unsigned)(2 * pairs));
     return launch_cached(kern, (int)tc2::SMEM_BYTES,

@@ -200,7 +200,7 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
     switch (algo) {
     case FCV_ALGO_AUTO:
         if (fcv::conv1d_tc2_preferred(C, T, O, K, stride, x, pw_w))
-            return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, s);
+            return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
         if (fcv::conv1d_tcx_supported(C, T, O, K, stride, x, pw_w))
             return fcv::launch_dwsep_conv1d_tcx(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
         if (fcv::conv1d_tc_supported(C, O, K, stride, pw_w)) {
@@ -209,7 +209,7 @@ int fcv_dwsep_conv1d_ex(const float* x, const float* dw_w, const float* pw_w, co
         return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     case FCV_CONV1D_TC2_3XTF32:
         if (!fcv::conv1d_tc2_supported(C, T, O, K, stride, x, pw_w)) return FCV_ERR_UNSUPPORTED;
-        return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, s);
+        return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     case FCV_CONV1D_FMA:
         return fcv::launch_dwsep_conv1d_fma(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out, s);
     case FCV_CONV1D_TC_3XTF32:
@@ -277,12 +277,12 @@ int fcv_selftest_conv1d_pair_stall(const float* x, const float* dw_w, const floa
     int st = check_conv1d(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, out, &To);
     if (st != FCV_OK) return st;
     if (role < 1 || role > 6 || rank < 0 || rank > 1 || (role == 3 && rank != 0) || (role == 6 && rank != 1) ||
-        at_tile < 0 || limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000)
+        (role == 5 && stride != 1) || at_tile < 0 || limit_ns == 0 || limit_ns > 10ull * 1000 * 1000 * 1000)
         return FCV_ERR_INVALID_ARG;
     if (!fcv::conv1d_tc2_supported(C, T, O, K, stride, x, pw_w)) return FCV_ERR_UNSUPPORTED;
     if (N == 0) return FCV_OK;
-    return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, pad, To, out, fcv::as_stream(stream),
-                                        role, at_tile, rank, limit_ns);
+    return fcv::launch_dwsep_conv1d_tc2(x, dw_w, pw_w, bias, N, C, T, O, K, stride, pad, To, out,
+                                        fcv::as_stream(stream), role, at_tile, rank, limit_ns);
 }
 
 int fcv_conv2d_auto_algo(int N, int Cin, int H, int W, int Cout, int pool, int* algo)

@@ -94,7 +94,7 @@ typedef enum {
     FCV_CONV1D_FMA = 20,          /* depthwise + pointwise on FP32 FMA */
     FCV_CONV1D_TC_3XTF32 = 21,    /* pointwise on tcgen05 tensor cores, 3xTF32 split, one SM per tile */
     FCV_CONV1D_TC2_3XTF32 = 22,   /* SM pairs (tcgen05 cta_group::2, 256x256 tiles), input halo
-                                     and pw by TMA; stride 1, T % 4 == 0, 16-byte aligned x */
+                                     and pw by TMA; stride 1 or 2, T % 4 == 0, 16-byte aligned x */
     FCV_CONV1D_TC_TMA_3XTF32 = 23 /* one SM per tile, input halo staged by TMA; stride 1 or 2,
                                      T % 4 == 0 and a 16-byte aligned x */
 } fcv_algo;
@@ -198,9 +198,10 @@ int fcv_conv2d_pool_tap(const float* x, const float* w, const float* b,
  * The depthwise result lives only in on-chip memory.  Every algorithm is
  * fp32-accurate (FP32 FMA, or tensor cores through a 3xTF32 split); results
  * are deterministic run to run.
- * FCV_ALGO_AUTO takes FCV_CONV1D_TC2_3XTF32 when stride is 1, C >= 256,
- * O >= 256, K <= 13, C % 4 == 0, T % 4 == 0, x and pw_w are 16-byte aligned
- * and 32*ceil(C/32)*K <= 8192 (where the SM pair measured faster); else
+ * FCV_ALGO_AUTO takes FCV_CONV1D_TC2_3XTF32 when C >= 256 and either stride
+ * is 2 or stride is 1 and O >= 256, with K <= 13, C % 4 == 0, T % 4 == 0, x
+ * and pw_w 16-byte aligned and 32*ceil(C/32)*K <= 8192 (where the SM pair
+ * measured faster); else
  * FCV_CONV1D_TC_TMA_3XTF32 when stride is 1 or 2, K <= 13, C % 4 == 0,
  * T % 4 == 0, x and pw_w are 16-byte aligned and 32*ceil(C/32)*K <= 8192;
  * else FCV_CONV1D_TC_3XTF32 when stride == 1, K <= 13, C % 4 == 0,

@@ -113,16 +113,17 @@ def stall1d_pair(lib, role=1, at=0, rank=0, limit=1000, **kw):
                                      (dict(rank=-1), "inv"), (dict(role=3, rank=1), "inv"),
                                      (dict(role=6, rank=0), "inv"), (dict(at=-1), "inv"), (dict(limit=0), "inv"),
                                      (dict(limit=11 * 10**9), "inv"), (dict(N=0), "ok"),
-                                     (dict(role=6, rank=1, N=0), "ok"), (dict(role=5, rank=1, N=0), "ok")])
+                                     (dict(role=6, rank=1, N=0), "ok"), (dict(role=5, rank=1, N=0), "ok"),
+                                     (dict(role=5, s=2), "inv"), (dict(role=6, rank=1, s=2, N=0), "ok")])
 def test_pair_stall_selftest_validates_on_the_host(lib, kw, want):
     """The SM-pair failure-path entry point rejects bad roles, ranks (the
-    MMA issuer lives in rank 0, the relay in rank 1), tiles and limits before
-    any CUDA call."""
+    MMA issuer lives in rank 0, the relay in rank 1; the pw split warps work
+    at stride 1 only), tiles and limits before any CUDA call."""
     assert stall1d_pair(lib, **kw) == {"inv": INVALID, "ok": OK}[want]
 
 
 def test_stall_selftests_outside_their_kernels(lib):
-    assert stall1d_pair(lib, s=2) == UNSUPPORTED
+    assert stall1d_pair(lib, s=3) == UNSUPPORTED
     assert stall1d_pair(lib, T=66) == UNSUPPORTED
     assert stall2d(lib, Cin=20) == UNSUPPORTED
     assert stall1d(lib, s=3) == UNSUPPORTED
@@ -226,8 +227,8 @@ def test_auto_algo_conv2d(lib):
 
 
 def test_auto_algo_conv1d(lib):
-    """AUTO: the SM-pair kernel for C >= 256 and O >= 256 (stride 1, aligned
-    x/pw, T % 4 == 0), then TMA-halo tensor cores for aligned x/pw, T % 4 == 0
+    """AUTO: the SM-pair kernel for C >= 256 with O >= 256 at stride 1 or any O
+    at stride 2 (aligned x/pw, T % 4 == 0), then TMA-halo tensor cores for aligned x/pw, T % 4 == 0
     and stride 1 or 2, then the register-halo tensor-core kernel (stride 1),
     then FMA."""
     a = ctypes.c_int()
@@ -237,7 +238,9 @@ def test_auto_algo_conv1d(lib):
     assert q(X, PW, 8, 384, 1000, 768, 3, 1, 1, ctypes.byref(a)) == OK and a.value == 22   # SM pair
     assert q(X, PW, 8, 64, 1000, 768, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 23    # C < 256
     assert q(X, PW, 8, 384, 1000, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 23   # O < 256
-    assert q(X, PW, 8, 384, 1000, 768, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 23   # stride 2
+    assert q(X, PW, 8, 384, 1000, 768, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 22   # stride 2, SM pair
+    assert q(X, PW, 8, 384, 1000, 128, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 22   # stride 2, O = 128
+    assert q(X, PW, 8, 64, 1000, 768, 9, 2, 4, ctypes.byref(a)) == OK and a.value == 23    # stride 2, C < 256
     assert q(X, PW, 8, 384, 1001, 768, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21   # T % 4 != 0
     assert q(P(0x10004), PW, 8, 384, 1000, 768, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21  # x misaligned
     assert q(X, PW, 2, 64, 1001, 128, 9, 1, 4, ctypes.byref(a)) == OK and a.value == 21    # T % 4 != 0

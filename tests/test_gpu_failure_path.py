@@ -93,20 +93,22 @@ def test_conv1d_stall_every_role(lib, stride):
         assert_close(got[bi:bi + 1], want, f"out[{bi}]")
 
 
-def test_conv1d_pair_stall_every_role(lib):
+@pytest.mark.parametrize("stride", [1, 2])
+def test_conv1d_pair_stall_every_role(lib, stride):
     """The SM-pair kernel: one role of one CTA of every pair stalls; that CTA
     gives up, its peer sees the abort flag through distributed shared memory,
     both drain what is in flight and free tensor memory, and the next normal
     call matches the oracle.  Roles: 1 TMA warp, 2 producers, 3 MMA issuer
     (rank 0 only), 4 epilogue, 5 pw split, 6 relay (rank 1 only)."""
     # 40 x 4 x 2 = 320 pair tiles on 74 pairs: every pair has >= 4
-    case = wl.Conv1dCase("pair_stall", 40, 256, 1024, 512, 9, 1, 4, seed=37)
+    case = wl.Conv1dCase("pair_stall", 40, 256, 1024 * stride, 512, 9, stride, 4, seed=37 + stride)
     x, dw, pw, bias = [t.cuda() for t in wl.conv1d_inputs(case)]
     To = binding.conv1d_out_len(case.T, case.K, case.stride, case.pad)
     out = torch.empty((case.N, case.O, To), device="cuda")
     sp = P(torch.cuda.current_stream().cuda_stream)
     assert lib.fcv_device_error(sp) == 0
-    for role, ranks in ((1, (0, 1)), (2, (0, 1)), (3, (0,)), (4, (0, 1)), (5, (0, 1)), (6, (1,))):
+    roles = ((1, (0, 1)), (2, (0, 1)), (3, (0,)), (4, (0, 1)), (5, (0, 1)), (6, (1,)))
+    for role, ranks in roles if stride == 1 else [r for r in roles if r[0] != 5]:  # no split warps at stride 2
         for rank in ranks:
             for at in (0, 2):
                 st = lib.fcv_selftest_conv1d_pair_stall(_p(x), _p(dw), _p(pw), _p(bias), case.N, case.C, case.T,

@@ -763,8 +763,10 @@ def conv1d_pair_abort_kernel(T, NK, stages=3, npw=8, split=2):
             tma += [("wait", f"empty{st}@{r}", (k & 1) ^ 1, k, f"tma{r}"), ("owns", f"empty{st}@{r}", k, f"tma{r}"),
                     ("enqueue", f"box{r}", [("arrive", f"tma{st}@{r}", k, 1, f"box{r}")]), ("mark2", r, seq, stages)]
             prod += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"producers{r}"),
-                     ("owns", f"empty{st}@{r}", k, f"producers{r}"), ("write", f"A{st}@{r}", k),
-                     ("arrive", target.format(st), k, npw, f"producers{r}")]
+                     ("owns", f"empty{st}@{r}", k, f"producers{r}"), ("write", f"A{st}@{r}", k)]
+            if not split:  # stride 2: the producers form B_lo after their halo barrier
+                prod.append(("write", f"B{st}@{r}", k))
+            prod.append(("arrive", target.format(st), k, npw, f"producers{r}"))
             spl += [("wait", f"tma{st}@{r}", k & 1, k + 1, f"split{r}"),
                     ("owns", f"empty{st}@{r}", k, f"split{r}"), ("write", f"B{st}@{r}", k),
                     ("arrive", target.format(st), k, split, f"split{r}")]
@@ -776,7 +778,8 @@ def conv1d_pair_abort_kernel(T, NK, stages=3, npw=8, split=2):
             if t == T - 1:
                 epi.append(("arrive", f"last@{r}", 0, 4, f"epilogue{r}"))
             epi.append(("arrive", f"aempty{buf}@0", bk, 4, f"epilogue{r}"))
-        sim.roles += [(tma, [("tma_drain2", r, stages, f"tma{r}")]), (prod, []), (spl, []), (epi, [])]
+        sim.roles += [(tma, [("tma_drain2", r, stages, f"tma{r}")]), (prod, [])] + ([(spl, [])] if split else []) + \
+            [(epi, [])]
     rel = []
     for seq in range(n):
         st, k = seq % stages, seq // stages
@@ -808,8 +811,9 @@ def test_conv1d_pair_abort_leaves_nothing_in_flight(T, NK):
     MMA is in flight; without an abort the protocol runs to the end."""
     aborted = 0
     for seed in range(40):
-        conv1d_pair_abort_kernel(T, NK).run(seed)
-        aborted += conv1d_pair_abort_kernel(T, NK).run(seed, p_abort=0.05)
+        for split in (2, 0):  # stride 1 (pw split warps) and stride 2 (the producers form B_lo)
+            conv1d_pair_abort_kernel(T, NK, split=split).run(seed)
+            aborted += conv1d_pair_abort_kernel(T, NK, split=split).run(seed, p_abort=0.05)
     assert aborted > 0
 
 
