@@ -637,7 +637,7 @@ def run_gpu(args):
                                               CASE_B.pad)
             achieved = 2 * pw_macs_b / tb_s / 1e12
             if algo_b == fcv.CONV1D_TC2_3XTF32:
-                kname, tkey = "tc2::dwsep_conv1d_tc2_kernel<9, 0>", "dwsep_conv1d_tc2"
+                kname, tkey = "tc2::dwsep_conv1d_tc2_kernel<9, 0, 1>", "dwsep_conv1d_tc2"
             else:
                 kname, tkey = "tcx::dwsep_conv1d_tcx_kernel<9, 0, 1, 256>", "dwsep_conv1d"
             roof = {"kernel": kname, "bound": "tensor", "achieved": achieved,
